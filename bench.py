@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE expert-MLP + Split-LoRA layer, forward + backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one pass of the whole hot path on one batch: top-k routing,
+counting-sort permute, grouped GEMM forward (gate_up + SwiGLU, down, Split-LoRA
+fused), weighted combine, grouped GEMM backward (dX, dA, dB with W frozen) and
+the dX combine.  Default workload: the Qwen3-30B-A3B-shaped layer (T=4096,
+m=2048, n=768, E=128, k=8, r=16), synthetic seeded inputs resident in HBM.
+
+N > 1 (torchrun, one process per GPU): data parallel.  Every rank runs its own
+batch of T tokens against the same expert weights and the adapter gradients
+are summed across ranks with one NCCL all-reduce per step (weak scaling).
+
+Rank 0 prints ONE JSON line.  `--impl reference` times the fp64 CPU oracle on
+bounded token samples of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from moe_inputs import CONFIGS, generate, generate_tokens  # noqa: E402
+from mixture_experts_lora_b200 import accounting as acc  # noqa: E402
+
+METRIC = "MoE-layer fwd+bwd tokens/s and TFLOP/s as % of B200 bf16 dense peak"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20          # > 126 MB L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="qwen3_30b_a3b", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=0,
+                    help="tokens per oracle sample (0: sized for ~15 s)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_name(cfg):
+    return (f"{cfg.name}: MoE expert-MLP + Split-LoRA layer fwd+bwd, T={cfg.T} m={cfg.m} "
+            f"n={cfg.n} E={cfg.E} k={cfg.k} r={cfg.r} alpha={cfg.alpha:g}")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                             "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                             "sw_power": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ---------------------------------------------------------------- accounting
+def kernel_work(cfg):
+    """Algorithmic work of each kernel kind for one step: (unit, amount per step)."""
+    T, m, n, E, k, r = cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r
+    P = T * k
+    wgrad_bytes = 2 * (P * n + P * m + P * 2 * n + P * m) + 4 * P * r * 2 + E * r * (2 * m + 3 * n) * 2
+    return {
+        "gemm_gateup_fwd": ("flop", acc.flops_gemm_gate_up_fwd(T, m, n, k, r)),
+        "gemm_down_fwd": ("flop", acc.flops_gemm_down_fwd(T, m, n, k, r)),
+        "gemm_down_bwd": ("flop", acc.flops_gemm_down_bwd(T, m, n, k, r)),
+        "gemm_gateup_bwd": ("flop", acc.flops_gemm_gate_up_bwd(T, m, n, k, r)),
+        "lora_wgrad": ("byte", wgrad_bytes),
+        "route_topk": ("byte", acc.bytes_route(T, E, k)),
+        "gather_rows": ("byte", 3 * acc.bytes_gather(T, m, k)),       # X fwd, w*dY and X bwd
+        "unpermute_combine": ("byte", 2 * acc.bytes_combine(T, m, k)),  # Y and dX
+    }
+
+
+def src_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixture_experts_lora_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, cfg_name: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, or None if
+    there is none for this workload or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("src_hash") != src_hash():
+        return None
+    ent = d.get("kernels", {}).get(cfg_name, {}).get(kernel)
+    return None if ent is None else ent.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        nums = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if nums:
+            return max(nums)
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle_sample(cfg, cpu_inp, W64, tok0, ntok):
+    """Forward + backward of the oracle on tokens [tok0, tok0 + ntok) of the workload."""
+    import numpy as np
+    import oracle.moe_lora_oracle as O
+    sl = slice(tok0, tok0 + ntok)
+    inp = dict(W64)
+    inp["logits"] = cpu_inp["logits"][sl].numpy().astype(np.float32)
+    inp["X"] = O.to64(cpu_inp["X"][sl])
+    dY = O.to64(cpu_inp["dY"][sl])
+    t0 = time.perf_counter()
+    Y, aux = O.moe_forward(inp, cfg.k, cfg.scale)
+    O.moe_backward(inp, aux, dY, cfg.k, cfg.scale)
+    return time.perf_counter() - t0
+
+
+def oracle_setup(cfg, cpu_inp):
+    import oracle.moe_lora_oracle as O
+    return {k: O.to64(cpu_inp[k]) for k in ("W_gu", "W_d", "A_gu", "B_gu", "A_d", "B_d")}
+
+
+def pick_sample_tokens(cfg, cpu_inp, W64, target_s, requested):
+    if requested > 0:
+        return requested
+    t = time_oracle_sample(cfg, cpu_inp, W64, 0, 8)
+    per_tok = max(t / 8, 1e-4)
+    return int(max(8, min(cfg.T, target_s / per_tok)))
+
+
+def cpu_baseline(cfg, cpu_inp, requested, target_s=15.0):
+    W64 = oracle_setup(cfg, cpu_inp)
+    ntok = pick_sample_tokens(cfg, cpu_inp, W64, target_s, requested)
+    dt = time_oracle_sample(cfg, cpu_inp, W64, 0, ntok)
+    return {"value": ntok / dt, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle fwd+bwd on the first {ntok} of {cfg.T} tokens of the "
+                      f"same workload (all {cfg.E} experts' weights), {dt:.1f} s wall clock; "
+                      f"fp64 weight conversion done once outside the timing"}
+
+
+def run_reference(args, cfg):
+    """The oracle arm: rank 0 only; other ranks exit without work."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    cpu = generate(cfg, seed=0, device="cpu")
+    W64 = oracle_setup(cfg, cpu)
+    ntok = pick_sample_tokens(cfg, cpu, W64, 2.0, args.cpu_sample_tokens)
+    for s in range(args.warmup):
+        time_oracle_sample(cfg, cpu, W64, (s * ntok) % max(1, cfg.T - ntok), ntok)
+    times = []
+    for s in range(args.steps):
+        times.append(time_oracle_sample(cfg, cpu, W64, (s * ntok) % max(1, cfg.T - ntok), ntok))
+    step_s = statistics.mean(times)
+    value = ntok / step_s
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_name(cfg),
+                                        "tokens_per_step_sample": ntok},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{ntok} tokens per step of the {cfg.T}-token workload"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, cfg):
+    import torch.distributed as dist
+    import mixture_experts_lora_b200 as ml
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    ml.lib()  # fails loudly if the CUDA library is missing
+
+    # inputs: weights shared by every rank (seed 0), tokens per rank
+    inp = generate(cfg, seed=0, device=str(dev))
+    if rank > 0:
+        inp.update(generate_tokens(cfg, seed=1000 + rank, device=str(dev)))
+    buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale, device=dev)
+    grads = (buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ml.layer_step(inp, cfg.k, cfg.scale, buf)
+        if world > 1:
+            for g in grads:
+                dist.all_reduce(g)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = ml.moe_get_device_error()
+    if st != ml.MOE_OK:
+        raise SystemExit(f"device error after warm-up: {ml.status_string(st)}")
+
+    # ---- timed region (device time, CUDA events per step, L2 flushed before each step)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ml.moe_profile_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ml.moe_profile_enable(False)
+    prof = ml.moe_profile_read()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    mean_ms = statistics.mean(step_ms)
+    if world > 1:
+        t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = float(t.item())
+    st = ml.moe_get_device_error()
+    if st != ml.MOE_OK:
+        raise SystemExit(f"device error in timed region: {ml.status_string(st)}")
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        h_in = {k: inp[k].cpu().pin_memory() for k in ("logits", "X", "dY")}
+        d_in = dict(inp)
+        d_in.update({k: torch.empty_like(inp[k]) for k in ("logits", "X", "dY")})
+        outs = (buf.Y, buf.dX) + grads
+        h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(t.numel() * t.element_size() for t in h_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+
+        def e2e_step():
+            for k, v in h_in.items():
+                d_in[k].copy_(v, non_blocking=True)
+            ml.layer_step(d_in, cfg.k, cfg.scale, buf)
+            if world > 1:
+                for g in grads:
+                    dist.all_reduce(g)
+            for o, h in zip(outs, h_out):
+                h.copy_(o, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * cfg.T / (e_ms / 1e3), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    # ---- report
+    peaks, peak_src = load_peaks()
+    flops = acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r)
+    tflops = flops / (mean_ms / 1e3) / 1e12
+    work = kernel_work(cfg)
+    kernels = {}
+    for name, (launches, tot_ms) in prof.items():
+        per_launch_ms = tot_ms / launches
+        ent = {"launches": launches, "ms_per_step": tot_ms / args.steps,
+               "share": tot_ms / max(1e-9, sum(v[1] for v in prof.values()))}
+        if name in work:
+            unit, amount = work[name]
+            per_launch = amount * args.steps / launches
+            if unit == "flop":
+                ent.update(bound="tensor", achieved=per_launch / (per_launch_ms / 1e3) / 1e12,
+                           unit="TFLOP/s", peak=peaks["bf16_tflops_sustained"])
+            else:
+                ent.update(bound="hbm", achieved=per_launch / (per_launch_ms / 1e3) / 1e9,
+                           unit="GB/s", peak=peaks["hbm_gbs"])
+            ent["frac"] = ent["achieved"] / ent["peak"]
+            ent["algorithmic_per_launch"] = per_launch
+        kernels[name] = ent
+    top = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
+    roof = None
+    if top is not None and "bound" in kernels[top]:
+        kt = kernels[top]
+        roof = {"kernel": top, "bound": kt["bound"], "achieved": kt["achieved"], "peak": kt["peak"],
+                "unit": kt["unit"], "frac": kt["frac"],
+                "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kt['bound'] == 'tensor' else 'hbm_gbs'}, MEASURED_PEAKS.json)",
+                "traffic": ncu_traffic(top, cfg.name)}
+    launches_total = sum(v[0] for v in prof.values())
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu_inp = {k: v.cpu() for k, v in inp.items()}
+        cpu = cpu_baseline(cfg, cpu_inp, args.cpu_sample_tokens)
+    line = {
+        "metric": METRIC, "value": world * cfg.T / (mean_ms / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; layer shapes of the named model family, random weights)",
+        "config": {"workload": workload_name(cfg), "tokens_per_rank": cfg.T,
+                   "global_tokens": world * cfg.T, "parallelism": f"dp{world}",
+                   "l2": "flushed before every timed step (256 MiB write outside the step events)",
+                   "lora_scale": cfg.scale},
+        "tflops": tflops,
+        "pct_bf16_peak": {"burst": tflops / peaks["bf16_tflops"],
+                          "sustained": tflops / peaks["bf16_tflops_sustained"],
+                          "source": peak_src},
+        "algorithmic_flop_per_step": flops,
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": launches_total,
+        "step_ms_min_max": [min(step_ms), max(step_ms)],
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    cfg = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

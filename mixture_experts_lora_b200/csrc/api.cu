@@ -1,0 +1,340 @@
+// C ABI of the layer (include/moelora.h): argument checks, workspace layout and
+// the launch sequence of each call.  Every call is asynchronous on the caller's
+// stream; the library allocates nothing.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// Device status word (one per device); kernels set it with atomicCAS, the host
+// reads and clears it in moe_get_device_error().
+__device__ int g_moe_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kTileRows = 128;
+
+int* status_ptr() {
+  static int* ptrs[kMaxDevices] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int device_sms() {
+  static int sms[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (sms[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
+inline int rank_padded(int r) { return r <= 16 ? 16 : 32; }
+
+inline int64_t chunk_rows_for(int64_t P) {
+  if (P <= 65536) return 256;
+  if (P <= 131072) return 1024;
+  return 2048;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_dims(const moe_dims_t* d) {
+  if (d == nullptr) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0) return MOE_ERR_INVALID_ARG;
+  if (!std::isfinite(d->scale)) return MOE_ERR_INVALID_ARG;
+  if (d->k < 1 || d->k > 32 || d->E < d->k || d->E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (d->m < 16 || d->n < 16 || d->m % 16 != 0 || d->n % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->r < 8 || d->r > 32 || d->r % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->T * (int64_t)d->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  // largest row index times the widest row must stay within 32-bit tile coordinates
+  if ((int64_t)d->m > (1 << 20) || (int64_t)d->n > (1 << 19)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Workspace regions (byte offsets), one layout for every call.
+struct Layout {
+  int64_t P;
+  int rp;
+  int max_row_tiles, max_chunks, chunk_rows, perm_chunks;
+  size_t hist, tiles, n_tiles, chunks, n_chunks, chunk_start;
+  size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
+  size_t rows, dgu, t1, t2, partial;
+  size_t total;
+};
+
+Layout make_layout(const moe_dims_t& d) {
+  Layout L{};
+  L.P = d.T * d.k;
+  L.rp = rank_padded(d.r);
+  L.max_row_tiles = (int)((L.P + kTileRows - 1) / kTileRows) + d.E;
+  L.chunk_rows = (int)chunk_rows_for(L.P);
+  L.max_chunks = (int)((L.P + L.chunk_rows - 1) / L.chunk_rows) + d.E;
+  L.perm_chunks = (int)((L.P + kPermuteChunk - 1) / kPermuteChunk);
+  const bool pad = d.r != L.rp;
+  const size_t E = d.E, m = d.m, n = d.n, rp = L.rp, P = (size_t)L.P;
+  const size_t dmax = m > 2 * n ? m : 2 * n;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  L.hist = take((size_t)L.perm_chunks * E * 4 + 4);
+  L.tiles = take((size_t)L.max_row_tiles * sizeof(TileInfo));
+  L.n_tiles = take(4);
+  L.chunks = take((size_t)L.max_chunks * sizeof(TileInfo));
+  L.n_chunks = take(4);
+  L.chunk_start = take((E + 1) * 4);
+  L.pad_A_gu = take(pad ? E * m * rp * 2 : 0);
+  L.pad_B_gu = take(pad ? E * rp * 2 * n * 2 : 0);
+  L.pad_A_d = take(pad ? E * n * rp * 2 : 0);
+  L.pad_B_d = take(pad ? E * rp * m * 2 : 0);
+  L.rows = take(P * m * 2);
+  L.dgu = take(P * 2 * n * 2);
+  L.t1 = take(P * rp * 2);
+  L.t2 = take(P * rp * 2);
+  L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
+  L.total = off;
+  return L;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                                  \
+  do {                                                 \
+    cudaError_t e_ = (expr);                           \
+    if (e_ != cudaSuccess) return MOE_ERR_CUDA;        \
+  } while (0)
+
+// Common set-up of the grouped GEMMs: tables, padded adapters, operand pointers.
+moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32_t* offsets,
+                     const uint16_t* W_gu, const uint16_t* W_d, const uint16_t* A_gu,
+                     const uint16_t* B_gu, const uint16_t* A_d, const uint16_t* B_d,
+                     bool with_chunks, cudaStream_t s, GemmShape* g, LayerPtrs* w) {
+  int* err = status_ptr();
+  if (err == nullptr) return MOE_ERR_CUDA;
+  MOE_TRY(launch_build_tables(offsets, d.E, kTileRows, at<TileInfo>(ws, L.tiles),
+                              at<int>(ws, L.n_tiles), L.chunk_rows,
+                              with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
+                              at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start), s));
+  w->W_gu = W_gu;
+  w->W_d = W_d;
+  if (d.r != L.rp) {
+    uint16_t* pa = at<uint16_t>(ws, L.pad_A_gu);
+    uint16_t* pb = at<uint16_t>(ws, L.pad_B_gu);
+    uint16_t* pc = at<uint16_t>(ws, L.pad_A_d);
+    uint16_t* pd = at<uint16_t>(ws, L.pad_B_d);
+    MOE_TRY(launch_pad3(A_gu, d.E, d.m, d.r, d.m, L.rp, pa, s));
+    MOE_TRY(launch_pad3(B_gu, d.E, d.r, 2 * d.n, L.rp, 2 * d.n, pb, s));
+    MOE_TRY(launch_pad3(A_d, d.E, d.n, d.r, d.n, L.rp, pc, s));
+    MOE_TRY(launch_pad3(B_d, d.E, d.r, d.m, L.rp, d.m, pd, s));
+    w->A_gu = pa; w->B_gu = pb; w->A_d = pc; w->B_d = pd;
+  } else {
+    w->A_gu = A_gu; w->B_gu = B_gu; w->A_d = A_d; w->B_d = B_d;
+  }
+  g->P = L.P;
+  g->m = d.m;
+  g->n = d.n;
+  g->E = d.E;
+  g->r = d.r;
+  g->rp = L.rp;
+  g->scale = d.scale;
+  g->max_row_tiles = L.max_row_tiles;
+  g->tiles = at<TileInfo>(ws, L.tiles);
+  g->n_row_tiles = at<int>(ws, L.n_tiles);
+  g->err = err;
+  g->num_sms = device_sms();
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_dims_t* dims) {
+  if (check_dims(dims) != MOE_OK) return 0;
+  return make_layout(*dims).total;
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_INDEX: return "expert id out of range (device)";
+    case MOE_ERR_TIMEOUT: return "bounded wait expired (device)";
+  }
+  return "unknown status";
+}
+
+moe_status_t moe_get_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int* p = status_ptr();
+  if (p == nullptr) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status_t>(v);
+}
+
+moe_status_t moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k,
+                            int32_t* topk_ids, float* topk_w, void* stream) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > 32 || E < k || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route_topk(logits, T, E, k, topk_ids, topk_w, status_ptr(),
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E, int32_t* counts,
+                         int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > 32 || E < k || E > 1024) return MOE_ERR_UNSUPPORTED;
+  const int64_t P = T * (int64_t)k;
+  if (P >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if (P > 0 && (topk_ids == nullptr || sorted_pairs == nullptr || pair_pos == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = align256((size_t)((P + kPermuteChunk - 1) / kPermuteChunk) * E * 4 + 4);
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  int* err = status_ptr();
+  if (err == nullptr) return MOE_ERR_CUDA;
+  return cuda_status(launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos,
+                                    static_cast<int32_t*>(ws), err,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t* X,
+                                       const int32_t* sorted_pairs, const int32_t* offsets,
+                                       const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
+                                       const moe_bf16_t* A_gu, const moe_bf16_t* B_gu,
+                                       const moe_bf16_t* A_d, const moe_bf16_t* B_d,
+                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_GU,
+                                       moe_bf16_t* save_H, moe_bf16_t* save_XA,
+                                       moe_bf16_t* save_HA, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t d = *dims;
+  if (d.T == 0) return MOE_OK;
+  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_GU, save_H, save_XA,
+                        save_HA, ws};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  GemmShape g;
+  LayerPtrs w;
+  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, s, &g, &w);
+  if (st != MOE_OK) return st;
+  uint16_t* xs = at<uint16_t>(ws, L.rows);
+  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, xs, s));
+  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, save_GU, save_H, save_XA, s));
+  MOE_TRY(launch_gemm_down_fwd(g, w, save_H, Y_sorted, save_HA, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_grouped_gemm_lora_bwd(
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
+    const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
+    moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
+    size_t ws_bytes, void* stream) {
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t d = *dims;
+  const void* outs[] = {dA_gu, dB_gu, dA_d, dB_d};
+  for (const void* p : outs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t E = d.E, m = d.m, n = d.n, r = d.r;
+  if (d.T == 0) {
+    MOE_TRY(launch_zero(dA_gu, E * m * r * 2, s));
+    MOE_TRY(launch_zero(dB_gu, E * r * 2 * n * 2, s));
+    MOE_TRY(launch_zero(dA_d, E * n * r * 2, s));
+    MOE_TRY(launch_zero(dB_d, E * r * m * 2, s));
+    return MOE_OK;
+  }
+  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA, save_HA,
+                       dX_sorted, ws};
+  for (const void* p : ins)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (topk_w == nullptr || sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  GemmShape g;
+  LayerPtrs w;
+  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, s, &g, &w);
+  if (st != MOE_OK) return st;
+  uint16_t* rows = at<uint16_t>(ws, L.rows);
+  uint16_t* dgu = at<uint16_t>(ws, L.dgu);
+  uint16_t* t1 = at<uint16_t>(ws, L.t1);
+  uint16_t* t2 = at<uint16_t>(ws, L.t2);
+  float* partial = at<float>(ws, L.partial);
+  const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
+  const int* n_chunks = at<int>(ws, L.n_chunks);
+  const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
+  // dy = w * dY[t] in sorted order
+  MOE_TRY(launch_gather_rows(dY, sorted_pairs, topk_w, L.P, d.k, d.m, rows, s));
+  // down projection: dGU (SwiGLU backward fused), T1 = dy B_d^T
+  MOE_TRY(launch_gemm_down_bwd(g, w, rows, save_GU, dgu, t1, s));
+  // dA_d = c H^T T1 ; dB_d = c HA^T dy
+  MOE_TRY(launch_lora_wgrad(g, save_H, d.n, t1, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
+                            partial, false, dA_d, s));
+  MOE_TRY(launch_lora_wgrad(g, rows, d.m, save_HA, d.r, chunks, n_chunks, L.max_chunks,
+                            chunk_start, partial, true, dB_d, s));
+  // gate_up projection: dX_sorted, T2 = dGU B_gu^T
+  MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, dX_sorted, t2, s));
+  // dB_gu = c XA^T dGU
+  MOE_TRY(launch_lora_wgrad(g, dgu, 2 * d.n, save_XA, d.r, chunks, n_chunks, L.max_chunks,
+                            chunk_start, partial, true, dB_gu, s));
+  // dA_gu = c X^T T2 (X re-gathered into the row buffer, dy no longer needed)
+  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
+  MOE_TRY(launch_lora_wgrad(g, rows, d.m, t2, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
+                            partial, false, dA_gu, s));
+  return MOE_OK;
+}
+
+moe_status_t moe_unpermute_combine(const moe_bf16_t* Y_sorted, const float* topk_w,
+                                   const int32_t* pair_pos, int64_t T, int32_t k, int32_t m,
+                                   moe_bf16_t* Y, void* stream) {
+  if (T < 0 || k < 1 || m < 8) return MOE_ERR_INVALID_ARG;
+  if (m % 8 != 0 || k > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!aligned16(Y_sorted) || !aligned16(Y) || pair_pos == nullptr) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_combine(Y_sorted, topk_w, pair_pos, T, k, m, Y, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

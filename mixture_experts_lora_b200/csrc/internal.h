@@ -1,0 +1,95 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moelora.h"
+
+namespace moe {
+
+struct TileInfo;
+
+// ---- kernel timing (profile.cu): while enabled, each launch is bracketed by
+// CUDA events on its stream and attributed to one of these kinds.
+enum KernelKind : int {
+  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
+  K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
+  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_NUM_KINDS
+};
+extern const char* const kKernelNames[K_NUM_KINDS];
+bool prof_enabled();
+void* prof_begin(int kind, cudaStream_t s);   // returns a record token (or nullptr)
+void prof_end(void* token, cudaStream_t s);
+
+struct ProfScope {
+  void* tok;
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t st) : tok(prof_enabled() ? prof_begin(kind, st) : nullptr), s(st) {}
+  ~ProfScope() { if (tok) prof_end(tok, s); }
+};
+
+// ---- SIMT kernels (simt_kernels.cu)
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
+                              float* w, int* err, cudaStream_t s);
+// per-warp chunks of kPermuteChunk pairs; hist holds n_chunks * E ints
+constexpr int kPermuteChunk = 1024;
+cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
+                           int32_t* hist, int* err, cudaStream_t s);
+// Row tiles of `tile_rows` rows per expert (grouped GEMMs) and row chunks of
+// `chunk_rows` rows per expert (adapter gradients), from offsets[E+1].
+cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
+                                int* n_tiles, int chunk_rows, TileInfo* chunks, int* n_chunks,
+                                int32_t* chunk_start, cudaStream_t s);
+// out[q] = (w ? bf16(w[p] * src[p / k]) : src[p / k]),  p = sorted_pairs[q]
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
+                               int64_t P, int k, int m, uint16_t* out, cudaStream_t s);
+cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_t* pair_pos,
+                           int64_t T, int k, int m, uint16_t* y, cudaStream_t s);
+// out [E, Ro, Co] = in [E, Ri, Ci] zero-padded (Ro >= Ri, Co >= Ci)
+cudaError_t launch_pad3(const uint16_t* in, int E, int Ri, int Ci, int Ro, int Co, uint16_t* out,
+                        cudaStream_t s);
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t s);
+
+// ---- tcgen05 GEMMs (gemm_launch.cu)
+struct LayerPtrs {
+  const uint16_t* W_gu;   // [E, m, 2n]
+  const uint16_t* W_d;    // [E, n, m]
+  const uint16_t* A_gu;   // [E, m, rp]   (padded copies when r < rp)
+  const uint16_t* B_gu;   // [E, rp, 2n]
+  const uint16_t* A_d;    // [E, n, rp]
+  const uint16_t* B_d;    // [E, rp, m]
+};
+
+struct GemmShape {
+  int64_t P;
+  int m, n, E, r, rp;
+  float scale;
+  int max_row_tiles;
+  const TileInfo* tiles;
+  const int* n_row_tiles;
+  int* err;
+  int num_sms;
+};
+
+// GU = Xs W_gu + c (Xs A_gu) B_gu; writes GU, H = silu(g) u, XA
+cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
+                                   uint16_t* GU, uint16_t* H, uint16_t* XA, cudaStream_t s);
+// Yp = H W_d + c (H A_d) B_d; writes Yp, HA
+cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
+                                 uint16_t* Yp, uint16_t* HA, cudaStream_t s);
+// dH = dy W_d^T + c (dy B_d^T) A_d^T -> dGU via SwiGLU backward with GU; writes T1 [P, rp]
+cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
+                                 const uint16_t* GU, uint16_t* dGU, uint16_t* T1, cudaStream_t s);
+// dXp = dGU W_gu^T + c (dGU B_gu^T) A_gu^T; writes dXp, T2 [P, rp]
+cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
+                                   uint16_t* dXp, uint16_t* T2, cudaStream_t s);
+// out = scale * sum_rows Big^T Small per expert, out [E, D, r] or (transpose) [E, r, D]
+cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, const uint16_t* small,
+                              int ld_small, const TileInfo* chunks, const int* n_chunks,
+                              int max_chunks, const int32_t* chunk_start, float* partial,
+                              bool transpose, uint16_t* out, cudaStream_t s);
+
+}  // namespace moe

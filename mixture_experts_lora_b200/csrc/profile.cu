@@ -1,0 +1,107 @@
+// Kernel timing for the benchmark and for tracing: while enabled, every launch
+// the library makes is bracketed by a pair of CUDA events recorded on the
+// launch stream.  moe_profile_read() waits for the events and reports, per
+// kernel kind, the number of launches and their summed device time.  Events
+// come from a pool that grows on demand and is reused; no device memory is
+// allocated.
+#include <mutex>
+#include <string.h>
+#include <vector>
+
+#include "internal.h"
+
+namespace moe {
+
+const char* const kKernelNames[K_NUM_KINDS] = {
+    "route_topk",        "permute_hist",      "permute_scan",     "permute_scatter",
+    "build_tables",      "pad_lora",          "gather_rows",      "gemm_gateup_fwd",
+    "gemm_down_fwd",     "gemm_down_bwd",     "gemm_gateup_bwd",  "lora_wgrad",
+    "lora_wgrad_reduce", "unpermute_combine", "memset"};
+
+namespace {
+struct Rec {
+  int kind;
+  cudaEvent_t a, b;
+  bool closed;
+};
+std::mutex g_mu;
+bool g_on = false;
+std::vector<Rec*> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+}  // namespace
+
+bool prof_enabled() { return g_on; }
+
+void* prof_begin(int kind, cudaStream_t s) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  Rec* r = new Rec{kind, take_event(), take_event(), false};
+  if (r->a == nullptr || r->b == nullptr) { delete r; return nullptr; }
+  cudaEventRecord(r->a, s);
+  g_recs.push_back(r);
+  return r;
+}
+
+void prof_end(void* token, cudaStream_t s) {
+  Rec* r = static_cast<Rec*>(token);
+  cudaEventRecord(r->b, s);
+  std::lock_guard<std::mutex> lk(g_mu);
+  r->closed = true;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+void moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_on = on != 0;
+}
+
+int moe_profile_read(int max_kinds, char* names, int name_len, int* launches, double* total_ms) {
+  std::vector<int> cnt(K_NUM_KINDS, 0);
+  std::vector<double> ms(K_NUM_KINDS, 0.0);
+  std::vector<Rec*> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    recs.swap(g_recs);
+  }
+  for (Rec* r : recs) {
+    float t = 0.f;
+    if (r->closed && cudaEventSynchronize(r->b) == cudaSuccess &&
+        cudaEventElapsedTime(&t, r->a, r->b) == cudaSuccess) {
+      cnt[r->kind] += 1;
+      ms[r->kind] += t;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_pool.push_back(r->a);
+    g_pool.push_back(r->b);
+    delete r;
+  }
+  int w = 0;
+  for (int k = 0; k < K_NUM_KINDS && w < max_kinds; ++k) {
+    if (cnt[k] == 0) continue;
+    if (names != nullptr && name_len > 0) {
+      strncpy(names + (size_t)w * name_len, kKernelNames[k], name_len - 1);
+      names[(size_t)w * name_len + name_len - 1] = 0;
+    }
+    if (launches) launches[w] = cnt[k];
+    if (total_ms) total_ms[w] = ms[k];
+    ++w;
+  }
+  return w;
+}
+
+}  // extern "C"

@@ -1,0 +1,401 @@
+// SIMT kernels of the layer: top-k routing, the stable counting-sort permute,
+// tile tables, row gather, weighted un-permute combine and LoRA padding.
+// All are HBM- or latency-bound; they use coalesced 16-byte accesses and warp
+// primitives, no floating-point atomics.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ routing
+// One warp per token.  Each lane holds logits e = lane + 32 i in shared memory;
+// k rounds of a warp arg-max on (value, lower index wins ties) pick the experts
+// in descending order; the weights are a softmax over the k picked logits.
+// Router equation: "Accelerating Mixture-of-Experts Fine-Tuning", section "The
+// Dynamic Dispatch Bottleneck in Mixture-of-Experts Architectures".
+__global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+                                  int32_t* __restrict__ ids, float* __restrict__ wout) {
+  extern __shared__ float s_logits[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;
+  float* row = s_logits + warp * E;
+  const float* src = logits + t * E;
+  for (int e = lane; e < E; e += 32) row[e] = src[e];
+  __syncwarp();
+  const int per_lane = (E + 31) >> 5;
+  uint32_t taken = 0;
+  float my_val = 0.f;
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    bool found = false;
+    float bv = 0.f;
+    int bi = 0x7fffffff;
+    for (int i = 0; i < per_lane; ++i) {
+      const int e = lane + 32 * i;
+      if (e >= E || ((taken >> i) & 1u)) continue;
+      const float v = row[e];
+      if (!found || v > bv) { bv = v; bi = e; found = true; }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      const bool of = __shfl_xor_sync(0xffffffffu, (int)found, off) != 0;
+      if (of && (!found || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; found = true; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) { my_val = bv; my_id = bi; }
+  }
+  const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
+  const float z = lane < k ? expf(my_val - vmax) : 0.f;
+  float sum = z;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < k) {
+    ids[t * k + lane] = my_id;
+    wout[t * k + lane] = z / sum;
+  }
+}
+
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w,
+                              int* err, cudaStream_t s) {
+  (void)err;
+  if (T == 0) return cudaSuccess;
+  const int warps = 8;
+  const int64_t blocks = (T + warps - 1) / warps;
+  const size_t smem = (size_t)warps * E * sizeof(float);
+  ProfScope ps(K_ROUTE, s);
+  route_topk_kernel<<<(unsigned)blocks, warps * 32, smem, s>>>(logits, T, E, k, ids, w);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ permute
+// Counting sort in three launches.  Pairs are cut into chunks of kPermuteChunk
+// consecutive pair indices, one warp per chunk:
+//   1. histogram of each chunk                       -> hist[c][e]
+//   2. one block: counts, exclusive offsets, and the first sorted position of
+//      each (chunk, expert) = offsets[e] + sum of earlier chunks  -> hist[c][e]
+//   3. each warp walks its chunk in pair order, 32 pairs at a time; lanes with
+//      the same expert are ranked with __match_any_sync, so positions are stable
+//      (ascending pair index inside every expert segment).
+// Replaces the per-expert mask lookup of the loop form ("What is
+// torch._grouped_mm?", Unsloth faster-moe docs).
+__global__ void permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E,
+                                    int32_t* __restrict__ hist, int* err) {
+  extern __shared__ int s_hist[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t chunk = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
+  if (chunk >= n_chunks) return;
+  int* h = s_hist + warp * E;
+  for (int e = lane; e < E; e += 32) h[e] = 0;
+  __syncwarp();
+  const int64_t p0 = chunk * kPermuteChunk;
+  const int64_t p1 = p0 + kPermuteChunk < P ? p0 + kPermuteChunk : P;
+  for (int64_t p = p0 + lane; p < p1; p += 32) {
+    const int e = ids[p];
+    if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+    else report_error(err, MOE_ERR_DEVICE_INDEX);
+  }
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) hist[chunk * E + e] = h[e];
+}
+
+__global__ void permute_scan_kernel(int32_t* __restrict__ hist, int64_t n_chunks, int E, int64_t P,
+                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int s_warp[32];
+  const int e = threadIdx.x;  // blockDim.x = 1024 >= E
+  int total = 0;
+  if (e < E) {
+    for (int64_t c = 0; c < n_chunks; ++c) {
+      const int v = hist[c * E + e];
+      hist[c * E + e] = total;
+      total += v;
+    }
+  }
+  // block exclusive scan of `total`
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = total;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = s_warp[lane];
+    int inc2 = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
+      if (lane >= off) inc2 += u;
+    }
+    s_warp[lane] = inc2 - v;
+  }
+  __syncthreads();
+  const int excl = incl - total + s_warp[warp];
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = excl;
+    for (int64_t c = 0; c < n_chunks; ++c) hist[c * E + e] += excl;
+  }
+  if (e == 0) offsets[E] = (int32_t)P;
+}
+
+__global__ void permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E,
+                                       const int32_t* __restrict__ base,
+                                       int32_t* __restrict__ sorted_pairs,
+                                       int32_t* __restrict__ pair_pos) {
+  extern __shared__ int s_run[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t chunk = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
+  if (chunk >= n_chunks) return;
+  int* run = s_run + warp * E;
+  for (int e = lane; e < E; e += 32) run[e] = base[chunk * E + e];
+  __syncwarp();
+  const int64_t p0 = chunk * kPermuteChunk;
+  const int64_t p1 = p0 + kPermuteChunk < P ? p0 + kPermuteChunk : P;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int64_t pb = p0; pb < p1; pb += 32) {
+    const int64_t p = pb + lane;
+    int e = -1;
+    if (p < p1) e = ids[p];
+    const bool ok = p < p1 && e >= 0 && e < E;
+    const int key = ok ? e : -1 - lane;  // invalid lanes never group
+    const unsigned grp = __match_any_sync(0xffffffffu, key);
+    int pos = 0;
+    if (ok) pos = run[e] + __popc(grp & lt_mask);
+    __syncwarp();
+    if (ok && (31 - __clz(grp)) == lane) run[e] += __popc(grp);
+    __syncwarp();
+    if (ok) {
+      sorted_pairs[pos] = (int32_t)p;
+      pair_pos[p] = pos;
+    }
+  }
+}
+
+cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* sorted_pairs, int32_t* pair_pos, int32_t* hist, int* err,
+                           cudaStream_t s) {
+  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
+  const int warps = 4;
+  const size_t smem = (size_t)warps * E * sizeof(int);
+  const unsigned blocks = (unsigned)((n_chunks + warps - 1) / warps);
+  if (n_chunks > 0) {
+    ProfScope ps(K_PERM_HIST, s);
+    permute_hist_kernel<<<blocks, warps * 32, smem, s>>>(ids, P, E, hist, err);
+    cudaError_t st = cudaGetLastError();
+    if (st != cudaSuccess) return st;
+  }
+  {
+    ProfScope ps(K_PERM_SCAN, s);
+    permute_scan_kernel<<<1, 1024, 0, s>>>(hist, n_chunks, E, P, counts, offsets);
+  }
+  cudaError_t st = cudaGetLastError();
+  if (st != cudaSuccess || n_chunks == 0) return st;
+  ProfScope ps(K_PERM_SCATTER, s);
+  permute_scatter_kernel<<<blocks, warps * 32, smem, s>>>(ids, P, E, hist, sorted_pairs, pair_pos);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ tile tables
+// From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
+// experts (grouped GEMMs), and row chunks of `chunk_rows` rows (adapter
+// gradients) with chunk_start[e] = first chunk of expert e.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int* total_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = s_warp[lane];
+    int inc2 = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
+      if (lane >= off) inc2 += u;
+    }
+    s_warp[lane] = inc2 - w;
+    if (lane == 31) s_warp[32] = inc2;
+  }
+  __syncthreads();
+  *total_out = s_warp[32];
+  return incl - v + s_warp[warp];
+}
+
+__global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, int tile_rows,
+                                    TileInfo* __restrict__ tiles, int* __restrict__ n_tiles,
+                                    int chunk_rows, TileInfo* __restrict__ chunks,
+                                    int* __restrict__ n_chunks, int32_t* __restrict__ chunk_start) {
+  __shared__ int s_warp[33];
+  const int e = threadIdx.x;
+  int lo = 0, hi = 0;
+  if (e < E) { lo = offsets[e]; hi = offsets[e + 1]; }
+  const int cnt = hi - lo;
+  int total;
+  const int nt = (cnt + tile_rows - 1) / tile_rows;
+  const int t0 = block_exclusive_scan_1024(nt, s_warp, &total);
+  for (int i = 0; i < nt; ++i) {
+    TileInfo ti;
+    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = hi; ti.pad = 0;
+    tiles[t0 + i] = ti;
+  }
+  if (threadIdx.x == 0) *n_tiles = total;
+  if (chunks != nullptr) {
+    const int nc = (cnt + chunk_rows - 1) / chunk_rows;
+    int ctotal;
+    const int c0 = block_exclusive_scan_1024(nc, s_warp, &ctotal);
+    for (int i = 0; i < nc; ++i) {
+      TileInfo ti;
+      ti.e = e;
+      ti.row0 = lo + i * chunk_rows;
+      ti.row_end = min(hi, lo + (i + 1) * chunk_rows);
+      ti.pad = 0;
+      chunks[c0 + i] = ti;
+    }
+    if (e < E) chunk_start[e] = c0;
+    if (threadIdx.x == 0) { *n_chunks = ctotal; chunk_start[E] = ctotal; }
+  }
+}
+
+cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
+                                int* n_tiles, int chunk_rows, TileInfo* chunks, int* n_chunks,
+                                int32_t* chunk_start, cudaStream_t s) {
+  ProfScope ps(K_TABLES, s);
+  build_tables_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_rows, tiles, n_tiles, chunk_rows, chunks,
+                                         n_chunks, chunk_start);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ gather
+// out[q, :] = src[p / k, :] (optionally scaled by w[p] before the bf16 rounding),
+// p = sorted_pairs[q].  One thread per 16-byte vector.
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ sp,
+                                   const float* __restrict__ w, int64_t P, int k, int vpr,
+                                   uint4* __restrict__ out) {
+  const int64_t total = P * vpr;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t q = i / vpr;
+    const int v = (int)(i - q * vpr);
+    const int p = sp[q];
+    uint4 x = src[(int64_t)(p / k) * vpr + v];
+    if (w != nullptr) {
+      const float s = w[p];
+      x.x = pack_bf16x2(s * bf16_lo(x.x), s * bf16_hi(x.x));
+      x.y = pack_bf16x2(s * bf16_lo(x.y), s * bf16_hi(x.y));
+      x.z = pack_bf16x2(s * bf16_lo(x.z), s * bf16_hi(x.z));
+      x.w = pack_bf16x2(s * bf16_lo(x.w), s * bf16_hi(x.w));
+    }
+    out[i] = x;
+  }
+}
+
+static int g_num_sms_cache = 0;
+static int num_sms() {
+  if (g_num_sms_cache == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms_cache, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms_cache <= 0) g_num_sms_cache = 148;
+  }
+  return g_num_sms_cache;
+}
+
+static unsigned grid_for(int64_t work, int threads) {
+  const int64_t want = (work + threads - 1) / threads;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  return (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
+                               int64_t P, int k, int m, uint16_t* out, cudaStream_t s) {
+  if (P == 0) return cudaSuccess;
+  const int vpr = m / 8;
+  ProfScope ps(K_GATHER, s);
+  gather_rows_kernel<<<grid_for(P * vpr, 256), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(src), sorted_pairs, w, P, k, vpr, reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ combine
+// y[t, :] = sum_j w[t, j] ysorted[pair_pos[t k + j], :], fp32 over ascending j,
+// one bf16 rounding; w == nullptr means every weight is 1.
+__global__ void combine_kernel(const uint4* __restrict__ ys, const float* __restrict__ w,
+                               const int32_t* __restrict__ pos, int64_t T, int k, int vpr,
+                               uint4* __restrict__ y) {
+  const int64_t total = T * vpr;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / vpr;
+    const int v = (int)(i - t * vpr);
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int64_t p = t * k + j;
+      const float s = w != nullptr ? w[p] : 1.0f;
+      const uint4 x = ys[(int64_t)pos[p] * vpr + v];
+      acc[0] += s * bf16_lo(x.x); acc[1] += s * bf16_hi(x.x);
+      acc[2] += s * bf16_lo(x.y); acc[3] += s * bf16_hi(x.y);
+      acc[4] += s * bf16_lo(x.z); acc[5] += s * bf16_hi(x.z);
+      acc[6] += s * bf16_lo(x.w); acc[7] += s * bf16_hi(x.w);
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    y[i] = o;
+  }
+}
+
+cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_t* pair_pos,
+                           int64_t T, int k, int m, uint16_t* y, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int vpr = m / 8;
+  ProfScope ps(K_COMBINE, s);
+  combine_kernel<<<grid_for(T * vpr, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(ysorted), w,
+                                                        pair_pos, T, k, vpr,
+                                                        reinterpret_cast<uint4*>(y));
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ pad
+__global__ void pad3_kernel(const uint16_t* __restrict__ in, int E, int Ri, int Ci, int Ro, int Co,
+                            uint16_t* __restrict__ out) {
+  const int64_t total = (int64_t)E * Ro * Co;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % Co);
+    const int64_t rr = i / Co;
+    const int r = (int)(rr % Ro);
+    const int64_t e = rr / Ro;
+    out[i] = (r < Ri && c < Ci) ? in[(e * Ri + r) * Ci + c] : (uint16_t)0;
+  }
+}
+
+cudaError_t launch_pad3(const uint16_t* in, int E, int Ri, int Ci, int Ro, int Co, uint16_t* out,
+                        cudaStream_t s) {
+  ProfScope ps(K_PAD, s);
+  pad3_kernel<<<grid_for((int64_t)E * Ro * Co, 256), 256, 0, s>>>(in, E, Ri, Ci, Ro, Co, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t s) {
+  if (bytes == 0) return cudaSuccess;
+  ProfScope ps(K_MEMSET, s);
+  return cudaMemsetAsync(p, 0, bytes, s);
+}
+
+}  // namespace moe

@@ -109,3 +109,19 @@ def generate(cfg: LayerConfig | str, seed: int = 0, device: str = "cpu",
 def small_config(T=64, m=64, n=32, E=4, k=2, r=8, alpha=16.0, name="custom") -> LayerConfig:
     """A free-form small configuration (oracle pins, edge cases)."""
     return LayerConfig(name, T=T, m=m, n=n, E=E, k=k, r=r, alpha=alpha)
+
+
+def generate_tokens(cfg: LayerConfig | str, seed: int, device: str = "cpu") -> dict:
+    """Per-token inputs only (logits, X, dY) from their own seeded generator, with
+    the same distributions as generate(); used to give data-parallel ranks their
+    own batch while the expert weights stay shared."""
+    if isinstance(cfg, str):
+        cfg = CONFIGS[cfg]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    logits = _normal(gen, (cfg.T, cfg.E), 1.0, device)
+    if cfg.zipf_s > 0:
+        logits = logits + zipf_logit_bias(cfg.E, cfg.zipf_s, cfg.bias_scale).to(device)
+    return {"logits": logits.contiguous(),
+            "X": _normal(gen, (cfg.T, cfg.m), 1.0, device).to(torch.bfloat16),
+            "dY": _normal(gen, (cfg.T, cfg.m), 1.0, device).to(torch.bfloat16)}

@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bit-exact: expert ids, counts, offsets, sorted_pairs, pair_pos.
+Floating point: max|gpu - oracle| / max|oracle| <= 1e-2 per bf16 output tensor
+(fp32 accumulation, bf16 storage), routing weights within 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mixture_experts_lora_b200 as ml
+import oracle.moe_lora_oracle as O
+from moe_inputs import CONFIGS, small_config, generate
+
+from gpu_common import (TOL, TOL_W, check_full_parity, check_sampled_parity, ensure_built,
+                        inputs_on, rel_err, run_layer, to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    ensure_built()
+
+
+# ------------------------------------------------------------------ routing
+@pytest.mark.parametrize("T,E,k", [(300, 64, 8), (37, 8, 8), (64, 1024, 32), (5, 128, 1), (129, 33, 3)])
+def test_route_topk_bitexact_with_ties(T, E, k):
+    g = torch.Generator().manual_seed(T * 1000 + E)
+    logits = (torch.randn(T, E, generator=g) * 2).round() / 2        # many exact ties
+    logits[0] = 0.0                                                  # a fully tied row
+    ids = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    ml.moe_route_topk(logits.cuda(), k, ids, w)
+    torch.cuda.synchronize()
+    rid, rw = O.route_topk(logits.numpy(), k)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    assert rel_err(to_np(w), rw) <= TOL_W
+    assert np.array_equal(ids[0].cpu().numpy(), np.arange(k))
+
+
+# ------------------------------------------------------------------ permute
+@pytest.mark.parametrize("T,k,E,hot", [(1500, 3, 7, True), (4096, 8, 128, False), (33, 1, 1024, False),
+                                        (2000, 4, 16, True)])
+def test_permute_bitexact(T, k, E, hot):
+    rng = np.random.default_rng(T + E)
+    ids = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    if hot:
+        ids[:, 0] = 1
+        ids[:, 1:][ids[:, 1:] == 1] = 0
+    ids_d = torch.from_numpy(ids).cuda()
+    P = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(P, dtype=torch.int32, device="cuda")
+    pos = torch.empty(P, dtype=torch.int32, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    ml.moe_permute(ids_d, E, counts, offsets, sp, pos, ws)
+    assert ml.moe_get_device_error() == ml.MOE_OK
+    rc, ro, rsp, rpos = O.permute(ids, E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(sp.cpu().numpy(), rsp)
+    assert np.array_equal(pos.cpu().numpy(), rpos)
+
+
+def test_permute_reports_bad_expert_id_without_faulting():
+    ids = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device="cuda")   # 7 >= E
+    E = 4
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sp = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    pos = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    ws = torch.empty(1 << 16, dtype=torch.uint8, device="cuda")
+    ml.moe_permute(ids, E, counts, offsets, sp, pos, ws)
+    assert ml.moe_get_device_error() == ml.MOE_ERR_DEVICE_INDEX
+    assert ml.moe_get_device_error() == ml.MOE_OK        # cleared after reading
+    assert counts.cpu().tolist() == [1, 1, 1, 0]
+
+
+# ------------------------------------------------------------------ combine
+@pytest.mark.parametrize("weighted", [True, False])
+def test_unpermute_combine(weighted):
+    T, k, m = 333, 4, 200
+    g = torch.Generator().manual_seed(7)
+    ys = torch.randn(T * k, m, generator=g).to(torch.bfloat16)
+    w = torch.rand(T, k, generator=g)
+    pos = torch.randperm(T * k, generator=g).to(torch.int32)
+    y = torch.empty(T, m, dtype=torch.bfloat16, device="cuda")
+    ml.moe_unpermute_combine(ys.cuda(), w.cuda() if weighted else None, pos.cuda(), T, k, m, y)
+    torch.cuda.synchronize()
+    ys64 = ys.double().numpy()
+    pos_n = pos.numpy().astype(np.int64)
+    ref = np.zeros((T, m))
+    for j in range(k):
+        wj = w[:, j].double().numpy()[:, None] if weighted else 1.0
+        ref += wj * ys64[pos_n[np.arange(T) * k + j]]
+    # one bf16 rounding of an fp32 sum: within one bf16 ulp of the value
+    assert np.all(np.abs(to_np(y) - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+
+
+# ------------------------------------------------------------------ whole layer, tiny + edges
+def _layer_case(cfg, mutate=None, seed=0):
+    inp, cpu = inputs_on(cfg, seed=seed)
+    if mutate is not None:
+        mutate(cpu)
+        inp = {k: v.cuda().contiguous() for k, v in cpu.items()}
+    buf = run_layer(inp, cfg)
+    return check_full_parity(buf, cpu, cfg), buf
+
+
+def test_tiny_config_full_parity():
+    errs, _ = _layer_case(CONFIGS["tiny"])
+    print("tiny parity", errs)
+
+
+EDGE = {
+    "one_token": small_config(T=1, m=128, n=64, E=8, k=2, r=8, alpha=16),
+    "ragged_odd_dims_r16": small_config(T=100, m=144, n=80, E=6, k=2, r=16, alpha=16),
+    "partial_gate_tile": small_config(T=150, m=64, n=208, E=4, k=2, r=16, alpha=32),
+    "rank32": small_config(T=200, m=128, n=96, E=8, k=2, r=32, alpha=32),
+    "rank24_padded": small_config(T=90, m=96, n=48, E=5, k=3, r=24, alpha=48),
+    "k_equals_E": small_config(T=70, m=64, n=32, E=8, k=8, r=8, alpha=8),
+    "long_K": small_config(T=130, m=1024, n=320, E=4, k=2, r=16, alpha=16),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_case_full_parity(name):
+    errs, _ = _layer_case(EDGE[name])
+    print(name, errs)
+
+
+def test_hot_expert_and_empty_experts():
+    cfg = small_config(T=300, m=128, n=64, E=8, k=2, r=8, alpha=16)
+
+    def mutate(cpu):
+        cpu["logits"][:, 3] += 20.0          # every token picks expert 3 first
+        cpu["logits"][:, 5:] -= 20.0         # experts 5..7 get nothing
+    errs, buf = _layer_case(cfg, mutate)
+    counts = buf.counts.cpu().numpy()
+    assert counts[3] == 300 and counts[5:].sum() == 0
+
+
+def test_tied_logits_route_to_lowest_indices():
+    cfg = small_config(T=64, m=64, n=32, E=6, k=2, r=8, alpha=16)
+
+    def mutate(cpu):
+        cpu["logits"][:] = 0.0
+    errs, buf = _layer_case(cfg, mutate)
+    assert np.array_equal(buf.ids.cpu().numpy(), np.tile([0, 1], (64, 1)))
+
+
+def test_deterministic_bitwise():
+    cfg = CONFIGS["tiny"]
+    inp, cpu = inputs_on(cfg)
+    a = run_layer(inp, cfg)
+    snap = {k: getattr(a, k).clone() for k in ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU")}
+    b = run_layer(inp, cfg, buf=a)
+    for k, v in snap.items():
+        assert torch.equal(v.view(torch.int16) if v.dtype == torch.bfloat16 else v,
+                           getattr(b, k).view(torch.int16) if v.dtype == torch.bfloat16 else getattr(b, k)), k
+
+
+def test_empty_input():
+    cfg = small_config(T=0, m=64, n=32, E=4, k=2, r=8, alpha=16)
+    inp, cpu = inputs_on(cfg)
+    buf = ml.alloc_buffers(0, 64, 32, 4, 2, 8, 2.0)
+    buf.dA_gu.fill_(1.0)
+    ml.layer_step(inp, 2, 2.0, buf)
+    assert ml.moe_get_device_error() == ml.MOE_OK
+    assert buf.offsets.cpu().tolist() == [0] * 5
+    assert not torch.any(buf.dA_gu != 0)
+
+
+# ------------------------------------------------------------------ full sizes (sampled)
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b", "gpt_oss_20b", "qwen3_skewed"])
+def test_full_size_sampled_parity(name):
+    cfg = CONFIGS[name]
+    inp, cpu = inputs_on(cfg)
+    buf = run_layer(inp, cfg)
+    errs = check_sampled_parity(buf, cpu, cfg)
+    print(name, errs)
