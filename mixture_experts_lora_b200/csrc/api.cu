@@ -17,6 +17,7 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kTileRows = 128;
+constexpr int kGemmChunkRows = 256;
 
 int* status_ptr() {
   static int* ptrs[kMaxDevices] = {nullptr};
@@ -71,10 +72,10 @@ moe_status_t check_dims(const moe_dims_t* d) {
 struct Layout {
   int64_t P;
   int rp;
-  int max_row_tiles, max_chunks, chunk_rows, perm_chunks;
-  size_t hist, tiles, n_tiles, chunks, n_chunks, chunk_start;
+  int max_row_tiles, max_gchunks, max_chunks, chunk_rows, perm_chunks;
+  size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
   size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
-  size_t rows, dgu, t1, t2, partial;
+  size_t rows, dgu, t1, t2, lrc1, lrc2, partial;
   size_t total;
 };
 
@@ -83,6 +84,7 @@ Layout make_layout(const moe_dims_t& d) {
   L.P = d.T * d.k;
   L.rp = rank_padded(d.r);
   L.max_row_tiles = (int)((L.P + kTileRows - 1) / kTileRows) + d.E;
+  L.max_gchunks = (int)((L.P + kGemmChunkRows - 1) / kGemmChunkRows) + d.E;
   L.chunk_rows = (int)chunk_rows_for(L.P);
   L.max_chunks = (int)((L.P + L.chunk_rows - 1) / L.chunk_rows) + d.E;
   L.perm_chunks = (int)((L.P + kPermuteChunk - 1) / kPermuteChunk);
@@ -94,6 +96,8 @@ Layout make_layout(const moe_dims_t& d) {
   L.hist = take((size_t)L.perm_chunks * E * 4 + 4);
   L.tiles = take((size_t)L.max_row_tiles * sizeof(TileInfo));
   L.n_tiles = take(4);
+  L.gchunks = take((size_t)L.max_gchunks * sizeof(TileInfo));
+  L.n_gchunks = take(4);
   L.chunks = take((size_t)L.max_chunks * sizeof(TileInfo));
   L.n_chunks = take(4);
   L.chunk_start = take((E + 1) * 4);
@@ -105,6 +109,8 @@ Layout make_layout(const moe_dims_t& d) {
   L.dgu = take(P * 2 * n * 2);
   L.t1 = take(P * rp * 2);
   L.t2 = take(P * rp * 2);
+  L.lrc1 = take(P * rp * 2);
+  L.lrc2 = take(P * rp * 2);
   L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
   L.total = off;
   return L;
@@ -131,7 +137,8 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
   int* err = status_ptr();
   if (err == nullptr) return MOE_ERR_CUDA;
   MOE_TRY(launch_build_tables(offsets, d.E, kTileRows, at<TileInfo>(ws, L.tiles),
-                              at<int>(ws, L.n_tiles), L.chunk_rows,
+                              at<int>(ws, L.n_tiles), kGemmChunkRows, at<TileInfo>(ws, L.gchunks),
+                              at<int>(ws, L.n_gchunks), L.chunk_rows,
                               with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
                               at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start), s));
   w->W_gu = W_gu;
@@ -159,6 +166,9 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
   g->max_row_tiles = L.max_row_tiles;
   g->tiles = at<TileInfo>(ws, L.tiles);
   g->n_row_tiles = at<int>(ws, L.n_tiles);
+  g->max_gchunks = L.max_gchunks;
+  g->gchunks = at<TileInfo>(ws, L.gchunks);
+  g->n_gchunks = at<int>(ws, L.n_gchunks);
   g->err = err;
   g->num_sms = device_sms();
   return MOE_OK;
@@ -256,9 +266,15 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, s, &g, &w);
   if (st != MOE_OK) return st;
   uint16_t* xs = at<uint16_t>(ws, L.rows);
+  uint16_t* xac = at<uint16_t>(ws, L.lrc1);
+  uint16_t* hac = at<uint16_t>(ws, L.lrc2);
   MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, xs, s));
-  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, save_GU, save_H, save_XA, s));
-  MOE_TRY(launch_gemm_down_fwd(g, w, save_H, Y_sorted, save_HA, s));
+  // XA = X A_gu (saved) and bf16(c XA), then GU = X W_gu + (c XA) B_gu with SwiGLU
+  MOE_TRY(launch_lowrank(g, xs, d.m, w.A_gu, true, save_XA, d.r, d.r, xac, s));
+  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, xac, save_GU, save_H, s));
+  // HA = H A_d (saved) and bf16(c HA), then Y = H W_d + (c HA) B_d
+  MOE_TRY(launch_lowrank(g, save_H, d.n, w.A_d, true, save_HA, d.r, d.r, hac, s));
+  MOE_TRY(launch_gemm_down_fwd(g, w, save_H, hac, Y_sorted, s));
   return MOE_OK;
 }
 
@@ -304,17 +320,21 @@ moe_status_t moe_grouped_gemm_lora_bwd(
   const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
   const int* n_chunks = at<int>(ws, L.n_chunks);
   const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
+  uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
+  uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
   // dy = w * dY[t] in sorted order
   MOE_TRY(launch_gather_rows(dY, sorted_pairs, topk_w, L.P, d.k, d.m, rows, s));
-  // down projection: dGU (SwiGLU backward fused), T1 = dy B_d^T
-  MOE_TRY(launch_gemm_down_bwd(g, w, rows, save_GU, dgu, t1, s));
+  // T1 = dy B_d^T (saved for dA_d) and bf16(c T1); dH = dy W_d^T + (c T1) A_d^T -> dGU
+  MOE_TRY(launch_lowrank(g, rows, d.m, w.B_d, false, t1, L.rp, L.rp, lrc1, s));
+  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, save_GU, dgu, s));
   // dA_d = c H^T T1 ; dB_d = c HA^T dy
   MOE_TRY(launch_lora_wgrad(g, save_H, d.n, t1, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
                             partial, false, dA_d, s));
   MOE_TRY(launch_lora_wgrad(g, rows, d.m, save_HA, d.r, chunks, n_chunks, L.max_chunks,
                             chunk_start, partial, true, dB_d, s));
-  // gate_up projection: dX_sorted, T2 = dGU B_gu^T
-  MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, dX_sorted, t2, s));
+  // T2 = dGU B_gu^T and bf16(c T2); dX_sorted = dGU W_gu^T + (c T2) A_gu^T
+  MOE_TRY(launch_lowrank(g, dgu, 2 * d.n, w.B_gu, false, t2, L.rp, L.rp, lrc2, s));
+  MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
   // dB_gu = c XA^T dGU
   MOE_TRY(launch_lora_wgrad(g, dgu, 2 * d.n, save_XA, d.r, chunks, n_chunks, L.max_chunks,
                             chunk_start, partial, true, dB_gu, s));

@@ -7,6 +7,7 @@
 #include "grouped_gemm.cuh"
 #include "internal.h"
 #include "lora_wgrad.cuh"
+#include "lowrank.cuh"
 
 namespace moe {
 
@@ -72,115 +73,136 @@ cudaError_t ensure_smem(Kern kernel, int bytes) {
 }
 
 template <class C>
-cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& la, const CUtensorMap& lb, const GemmParams& p,
+cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap& tw, const CUtensorMap& ta,
+                        const CUtensorMap& tlw, const CUtensorMap& tlr, const GemmParams& p,
                         cudaStream_t s) {
   auto kern = moe_gemm_kernel<C>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
-  const int64_t tiles = (int64_t)g.max_row_tiles * p.n_tiles;
+  const int64_t tiles = (int64_t)g.max_gchunks * p.n_ftiles;
   const int grid = (int)(tiles < g.num_sms ? (tiles > 0 ? tiles : 1) : g.num_sms);
   ProfScope ps(kind, s);
-  kern<<<grid, 192, C::SMEM_BYTES, s>>>(a, b, la, lb, p);
+  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tw, ta, tlw, tlr, p);
   return cudaGetLastError();
 }
 
-GemmParams base_params(const GemmShape& g, int N, int K, int BN_tile) {
+GemmParams base_params(const GemmShape& g, int F, int K, int feat_per_tile) {
   GemmParams p{};
-  p.tiles = g.tiles;
-  p.n_row_tiles = g.n_row_tiles;
-  p.N = N;
+  p.chunks = g.gchunks;
+  p.n_chunks = g.n_gchunks;
+  p.F = F;
   p.K = K;
-  p.n_tiles = (N + BN_tile - 1) / BN_tile;
+  p.n_ftiles = (F + feat_per_tile - 1) / feat_per_tile;
   p.nk = (K + 63) / 64;
-  p.scale = g.scale;
   p.err = g.err;
   return p;
 }
 
 }  // namespace
 
-constexpr int kBnGateUpFwd = 192;   // 96 gate + 96 up columns
-constexpr int kBnDownFwd = 224;
-constexpr int kBnDownBwd = 192;
-constexpr int kBnGateUpBwd = 224;
+// Token-row operand boxes: 32 rows x 64 K (activations) or 32 rows x rp (LoRA operand).
+constexpr uint32_t kTokBox = 32;
 
 cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
-                                   uint16_t* GU, uint16_t* H, uint16_t* XA, cudaStream_t s) {
-  CUtensorMap a, b, la, lb;
+                                   const uint16_t* XAc, uint16_t* GU, uint16_t* H, cudaStream_t s) {
+  CUtensorMap tw, ta, tlw, tlr;
   const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode2d(&a, Xs, P, m, 128, 64) || !encode3d(&b, w.W_gu, E, m, 2 * n, 64, 32) ||
-      !encode3d(&la, w.A_gu, E, m, rp, 64, (uint32_t)rp) ||
-      !encode3d(&lb, w.B_gu, E, rp, 2 * n, (uint32_t)rp, 32))
+  if (!encode3d(&tw, w.W_gu, E, m, 2 * n, 64, 64) || !encode2d(&ta, Xs, P, m, kTokBox, 64) ||
+      !encode3d(&tlw, w.B_gu, E, rp, 2 * n, (uint32_t)rp, 64) ||
+      !encode2d(&tlr, XAc, P, rp, kTokBox, (uint32_t)rp))
     return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.n, g.m, kBnGateUpFwd / 2);
+  GemmParams p = base_params(g, g.n, g.m, 64);
   p.n_half = g.n;
   p.out0 = reinterpret_cast<__nv_bfloat16*>(GU);
   p.ld0 = 2 * g.n;
   p.out1 = reinterpret_cast<__nv_bfloat16*>(H);
   p.ld1 = g.n;
-  p.save_lr = reinterpret_cast<__nv_bfloat16*>(XA);
-  p.ld_lr = g.r;
-  p.r_lr = g.r;
-  if (g.rp == 16) return launch_gemm<GemmCfg<kBnGateUpFwd, true, 16, EPI_GATEUP_FWD>>(K_GEMM_GATEUP_FWD, g, a, b, la, lb, p, s);
-  return launch_gemm<GemmCfg<kBnGateUpFwd, true, 32, EPI_GATEUP_FWD>>(K_GEMM_GATEUP_FWD, g, a, b, la, lb, p, s);
+  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_GATEUP_FWD, true, 16>>(K_GEMM_GATEUP_FWD, g, tw, ta, tlw, tlr, p, s);
+  return launch_gemm<GemmCfg<EPI_GATEUP_FWD, true, 32>>(K_GEMM_GATEUP_FWD, g, tw, ta, tlw, tlr, p, s);
 }
 
 cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
-                                 uint16_t* Yp, uint16_t* HA, cudaStream_t s) {
-  CUtensorMap a, b, la, lb;
+                                 const uint16_t* HAc, uint16_t* Yp, cudaStream_t s) {
+  CUtensorMap tw, ta, tlw, tlr;
   const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode2d(&a, H, P, n, 128, 64) || !encode3d(&b, w.W_d, E, n, m, 64, 32) ||
-      !encode3d(&la, w.A_d, E, n, rp, 64, (uint32_t)rp) ||
-      !encode3d(&lb, w.B_d, E, rp, m, (uint32_t)rp, 32))
+  if (!encode3d(&tw, w.W_d, E, n, m, 64, 64) || !encode2d(&ta, H, P, n, kTokBox, 64) ||
+      !encode3d(&tlw, w.B_d, E, rp, m, (uint32_t)rp, 64) ||
+      !encode2d(&tlr, HAc, P, rp, kTokBox, (uint32_t)rp))
     return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.m, g.n, kBnDownFwd);
+  GemmParams p = base_params(g, g.m, g.n, 128);
   p.out0 = reinterpret_cast<__nv_bfloat16*>(Yp);
   p.ld0 = g.m;
-  p.save_lr = reinterpret_cast<__nv_bfloat16*>(HA);
-  p.ld_lr = g.r;
-  p.r_lr = g.r;
-  if (g.rp == 16) return launch_gemm<GemmCfg<kBnDownFwd, true, 16, EPI_STORE>>(K_GEMM_DOWN_FWD, g, a, b, la, lb, p, s);
-  return launch_gemm<GemmCfg<kBnDownFwd, true, 32, EPI_STORE>>(K_GEMM_DOWN_FWD, g, a, b, la, lb, p, s);
+  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_STORE, true, 16>>(K_GEMM_DOWN_FWD, g, tw, ta, tlw, tlr, p, s);
+  return launch_gemm<GemmCfg<EPI_STORE, true, 32>>(K_GEMM_DOWN_FWD, g, tw, ta, tlw, tlr, p, s);
 }
 
 cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
-                                 const uint16_t* GU, uint16_t* dGU, uint16_t* T1, cudaStream_t s) {
-  CUtensorMap a, b, la, lb;
+                                 const uint16_t* T1c, const uint16_t* GU, uint16_t* dGU,
+                                 cudaStream_t s) {
+  CUtensorMap tw, ta, tlw, tlr;
   const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode2d(&a, dys, P, m, 128, 64) || !encode3d(&b, w.W_d, E, n, m, kBnDownBwd, 64) ||
-      !encode3d(&la, w.B_d, E, rp, m, (uint32_t)rp, 64) ||
-      !encode3d(&lb, w.A_d, E, n, rp, kBnDownBwd, (uint32_t)rp))
+  if (!encode3d(&tw, w.W_d, E, n, m, 128, 64) || !encode2d(&ta, dys, P, m, kTokBox, 64) ||
+      !encode3d(&tlw, w.A_d, E, n, rp, 128, (uint32_t)rp) ||
+      !encode2d(&tlr, T1c, P, rp, kTokBox, (uint32_t)rp))
     return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.n, g.m, kBnDownBwd);
+  GemmParams p = base_params(g, g.n, g.m, 128);
   p.n_half = g.n;
   p.out0 = reinterpret_cast<__nv_bfloat16*>(dGU);
   p.ld0 = 2 * g.n;
   p.in0 = reinterpret_cast<const __nv_bfloat16*>(GU);
   p.ldi0 = 2 * g.n;
-  p.save_lr = reinterpret_cast<__nv_bfloat16*>(T1);
-  p.ld_lr = g.rp;
-  p.r_lr = g.rp;
-  if (g.rp == 16) return launch_gemm<GemmCfg<kBnDownBwd, false, 16, EPI_SWIGLU_BWD>>(K_GEMM_DOWN_BWD, g, a, b, la, lb, p, s);
-  return launch_gemm<GemmCfg<kBnDownBwd, false, 32, EPI_SWIGLU_BWD>>(K_GEMM_DOWN_BWD, g, a, b, la, lb, p, s);
+  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_SWIGLU_BWD, false, 16>>(K_GEMM_DOWN_BWD, g, tw, ta, tlw, tlr, p, s);
+  return launch_gemm<GemmCfg<EPI_SWIGLU_BWD, false, 32>>(K_GEMM_DOWN_BWD, g, tw, ta, tlw, tlr, p, s);
 }
 
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
-                                   uint16_t* dXp, uint16_t* T2, cudaStream_t s) {
-  CUtensorMap a, b, la, lb;
+                                   const uint16_t* T2c, uint16_t* dXp, cudaStream_t s) {
+  CUtensorMap tw, ta, tlw, tlr;
   const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode2d(&a, dGU, P, 2 * n, 128, 64) || !encode3d(&b, w.W_gu, E, m, 2 * n, kBnGateUpBwd, 64) ||
-      !encode3d(&la, w.B_gu, E, rp, 2 * n, (uint32_t)rp, 64) ||
-      !encode3d(&lb, w.A_gu, E, m, rp, kBnGateUpBwd, (uint32_t)rp))
+  if (!encode3d(&tw, w.W_gu, E, m, 2 * n, 128, 64) || !encode2d(&ta, dGU, P, 2 * n, kTokBox, 64) ||
+      !encode3d(&tlw, w.A_gu, E, m, rp, 128, (uint32_t)rp) ||
+      !encode2d(&tlr, T2c, P, rp, kTokBox, (uint32_t)rp))
     return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.m, 2 * g.n, kBnGateUpBwd);
+  GemmParams p = base_params(g, g.m, 2 * g.n, 128);
   p.out0 = reinterpret_cast<__nv_bfloat16*>(dXp);
   p.ld0 = g.m;
-  p.save_lr = reinterpret_cast<__nv_bfloat16*>(T2);
-  p.ld_lr = g.rp;
-  p.r_lr = g.rp;
-  if (g.rp == 16) return launch_gemm<GemmCfg<kBnGateUpBwd, false, 16, EPI_STORE>>(K_GEMM_GATEUP_BWD, g, a, b, la, lb, p, s);
-  return launch_gemm<GemmCfg<kBnGateUpBwd, false, 32, EPI_STORE>>(K_GEMM_GATEUP_BWD, g, a, b, la, lb, p, s);
+  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_STORE, false, 16>>(K_GEMM_GATEUP_BWD, g, tw, ta, tlw, tlr, p, s);
+  return launch_gemm<GemmCfg<EPI_STORE, false, 32>>(K_GEMM_GATEUP_BWD, g, tw, ta, tlw, tlr, p, s);
+}
+
+template <int RP, bool L_MN>
+static cudaError_t lowrank_rp(const GemmShape& g, const CUtensorMap& ta, const CUtensorMap& tl,
+                              const LowrankParams& lp, cudaStream_t s) {
+  using C = LowrankCfg<RP, L_MN>;
+  auto kern = lowrank_kernel<RP, L_MN>;
+  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
+  if (st != cudaSuccess) return st;
+  ProfScope ps(K_LOWRANK, s);
+  kern<<<g.max_row_tiles, 128, C::SMEM_BYTES, s>>>(ta, tl, lp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const uint16_t* L,
+                           bool L_mn, uint16_t* save, int ld_save, int r_save, uint16_t* outc,
+                           cudaStream_t s) {
+  CUtensorMap ta, tl;
+  const uint64_t E = g.E, rp = g.rp;
+  bool ok = encode2d(&ta, act, (uint64_t)g.P, (uint64_t)K, 128, 64);
+  ok = ok && (L_mn ? encode3d(&tl, L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
+                   : encode3d(&tl, L, E, rp, (uint64_t)K, (uint32_t)rp, 64));
+  if (!ok) return cudaErrorInvalidValue;
+  LowrankParams lp{};
+  lp.tiles = g.tiles;
+  lp.n_tiles = g.n_row_tiles;
+  lp.nk = (K + 63) / 64;
+  lp.scale = g.scale;
+  lp.save = reinterpret_cast<__nv_bfloat16*>(save);
+  lp.ld_save = ld_save;
+  lp.r_save = r_save;
+  lp.outc = reinterpret_cast<__nv_bfloat16*>(outc);
+  lp.err = g.err;
+  if (g.rp == 16) return L_mn ? lowrank_rp<16, true>(g, ta, tl, lp, s) : lowrank_rp<16, false>(g, ta, tl, lp, s);
+  return L_mn ? lowrank_rp<32, true>(g, ta, tl, lp, s) : lowrank_rp<32, false>(g, ta, tl, lp, s);
 }
 
 template <int RP>

@@ -16,7 +16,7 @@ struct TileInfo;
 enum KernelKind : int {
   K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
-  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_NUM_KINDS
+  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_LOWRANK, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
 bool prof_enabled();
@@ -38,10 +38,14 @@ constexpr int kPermuteChunk = 1024;
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
                            int32_t* hist, int* err, cudaStream_t s);
-// Row tiles of `tile_rows` rows per expert (grouped GEMMs) and row chunks of
-// `chunk_rows` rows per expert (adapter gradients), from offsets[E+1].
+// From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
+// experts (low-rank kernel), token chunks of at most `gchunk_rows` rows split
+// evenly inside each expert (grouped GEMMs; all but the last chunk of an expert
+// are multiples of 16), and row chunks of `chunk_rows` rows (adapter gradients)
+// with chunk_start[e] = first chunk of expert e.
 cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
-                                int* n_tiles, int chunk_rows, TileInfo* chunks, int* n_chunks,
+                                int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
+                                int chunk_rows, TileInfo* chunks, int* n_chunks,
                                 int32_t* chunk_start, cudaStream_t s);
 // out[q] = (w ? bf16(w[p] * src[p / k]) : src[p / k]),  p = sorted_pairs[q]
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
@@ -67,25 +71,34 @@ struct GemmShape {
   int64_t P;
   int m, n, E, r, rp;
   float scale;
-  int max_row_tiles;
+  int max_row_tiles;          // 128-row tiles (low-rank kernel)
   const TileInfo* tiles;
   const int* n_row_tiles;
+  int max_gchunks;            // token chunks of at most 256 rows (grouped GEMMs)
+  const TileInfo* gchunks;
+  const int* n_gchunks;
   int* err;
   int num_sms;
 };
 
-// GU = Xs W_gu + c (Xs A_gu) B_gu; writes GU, H = silu(g) u, XA
+// LR = Act L[e] per expert segment; save = LR (first r_save columns, ld_save),
+// outc = bf16(scale * LR) [P, rp].  L_mn: L stored [E, K, rp]; else [E, rp, K].
+cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const uint16_t* L,
+                           bool L_mn, uint16_t* save, int ld_save, int r_save, uint16_t* outc,
+                           cudaStream_t s);
+// GU = Xs W_gu + XAc B_gu (XAc = c X A_gu); writes GU and H = silu(g) u
 cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
-                                   uint16_t* GU, uint16_t* H, uint16_t* XA, cudaStream_t s);
-// Yp = H W_d + c (H A_d) B_d; writes Yp, HA
+                                   const uint16_t* XAc, uint16_t* GU, uint16_t* H, cudaStream_t s);
+// Yp = H W_d + HAc B_d
 cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
-                                 uint16_t* Yp, uint16_t* HA, cudaStream_t s);
-// dH = dy W_d^T + c (dy B_d^T) A_d^T -> dGU via SwiGLU backward with GU; writes T1 [P, rp]
+                                 const uint16_t* HAc, uint16_t* Yp, cudaStream_t s);
+// dH = dy W_d^T + T1c A_d^T -> dGU via the SwiGLU backward with GU
 cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
-                                 const uint16_t* GU, uint16_t* dGU, uint16_t* T1, cudaStream_t s);
-// dXp = dGU W_gu^T + c (dGU B_gu^T) A_gu^T; writes dXp, T2 [P, rp]
+                                 const uint16_t* T1c, const uint16_t* GU, uint16_t* dGU,
+                                 cudaStream_t s);
+// dXp = dGU W_gu^T + T2c A_gu^T
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
-                                   uint16_t* dXp, uint16_t* T2, cudaStream_t s);
+                                   const uint16_t* T2c, uint16_t* dXp, cudaStream_t s);
 // out = scale * sum_rows Big^T Small per expert, out [E, D, r] or (transpose) [E, r, D]
 cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, const uint16_t* small,
                               int ld_small, const TileInfo* chunks, const int* n_chunks,

@@ -235,22 +235,38 @@ __device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int
 
 __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, int tile_rows,
                                     TileInfo* __restrict__ tiles, int* __restrict__ n_tiles,
-                                    int chunk_rows, TileInfo* __restrict__ chunks,
-                                    int* __restrict__ n_chunks, int32_t* __restrict__ chunk_start) {
+                                    int gchunk_rows, TileInfo* __restrict__ gchunks,
+                                    int* __restrict__ n_gchunks, int chunk_rows,
+                                    TileInfo* __restrict__ chunks, int* __restrict__ n_chunks,
+                                    int32_t* __restrict__ chunk_start) {
   __shared__ int s_warp[33];
   const int e = threadIdx.x;
   int lo = 0, hi = 0;
   if (e < E) { lo = offsets[e]; hi = offsets[e + 1]; }
   const int cnt = hi - lo;
   int total;
+  // row tiles of exactly tile_rows rows (the last one of an expert may be short)
   const int nt = (cnt + tile_rows - 1) / tile_rows;
   const int t0 = block_exclusive_scan_1024(nt, s_warp, &total);
   for (int i = 0; i < nt; ++i) {
     TileInfo ti;
-    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = hi; ti.pad = 0;
+    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = min(hi, lo + (i + 1) * tile_rows); ti.pad = 0;
     tiles[t0 + i] = ti;
   }
   if (threadIdx.x == 0) *n_tiles = total;
+  // token chunks: ceil(cnt / gchunk_rows) chunks of equal size rounded up to 16
+  if (gchunks != nullptr) {
+    const int ng = (cnt + gchunk_rows - 1) / gchunk_rows;
+    int gtotal;
+    const int g0 = block_exclusive_scan_1024(ng, s_warp, &gtotal);
+    const int sz = ng > 0 ? (((cnt + ng - 1) / ng + 15) & ~15) : 0;
+    for (int i = 0; i < ng; ++i) {
+      TileInfo ti;
+      ti.e = e; ti.row0 = lo + i * sz; ti.row_end = min(hi, lo + (i + 1) * sz); ti.pad = 0;
+      gchunks[g0 + i] = ti;
+    }
+    if (threadIdx.x == 0) *n_gchunks = gtotal;
+  }
   if (chunks != nullptr) {
     const int nc = (cnt + chunk_rows - 1) / chunk_rows;
     int ctotal;
@@ -269,11 +285,12 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
 }
 
 cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
-                                int* n_tiles, int chunk_rows, TileInfo* chunks, int* n_chunks,
+                                int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
+                                int chunk_rows, TileInfo* chunks, int* n_chunks,
                                 int32_t* chunk_start, cudaStream_t s) {
   ProfScope ps(K_TABLES, s);
-  build_tables_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_rows, tiles, n_tiles, chunk_rows, chunks,
-                                         n_chunks, chunk_start);
+  build_tables_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_rows, tiles, n_tiles, gchunk_rows, gchunks,
+                                         n_gchunks, chunk_rows, chunks, n_chunks, chunk_start);
   return cudaGetLastError();
 }
 
