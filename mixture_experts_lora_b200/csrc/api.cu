@@ -45,11 +45,9 @@ int device_sms() {
 
 inline int rank_padded(int r) { return r <= 16 ? 16 : 32; }
 
-inline int64_t chunk_rows_for(int64_t P) {
-  if (P <= 65536) return 256;
-  if (P <= 131072) return 1024;
-  return 2048;
-}
+// Row chunk of the adapter-gradient kernel: one chunk covers a whole expert at
+// the shapes served here, so most experts need no second reduction pass.
+inline int64_t chunk_rows_for(int64_t) { return 1024; }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -75,7 +73,7 @@ struct Layout {
   int max_row_tiles, max_gchunks, max_chunks, chunk_rows, perm_chunks;
   size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
   size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
-  size_t rows, dgu, t1, t2, lrc1, lrc2, partial;
+  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial;
   size_t total;
 };
 
@@ -107,6 +105,7 @@ Layout make_layout(const moe_dims_t& d) {
   L.pad_B_d = take(pad ? E * rp * m * 2 : 0);
   L.rows = take(P * m * 2);
   L.dgu = take(P * 2 * n * 2);
+  L.dh = take(P * n * 2);
   L.t1 = take(P * rp * 2);
   L.t2 = take(P * rp * 2);
   L.lrc1 = take(P * rp * 2);
@@ -268,12 +267,15 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   uint16_t* xs = at<uint16_t>(ws, L.rows);
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
-  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, xs, s));
-  // XA = X A_gu (saved) and bf16(c XA), then GU = X W_gu + (c XA) B_gu with SwiGLU
-  MOE_TRY(launch_lowrank(g, xs, d.m, w.A_gu, true, save_XA, d.r, d.r, xac, s));
-  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, xac, save_GU, save_H, s));
-  // HA = H A_d (saved) and bf16(c HA), then Y = H W_d + (c HA) B_d
-  MOE_TRY(launch_lowrank(g, save_H, d.n, w.A_d, true, save_HA, d.r, d.r, hac, s));
+  // X rows in expert order, XA = X A_gu (saved) and bf16(c XA)
+  MOE_TRY(launch_rows_lowrank(g, 0, d.m, X, sorted_pairs, nullptr, d.k, nullptr, nullptr, w.A_gu,
+                              true, xs, save_XA, d.r, d.r, xac, s));
+  // GU = X W_gu + (c XA) B_gu
+  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, xac, save_GU, s));
+  // H = silu(g) u, HA = H A_d (saved) and bf16(c HA)
+  MOE_TRY(launch_rows_lowrank(g, 1, d.n, nullptr, nullptr, nullptr, d.k, save_GU, nullptr, w.A_d,
+                              true, save_H, save_HA, d.r, d.r, hac, s));
+  // Y = H W_d + (c HA) B_d
   MOE_TRY(launch_gemm_down_fwd(g, w, save_H, hac, Y_sorted, s));
   return MOE_OK;
 }
@@ -322,18 +324,21 @@ moe_status_t moe_grouped_gemm_lora_bwd(
   const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
   uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
   uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
-  // dy = w * dY[t] in sorted order
-  MOE_TRY(launch_gather_rows(dY, sorted_pairs, topk_w, L.P, d.k, d.m, rows, s));
-  // T1 = dy B_d^T (saved for dA_d) and bf16(c T1); dH = dy W_d^T + (c T1) A_d^T -> dGU
-  MOE_TRY(launch_lowrank(g, rows, d.m, w.B_d, false, t1, L.rp, L.rp, lrc1, s));
-  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, save_GU, dgu, s));
+  uint16_t* dh = at<uint16_t>(ws, L.dh);
+  // dy = w * dY[t] in expert order, T1 = dy B_d^T (kept for dA_d) and bf16(c T1)
+  MOE_TRY(launch_rows_lowrank(g, 0, d.m, dY, sorted_pairs, topk_w, d.k, nullptr, nullptr, w.B_d,
+                              false, rows, t1, L.rp, L.rp, lrc1, s));
+  // dH = dy W_d^T + (c T1) A_d^T
+  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
   // dA_d = c H^T T1 ; dB_d = c HA^T dy
   MOE_TRY(launch_lora_wgrad(g, save_H, d.n, t1, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
                             partial, false, dA_d, s));
   MOE_TRY(launch_lora_wgrad(g, rows, d.m, save_HA, d.r, chunks, n_chunks, L.max_chunks,
                             chunk_start, partial, true, dB_d, s));
-  // T2 = dGU B_gu^T and bf16(c T2); dX_sorted = dGU W_gu^T + (c T2) A_gu^T
-  MOE_TRY(launch_lowrank(g, dgu, 2 * d.n, w.B_gu, false, t2, L.rp, L.rp, lrc2, s));
+  // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
+  MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
+                              false, dgu, t2, L.rp, L.rp, lrc2, s));
+  // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
   // dB_gu = c XA^T dGU
   MOE_TRY(launch_lora_wgrad(g, dgu, 2 * d.n, save_XA, d.r, chunks, n_chunks, L.max_chunks,

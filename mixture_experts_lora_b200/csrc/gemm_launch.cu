@@ -8,6 +8,7 @@
 #include "internal.h"
 #include "lora_wgrad.cuh"
 #include "lowrank.cuh"
+#include "rows_lowrank.cuh"
 
 namespace moe {
 
@@ -73,101 +74,140 @@ cudaError_t ensure_smem(Kern kernel, int bytes) {
 }
 
 template <class C>
-cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap& tw, const CUtensorMap& ta,
-                        const CUtensorMap& tlw, const CUtensorMap& tlr, const GemmParams& p,
+cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap* maps, const GemmParams& p,
                         cudaStream_t s) {
   auto kern = moe_gemm_kernel<C>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
   const int64_t tiles = (int64_t)g.max_gchunks * p.n_ftiles;
-  const int grid = (int)(tiles < g.num_sms ? (tiles > 0 ? tiles : 1) : g.num_sms);
+  const int pairs_max = g.num_sms / 2 > 0 ? g.num_sms / 2 : 1;
+  const int pairs = (int)(tiles < pairs_max ? (tiles > 0 ? tiles : 1) : pairs_max);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   ProfScope ps(kind, s);
-  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tw, ta, tlw, tlr, p);
+  st = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+  if (st != cudaSuccess) return st;
   return cudaGetLastError();
 }
 
-GemmParams base_params(const GemmShape& g, int F, int K, int feat_per_tile) {
+// One grouped GEMM: out [P, F] = act [P, K] x W[e] (+ LoRA block), features on M.
+// w_fk: W stored [E, F, K] (K-major A) instead of [E, K, F] (MN-major A);
+// lw: L_B^T stored [E, rp, F] (forward) or [E, F, rp] (backward).
+cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk, int F, int K,
+                     const uint16_t* act, const uint16_t* lw, const uint16_t* lrc, uint16_t* out,
+                     cudaStream_t s) {
+  CUtensorMap mp[4];
+  const uint64_t P = g.P, E = g.E, rp = g.rp;
+  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, 32, 64) &&
+            encode2d(&mp[3], lrc, P, rp, 32, (uint32_t)rp);
+  if (w_fk) {
+    ok = ok && encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64) &&
+         encode3d(&mp[2], lw, E, (uint64_t)F, rp, 128, (uint32_t)rp);
+  } else {
+    ok = ok && encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64, 64) &&
+         encode3d(&mp[2], lw, E, rp, (uint64_t)F, (uint32_t)rp, 64);
+  }
+  if (!ok) return cudaErrorInvalidValue;
   GemmParams p{};
   p.chunks = g.gchunks;
   p.n_chunks = g.n_gchunks;
   p.F = F;
-  p.K = K;
-  p.n_ftiles = (F + feat_per_tile - 1) / feat_per_tile;
+  p.n_ftiles = (F + 255) / 256;
   p.nk = (K + 63) / 64;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.err = g.err;
-  return p;
+  if (w_fk) {
+    if (g.rp == 16) return launch_gemm<GemmCfg<false, 16>>(kind, g, mp, p, s);
+    return launch_gemm<GemmCfg<false, 32>>(kind, g, mp, p, s);
+  }
+  if (g.rp == 16) return launch_gemm<GemmCfg<true, 16>>(kind, g, mp, p, s);
+  return launch_gemm<GemmCfg<true, 32>>(kind, g, mp, p, s);
 }
 
 }  // namespace
 
-// Token-row operand boxes: 32 rows x 64 K (activations) or 32 rows x rp (LoRA operand).
-constexpr uint32_t kTokBox = 32;
-
 cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
-                                   const uint16_t* XAc, uint16_t* GU, uint16_t* H, cudaStream_t s) {
-  CUtensorMap tw, ta, tlw, tlr;
-  const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode3d(&tw, w.W_gu, E, m, 2 * n, 64, 64) || !encode2d(&ta, Xs, P, m, kTokBox, 64) ||
-      !encode3d(&tlw, w.B_gu, E, rp, 2 * n, (uint32_t)rp, 64) ||
-      !encode2d(&tlr, XAc, P, rp, kTokBox, (uint32_t)rp))
-    return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.n, g.m, 64);
-  p.n_half = g.n;
-  p.out0 = reinterpret_cast<__nv_bfloat16*>(GU);
-  p.ld0 = 2 * g.n;
-  p.out1 = reinterpret_cast<__nv_bfloat16*>(H);
-  p.ld1 = g.n;
-  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_GATEUP_FWD, true, 16>>(K_GEMM_GATEUP_FWD, g, tw, ta, tlw, tlr, p, s);
-  return launch_gemm<GemmCfg<EPI_GATEUP_FWD, true, 32>>(K_GEMM_GATEUP_FWD, g, tw, ta, tlw, tlr, p, s);
+                                   const uint16_t* XAc, uint16_t* GU, cudaStream_t s) {
+  return gemm_any(K_GEMM_GATEUP_FWD, g, w.W_gu, false, 2 * g.n, g.m, Xs, w.B_gu, XAc, GU, s);
 }
 
 cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
                                  const uint16_t* HAc, uint16_t* Yp, cudaStream_t s) {
-  CUtensorMap tw, ta, tlw, tlr;
-  const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode3d(&tw, w.W_d, E, n, m, 64, 64) || !encode2d(&ta, H, P, n, kTokBox, 64) ||
-      !encode3d(&tlw, w.B_d, E, rp, m, (uint32_t)rp, 64) ||
-      !encode2d(&tlr, HAc, P, rp, kTokBox, (uint32_t)rp))
-    return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.m, g.n, 128);
-  p.out0 = reinterpret_cast<__nv_bfloat16*>(Yp);
-  p.ld0 = g.m;
-  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_STORE, true, 16>>(K_GEMM_DOWN_FWD, g, tw, ta, tlw, tlr, p, s);
-  return launch_gemm<GemmCfg<EPI_STORE, true, 32>>(K_GEMM_DOWN_FWD, g, tw, ta, tlw, tlr, p, s);
+  return gemm_any(K_GEMM_DOWN_FWD, g, w.W_d, false, g.m, g.n, H, w.B_d, HAc, Yp, s);
 }
 
 cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
-                                 const uint16_t* T1c, const uint16_t* GU, uint16_t* dGU,
-                                 cudaStream_t s) {
-  CUtensorMap tw, ta, tlw, tlr;
-  const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode3d(&tw, w.W_d, E, n, m, 128, 64) || !encode2d(&ta, dys, P, m, kTokBox, 64) ||
-      !encode3d(&tlw, w.A_d, E, n, rp, 128, (uint32_t)rp) ||
-      !encode2d(&tlr, T1c, P, rp, kTokBox, (uint32_t)rp))
-    return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.n, g.m, 128);
-  p.n_half = g.n;
-  p.out0 = reinterpret_cast<__nv_bfloat16*>(dGU);
-  p.ld0 = 2 * g.n;
-  p.in0 = reinterpret_cast<const __nv_bfloat16*>(GU);
-  p.ldi0 = 2 * g.n;
-  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_SWIGLU_BWD, false, 16>>(K_GEMM_DOWN_BWD, g, tw, ta, tlw, tlr, p, s);
-  return launch_gemm<GemmCfg<EPI_SWIGLU_BWD, false, 32>>(K_GEMM_DOWN_BWD, g, tw, ta, tlw, tlr, p, s);
+                                 const uint16_t* T1c, uint16_t* dH, cudaStream_t s) {
+  return gemm_any(K_GEMM_DOWN_BWD, g, w.W_d, true, g.n, g.m, dys, w.A_d, T1c, dH, s);
 }
 
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
                                    const uint16_t* T2c, uint16_t* dXp, cudaStream_t s) {
-  CUtensorMap tw, ta, tlw, tlr;
-  const uint64_t P = g.P, m = g.m, n = g.n, E = g.E, rp = g.rp;
-  if (!encode3d(&tw, w.W_gu, E, m, 2 * n, 128, 64) || !encode2d(&ta, dGU, P, 2 * n, kTokBox, 64) ||
-      !encode3d(&tlw, w.A_gu, E, m, rp, 128, (uint32_t)rp) ||
-      !encode2d(&tlr, T2c, P, rp, kTokBox, (uint32_t)rp))
-    return cudaErrorInvalidValue;
-  GemmParams p = base_params(g, g.m, 2 * g.n, 128);
-  p.out0 = reinterpret_cast<__nv_bfloat16*>(dXp);
-  p.ld0 = g.m;
-  if (g.rp == 16) return launch_gemm<GemmCfg<EPI_STORE, false, 16>>(K_GEMM_GATEUP_BWD, g, tw, ta, tlw, tlr, p, s);
-  return launch_gemm<GemmCfg<EPI_STORE, false, 32>>(K_GEMM_GATEUP_BWD, g, tw, ta, tlw, tlr, p, s);
+  return gemm_any(K_GEMM_GATEUP_BWD, g, w.W_gu, true, g.m, 2 * g.n, dGU, w.A_gu, T2c, dXp, s);
+}
+
+template <int MODE, int RP, bool L_MN>
+static cudaError_t rows_rp(const GemmShape& g, const CUtensorMap& tl, const RowsParams& rp_,
+                           cudaStream_t s) {
+  using C = RowsCfg<MODE, RP, L_MN>;
+  auto kern = rows_lowrank_kernel<MODE, RP, L_MN>;
+  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
+  if (st != cudaSuccess) return st;
+  ProfScope ps(MODE == ROWS_GATHER ? K_ROWS_GATHER : (MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD), s);
+  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl, rp_);
+  return cudaGetLastError();
+}
+
+template <int MODE, bool L_MN>
+static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap& tl, const RowsParams& rp_,
+                             cudaStream_t s) {
+  if (g.rp == 16) return rows_rp<MODE, 16, L_MN>(g, tl, rp_, s);
+  return rows_rp<MODE, 32, L_MN>(g, tl, rp_, s);
+}
+
+cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint16_t* src,
+                                const int32_t* sorted_pairs, const float* w, int k,
+                                const uint16_t* gu, const uint16_t* dh, const uint16_t* L,
+                                bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
+                                int r_save, uint16_t* outc, cudaStream_t s) {
+  CUtensorMap tl;
+  const uint64_t E = g.E, rp = g.rp;
+  const bool ok = L_mn ? encode3d(&tl, L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
+                       : encode3d(&tl, L, E, rp, (uint64_t)K, (uint32_t)rp, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  RowsParams p{};
+  p.tiles = g.tiles;
+  p.n_tiles = g.n_row_tiles;
+  p.K = K;
+  p.nk = (K + 63) / 64;
+  p.src = reinterpret_cast<const __nv_bfloat16*>(src);
+  p.sorted_pairs = sorted_pairs;
+  p.w = w;
+  p.k = k;
+  p.gu = reinterpret_cast<const __nv_bfloat16*>(gu);
+  p.dh = reinterpret_cast<const __nv_bfloat16*>(dh);
+  p.n = g.n;
+  p.rows_out = reinterpret_cast<__nv_bfloat16*>(rows_out);
+  p.scale = g.scale;
+  p.save = reinterpret_cast<__nv_bfloat16*>(save);
+  p.ld_save = ld_save;
+  p.r_save = r_save;
+  p.outc = reinterpret_cast<__nv_bfloat16*>(outc);
+  p.err = g.err;
+  if (mode == ROWS_GATHER)
+    return L_mn ? rows_mode<ROWS_GATHER, true>(g, tl, p, s) : rows_mode<ROWS_GATHER, false>(g, tl, p, s);
+  if (mode == ROWS_SWIGLU) return rows_mode<ROWS_SWIGLU, true>(g, tl, p, s);
+  return rows_mode<ROWS_SWIGLU_BWD, false>(g, tl, p, s);
 }
 
 template <int RP, bool L_MN>
@@ -206,25 +246,24 @@ cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const
 }
 
 template <int RP>
-static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap& tm, const WgradParams& wp, int D,
-                            int max_chunks, const int32_t* chunk_start, bool transpose,
-                            uint16_t* out, cudaStream_t s) {
+static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap& tm, const WgradParams& wp,
+                            int max_chunks, cudaStream_t s) {
   using C = WgradCfg<RP>;
   auto kern = lora_wgrad_kernel<RP>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
-  if (max_chunks > 0) {
-    dim3 grid((D + 127) / 128, max_chunks);
+  const int64_t units = (int64_t)max_chunks * wp.n_dtiles;
+  if (units > 0) {
+    const int grid = (int)(units < g.num_sms ? units : g.num_sms);
     ProfScope ps(K_WGRAD, s);
-    kern<<<grid, 128, C::SMEM_BYTES, s>>>(tm, wp);
+    kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm, wp);
     st = cudaGetLastError();
     if (st != cudaSuccess) return st;
   }
-  const int64_t total = (int64_t)g.E * D;
+  const int64_t total = (int64_t)g.E * wp.D;
   ProfScope ps(K_WGRAD_REDUCE, s);
   lora_wgrad_reduce_kernel<RP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-      wp.partial, chunk_start, g.E, D, g.r, g.scale, transpose,
-      reinterpret_cast<__nv_bfloat16*>(out));
+      wp.partial, wp.chunk_start, g.E, wp.D, g.r, g.scale, wp.transpose, wp.out);
   return cudaGetLastError();
 }
 
@@ -241,11 +280,17 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, co
   wp.r_small = ld_small;  // the caller's buffer has exactly ld_small columns
   wp.chunks = chunks;
   wp.n_chunks = n_chunks;
+  wp.chunk_start = chunk_start;
   wp.D = D;
+  wp.n_dtiles = (D + 127) / 128;
+  wp.r = g.r;
+  wp.scale = g.scale;
+  wp.transpose = transpose;
+  wp.out = reinterpret_cast<__nv_bfloat16*>(out);
   wp.partial = partial;
   wp.err = g.err;
-  if (g.rp == 16) return wgrad_rp<16>(g, tm, wp, D, max_chunks, chunk_start, transpose, out, s);
-  return wgrad_rp<32>(g, tm, wp, D, max_chunks, chunk_start, transpose, out, s);
+  if (g.rp == 16) return wgrad_rp<16>(g, tm, wp, max_chunks, s);
+  return wgrad_rp<32>(g, tm, wp, max_chunks, s);
 }
 
 }  // namespace moe

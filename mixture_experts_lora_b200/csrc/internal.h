@@ -16,7 +16,8 @@ struct TileInfo;
 enum KernelKind : int {
   K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
-  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_LOWRANK, K_NUM_KINDS
+  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_LOWRANK, K_ROWS_GATHER, K_ROWS_SWIGLU,
+  K_ROWS_SWIGLU_BWD, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
 bool prof_enabled();
@@ -86,19 +87,29 @@ struct GemmShape {
 cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const uint16_t* L,
                            bool L_mn, uint16_t* save, int ld_save, int r_save, uint16_t* outc,
                            cudaStream_t s);
-// GU = Xs W_gu + XAc B_gu (XAc = c X A_gu); writes GU and H = silu(g) u
+// Grouped GEMMs (features on M, expert tokens on N, CTA pairs); each writes
+// out [P, F] in sorted token order.
+// GU = Xs W_gu + XAc B_gu             (XAc = bf16(c X A_gu))
 cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
-                                   const uint16_t* XAc, uint16_t* GU, uint16_t* H, cudaStream_t s);
+                                   const uint16_t* XAc, uint16_t* GU, cudaStream_t s);
 // Yp = H W_d + HAc B_d
 cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
                                  const uint16_t* HAc, uint16_t* Yp, cudaStream_t s);
-// dH = dy W_d^T + T1c A_d^T -> dGU via the SwiGLU backward with GU
+// dH = dy W_d^T + T1c A_d^T
 cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
-                                 const uint16_t* T1c, const uint16_t* GU, uint16_t* dGU,
-                                 cudaStream_t s);
+                                 const uint16_t* T1c, uint16_t* dH, cudaStream_t s);
 // dXp = dGU W_gu^T + T2c A_gu^T
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
                                    const uint16_t* T2c, uint16_t* dXp, cudaStream_t s);
+// Row producer + rank-r product (rows_lowrank.cuh); mode: 0 gather (src rows by
+// sorted pair, times w if given), 1 SwiGLU from gu, 2 SwiGLU backward from dh and gu.
+// Writes rows_out [P, K] (if not null), save = LR (first r_save columns, ld_save)
+// and outc = bf16(scale * LR) [P, rp].
+cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint16_t* src,
+                                const int32_t* sorted_pairs, const float* w, int k,
+                                const uint16_t* gu, const uint16_t* dh, const uint16_t* L,
+                                bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
+                                int r_save, uint16_t* outc, cudaStream_t s);
 // out = scale * sum_rows Big^T Small per expert, out [E, D, r] or (transpose) [E, r, D]
 cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, const uint16_t* small,
                               int ld_small, const TileInfo* chunks, const int* n_chunks,

@@ -2,18 +2,22 @@
 //
 // For expert e with sorted rows R_e the four adapter gradients all have the form
 //     G_e [D, r] = sum_{q in R_e} Big[q, :]^T Small[q, :]
-// (Big = H, dy, dGU or X with D = n, m, 2n or m; Small = T1, HA, XA or T2 with r
-// columns).  dA_d = c G (Big = H, Small = T1), dB_d = c G^T (Big = w*dY, Small =
-// HA), dA_gu = c G (Big = X, Small = T2), dB_gu = c G^T (Big = dGU, Small = XA).
+// dA_d = c G (Big = H, Small = T1), dB_d = c G^T (Big = w*dY, Small = HA),
+// dA_gu = c G (Big = X, Small = T2), dB_gu = c G^T (Big = dGU, Small = XA):
+// the chain rule through Y = XW + (alpha/r)(XA)B with W frozen ("Accelerating
+// Mixture-of-Experts Fine-Tuning", Mathematical Formulation section 2; Unsloth
+// docs "Implementation details": only the m*r + r*n adapter parameters train).
 //
-// Work is split into (row chunk, 128-wide D tile) units; each unit is one CTA:
+// Units are (row chunk of one expert, 128-wide D tile); a persistent CTA walks
+// its units with one continuous TMA/MMA pipeline:
 //   M = 128 columns of Big (MN-major A operand, TMA, 128-byte swizzle),
 //   N = RP (Small, MN-major, no swizzle, written by the producer warp with rows
 //       outside the chunk zeroed, so a ragged tail contributes nothing),
 //   K = rows of the chunk, 64 per stage.
-// Each unit writes an fp32 partial; a second kernel sums a fixed sequence of
-// partials per expert (deterministic, no atomics) and applies c, the bf16
-// rounding and the output orientation.
+// The accumulator is double buffered in TMEM.  A unit of an expert whose rows fit
+// in one chunk writes the final bf16 gradient (scaled, in its output orientation);
+// otherwise it writes an fp32 partial and a second kernel sums the expert's
+// partials in chunk order (deterministic, no atomics).
 #pragma once
 
 #include "common.cuh"
@@ -26,50 +30,55 @@ struct WgradParams {
   int r_small;                 // columns of `small` to read (rest zero)
   const TileInfo* chunks;      // row chunks {e, row0, row_end}
   const int* n_chunks;
+  const int32_t* chunk_start;  // [E+1]
   int D;
+  int n_dtiles;
+  int r;                       // output rank
+  float scale;
+  bool transpose;              // out [E, r, D] instead of [E, D, r]
+  __nv_bfloat16* out;
   float* partial;              // [max_chunks, D, RP]
   int* err;
 };
 
 template <int RP>
 struct WgradCfg {
-  static constexpr int BM = 128, BK = 64, STAGES = 4;
+  static constexpr int BM = 128, BK = 64, STAGES = 8;
   static constexpr int BIG_BYTES = BM * BK * 2;   // two 64-column boxes
   static constexpr int SMALL_BYTES = RP * BK * 2;
   static constexpr int STAGE_BYTES = BIG_BYTES + SMALL_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
-  static constexpr int TMEM_COLS = 32;
+  static constexpr int TMEM_COLS = 64;            // 2 x RP fp32 columns (RP <= 32)
 };
 
 template <int RP>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(192, 1)
     lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig, const WgradParams p) {
   using C = WgradCfg<RP>;
-  const int j = blockIdx.y;
-  if (j >= *p.n_chunks) return;
-  const TileInfo ch = p.chunks[j];
-  const int d0 = blockIdx.x * C::BM;
-  const int nrows = ch.row_end - ch.row0;
-  const int nk = (nrows + C::BK - 1) / C::BK;
-
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + C::STAGES;
-  uint64_t* done = bars + 2 * C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * C::STAGES + 2);
+  uint64_t* full = bars;                     // [STAGES]: TMA bytes + producer stores
+  uint64_t* empty = bars + C::STAGES;        // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES; // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* drain = acc_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_full + 6);
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 2);   // TMA (expect_tx) + producer's shared stores
+      mbar_init(smem_u32(&full[s]), 2);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(done), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmBig);
@@ -82,40 +91,47 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int total = (*p.n_chunks) * p.n_dtiles;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
+    // ---------------------------------------------------------- producer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int ks = 0; ks < nk; ++ks) {
-      bool w = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-      const uint32_t fb = smem_u32(&full[stage]);
-      const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
-      const int r0 = ch.row0 + ks * C::BK;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(fb, C::BIG_BYTES);
-        tma_load_2d(&tmBig, fb, sbig, d0, r0);
-        tma_load_2d(&tmBig, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
-      }
-      // Small tile [64 rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
-      // columns (128 B), row groups 128 B apart, column groups 1024 B apart.
-      uint8_t* ssm = smem + stage * C::STAGE_BYTES + C::BIG_BYTES;
-      constexpr int CG = RP / 8;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const int c = t / p.n_dtiles, dt = t % p.n_dtiles;
+      const TileInfo ch = p.chunks[c];
+      const int d0 = dt * C::BM;
+      const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
+      for (int ks = 0; ks < nk; ++ks) {
+        bool w = !(*abort_flag) && mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        const uint32_t fb = smem_u32(&full[stage]);
+        const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
+        const int r0 = ch.row0 + ks * C::BK;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(fb, C::BIG_BYTES);
+          tma_load_2d(&tmBig, fb, sbig, d0, r0);
+          tma_load_2d(&tmBig, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
+        }
+        // Small tile [64 rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
+        // columns (128 B), row groups 128 B apart, column groups 1024 B apart.
+        uint8_t* ssm = smem + stage * C::STAGE_BYTES + C::BIG_BYTES;
+        constexpr int CG = RP / 8;
 #pragma unroll
-      for (int i = lane; i < C::BK * CG; i += 32) {
-        const int rr = i / CG, cg = i % CG;
-        const int row = r0 + rr;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < ch.row_end && cg * 8 < p.r_small)
-          v = *reinterpret_cast<const uint4*>(p.small + (size_t)row * p.ld_small + cg * 8);
-        *reinterpret_cast<uint4*>(ssm + cg * 1024 + (rr & 7) * 16 + (rr >> 3) * 128) = v;
+        for (int i = lane; i < C::BK * CG; i += 32) {
+          const int rr = i / CG, cg = i % CG;
+          const int row = r0 + rr;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (row < ch.row_end && cg * 8 < p.r_small)
+            v = *reinterpret_cast<const uint4*>(p.small + (size_t)row * p.ld_small + cg * 8);
+          *reinterpret_cast<uint4*>(ssm + cg * 1024 + (rr & 7) * 16 + (rr >> 3) * 128) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(fb);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(fb);
-      if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
     }
     if (!ok) *abort_flag = 1;
   } else if (warp == 1) {
@@ -124,63 +140,104 @@ __global__ void __launch_bounds__(128)
       const uint32_t idesc = idesc_bf16(128, RP, 1, 1);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
-      for (int ks = 0; ks < nk; ++ks) {
-        if (*abort_flag) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+      int it = 0;
+      bool ok = true, issued_any = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const int c = t / p.n_dtiles;
+        const TileInfo ch = p.chunks[c];
+        const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
+        const int b = it & 1;
+        if (!mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
-        const uint32_t ssm = sbig + C::BIG_BYTES;
+        const uint32_t d = tmem + b * 32;
+        for (int ks = 0; ks < nk; ++ks) {
+          if (*abort_flag) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
+          const uint32_t ssm = sbig + C::BIG_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk) {
-          // Big^T: MN-major, 128-byte swizzle, 64-column atoms 8 KB apart, 8-row groups 1 KB apart
-          const uint64_t ad = smem_desc(sbig + kk * 16 * 128, C::BIG_BYTES / 2, 1024, kSw128);
-          // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at 1024 B
-          const uint64_t bd = smem_desc(ssm + kk * 256, 128, 1024, kSwNone);
-          umma_bf16(tmem, ad, bd, idesc, (ks | kk) ? 1u : 0u);
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            // Big^T: MN-major, 128-byte swizzle, 64-column atoms 8 KB apart, 8-row groups 1 KB apart
+            const uint64_t ad = smem_desc(sbig + kk * 16 * 128, C::BIG_BYTES / 2, 1024, kSw128);
+            // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at 1024 B
+            const uint64_t bd = smem_desc(ssm + kk * 256, 128, 1024, kSwNone);
+            umma_bf16(d, ad, bd, idesc, (ks | kk) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&empty[stage]));
+          issued_any = true;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
-        umma_commit(smem_u32(&empty[stage]));
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        if (!ok) break;
+        umma_commit(smem_u32(&acc_full[b]));
       }
       if (!ok) *abort_flag = 1;
-      umma_commit(smem_u32(done));
+      if (issued_any) {
+        umma_commit(smem_u32(drain));
+        mbar_wait(smem_u32(drain), 0, p.err);
+      }
     }
     __syncwarp();
+  } else {
+    // ---------------------------------------------------------- epilogue (warps 2..5)
+    const int q = warp & 3;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const int c = t / p.n_dtiles, dt = t % p.n_dtiles;
+      const TileInfo ch = p.chunks[c];
+      const int b = it & 1;
+      bool ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
+      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      float v[RP];
+      if constexpr (RP == 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + b * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+      } else {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+      const int d = dt * C::BM + q * 32 + lane;
+      if (d < p.D) {
+        const bool single = p.chunk_start[ch.e + 1] - p.chunk_start[ch.e] == 1;
+        if (single) {
+          if (p.transpose) {
+#pragma unroll
+            for (int i = 0; i < RP; ++i)
+              if (i < p.r) p.out[((size_t)ch.e * p.r + i) * p.D + d] = __float2bfloat16_rn(p.scale * v[i]);
+          } else {
+            __nv_bfloat16* dst = p.out + ((size_t)ch.e * p.D + d) * p.r;
+#pragma unroll
+            for (int g = 0; g < RP / 8; ++g) {
+              if (g * 8 < p.r) {
+                uint4 o;
+                o.x = pack_bf16x2(p.scale * v[8 * g + 0], p.scale * v[8 * g + 1]);
+                o.y = pack_bf16x2(p.scale * v[8 * g + 2], p.scale * v[8 * g + 3]);
+                o.z = pack_bf16x2(p.scale * v[8 * g + 4], p.scale * v[8 * g + 5]);
+                o.w = pack_bf16x2(p.scale * v[8 * g + 6], p.scale * v[8 * g + 7]);
+                *reinterpret_cast<uint4*>(dst + 8 * g) = o;
+              }
+            }
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)c * p.D + d) * RP);
+#pragma unroll
+          for (int i = 0; i < RP / 4; ++i)
+            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    }
   }
 
-  // ---------------------------------------------------------- epilogue (all warps)
-  __syncthreads();
-  {
-    bool ok = mbar_wait(smem_u32(done), 0, p.err);
-    ok = __all_sync(0xffffffffu, ok);
-    tc_fence_after();
-    const int d = d0 + warp * 32 + lane;
-    uint32_t v[RP];
-    if constexpr (RP == 16) {
-      uint32_t r[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = r[i];
-    } else {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16), r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = r[i];
-    }
-    if (ok && nk > 0 && d < p.D) {
-      float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)j * p.D + d) * RP);
-#pragma unroll
-      for (int i = 0; i < RP / 4; ++i)
-        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-    } else if (d < p.D) {
-      float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)j * p.D + d) * RP);
-#pragma unroll
-      for (int i = 0; i < RP / 4; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -189,8 +246,9 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-// out[e] = bf16(scale * sum over the chunks of e, in chunk order, of partial)
-// transpose = false: out [E, D, r];  transpose = true: out [E, r, D].
+// Experts with 0 chunks get zeros; experts with 2+ chunks get
+// bf16(scale * sum of their partials in chunk order).  Single-chunk experts were
+// written by lora_wgrad_kernel.  transpose = false: out [E, D, r]; true: [E, r, D].
 template <int RP>
 __global__ void lora_wgrad_reduce_kernel(const float* __restrict__ partial,
                                          const int* __restrict__ chunk_start, int E, int D, int r,
@@ -199,10 +257,11 @@ __global__ void lora_wgrad_reduce_kernel(const float* __restrict__ partial,
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)E * D) return;
   const int e = (int)(idx / D), d = (int)(idx % D);
+  const int c0 = chunk_start[e], c1 = chunk_start[e + 1];
+  if (c1 - c0 == 1) return;
   float acc[RP];
 #pragma unroll
   for (int i = 0; i < RP; ++i) acc[i] = 0.f;
-  const int c0 = chunk_start[e], c1 = chunk_start[e + 1];
   for (int c = c0; c < c1; ++c) {
     const float4* src = reinterpret_cast<const float4*>(partial + ((size_t)c * D + d) * RP);
 #pragma unroll
@@ -214,11 +273,13 @@ __global__ void lora_wgrad_reduce_kernel(const float* __restrict__ partial,
       acc[4 * i + 3] += v.w;
     }
   }
-  if (transpose) {
-    for (int i = 0; i < r; ++i) out[((size_t)e * r + i) * D + d] = __float2bfloat16_rn(scale * acc[i]);
-  } else {
-    __nv_bfloat16* dst = out + ((size_t)e * D + d) * r;
-    for (int i = 0; i < r; ++i) dst[i] = __float2bfloat16_rn(scale * acc[i]);
+#pragma unroll
+  for (int i = 0; i < RP; ++i) {
+    if (i < r) {
+      const __nv_bfloat16 o = __float2bfloat16_rn(scale * acc[i]);
+      if (transpose) out[((size_t)e * r + i) * D + d] = o;
+      else out[((size_t)e * D + d) * r + i] = o;
+    }
   }
 }
 

@@ -181,3 +181,14 @@ def test_full_size_sampled_parity(name):
     buf = run_layer(inp, cfg)
     errs = check_sampled_parity(buf, cpu, cfg)
     print(name, errs)
+
+
+def test_expert_spanning_several_chunks():
+    # 1500 rows on one expert: several token chunks in the grouped GEMMs and two
+    # row chunks in the adapter-gradient reduction
+    cfg = small_config(T=1500, m=64, n=48, E=4, k=1, r=16, alpha=16)
+
+    def mutate(cpu):
+        cpu["logits"][:, 0] += 30.0
+    errs, buf = _layer_case(cfg, mutate)
+    assert buf.counts.cpu().tolist()[0] == 1500
