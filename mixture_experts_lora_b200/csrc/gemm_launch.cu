@@ -157,19 +157,19 @@ cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const
 }
 
 template <int MODE, int RP, bool L_MN>
-static cudaError_t rows_rp(const GemmShape& g, const CUtensorMap& tl, const RowsParams& rp_,
+static cudaError_t rows_rp(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
                            cudaStream_t s) {
   using C = RowsCfg<MODE, RP, L_MN>;
   auto kern = rows_lowrank_kernel<MODE, RP, L_MN>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
   ProfScope ps(MODE == ROWS_GATHER ? K_ROWS_GATHER : (MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD), s);
-  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl, rp_);
+  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
   return cudaGetLastError();
 }
 
 template <int MODE, bool L_MN>
-static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap& tl, const RowsParams& rp_,
+static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
                              cudaStream_t s) {
   if (g.rp == 16) return rows_rp<MODE, 16, L_MN>(g, tl, rp_, s);
   return rows_rp<MODE, 32, L_MN>(g, tl, rp_, s);
@@ -180,10 +180,19 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
                                 const uint16_t* gu, const uint16_t* dh, const uint16_t* L,
                                 bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
                                 int r_save, uint16_t* outc, cudaStream_t s) {
-  CUtensorMap tl;
-  const uint64_t E = g.E, rp = g.rp;
-  const bool ok = L_mn ? encode3d(&tl, L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
-                       : encode3d(&tl, L, E, rp, (uint64_t)K, (uint32_t)rp, 64);
+  CUtensorMap tl[3];
+  const uint64_t E = g.E, rp = g.rp, P = g.P, n = g.n;
+  bool ok = L_mn ? encode3d(&tl[0], L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
+                 : encode3d(&tl[0], L, E, rp, (uint64_t)K, (uint32_t)rp, 64);
+  // input tiles of 128 rows x 64 columns, no swizzle (the threads read them back)
+  auto plain = [&](CUtensorMap* m, const void* base, uint64_t cols) {
+    const uint64_t dims[2] = {cols, P};
+    const uint64_t str[1] = {cols * 2};
+    const uint32_t box[2] = {64, 128};
+    return encode(m, base, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  };
+  ok = ok && plain(&tl[1], gu != nullptr ? gu : L, gu != nullptr ? 2 * n : 64);
+  ok = ok && plain(&tl[2], dh != nullptr ? dh : L, dh != nullptr ? n : 64);
   if (!ok) return cudaErrorInvalidValue;
   RowsParams p{};
   p.tiles = g.tiles;

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 2);
+      mbar_init(smem_u32(&full[s]), 33);   // TMA expect_tx arrive + 32 cp.async arrivals
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -116,20 +116,19 @@ __global__ void __launch_bounds__(192, 1)
         }
         // Small tile [64 rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
         // columns (128 B), row groups 128 B apart, column groups 1024 B apart.
-        uint8_t* ssm = smem + stage * C::STAGE_BYTES + C::BIG_BYTES;
+        // Rows outside the chunk (and columns past r_small) are zero-filled.
+        const uint32_t ssm = sbig + C::BIG_BYTES;
         constexpr int CG = RP / 8;
 #pragma unroll
         for (int i = lane; i < C::BK * CG; i += 32) {
           const int rr = i / CG, cg = i % CG;
           const int row = r0 + rr;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (row < ch.row_end && cg * 8 < p.r_small)
-            v = *reinterpret_cast<const uint4*>(p.small + (size_t)row * p.ld_small + cg * 8);
-          *reinterpret_cast<uint4*>(ssm + cg * 1024 + (rr & 7) * 16 + (rr >> 3) * 128) = v;
+          const bool valid = row < ch.row_end && cg * 8 < p.r_small;
+          const void* src = valid ? (const void*)(p.small + (size_t)row * p.ld_small + cg * 8)
+                                  : (const void*)p.small;
+          cp_async_16(ssm + cg * 1024 + (rr & 7) * 16 + (rr >> 3) * 128, src, valid ? 16u : 0u);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(fb);
+        cp_async_mbar_arrive(fb);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
@@ -153,6 +152,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int ks = 0; ks < nk; ++ks) {
           if (*abort_flag) { ok = false; break; }
           if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+          fence_proxy_async_smem();   // cp.async writes -> tcgen05 reads
           tc_fence_after();
           const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
           const uint32_t ssm = sbig + C::BIG_BYTES;

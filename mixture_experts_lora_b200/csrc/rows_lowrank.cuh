@@ -49,12 +49,18 @@ struct RowsParams {
 
 template <int MODE, int RP, bool L_MN>
 struct RowsCfg {
-  static constexpr int BM = 128, BK = 64, THREADS = 256;
+  static constexpr int BM = 128, BK = 64, THREADS = 512, PASSES = BM * 8 / THREADS;
   static constexpr int HALVES = MODE == ROWS_SWIGLU_BWD ? 2 : 1;   // dg and du chunks together
   static constexpr int A_BYTES = HALVES * BM * BK * 2;
   static constexpr int L_BYTES = HALVES * RP * BK * 2;
-  static constexpr int BUF_BYTES = A_BYTES + L_BYTES;
-  static constexpr int SMEM_BYTES = 2 * BUF_BYTES + 256 + 1024;
+  static constexpr int L_RING = 4;                     // L chunks loaded two iterations ahead
+  static constexpr int BUF_BYTES = A_BYTES;
+  static constexpr int NT = MODE == ROWS_GATHER ? 1 : (MODE == ROWS_SWIGLU ? 2 : 3);  // input tensors
+  static constexpr int TILE_BYTES = BM * BK * 2;
+  static constexpr int IN_STAGES = 2;
+  static_assert(IN_STAGES >= 2, "input ring");
+  static constexpr int IN_BYTES = IN_STAGES * NT * TILE_BYTES;
+  static constexpr int SMEM_BYTES = 2 * A_BYTES + L_RING * L_BYTES + IN_BYTES + 256 + 1024;
   static constexpr int TMEM_COLS = 32;
 };
 
@@ -74,8 +80,9 @@ __device__ __forceinline__ void unpack8(uint4 v, float (&x)[8]) {
 }
 
 template <int MODE, int RP, bool L_MN>
-__global__ void __launch_bounds__(256)
-    rows_lowrank_kernel(const __grid_constant__ CUtensorMap tmL, const RowsParams p) {
+__global__ void __launch_bounds__(512)
+    rows_lowrank_kernel(const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmGU,
+                        const __grid_constant__ CUtensorMap tmDH, const RowsParams p) {
   using C = RowsCfg<MODE, RP, L_MN>;
   const int tile = blockIdx.x;
   if (tile >= *p.n_tiles) return;
@@ -84,19 +91,23 @@ __global__ void __launch_bounds__(256)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * C::BUF_BYTES);
-  uint64_t* lfull = bars;        // [2] L chunk landed
-  uint64_t* mdone = bars + 2;    // [2] MMAs reading buffer b finished
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint8_t* lring = smem + 2 * C::A_BYTES;
+  uint8_t* in_ring = lring + C::L_RING * C::L_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(in_ring + C::IN_BYTES);
+  uint64_t* lfull = bars;        // [L_RING] L chunk landed
+  uint64_t* mdone = bars + C::L_RING;    // [2] MMAs of iteration it (parity it/2) finished
+  uint64_t* infull = bars + C::L_RING + 2;  // [IN_STAGES] input tiles landed (TMA modes)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::L_RING + 2 + C::IN_STAGES);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   if (tid == 0) {
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&lfull[b]), 1);
-      mbar_init(smem_u32(&mdone[b]), 1);
-    }
+    for (int b = 0; b < C::L_RING; ++b) mbar_init(smem_u32(&lfull[b]), 1);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&mdone[b]), 1);
+    for (int b = 0; b < C::IN_STAGES; ++b) mbar_init(smem_u32(&infull[b]), 1);
     mbar_fence_init();
     tma_prefetch_desc(&tmL);
+    if constexpr (MODE != ROWS_GATHER) tma_prefetch_desc(&tmGU);
+    if constexpr (MODE == ROWS_SWIGLU_BWD) tma_prefetch_desc(&tmDH);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -108,23 +119,23 @@ __global__ void __launch_bounds__(256)
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = idesc_bf16(128, RP, 0, L_MN ? 1 : 0);
 
-  // thread -> (row, 16-byte column group) of the 128 x 64 chunk, 4 passes of 32 rows
+  // thread -> (row, 16-byte column group) of the 128 x 64 chunk, PASSES passes of 64 rows
   const int cv = tid & 7;
   const int rbase = tid >> 3;
   bool ok = true;
   // iterations: 64 columns each (SWIGLU_BWD: 64 gate + the matching 64 up columns)
   const int n_it = MODE == ROWS_SWIGLU_BWD ? (p.n + C::BK - 1) / C::BK : p.nk;
 
-  // source rows of this thread's 4 rows (hoisted out of the column loop)
-  const __nv_bfloat16* srow[4];
-  float wrow[4];
-  bool rvalid[4];
+  // source rows of this thread's rows (hoisted out of the column loop)
+  const __nv_bfloat16* srow[C::PASSES];
+  float wrow[C::PASSES];
+  bool rvalid[C::PASSES];
 #pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-    const int q = ti.row0 + rbase + pass * 32;
+  for (int pass = 0; pass < C::PASSES; ++pass) {
+    const int q = ti.row0 + rbase + pass * 64;
     rvalid[pass] = q < ti.row_end;
     wrow[pass] = 1.0f;
-    srow[pass] = nullptr;
+    srow[pass] = p.gu != nullptr ? p.gu : p.src;
     if constexpr (MODE == ROWS_GATHER) {
       if (rvalid[pass]) {
         const int pr = p.sorted_pairs[q];
@@ -134,8 +145,9 @@ __global__ void __launch_bounds__(256)
     }
   }
 
-  auto load_l = [&](int it, int b) {   // L chunk(s) of iteration it into buffer b (thread 0)
-    const uint32_t lb = smem_u32(smem + b * C::BUF_BYTES + C::A_BYTES);
+  auto load_l = [&](int it) {   // L chunk(s) of iteration it into ring slot it % L_RING (thread 0)
+    const int b = it % C::L_RING;
+    const uint32_t lb = smem_u32(lring + b * C::L_BYTES);
     mbar_arrive_expect_tx(smem_u32(&lfull[b]), C::L_BYTES);
 #pragma unroll
     for (int h = 0; h < C::HALVES; ++h) {
@@ -146,54 +158,69 @@ __global__ void __launch_bounds__(256)
     }
   };
 
-  // registers holding the loads of one iteration: [pass][tensor]
-  constexpr int NT = MODE == ROWS_GATHER ? 1 : (MODE == ROWS_SWIGLU ? 2 : 3);
-  uint4 cur[4][NT], nxt[4][NT];
-  auto issue_loads = [&](int it, uint4 (&dst)[4][NT]) {
+  // Input ring: IN_STAGES x NT tensors x [128 rows][64 columns] (no swizzle); each
+  // thread copies and later reads back only its own 16-byte pieces, so its
+  // cp.async groups need no block-level synchronisation.
+  auto issue_loads = [&](int it) {
     const int col = it * C::BK + cv * 8;
+    uint8_t* st = in_ring + (it % C::IN_STAGES) * (C::NT * C::TILE_BYTES);
+    if constexpr (MODE == ROWS_GATHER) {
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int q = ti.row0 + rbase + pass * 32;
-#pragma unroll
-      for (int j = 0; j < NT; ++j) dst[pass][j] = make_uint4(0, 0, 0, 0);
-      if constexpr (MODE == ROWS_GATHER) {
-        if (rvalid[pass] && col < p.K) dst[pass][0] = *reinterpret_cast<const uint4*>(srow[pass] + col);
-      } else if constexpr (MODE == ROWS_SWIGLU) {
-        if (rvalid[pass] && col < p.n) {
-          dst[pass][0] = *reinterpret_cast<const uint4*>(p.gu + (size_t)q * 2 * p.n + col);
-          dst[pass][1] = *reinterpret_cast<const uint4*>(p.gu + (size_t)q * 2 * p.n + p.n + col);
-        }
+      for (int pass = 0; pass < C::PASSES; ++pass) {
+        const int r = rbase + pass * 64;
+        const uint32_t off = r * 128 + cv * 16;
+        const bool v = rvalid[pass] && col < p.K;
+        cp_async_16(smem_u32(st + off), v ? (const void*)(srow[pass] + col) : (const void*)p.src, v ? 16u : 0u);
+      }
+    } else if (tid == 0) {
+      // whole 128 x 64 tiles of the expert-sorted rows (rows past P read as zero)
+      const uint32_t fb = smem_u32(&infull[it % C::IN_STAGES]);
+      const int c0 = it * C::BK;
+      mbar_arrive_expect_tx(fb, C::NT * C::TILE_BYTES);
+      if constexpr (MODE == ROWS_SWIGLU) {
+        tma_load_2d(&tmGU, fb, smem_u32(st), c0, ti.row0);
+        tma_load_2d(&tmGU, fb, smem_u32(st + C::TILE_BYTES), p.n + c0, ti.row0);
       } else {
-        if (rvalid[pass] && col < p.n) {
-          dst[pass][0] = *reinterpret_cast<const uint4*>(p.dh + (size_t)q * p.n + col);
-          dst[pass][1] = *reinterpret_cast<const uint4*>(p.gu + (size_t)q * 2 * p.n + col);
-          dst[pass][2] = *reinterpret_cast<const uint4*>(p.gu + (size_t)q * 2 * p.n + p.n + col);
-        }
+        tma_load_2d(&tmDH, fb, smem_u32(st), c0, ti.row0);
+        tma_load_2d(&tmGU, fb, smem_u32(st + C::TILE_BYTES), c0, ti.row0);
+        tma_load_2d(&tmGU, fb, smem_u32(st + 2 * C::TILE_BYTES), p.n + c0, ti.row0);
       }
     }
   };
 
-  if (tid == 0) load_l(0, 0);
-  issue_loads(0, cur);
+  if (tid == 0) {
+    load_l(0);
+    if (n_it > 1) load_l(1);
+  }
+#pragma unroll
+  for (int j = 0; j < C::IN_STAGES - 1; ++j) {
+    if (j < n_it) issue_loads(j);
+    if constexpr (MODE == ROWS_GATHER) cp_async_commit();
+  }
 
   for (int it = 0; it < n_it; ++it) {
     const int b = it & 1;
-    uint8_t* abuf = smem + b * C::BUF_BYTES;
-    if (it + 1 < n_it) issue_loads(it + 1, nxt);     // in flight while this chunk is written
-    // buffer b was last read by the MMAs of iteration it - 2
-    if (it >= 2) ok = mbar_wait(smem_u32(&mdone[b]), ((it - 2) >> 1) & 1, p.err) && ok;
-    if (tid == 0 && it + 1 < n_it) {
-      if (it >= 1) ok = mbar_wait(smem_u32(&mdone[b ^ 1]), ((it - 1) >> 1) & 1, p.err) && ok;
-      load_l(it + 1, b ^ 1);
+    uint8_t* abuf = smem + b * C::A_BYTES;
+    if (it + C::IN_STAGES - 1 < n_it) issue_loads(it + C::IN_STAGES - 1);
+    if constexpr (MODE == ROWS_GATHER) {
+      cp_async_commit();
+      cp_async_wait<C::IN_STAGES - 1>();               // this thread's pieces have landed
+    } else {
+      ok = mbar_wait(smem_u32(&infull[it % C::IN_STAGES]), (it / C::IN_STAGES) & 1, p.err) && ok;
     }
+    // A buffer b and L slot (it + 2) % L_RING were last read by the MMAs of iteration it - 2
+    if (it >= 2) ok = mbar_wait(smem_u32(&mdone[b]), ((it - 2) >> 1) & 1, p.err) && ok;
+    if (tid == 0 && it + 2 < n_it) load_l(it + 2);
     const int col = it * C::BK + cv * 8;
+    const uint8_t* st = in_ring + (it % C::IN_STAGES) * (C::NT * C::TILE_BYTES);
+    uint4 out0[C::PASSES], out1[C::PASSES];
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int r = rbase + pass * 32;
-      const int q = ti.row0 + r;
+    for (int pass = 0; pass < C::PASSES; ++pass) {
+      const int r = rbase + pass * 64;
+      const uint32_t off = r * 128 + cv * 16;
       uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
       if constexpr (MODE == ROWS_GATHER) {
-        o0 = cur[pass][0];
+        o0 = *reinterpret_cast<const uint4*>(st + off);
         if (wrow[pass] != 1.0f) {
           float x[8];
           unpack8(o0, x);
@@ -201,34 +228,29 @@ __global__ void __launch_bounds__(256)
           for (int i = 0; i < 8; ++i) x[i] *= wrow[pass];
           o0 = pack8(x);
         }
-        if (rvalid[pass] && col < p.K && p.rows_out != nullptr)
-          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.K + col) = o0;
       } else if constexpr (MODE == ROWS_SWIGLU) {
         float g[8], u[8], h[8];
-        unpack8(cur[pass][0], g);
-        unpack8(cur[pass][1], u);
+        unpack8(*reinterpret_cast<const uint4*>(st + off), g);
+        unpack8(*reinterpret_cast<const uint4*>(st + C::TILE_BYTES + off), u);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) h[i] = g[i] / (1.0f + __expf(-g[i])) * u[i];
+        for (int i = 0; i < 8; ++i) h[i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * u[i];
         o0 = pack8(h);
-        if (rvalid[pass] && col < p.n) *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.n + col) = o0;
       } else {
         float d[8], g[8], u[8], dg[8], du[8];
-        unpack8(cur[pass][0], d);
-        unpack8(cur[pass][1], g);
-        unpack8(cur[pass][2], u);
+        unpack8(*reinterpret_cast<const uint4*>(st + off), d);
+        unpack8(*reinterpret_cast<const uint4*>(st + C::TILE_BYTES + off), g);
+        unpack8(*reinterpret_cast<const uint4*>(st + 2 * C::TILE_BYTES + off), u);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float s = 1.0f / (1.0f + __expf(-g[i]));
+          const float s = __fdividef(1.0f, 1.0f + __expf(-g[i]));
           dg[i] = d[i] * u[i] * s * (1.0f + g[i] * (1.0f - s));
           du[i] = d[i] * g[i] * s;
         }
         o0 = pack8(dg);
         o1 = pack8(du);
-        if (rvalid[pass] && col < p.n) {
-          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + col) = o0;
-          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + p.n + col) = o1;
-        }
       }
+      out0[pass] = o0;
+      out1[pass] = o1;
       // K-major, 128-byte swizzle: 16-byte group cv of row r lands at group cv ^ (r & 7)
       *reinterpret_cast<uint4*>(abuf + r * 128 + ((cv ^ (r & 7)) << 4)) = o0;
       if constexpr (C::HALVES == 2)
@@ -237,12 +259,12 @@ __global__ void __launch_bounds__(256)
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      ok = mbar_wait(smem_u32(&lfull[b]), (it >> 1) & 1, p.err) && ok;
+      ok = mbar_wait(smem_u32(&lfull[it % C::L_RING]), (it / C::L_RING) & 1, p.err) && ok;
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < C::HALVES; ++h) {
         const uint32_t sa = smem_u32(abuf) + h * (C::BM * C::BK * 2);
-        const uint32_t sl = smem_u32(abuf) + C::A_BYTES + h * (RP * C::BK * 2);
+        const uint32_t sl = smem_u32(lring + (it % C::L_RING) * C::L_BYTES) + h * (RP * C::BK * 2);
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk) {
           const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024, kSw128);
@@ -258,11 +280,21 @@ __global__ void __launch_bounds__(256)
       }
       umma_commit(smem_u32(&mdone[b]));
     }
-    if (it + 1 < n_it) {
+    // the rows themselves go to HBM after the shared-memory hand-off
 #pragma unroll
-      for (int pass = 0; pass < 4; ++pass)
-#pragma unroll
-        for (int j = 0; j < NT; ++j) cur[pass][j] = nxt[pass][j];
+    for (int pass = 0; pass < C::PASSES; ++pass) {
+      const int q = ti.row0 + rbase + pass * 64;
+      if constexpr (MODE == ROWS_GATHER) {
+        if (rvalid[pass] && col < p.K && p.rows_out != nullptr)
+          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.K + col) = out0[pass];
+      } else if constexpr (MODE == ROWS_SWIGLU) {
+        if (rvalid[pass] && col < p.n) *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.n + col) = out0[pass];
+      } else {
+        if (rvalid[pass] && col < p.n) {
+          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + col) = out0[pass];
+          *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + p.n + col) = out1[pass];
+        }
+      }
     }
   }
 
