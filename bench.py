@@ -127,9 +127,12 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- accounting
 def kernel_work(cfg):
-    """Algorithmic work of each kernel kind for one step: (unit, amount per step)."""
+    """Algorithmic work of each kernel kind for one step: (unit, amount per step).
+    Byte counts read and write each tensor once (rank-r outputs included)."""
     T, m, n, E, k, r = cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r
     P = T * k
+    rp = 16 if r <= 16 else 32
+    lr_out = P * r * 2 + P * rp * 2                       # saved LR + bf16(c LR)
     wgrad_bytes = 2 * (P * n + P * m + P * 2 * n + P * m) + 4 * P * r * 2 + E * r * (2 * m + 3 * n) * 2
     return {
         "gemm_gateup_fwd": ("flop", acc.flops_gemm_gate_up_fwd(T, m, n, k, r)),
@@ -138,7 +141,11 @@ def kernel_work(cfg):
         "gemm_gateup_bwd": ("flop", acc.flops_gemm_gate_up_bwd(T, m, n, k, r)),
         "lora_wgrad": ("byte", wgrad_bytes),
         "route_topk": ("byte", acc.bytes_route(T, E, k)),
-        "gather_rows": ("byte", 3 * acc.bytes_gather(T, m, k)),       # X fwd, w*dY and X bwd
+        # X rows (forward) and w*dY rows (backward): gather + rank-r product
+        "rows_gather": ("byte", 2 * (acc.bytes_gather(T, m, k) + P * 4 + lr_out)),
+        "rows_swiglu": ("byte", P * 2 * n * 2 + P * n * 2 + lr_out),
+        "rows_swiglu_bwd": ("byte", P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + lr_out),
+        "gather_rows": ("byte", acc.bytes_gather(T, m, k)),       # X again for dA_gu
         "unpermute_combine": ("byte", 2 * acc.bytes_combine(T, m, k)),  # Y and dX
     }
 
