@@ -160,6 +160,24 @@ moe_status_t moe_grouped_gemm_lora_bwd(
     moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream);
 
+/* The same permutation as moe_permute(), for callers that cannot allocate device
+ * memory: plug-ins hosted inside another framework that owns all device memory
+ * and hands them no allocator, or code that must run with a fixed device-memory
+ * footprint decided before it starts.  It takes no workspace; its scratch (the
+ * per-chunk histograms) is a 1 MiB array built into the library, which every GPU
+ * that loads the library holds until the process exits.  There is no
+ * counterpart on the pages: this is an interface convenience.
+ * Limit: ceil(T*k / 1024) * E <= 262144 (e.g. T*k <= 2^21 pairs at E = 128);
+ * larger problems return MOE_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  All calls share the one array: calls that overlap on the
+ * GPU (different streams, no ordering between them) race and must be avoided.
+ * Arguments, outputs and errors otherwise as moe_permute(). */
+moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                                 int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
+                                 int32_t* pair_pos, void* stream);
+
 /* Weighted un-permute: Y[t] = sum_{j=0..k-1} w[t,j] * Y_sorted[pair_pos[t*k+j]],
  * summed in fp32 over ascending j and rounded once to bf16.  With topk_w = NULL
  * every weight is 1 (the dX reduction of the backward).

@@ -30,7 +30,7 @@ MOE_ERR_TIMEOUT = 6
 EXPORTED = (
     "moe_workspace_bytes", "moe_route_topk", "moe_permute", "moe_grouped_gemm_lora_fwd",
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
-    "moe_status_string", "moe_profile_enable", "moe_profile_read",
+    "moe_status_string", "moe_profile_enable", "moe_profile_read", "moe_permute_noalloc",
 )
 
 
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         h.moe_workspace_bytes.restype = SZ
         h.moe_route_topk.argtypes = [P, I64, I32, I32, P, P, P]
         h.moe_permute.argtypes = [P, I64, I32, I32, P, P, P, P, P, SZ, P]
+        h.moe_permute_noalloc.argtypes = [P, I64, I32, I32, P, P, P, P, P]
         h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 15 + [SZ, P]
         h.moe_grouped_gemm_lora_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
         h.moe_unpermute_combine.argtypes = [P, P, P, I64, I32, I32, P, P]
@@ -120,6 +121,14 @@ def moe_permute(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, ws, stream
                                             _ptr(offsets), _ptr(sorted_pairs), _ptr(pair_pos),
                                             _ptr(ws), ws.numel() * ws.element_size(),
                                             _stream(stream)))
+
+
+def moe_permute_noalloc(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream=None):
+    """moe_permute without a workspace (scratch built into the library)."""
+    T, k = topk_ids.shape
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(
+        _ptr(topk_ids), T, k, int(E), _ptr(counts), _ptr(offsets), _ptr(sorted_pairs),
+        _ptr(pair_pos), _stream(stream)))
 
 
 def moe_grouped_gemm_lora_fwd(dims, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,

@@ -174,6 +174,9 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
 }
 
 }  // namespace
+
+int* moe_status_word() { return status_ptr(); }
+
 }  // namespace moe
 
 using namespace moe;

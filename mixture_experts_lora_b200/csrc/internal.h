@@ -31,6 +31,9 @@ struct ProfScope {
   ~ProfScope() { if (tok) prof_end(tok, s); }
 };
 
+// Device address of the status word of the current device (api.cu), or nullptr.
+int* moe_status_word();
+
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
