@@ -32,7 +32,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from moe_inputs import CONFIGS, generate, generate_tokens  # noqa: E402
+from moe_inputs import CONFIGS, generate  # noqa: E402
 from mixture_experts_lora_b200 import accounting as acc  # noqa: E402
 
 METRIC = "MoE-layer fwd+bwd tokens/s and TFLOP/s as % of B200 bf16 dense peak"
@@ -277,9 +277,8 @@ def run_ours(args, cfg):
     ml.lib()  # fails loudly if the CUDA library is missing
 
     # inputs: weights shared by every rank (seed 0), tokens per rank
-    inp = generate(cfg, seed=0, device=str(dev))
-    if rank > 0:
-        inp.update(generate_tokens(cfg, seed=1000 + rank, device=str(dev)))
+    from mixture_experts_lora_b200 import dp
+    inp = dp.rank_inputs(cfg, rank, device=dev)
     buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale, device=dev)
     grads = (buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -287,9 +286,7 @@ def run_ours(args, cfg):
 
     def step():
         ml.layer_step(inp, cfg.k, cfg.scale, buf)
-        if world > 1:
-            for g in grads:
-                dist.all_reduce(g)
+        dp.allreduce_adapter_grads(grads)
 
     for _ in range(args.warmup):
         step()
@@ -344,9 +341,7 @@ def run_ours(args, cfg):
             for k, v in h_in.items():
                 d_in[k].copy_(v, non_blocking=True)
             ml.layer_step(d_in, cfg.k, cfg.scale, buf)
-            if world > 1:
-                for g in grads:
-                    dist.all_reduce(g)
+            dp.allreduce_adapter_grads(grads)
             for o, h in zip(outs, h_out):
                 h.copy_(o, non_blocking=True)
 
