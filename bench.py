@@ -126,28 +126,58 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- accounting
-def kernel_work(cfg):
-    """Algorithmic work of each kernel kind for one step: (unit, amount per step).
-    Byte counts read and write each tensor once (rank-r outputs included)."""
+def kernel_work(cfg, active_experts=None):
+    """Algorithmic work of each kernel kind for one step: {kind: {"flop": F, "byte": B}}.
+    Byte counts read and write each tensor once (rank-r outputs included); a GEMM
+    reads the frozen weights of the experts that received tokens once."""
     T, m, n, E, k, r = cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r
+    Ea = E if active_experts is None else active_experts
     P = T * k
     rp = 16 if r <= 16 else 32
     lr_out = P * r * 2 + P * rp * 2                       # saved LR + bf16(c LR)
     wgrad_bytes = 2 * (P * n + P * m + P * 2 * n + P * m) + 4 * P * r * 2 + E * r * (2 * m + 3 * n) * 2
+    lrc = P * rp * 2
     return {
-        "gemm_gateup_fwd": ("flop", acc.flops_gemm_gate_up_fwd(T, m, n, k, r)),
-        "gemm_down_fwd": ("flop", acc.flops_gemm_down_fwd(T, m, n, k, r)),
-        "gemm_down_bwd": ("flop", acc.flops_gemm_down_bwd(T, m, n, k, r)),
-        "gemm_gateup_bwd": ("flop", acc.flops_gemm_gate_up_bwd(T, m, n, k, r)),
-        "lora_wgrad": ("byte", wgrad_bytes),
-        "route_topk": ("byte", acc.bytes_route(T, E, k)),
+        "gemm_gateup_fwd": {"flop": acc.flops_gemm_gate_up_fwd(T, m, n, k, r),
+                            "byte": Ea * m * 2 * n * 2 + P * m * 2 + lrc + Ea * rp * 2 * n * 2 + P * 2 * n * 2},
+        "gemm_down_fwd": {"flop": acc.flops_gemm_down_fwd(T, m, n, k, r),
+                          "byte": Ea * n * m * 2 + P * n * 2 + lrc + Ea * rp * m * 2 + P * m * 2},
+        "gemm_down_bwd": {"flop": acc.flops_gemm_down_bwd(T, m, n, k, r),
+                          "byte": Ea * n * m * 2 + P * m * 2 + lrc + Ea * n * rp * 2 + P * n * 2},
+        "gemm_gateup_bwd": {"flop": acc.flops_gemm_gate_up_bwd(T, m, n, k, r),
+                            "byte": Ea * m * 2 * n * 2 + P * 2 * n * 2 + lrc + Ea * m * rp * 2 + P * m * 2},
+        "lora_wgrad": {"byte": wgrad_bytes},
+        "route_topk": {"byte": acc.bytes_route(T, E, k)},
         # X rows (forward) and w*dY rows (backward): gather + rank-r product
-        "rows_gather": ("byte", 2 * (acc.bytes_gather(T, m, k) + P * 4 + lr_out)),
-        "rows_swiglu": ("byte", P * 2 * n * 2 + P * n * 2 + lr_out),
-        "rows_swiglu_bwd": ("byte", P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + lr_out),
-        "gather_rows": ("byte", acc.bytes_gather(T, m, k)),       # X again for dA_gu
-        "unpermute_combine": ("byte", 2 * acc.bytes_combine(T, m, k)),  # Y and dX
+        "rows_gather": {"byte": 2 * (acc.bytes_gather(T, m, k) + P * 4 + lr_out)},
+        "rows_swiglu": {"byte": P * 2 * n * 2 + P * n * 2 + lr_out},
+        "rows_swiglu_bwd": {"byte": P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + lr_out},
+        "gather_rows": {"byte": acc.bytes_gather(T, m, k)},       # X again for dA_gu
+        "unpermute_combine": {"byte": 2 * acc.bytes_combine(T, m, k)},  # Y and dX
     }
+
+
+def roof_entry(work, per_launch_ms, launches_per_step, peaks):
+    """Roofline of one kernel kind: achieved rate of each resource it uses and the
+    binding one (the larger ideal time at the measured peaks)."""
+    ent = {}
+    sec = per_launch_ms / 1e3
+    opts = []
+    if "flop" in work:
+        f = work["flop"] / launches_per_step
+        a = f / sec / 1e12
+        ent["tensor"] = {"achieved": a, "unit": "TFLOP/s", "peak": peaks["bf16_tflops_sustained"],
+                         "frac": a / peaks["bf16_tflops_sustained"], "per_launch": f}
+        opts.append(("tensor", f / (peaks["bf16_tflops_sustained"] * 1e12)))
+    if "byte" in work:
+        b = work["byte"] / launches_per_step
+        a = b / sec / 1e9
+        ent["hbm"] = {"achieved": a, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                      "frac": a / peaks["hbm_gbs"], "per_launch": b}
+        opts.append(("hbm", b / (peaks["hbm_gbs"] * 1e9)))
+    if opts:
+        ent["bound"] = max(opts, key=lambda o: o[1])[0]
+    return ent
 
 
 def src_hash():
@@ -295,7 +325,22 @@ def run_ours(args, cfg):
     if st != ml.MOE_OK:
         raise SystemExit(f"device error after warm-up: {ml.status_string(st)}")
 
-    # ---- timed region (device time, CUDA events per step, L2 flushed before each step)
+    # ---- traced pass (not the timed value): every kernel kind bracketed by CUDA
+    # events, for the per-kernel breakdown and to find the dominant kernel
+    ml.moe_profile_select(None)
+    ml.moe_profile_enable(True)
+    for _ in range(args.steps):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ml.moe_profile_enable(False)
+    prof_all = ml.moe_profile_read()
+    launches_per_step = sum(v[0] for v in prof_all.values()) / args.steps
+    top = max(prof_all, key=lambda k: prof_all[k][1]) if prof_all else None
+
+    # ---- timed region (device time, CUDA events per step, L2 flushed before each
+    # step); only the dominant kernel kind is traced, so its events add two
+    # records per launch and nothing to the other kernels
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -304,7 +349,9 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ml.moe_profile_enable(True)
+    if top is not None:
+        ml.moe_profile_select(top)
+        ml.moe_profile_enable(True)
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
@@ -312,12 +359,14 @@ def run_ours(args, cfg):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     ml.moe_profile_enable(False)
-    prof = ml.moe_profile_read()
+    prof_top = ml.moe_profile_read()
+    ml.moe_profile_select(None)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in evs]
     mean_ms = statistics.mean(step_ms)
+    median_ms = statistics.median(step_ms)
     if world > 1:
         t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -325,6 +374,7 @@ def run_ours(args, cfg):
     st = ml.moe_get_device_error()
     if st != ml.MOE_OK:
         raise SystemExit(f"device error in timed region: {ml.status_string(st)}")
+    active_experts = int((buf.counts > 0).sum().item())
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -374,33 +424,32 @@ def run_ours(args, cfg):
     peaks, peak_src = load_peaks()
     flops = acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r)
     tflops = flops / (mean_ms / 1e3) / 1e12
-    work = kernel_work(cfg)
+    work = kernel_work(cfg, active_experts)
+    total_traced = max(1e-9, sum(v[1] for v in prof_all.values()))
     kernels = {}
-    for name, (launches, tot_ms) in prof.items():
-        per_launch_ms = tot_ms / launches
-        ent = {"launches": launches, "ms_per_step": tot_ms / args.steps,
-               "share": tot_ms / max(1e-9, sum(v[1] for v in prof.values()))}
+    for name, (launches, tot_ms) in prof_all.items():
+        ent = {"launches": launches, "ms_per_step": tot_ms / args.steps, "share": tot_ms / total_traced}
         if name in work:
-            unit, amount = work[name]
-            per_launch = amount * args.steps / launches
-            if unit == "flop":
-                ent.update(bound="tensor", achieved=per_launch / (per_launch_ms / 1e3) / 1e12,
-                           unit="TFLOP/s", peak=peaks["bf16_tflops_sustained"])
-            else:
-                ent.update(bound="hbm", achieved=per_launch / (per_launch_ms / 1e3) / 1e9,
-                           unit="GB/s", peak=peaks["hbm_gbs"])
-            ent["frac"] = ent["achieved"] / ent["peak"]
-            ent["algorithmic_per_launch"] = per_launch
+            ent.update(roof_entry(work[name], tot_ms / launches, launches / args.steps, peaks))
         kernels[name] = ent
-    top = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
     roof = None
-    if top is not None and "bound" in kernels[top]:
-        kt = kernels[top]
-        roof = {"kernel": top, "bound": kt["bound"], "achieved": kt["achieved"], "peak": kt["peak"],
-                "unit": kt["unit"], "frac": kt["frac"],
-                "peak_source": f"{peak_src} ({'bf16_tflops_sustained' if kt['bound'] == 'tensor' else 'hbm_gbs'}, MEASURED_PEAKS.json)",
-                "traffic": ncu_traffic(top, cfg.name)}
-    launches_total = sum(v[0] for v in prof.values())
+    if top is not None and top in prof_top and top in work:
+        launches, tot_ms = prof_top[top]
+        re_ = roof_entry(work[top], tot_ms / launches, launches / args.steps, peaks)
+        b = re_["bound"]
+        pk = "bf16_tflops_sustained" if b == "tensor" else "hbm_gbs"
+        roof = {"kernel": top, "bound": b, "achieved": re_[b]["achieved"], "peak": re_[b]["peak"],
+                "unit": re_[b]["unit"], "frac": re_[b]["frac"],
+                "peak_source": f"{peak_src} ({pk}, MEASURED_PEAKS.json)",
+                "traffic": ncu_traffic(top, cfg.name),
+                "algorithmic_per_launch": re_[b]["per_launch"],
+                "ms_per_launch": tot_ms / launches,
+                "measured_in": "timed region (CUDA events on the launch stream around this kernel only)"}
+        other = "hbm" if b == "tensor" else "tensor"
+        if other in re_:
+            roof["other_resource"] = {"resource": other, "achieved": re_[other]["achieved"],
+                                      "unit": re_[other]["unit"], "frac": re_[other]["frac"]}
+    launches_total = int(round(launches_per_step * args.steps))
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         cpu_inp = {k: v.cpu() for k, v in inp.items()}
@@ -421,8 +470,11 @@ def run_ours(args, cfg):
         "algorithmic_flop_per_step": flops,
         "roofline": roof,
         "kernels": kernels,
+        "kernels_source": "separate traced pass of the same steps (every launch bracketed by CUDA events)",
         "gpu_launches": launches_total,
         "step_ms_min_max": [min(step_ms), max(step_ms)],
+        "step_ms_median": median_ms,
+        "active_experts": active_experts,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -201,6 +201,13 @@ const char* moe_status_string(moe_status_t status);
  * from a host-side pool, no device memory is allocated.  Off by default. */
 void moe_profile_enable(int on);
 
+/* Restricts the tracing to the kernel kinds named in `kinds`, a comma-separated
+ * list of the names moe_profile_read reports (e.g. "gemm_gateup_fwd,lora_wgrad");
+ * NULL or "" selects every kind (the default).  Returns the number of kinds
+ * selected, or -1 (selection unchanged) if a name is unknown.  Tracing one kernel
+ * kind keeps the event overhead out of the rest of a timed step. */
+int moe_profile_select(const char* kinds);
+
 /* Waits for the recorded events and reports, per kernel kind that ran since
  * the last read, its name (NUL-terminated, at most name_len bytes, row w of
  * `names`), its launch count and its summed device time in milliseconds.

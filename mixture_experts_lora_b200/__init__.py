@@ -30,7 +30,8 @@ MOE_ERR_TIMEOUT = 6
 EXPORTED = (
     "moe_workspace_bytes", "moe_route_topk", "moe_permute", "moe_grouped_gemm_lora_fwd",
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
-    "moe_status_string", "moe_profile_enable", "moe_profile_read", "moe_permute_noalloc",
+    "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
+    "moe_permute_noalloc",
 )
 
 
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
         h.moe_status_string.restype = ctypes.c_char_p
         h.moe_profile_enable.argtypes = [ctypes.c_int]
         h.moe_profile_enable.restype = None
+        h.moe_profile_select.argtypes = [ctypes.c_char_p]
         h.moe_profile_read.argtypes = [ctypes.c_int, ctypes.c_char_p, ctypes.c_int,
                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
         for name in EXPORTED:
@@ -162,6 +164,16 @@ def moe_get_device_error(stream=None) -> int:
 
 def moe_profile_enable(on: bool = True):
     lib().moe_profile_enable(1 if on else 0)
+
+
+def moe_profile_select(kinds=None) -> int:
+    """Trace only the named kernel kinds (a list or comma-separated string); None = all."""
+    if kinds is not None and not isinstance(kinds, str):
+        kinds = ",".join(kinds)
+    n = lib().moe_profile_select(None if not kinds else kinds.encode())
+    if n < 0:
+        raise ValueError(f"unknown kernel kind in {kinds!r}")
+    return n
 
 
 def moe_profile_read() -> dict:

@@ -21,13 +21,14 @@ enum KernelKind : int {
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
 bool prof_enabled();
+bool prof_traced(int kind);   // enabled and the kind is selected
 void* prof_begin(int kind, cudaStream_t s);   // returns a record token (or nullptr)
 void prof_end(void* token, cudaStream_t s);
 
 struct ProfScope {
   void* tok;
   cudaStream_t s;
-  ProfScope(int kind, cudaStream_t st) : tok(prof_enabled() ? prof_begin(kind, st) : nullptr), s(st) {}
+  ProfScope(int kind, cudaStream_t st) : tok(prof_traced(kind) ? prof_begin(kind, st) : nullptr), s(st) {}
   ~ProfScope() { if (tok) prof_end(tok, s); }
 };
 

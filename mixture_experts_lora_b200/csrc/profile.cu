@@ -4,6 +4,7 @@
 // kernel kind, the number of launches and their summed device time.  Events
 // come from a pool that grows on demand and is reused; no device memory is
 // allocated.
+#include <atomic>
 #include <mutex>
 #include <string.h>
 #include <vector>
@@ -26,7 +27,8 @@ struct Rec {
   bool closed;
 };
 std::mutex g_mu;
-bool g_on = false;
+std::atomic<bool> g_on{false};
+std::atomic<uint32_t> g_kinds{~0u};     // bit k set: launches of kind k are traced
 std::vector<Rec*> g_recs;
 std::vector<cudaEvent_t> g_pool;
 
@@ -42,7 +44,9 @@ cudaEvent_t take_event() {
 }
 }  // namespace
 
-bool prof_enabled() { return g_on; }
+bool prof_enabled() { return g_on.load(); }
+
+bool prof_traced(int kind) { return g_on.load() && ((g_kinds.load() >> kind) & 1u); }
 
 void* prof_begin(int kind, cudaStream_t s) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -69,6 +73,30 @@ extern "C" {
 void moe_profile_enable(int on) {
   std::lock_guard<std::mutex> lk(g_mu);
   g_on = on != 0;
+}
+
+int moe_profile_select(const char* kinds) {
+  uint32_t mask = 0;
+  int n = 0;
+  if (kinds == nullptr || kinds[0] == 0) {
+    mask = ~0u;
+  } else {
+    const char* p = kinds;
+    while (*p) {
+      const char* q = p;
+      while (*q && *q != ',') ++q;
+      const size_t len = (size_t)(q - p);
+      int found = -1;
+      for (int k = 0; k < K_NUM_KINDS; ++k)
+        if (strlen(kKernelNames[k]) == len && strncmp(kKernelNames[k], p, len) == 0) found = k;
+      if (found < 0) return -1;
+      mask |= 1u << found;
+      ++n;
+      p = *q ? q + 1 : q;
+    }
+  }
+  g_kinds.store(mask);
+  return kinds == nullptr || kinds[0] == 0 ? K_NUM_KINDS : n;
 }
 
 int moe_profile_read(int max_kinds, char* names, int name_len, int* launches, double* total_ms) {
