@@ -164,10 +164,10 @@ moe_status_t moe_grouped_gemm_lora_bwd(
  * memory: plug-ins hosted inside another framework that owns all device memory
  * and hands them no allocator, or code that must run with a fixed device-memory
  * footprint decided before it starts.  It takes no workspace; its scratch (the
- * per-chunk histograms) is a 1 MiB array built into the library, which every GPU
+ * per-chunk histograms) is a 2 MiB array built into the library, which every GPU
  * that loads the library holds until the process exits.  There is no
  * counterpart on the pages: this is an interface convenience.
- * Limit: ceil(T*k / 1024) * E <= 262144 (e.g. T*k <= 2^21 pairs at E = 128);
+ * Limit: ceil(T*k / 512) * E <= 524288 (e.g. T*k <= 2^21 pairs at E = 128);
  * larger problems return MOE_ERR_WORKSPACE before any launch.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before

@@ -38,8 +38,8 @@ int* moe_status_word();
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
-// per-warp chunks of kPermuteChunk pairs; hist holds n_chunks * E ints
-constexpr int kPermuteChunk = 1024;
+// one block per chunk of kPermuteChunk pairs; hist holds n_chunks * E ints
+constexpr int kPermuteChunk = 512;
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
                            int32_t* hist, int* err, cudaStream_t s);

@@ -14,8 +14,8 @@
 namespace moe {
 namespace {
 
-// 2^18 int32 = 1 MiB: room for ceil(T*k / 1024) * E histogram entries.
-constexpr size_t kPermuteScratchInts = size_t(1) << 18;
+// 2^19 int32 = 2 MiB: room for ceil(T*k / kPermuteChunk) * E histogram entries.
+constexpr size_t kPermuteScratchInts = size_t(1) << 19;
 __device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts];
 
 constexpr int kMaxDevices = 64;

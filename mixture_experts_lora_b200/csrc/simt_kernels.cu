@@ -7,12 +7,50 @@
 
 namespace moe {
 
+// ------------------------------------------------------------------ block scan
+// Exclusive scan of one int per thread over a block of up to 1024 threads;
+// *total_out receives the block total.  s_warp holds 33 ints.
+__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int* total_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
+    int inc2 = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
+      if (lane >= off) inc2 += u;
+    }
+    s_warp[lane] = inc2 - w;
+    if (lane == 31) s_warp[32] = inc2;
+  }
+  __syncthreads();
+  *total_out = s_warp[32];
+  return incl - v + s_warp[warp];
+}
+
 // ------------------------------------------------------------------ routing
-// One warp per token.  Each lane holds logits e = lane + 32 i in shared memory;
-// k rounds of a warp arg-max on (value, lower index wins ties) pick the experts
-// in descending order; the weights are a softmax over the k picked logits.
-// Router equation: "Accelerating Mixture-of-Experts Fine-Tuning", section "The
-// Dynamic Dispatch Bottleneck in Mixture-of-Experts Architectures".
+// One warp per token; the token's logits are staged in shared memory.  Each of
+// the k rounds picks the largest remaining logit, lower expert id on ties: every
+// lane proposes its best untaken candidate as (order-preserving key of the
+// value, lower id wins), two warp max-reductions (redux.sync) pick the winner.
+// The weights are a softmax over the k picked logits.  Router equation:
+// "Accelerating Mixture-of-Experts Fine-Tuning", section "The Dynamic Dispatch
+// Bottleneck in Mixture-of-Experts Architectures".
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;                       // -0 ties with +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // larger float -> larger key
+}
+
 __global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
                                   int32_t* __restrict__ ids, float* __restrict__ wout) {
   extern __shared__ float s_logits[];
@@ -28,24 +66,18 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, i
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    bool found = false;
-    float bv = 0.f;
-    int bi = 0x7fffffff;
+    uint32_t bkey = 0, blo = 0;          // blo = ~e of the lane's candidate (0: none)
     for (int i = 0; i < per_lane; ++i) {
       const int e = lane + 32 * i;
       if (e >= E || ((taken >> i) & 1u)) continue;
-      const float v = row[e];
-      if (!found || v > bv) { bv = v; bi = e; found = true; }
+      const uint32_t key = order_key(row[e]);
+      if (blo == 0 || key > bkey) { bkey = key; blo = ~(uint32_t)e; }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      const bool of = __shfl_xor_sync(0xffffffffu, (int)found, off) != 0;
-      if (of && (!found || ov > bv || (ov == bv && oi < bi))) { bv = ov; bi = oi; found = true; }
-    }
+    const uint32_t wkey = __reduce_max_sync(0xffffffffu, blo != 0 ? bkey : 0u);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, (blo != 0 && bkey == wkey) ? blo : 0u);
+    const int bi = (int)(~wlo);
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == j) { my_val = bv; my_id = bi; }
+    if (lane == j) { my_val = row[bi]; my_id = bi; }
   }
   const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
   const float z = lane < k ? expf(my_val - vmax) : 0.f;
@@ -72,122 +104,116 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 
 // ------------------------------------------------------------------ permute
 // Counting sort in three launches.  Pairs are cut into chunks of kPermuteChunk
-// consecutive pair indices, one warp per chunk:
-//   1. histogram of each chunk                       -> hist[c][e]
-//   2. one block: counts, exclusive offsets, and the first sorted position of
-//      each (chunk, expert) = offsets[e] + sum of earlier chunks  -> hist[c][e]
-//   3. each warp walks its chunk in pair order, 32 pairs at a time; lanes with
-//      the same expert are ranked with __match_any_sync, so positions are stable
-//      (ascending pair index inside every expert segment).
+// consecutive pair indices, one 512-thread block per chunk, one pair per thread:
+//   1. histogram of each chunk (shared-memory atomics)     -> hist[e][c]
+//   2. one block: per expert, an exclusive scan over the chunks (a warp per
+//      expert column), counts and offsets from a block scan over the experts,
+//      then hist[e][c] = offsets[e] + pairs of expert e in chunks before c
+//   3. each block ranks its pairs: __match_any_sync groups the lanes of a warp by
+//      expert (rank = earlier lanes of the group), a shared [warp][expert] table
+//      prefix-summed over the warps orders the warps, hist gives the chunk base;
+//      positions are therefore stable (ascending pair index inside every segment).
 // Replaces the per-expert mask lookup of the loop form ("What is
 // torch._grouped_mm?", Unsloth faster-moe docs).
-__global__ void permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E,
-                                    int32_t* __restrict__ hist, int* err) {
+constexpr int kPermThreads = kPermuteChunk;
+constexpr int kPermWarps = kPermThreads / 32;
+
+__global__ void __launch_bounds__(kPermThreads)
+    permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
+                        int32_t* __restrict__ hist, int* err) {
   extern __shared__ int s_hist[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t chunk = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
-  if (chunk >= n_chunks) return;
-  int* h = s_hist + warp * E;
-  for (int e = lane; e < E; e += 32) h[e] = 0;
-  __syncwarp();
-  const int64_t p0 = chunk * kPermuteChunk;
-  const int64_t p1 = p0 + kPermuteChunk < P ? p0 + kPermuteChunk : P;
-  for (int64_t p = p0 + lane; p < p1; p += 32) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int64_t p = (int64_t)blockIdx.x * kPermuteChunk + threadIdx.x;
+  if (p < P) {
     const int e = ids[p];
-    if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+    if (e >= 0 && e < E) atomicAdd(&s_hist[e], 1);
     else report_error(err, MOE_ERR_DEVICE_INDEX);
   }
-  __syncwarp();
-  for (int e = lane; e < E; e += 32) hist[chunk * E + e] = h[e];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    hist[(int64_t)e * n_chunks + blockIdx.x] = s_hist[e];
 }
 
-__global__ void permute_scan_kernel(int32_t* __restrict__ hist, int64_t n_chunks, int E, int64_t P,
-                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
-  __shared__ int s_warp[32];
-  const int e = threadIdx.x;  // blockDim.x = 1024 >= E
-  int total = 0;
-  if (e < E) {
-    for (int64_t c = 0; c < n_chunks; ++c) {
-      const int v = hist[c * E + e];
-      hist[c * E + e] = total;
-      total += v;
-    }
-  }
-  // block exclusive scan of `total`
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = total;
+__global__ void __launch_bounds__(1024)
+    permute_scan_kernel(int32_t* __restrict__ hist, int n_chunks, int E, int64_t P,
+                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int s_tot[1024];
+  __shared__ int s_warp[33];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = warp; e < E; e += 32) {
+    int32_t* col = hist + (int64_t)e * n_chunks;
+    int run = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int v = c < n_chunks ? col[c] : 0;
+      int incl = v;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int v = s_warp[lane];
-    int inc2 = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
-      if (lane >= off) inc2 += u;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+      }
+      if (c < n_chunks) col[c] = run + incl - v;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    s_warp[lane] = inc2 - v;
+    if (lane == 0) s_tot[e] = run;
   }
   __syncthreads();
-  const int excl = incl - total + s_warp[warp];
+  const int e = threadIdx.x;
+  const int tot = e < E ? s_tot[e] : 0;
+  int all;
+  const int excl = block_exclusive_scan_1024(tot, s_warp, &all);
   if (e < E) {
-    counts[e] = total;
+    counts[e] = tot;
     offsets[e] = excl;
-    for (int64_t c = 0; c < n_chunks; ++c) hist[c * E + e] += excl;
+    s_tot[e] = excl;
   }
   if (e == 0) offsets[E] = (int32_t)P;
+  __syncthreads();
+  const int64_t total = (int64_t)n_chunks * E;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) hist[i] += s_tot[i / n_chunks];
 }
 
-__global__ void permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E,
-                                       const int32_t* __restrict__ base,
-                                       int32_t* __restrict__ sorted_pairs,
-                                       int32_t* __restrict__ pair_pos) {
-  extern __shared__ int s_run[];
+__global__ void __launch_bounds__(kPermThreads)
+    permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
+                           const int32_t* __restrict__ base, int32_t* __restrict__ sorted_pairs,
+                           int32_t* __restrict__ pair_pos) {
+  extern __shared__ int s_cnt[];   // [kPermWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t chunk = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
-  if (chunk >= n_chunks) return;
-  int* run = s_run + warp * E;
-  for (int e = lane; e < E; e += 32) run[e] = base[chunk * E + e];
-  __syncwarp();
-  const int64_t p0 = chunk * kPermuteChunk;
-  const int64_t p1 = p0 + kPermuteChunk < P ? p0 + kPermuteChunk : P;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  for (int64_t pb = p0; pb < p1; pb += 32) {
-    const int64_t p = pb + lane;
-    int e = -1;
-    if (p < p1) e = ids[p];
-    const bool ok = p < p1 && e >= 0 && e < E;
-    const int key = ok ? e : -1 - lane;  // invalid lanes never group
-    const unsigned grp = __match_any_sync(0xffffffffu, key);
-    int pos = 0;
-    if (ok) pos = run[e] + __popc(grp & lt_mask);
-    __syncwarp();
-    if (ok && (31 - __clz(grp)) == lane) run[e] += __popc(grp);
-    __syncwarp();
-    if (ok) {
-      sorted_pairs[pos] = (int32_t)p;
-      pair_pos[p] = pos;
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_cnt[i] = 0;
+  __syncthreads();
+  const int64_t p = (int64_t)blockIdx.x * kPermuteChunk + threadIdx.x;
+  int e = -1;
+  if (p < P) e = ids[p];
+  const bool ok = p < P && e >= 0 && e < E;
+  const int key = ok ? e : -1 - lane;  // invalid lanes never group
+  const unsigned grp = __match_any_sync(0xffffffffu, key);
+  const int rank = __popc(grp & ((1u << lane) - 1u));
+  if (ok && (31 - __clz(grp)) == lane) s_cnt[warp * E + e] = __popc(grp);
+  __syncthreads();
+  for (int ee = threadIdx.x; ee < E; ee += blockDim.x) {
+    int run = base[(int64_t)ee * n_chunks + blockIdx.x];
+    for (int w = 0; w < kPermWarps; ++w) {
+      const int t = s_cnt[w * E + ee];
+      s_cnt[w * E + ee] = run;
+      run += t;
     }
+  }
+  __syncthreads();
+  if (ok) {
+    const int pos = s_cnt[warp * E + e] + rank;
+    sorted_pairs[pos] = (int32_t)p;
+    pair_pos[p] = pos;
   }
 }
 
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts, int32_t* offsets,
                            int32_t* sorted_pairs, int32_t* pair_pos, int32_t* hist, int* err,
                            cudaStream_t s) {
-  const int64_t n_chunks = (P + kPermuteChunk - 1) / kPermuteChunk;
-  const int warps = 4;
-  const size_t smem = (size_t)warps * E * sizeof(int);
-  const unsigned blocks = (unsigned)((n_chunks + warps - 1) / warps);
+  const int n_chunks = (int)((P + kPermuteChunk - 1) / kPermuteChunk);
   if (n_chunks > 0) {
     ProfScope ps(K_PERM_HIST, s);
-    permute_hist_kernel<<<blocks, warps * 32, smem, s>>>(ids, P, E, hist, err);
+    permute_hist_kernel<<<n_chunks, kPermThreads, E * sizeof(int), s>>>(ids, P, E, n_chunks, hist, err);
     cudaError_t st = cudaGetLastError();
     if (st != cudaSuccess) return st;
   }
@@ -197,8 +223,14 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
   }
   cudaError_t st = cudaGetLastError();
   if (st != cudaSuccess || n_chunks == 0) return st;
+  const int smem = kPermWarps * E * (int)sizeof(int);
+  if (smem > 48 * 1024) {
+    st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (st != cudaSuccess) return st;
+  }
   ProfScope ps(K_PERM_SCATTER, s);
-  permute_scatter_kernel<<<blocks, warps * 32, smem, s>>>(ids, P, E, hist, sorted_pairs, pair_pos);
+  permute_scatter_kernel<<<n_chunks, kPermThreads, smem, s>>>(ids, P, E, n_chunks, hist, sorted_pairs,
+                                                              pair_pos);
   return cudaGetLastError();
 }
 
@@ -206,33 +238,6 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
 // From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
 // experts (grouped GEMMs), and row chunks of `chunk_rows` rows (adapter
 // gradients) with chunk_start[e] = first chunk of expert e.
-__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int* total_out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += u;
-  }
-  __syncthreads();
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int w = s_warp[lane];
-    int inc2 = w;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
-      if (lane >= off) inc2 += u;
-    }
-    s_warp[lane] = inc2 - w;
-    if (lane == 31) s_warp[32] = inc2;
-  }
-  __syncthreads();
-  *total_out = s_warp[32];
-  return incl - v + s_warp[warp];
-}
-
 __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, int tile_rows,
                                     TileInfo* __restrict__ tiles, int* __restrict__ n_tiles,
                                     int gchunk_rows, TileInfo* __restrict__ gchunks,

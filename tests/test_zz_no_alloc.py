@@ -2,7 +2,7 @@
 
 moe_permute_noalloc serves callers that cannot allocate device memory (a plug-in
 inside a framework that owns all device memory, or code with a fixed footprint):
-it keeps its histogram scratch in a 1 MiB array inside the library instead of a
+it keeps its histogram scratch in a 2 MiB array inside the library instead of a
 caller workspace.  Its outputs must equal moe_permute's exactly (integers), on
 consecutive calls that reuse the built-in scratch.  This file is collected last
 so that a failure here does not hide the other tests.
@@ -50,7 +50,8 @@ def test_permute_noalloc_matches_permute_on_consecutive_calls(T, k, E):
 def test_permute_noalloc_rejects_oversized_problem():
     ensure_built()
     E, k = 1024, 8
-    T = (262144 // E + 1) * 1024 // k       # one chunk more than the built-in scratch holds
+    scratch_ints, chunk = 1 << 19, 512       # built-in scratch, pairs per histogram chunk
+    T = (scratch_ints // E + 1) * chunk // k  # one chunk more than the scratch holds
     ids = torch.zeros(T, k, dtype=torch.int32, device="cuda")
     outs = _outputs(T, k, E)
     with pytest.raises(ml.MoEError) as e:
