@@ -41,7 +41,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
             const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
   auto fn = encode_fn();
   if (fn == nullptr) return false;
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
                   reinterpret_cast<const cuuint64_t*>(dims),
                   reinterpret_cast<const cuuint64_t*>(strides_bytes),
@@ -66,6 +66,16 @@ bool encode3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t rows, uint6
   const uint64_t str[2] = {cols * 2, rows * cols * 2};
   const uint32_t box[3] = {box_cols, box_rows, 1};
   return encode(m, base, 3, dims, str, box, swz_for_bytes((int)box_cols * 2));
+}
+
+// W [E, K, F] row-major seen as [E][F/64 atoms][K][64]: box = two 64-feature atoms of
+// box_k K rows, so one copy fills an MN-major operand of 128 features (F % 64 == 0).
+bool encode_w_atoms(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t F,
+                    uint32_t box_k) {
+  const uint64_t dims[4] = {64, K, F / 64, E};
+  const uint64_t str[3] = {F * 2, 128, K * F * 2};
+  const uint32_t box[4] = {64, box_k, 2, 1};
+  return encode(m, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <class Kern>
@@ -108,13 +118,16 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
                      cudaStream_t s) {
   CUtensorMap mp[4];
   const uint64_t P = g.P, E = g.E, rp = g.rp;
-  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, 32, 64) &&
-            encode2d(&mp[3], lrc, P, rp, 32, (uint32_t)rp);
+  const uint32_t boxr = GemmCfg<true, 16>::BOXR;
+  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, boxr, 64) &&
+            encode2d(&mp[3], lrc, P, rp, boxr, (uint32_t)rp);
+  const bool w4 = !w_fk && F % 64 == 0;
   if (w_fk) {
     ok = ok && encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64) &&
          encode3d(&mp[2], lw, E, (uint64_t)F, rp, 128, (uint32_t)rp);
   } else {
-    ok = ok && encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64, 64) &&
+    ok = ok && (w4 ? encode_w_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64)
+                   : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64, 64)) &&
          encode3d(&mp[2], lw, E, rp, (uint64_t)F, (uint32_t)rp, 64);
   }
   if (!ok) return cudaErrorInvalidValue;
@@ -129,6 +142,10 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
   if (w_fk) {
     if (g.rp == 16) return launch_gemm<GemmCfg<false, 16>>(kind, g, mp, p, s);
     return launch_gemm<GemmCfg<false, 32>>(kind, g, mp, p, s);
+  }
+  if (w4) {
+    if (g.rp == 16) return launch_gemm<GemmCfg<true, 16, true>>(kind, g, mp, p, s);
+    return launch_gemm<GemmCfg<true, 32, true>>(kind, g, mp, p, s);
   }
   if (g.rp == 16) return launch_gemm<GemmCfg<true, 16>>(kind, g, mp, p, s);
   return launch_gemm<GemmCfg<true, 32>>(kind, g, mp, p, s);

@@ -26,10 +26,14 @@
 // tile overlaps the K-loop of the next.
 //
 // Shared-memory operands (canonical UMMA layouts, per CTA):
-//   A (weights)  forward, W stored [K][F]: MN-major, two 64-feature boxes of 64 K
-//                rows, 128-byte swizzle; backward, W stored [F][K]: K-major,
+//   A (weights)  forward, W stored [K][F]: MN-major, two 64-feature atoms of 64 K
+//                rows, 128-byte swizzle (one TMA copy through a 4-D view when
+//                F % 64 == 0); backward, W stored [F][K]: K-major,
 //                [128 features][64 K], 128-byte swizzle
-//   B (tokens)   [N/2 rows][64 K], K-major, 128-byte swizzle, boxes of 32 rows
+//   B (tokens)   [N/2 rows][64 K], K-major, 128-byte swizzle, boxes of 64 rows
+// Each stage costs the two issuing threads a fixed number of instructions
+// (waits, TMA copies, MMAs, a commit), so the loaders use as few copies per stage
+// as the layouts allow and the MMA descriptors are advanced by offsets.
 //   LoRA block   A: L_B^T (forward [r][F]: MN-major; backward [F][r]: K-major,
 //                32/64-byte swizzle); B: LRc [N/2 rows][r], K-major, 32/64-byte swizzle
 #pragma once
@@ -48,11 +52,15 @@ struct GemmParams {
   int* err;
 };
 
-template <bool A_MN_, int RP_>
+// A_MN: weights stored [K][F] (MN-major A); W4: the forward weight tile is one TMA
+// copy through a 4-D view (64-feature atom, K, atom index, expert), which needs F % 64
+// == 0; otherwise two 64-feature boxes.
+template <bool A_MN_, int RP_, bool W4_ = false>
 struct GemmCfg {
   static constexpr int RP = RP_;
   static constexpr bool A_MN = A_MN_;
-  static constexpr int BM = 128, BK = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 32;
+  static constexpr bool W4 = W4_;
+  static constexpr int BM = 128, BK = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 64;
   static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
   static constexpr int B_BYTES = NHALF * BK * 2;       // 16 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -66,7 +74,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int LA_BOX_BYTES = RP * 64 * 2;          // forward: 64 features x RP rows
   static constexpr int LA_BYTES = A_MN ? 2 * LA_BOX_BYTES : BM * RP * 2;
-  static constexpr int LR_BOX_BYTES = BOXR * RP * 2;        // 32 token rows x RP
+  static constexpr int LR_BOX_BYTES = BOXR * RP * 2;        // 64 token rows x RP
   static constexpr uint32_t LR_SWZ = RP == 16 ? kSw32 : kSw64;
   static constexpr uint32_t LR_SBO = RP == 16 ? 256 : 512;
   static_assert(RP == 16 || RP == 32, "RP");
@@ -149,27 +157,31 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      const uint32_t full_leader = mapa_smem(smem_u32(full), 0);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
-        const int c = t / p.n_ftiles, w = t % p.n_ftiles;
-        const TileInfo ch = p.chunks[c];
-        const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
-        const int nbh = (half + C::BOXR - 1) / C::BOXR;
-        const int r0 = ch.row0 + (int)rank * half;
-        for (int ks = 0; ks <= p.nk; ++ks) {
-          if (*abort_flag) { ok = false; break; }
-          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err)) { ok = false; break; }
+    // The whole warp waits (converged), lane 0 issues the copies.
+    const uint32_t full_leader = mapa_smem(smem_u32(full), 0);
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int t = pair; t < total && ok; t += npairs) {
+      const int c = t / p.n_ftiles, w = t % p.n_ftiles;
+      const TileInfo ch = p.chunks[c];
+      const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
+      const int nbh = (half + C::BOXR - 1) / C::BOXR;
+      const int r0 = ch.row0 + (int)rank * half;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+      for (int ks = 0; ks <= p.nk; ++ks) {
+        const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
+        if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
+        if (lane == 0) {
           const uint32_t fb = full_leader + stage * 8;
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           if (ks < p.nk) {
             const uint32_t bytes = C::A_BYTES + nbh * (C::BOXR * C::BK * 2);
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * bytes);
-            if constexpr (C::A_MN) {
+            if constexpr (C::W4) {
+              tma_load_4d_pair(&tmW, fb, sa, 0, ks * C::BK, feat_box(w, rank, 0) / 64, ch.e);
+            } else if constexpr (C::A_MN) {
               tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), ks * C::BK, ch.e);
               tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), ks * C::BK, ch.e);
             } else {
@@ -189,15 +201,25 @@ __global__ void __launch_bounds__(320, 1)
             for (int j = 0; j < nbh; ++j)
               tma_load_2d_pair(&tmLR, fb, sb + j * C::LR_BOX_BYTES, 0, r0 + j * C::BOXR);
           }
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
+        __syncwarp();
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) *abort_flag = 1;
     }
+    if (!ok && lane == 0) *abort_flag = 1;
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
-    if (lane == 0 && rank == 0) {
+    // The whole warp waits (converged); lane 0 issues every MMA and commit, so each
+    // commit tracks all MMAs issued before it.
+    if (rank == 0) {
+      // descriptors of stage 0, k-step 0 (A at the stage base, B after A)
+      const uint64_t a_desc0 = C::A_MN ? smem_desc(s_base, C::A_BYTES / 2, 1024, kSw128)
+                                       : smem_desc(s_base, 16, 1024, kSw128);
+      const uint64_t b_desc0 = smem_desc(s_base + C::A_BYTES, 16, 1024, kSw128);
+      const uint64_t la_desc0 = C::A_MN ? smem_desc(s_base, C::LA_BOX_BYTES, 1024, kSw128)
+                                        : smem_desc(s_base, 16, C::LR_SBO, C::LR_SWZ);
+      const uint64_t lr_desc0 = smem_desc(s_base + C::A_BYTES, 16, C::LR_SBO, C::LR_SWZ);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -209,42 +231,43 @@ __global__ void __launch_bounds__(320, 1)
         const int ncols = ((ch.row_end - ch.row0) + 15) & ~15;
         const uint32_t idesc = idesc_bf16(256, ncols, C::A_MN ? 1 : 0, 0);
         const int b = it & 1;
-        if (!mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
+        const bool aok = mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err);
+        if (!__all_sync(0xffffffffu, aok)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + b * C::NMAX;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
         for (int ks = 0; ks <= p.nk; ++ks) {
-          if (*abort_flag) { ok = false; break; }
-          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+          const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
+          if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = s_base + stage * C::STAGE_BYTES;
-          const uint32_t sb = sa + C::A_BYTES;
-          if (ks < p.nk) {
+          if (lane == 0) {
+            // descriptors: the 14-bit start-address field advances by (byte offset >> 4)
+            const uint32_t so = (uint32_t)(stage * C::STAGE_BYTES) >> 4;
+            if (ks < p.nk) {
 #pragma unroll
-            for (int kk = 0; kk < C::BK / 16; ++kk) {
-              const uint64_t ad = C::A_MN ? smem_desc(sa + kk * 2048, C::A_BYTES / 2, 1024, kSw128)
-                                          : smem_desc(sa + kk * 32, 16, 1024, kSw128);
-              const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, kSw128);
-              umma_bf16_pair(d, ad, bd, idesc, (ks | kk) ? 1u : 0u);
-            }
-          } else {
+              for (int kk = 0; kk < C::BK / 16; ++kk)
+                umma_bf16_pair(d, a_desc0 + so + kk * (C::A_MN ? 2048 / 16 : 32 / 16),
+                               b_desc0 + so + kk * (32 / 16), idesc, (ks | kk) ? 1u : 0u);
+            } else {
 #pragma unroll
-            for (int kk = 0; kk < C::RP / 16; ++kk) {
-              const uint64_t ad = C::A_MN ? smem_desc(sa + kk * 2048, C::LA_BOX_BYTES, 1024, kSw128)
-                                          : smem_desc(sa + kk * 32, 16, C::LR_SBO, C::LR_SWZ);
-              const uint64_t bd = smem_desc(sb + kk * 32, 16, C::LR_SBO, C::LR_SWZ);
-              umma_bf16_pair(d, ad, bd, idesc, 1u);
+              for (int kk = 0; kk < C::RP / 16; ++kk)
+                umma_bf16_pair(d, la_desc0 + so + kk * (C::A_MN ? 2048 / 16 : 32 / 16),
+                               lr_desc0 + so + kk * (32 / 16), idesc, 1u);
             }
+            umma_commit_pair(smem_u32(&empty[stage]), 0x3);
           }
-          umma_commit_pair(smem_u32(&empty[stage]), 0x3);
+          __syncwarp();
           issued_any = true;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit_pair(smem_u32(&acc_full[b]), 0x3);
+        if (lane == 0) umma_commit_pair(smem_u32(&acc_full[b]), 0x3);
+        __syncwarp();
       }
-      if (!ok) *abort_flag = 1;
+      if (!ok && lane == 0) *abort_flag = 1;
       if (issued_any) {
-        umma_commit_pair(smem_u32(drain), 0x1);
+        if (lane == 0) umma_commit_pair(smem_u32(drain), 0x1);
+        __syncwarp();
         mbar_wait(smem_u32(drain), 0, p.err);
       }
     }
