@@ -118,16 +118,16 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
                      cudaStream_t s) {
   CUtensorMap mp[4];
   const uint64_t P = g.P, E = g.E, rp = g.rp;
-  const uint32_t boxr = GemmCfg<true, 16>::BOXR;
-  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, boxr, 64) &&
-            encode2d(&mp[3], lrc, P, rp, boxr, (uint32_t)rp);
+  using C0 = GemmCfg<true, 16>;
+  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, C0::NHALF, C0::KA) &&
+            encode2d(&mp[3], lrc, P, rp, C0::BOXR, (uint32_t)rp);
   const bool w4 = !w_fk && F % 64 == 0;
   if (w_fk) {
     ok = ok && encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64) &&
          encode3d(&mp[2], lw, E, (uint64_t)F, rp, 128, (uint32_t)rp);
   } else {
-    ok = ok && (w4 ? encode_w_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64)
-                   : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, 64, 64)) &&
+    ok = ok && (w4 ? encode_w_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK)
+                   : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 64)) &&
          encode3d(&mp[2], lw, E, rp, (uint64_t)F, (uint32_t)rp, 64);
   }
   if (!ok) return cudaErrorInvalidValue;
@@ -136,7 +136,7 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
   p.n_chunks = g.n_gchunks;
   p.F = F;
   p.n_ftiles = (F + 255) / 256;
-  p.nk = (K + 63) / 64;
+  p.nk = (K + C0::BK - 1) / C0::BK;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.err = g.err;
   if (w_fk) {

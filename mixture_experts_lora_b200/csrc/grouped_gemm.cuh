@@ -30,7 +30,7 @@
 //                rows, 128-byte swizzle (one TMA copy through a 4-D view when
 //                F % 64 == 0); backward, W stored [F][K]: K-major,
 //                [128 features][64 K], 128-byte swizzle
-//   B (tokens)   [N/2 rows][64 K], K-major, 128-byte swizzle, boxes of 64 rows
+//   B (tokens)   two K atoms of [128 rows][64 K], K-major, 128-byte swizzle
 // Each stage costs the two issuing threads a fixed number of instructions
 // (waits, TMA copies, MMAs, a commit), so the loaders use as few copies per stage
 // as the layouts allow and the MMA descriptors are advanced by offsets.
@@ -47,7 +47,7 @@ struct GemmParams {
   const int* n_chunks;
   int F;                   // output features
   int n_ftiles;            // feature tiles (256 features per pair) per chunk
-  int nk;                  // K steps of 64 (the LoRA block is step nk)
+  int nk;                  // K steps of 128 (the LoRA block is step nk)
   __nv_bfloat16* out;      // [P, F] in sorted token order
   int* err;
 };
@@ -60,16 +60,20 @@ struct GemmCfg {
   static constexpr int RP = RP_;
   static constexpr bool A_MN = A_MN_;
   static constexpr bool W4 = W4_;
-  static constexpr int BM = 128, BK = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 64;
-  static constexpr int A_BYTES = BM * BK * 2;          // 16 KB
-  static constexpr int B_BYTES = NHALF * BK * 2;       // 16 KB
+  // BK = 128 per stage as two 64-wide K atoms (one 128-byte swizzle row each): a
+  // stage carries 8 MMAs per wait and commit.  BOXR: token rows per LoRA-block copy.
+  static constexpr int BM = 128, BK = 128, KA = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 64;
+  static constexpr int A_BYTES = BM * BK * 2;          // 32 KB
+  static constexpr int B_BYTES = NHALF * BK * 2;       // 32 KB
+  static constexpr int ATOM_A = BM * KA * 2;           // 16 KB: one K atom of a K-major A
+  static constexpr int ATOM_B = NHALF * KA * 2;        // 16 KB: one K atom of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BLK_BYTES = 32 * 32 * 2;        // one 32 x 32 bf16 staging block
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_BYTES = EPI_WARPS * BLK_BYTES;   // one transpose block per warp
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int STAGES_FIT = (SMEM_LIMIT - EPI_BYTES - 2048) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 2048;
   static constexpr int TMEM_COLS = 512;
   static constexpr int LA_BOX_BYTES = RP * 64 * 2;          // forward: 64 features x RP rows
@@ -78,7 +82,7 @@ struct GemmCfg {
   static constexpr uint32_t LR_SWZ = RP == 16 ? kSw32 : kSw64;
   static constexpr uint32_t LR_SBO = RP == 16 ? 256 : 512;
   static_assert(RP == 16 || RP == 32, "RP");
-  static_assert(STAGES >= 4, "pipeline depth");
+  static_assert(STAGES >= 3, "pipeline depth");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
 };
 
@@ -177,18 +181,21 @@ __global__ void __launch_bounds__(320, 1)
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           if (ks < p.nk) {
-            const uint32_t bytes = C::A_BYTES + nbh * (C::BOXR * C::BK * 2);
-            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * bytes);
+            // every copy is full-size (rows past the chunk are loaded and ignored,
+            // rows past P and K past the end read as zero)
+            const int k0 = ks * C::BK;
+            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + C::B_BYTES));
             if constexpr (C::W4) {
-              tma_load_4d_pair(&tmW, fb, sa, 0, ks * C::BK, feat_box(w, rank, 0) / 64, ch.e);
+              tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box(w, rank, 0) / 64, ch.e);
             } else if constexpr (C::A_MN) {
-              tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), ks * C::BK, ch.e);
-              tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), ks * C::BK, ch.e);
+              tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), k0, ch.e);
+              tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), k0, ch.e);
             } else {
-              tma_load_3d_pair(&tmW, fb, sa, ks * C::BK, feat_box(w, rank, 0), ch.e);
+              tma_load_3d_pair(&tmW, fb, sa, k0, feat_box(w, rank, 0), ch.e);
+              tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box(w, rank, 0), ch.e);
             }
-            for (int j = 0; j < nbh; ++j)
-              tma_load_2d_pair(&tmAct, fb, sb + j * (C::BOXR * C::BK * 2), ks * C::BK, r0 + j * C::BOXR);
+            tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
+            tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
           } else {
             const uint32_t bytes = C::LA_BYTES + nbh * C::LR_BOX_BYTES;
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * bytes);
@@ -245,9 +252,14 @@ __global__ void __launch_bounds__(320, 1)
             const uint32_t so = (uint32_t)(stage * C::STAGE_BYTES) >> 4;
             if (ks < p.nk) {
 #pragma unroll
-              for (int kk = 0; kk < C::BK / 16; ++kk)
-                umma_bf16_pair(d, a_desc0 + so + kk * (C::A_MN ? 2048 / 16 : 32 / 16),
-                               b_desc0 + so + kk * (32 / 16), idesc, (ks | kk) ? 1u : 0u);
+              for (int kk = 0; kk < C::BK / 16; ++kk) {
+                // K step kk: MN-major A advances 16 rows of 128 B; K-major operands
+                // advance 32 B inside a K atom, atoms ATOM_* bytes apart
+                const uint32_t ka = (uint32_t)((kk >> 2) * C::ATOM_A + (kk & 3) * 32) >> 4;
+                const uint32_t kb = (uint32_t)((kk >> 2) * C::ATOM_B + (kk & 3) * 32) >> 4;
+                umma_bf16_pair(d, a_desc0 + so + (C::A_MN ? kk * (2048 / 16) : ka), b_desc0 + so + kb,
+                               idesc, (ks | kk) ? 1u : 0u);
+              }
             } else {
 #pragma unroll
               for (int kk = 0; kk < C::RP / 16; ++kk)
