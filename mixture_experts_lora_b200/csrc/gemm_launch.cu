@@ -68,14 +68,15 @@ bool encode3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t rows, uint6
   return encode(m, base, 3, dims, str, box, swz_for_bytes((int)box_cols * 2));
 }
 
-// W [E, K, F] row-major seen as [E][F/64 atoms][K][64]: box = two 64-feature atoms of
-// box_k K rows, so one copy fills an MN-major operand of 128 features (F % 64 == 0).
-bool encode_w_atoms(CUtensorMap* m, const void* base, uint64_t E, uint64_t K, uint64_t F,
-                    uint32_t box_k) {
-  const uint64_t dims[4] = {64, K, F / 64, E};
-  const uint64_t str[3] = {F * 2, 128, K * F * 2};
-  const uint32_t box[4] = {64, box_k, 2, 1};
-  return encode(m, base, 4, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+// [E, R, C] row-major (C % 64 == 0) seen as [E][C/64 atoms][R][64]: a box of
+// `box_atoms` 64-wide atoms of `box_r` rows lands as atom-major 128-byte-swizzled
+// tiles, so one copy fills a whole operand tile.  E = 1 for a 2-D tensor.
+bool encode_atoms(CUtensorMap* m, const void* base, uint64_t E, uint64_t R, uint64_t C,
+                  uint32_t box_r, uint32_t box_atoms) {
+  const uint64_t dims[4] = {64, R, C / 64, E};
+  const uint64_t str[3] = {C * 2, 128, R * C * 2};
+  const uint32_t box[4] = {64, box_r, box_atoms, 1};
+  return encode(m, base, E > 1 ? 4 : 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <class Kern>
@@ -119,15 +120,19 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
   CUtensorMap mp[4];
   const uint64_t P = g.P, E = g.E, rp = g.rp;
   using C0 = GemmCfg<true, 16>;
-  bool ok = encode2d(&mp[1], act, P, (uint64_t)K, C0::NHALF, C0::KA) &&
+  // atom views (one copy per operand and stage) when the K (and MN-major F) extents
+  // are whole 64-wide atoms
+  const bool v = K % 64 == 0 && (w_fk || F % 64 == 0);
+  bool ok = (v ? encode_atoms(&mp[1], act, 1, P, (uint64_t)K, C0::NHALF, C0::BK / 64)
+               : encode2d(&mp[1], act, P, (uint64_t)K, C0::NHALF, C0::KA)) &&
             encode2d(&mp[3], lrc, P, rp, C0::BOXR, (uint32_t)rp);
-  const bool w4 = !w_fk && F % 64 == 0;
   if (w_fk) {
-    ok = ok && encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64) &&
+    ok = ok && (v ? encode_atoms(&mp[0], W, E, (uint64_t)F, (uint64_t)K, C0::BM, C0::BK / 64)
+                  : encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64)) &&
          encode3d(&mp[2], lw, E, (uint64_t)F, rp, 128, (uint32_t)rp);
   } else {
-    ok = ok && (w4 ? encode_w_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK)
-                   : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 64)) &&
+    ok = ok && (v ? encode_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 2)
+                  : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 64)) &&
          encode3d(&mp[2], lw, E, rp, (uint64_t)F, (uint32_t)rp, 64);
   }
   if (!ok) return cudaErrorInvalidValue;
@@ -140,10 +145,14 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.err = g.err;
   if (w_fk) {
+    if (v) {
+      if (g.rp == 16) return launch_gemm<GemmCfg<false, 16, true>>(kind, g, mp, p, s);
+      return launch_gemm<GemmCfg<false, 32, true>>(kind, g, mp, p, s);
+    }
     if (g.rp == 16) return launch_gemm<GemmCfg<false, 16>>(kind, g, mp, p, s);
     return launch_gemm<GemmCfg<false, 32>>(kind, g, mp, p, s);
   }
-  if (w4) {
+  if (v) {
     if (g.rp == 16) return launch_gemm<GemmCfg<true, 16, true>>(kind, g, mp, p, s);
     return launch_gemm<GemmCfg<true, 32, true>>(kind, g, mp, p, s);
   }
@@ -298,7 +307,7 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, co
                               int max_chunks, const int32_t* chunk_start, float* partial,
                               bool transpose, uint16_t* out, cudaStream_t s) {
   CUtensorMap tm;
-  if (!encode2d(&tm, big, (uint64_t)(g.P > 0 ? g.P : 1), (uint64_t)D, 64, 64))
+  if (!encode2d(&tm, big, (uint64_t)(g.P > 0 ? g.P : 1), (uint64_t)D, WgradCfg<16>::BK, 64))
     return cudaErrorInvalidValue;
   WgradParams wp{};
   wp.small = reinterpret_cast<const __nv_bfloat16*>(small);

@@ -52,14 +52,16 @@ struct GemmParams {
   int* err;
 };
 
-// A_MN: weights stored [K][F] (MN-major A); W4: the forward weight tile is one TMA
-// copy through a 4-D view (64-feature atom, K, atom index, expert), which needs F % 64
-// == 0; otherwise two 64-feature boxes.
-template <bool A_MN_, int RP_, bool W4_ = false>
+// A_MN: weights stored [K][F] (MN-major A).  V: operands through atom views, one
+// TMA copy per operand and stage: the weight tile via a 4-D view (64-wide atom,
+// rows, atom index, expert) and the token tile via a 3-D view (64-wide K atom,
+// rows, atom index); needs K % 64 == 0 (and F % 64 == 0 for MN-major weights).
+// Otherwise two copies per operand.
+template <bool A_MN_, int RP_, bool V_ = false>
 struct GemmCfg {
   static constexpr int RP = RP_;
   static constexpr bool A_MN = A_MN_;
-  static constexpr bool W4 = W4_;
+  static constexpr bool V = V_;
   // BK = 128 per stage as two 64-wide K atoms (one 128-byte swizzle row each): a
   // stage carries 8 MMAs per wait and commit.  BOXR: token rows per LoRA-block copy.
   static constexpr int BM = 128, BK = 128, KA = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 64;
@@ -185,17 +187,23 @@ __global__ void __launch_bounds__(320, 1)
             // rows past P and K past the end read as zero)
             const int k0 = ks * C::BK;
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + C::B_BYTES));
-            if constexpr (C::W4) {
-              tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box(w, rank, 0) / 64, ch.e);
-            } else if constexpr (C::A_MN) {
-              tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), k0, ch.e);
-              tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), k0, ch.e);
+            if constexpr (C::V) {
+              if constexpr (C::A_MN)
+                tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box(w, rank, 0) / 64, ch.e);
+              else
+                tma_load_4d_pair(&tmW, fb, sa, 0, feat_box(w, rank, 0), k0 / C::KA, ch.e);
+              tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
             } else {
-              tma_load_3d_pair(&tmW, fb, sa, k0, feat_box(w, rank, 0), ch.e);
-              tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box(w, rank, 0), ch.e);
+              if constexpr (C::A_MN) {
+                tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), k0, ch.e);
+                tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), k0, ch.e);
+              } else {
+                tma_load_3d_pair(&tmW, fb, sa, k0, feat_box(w, rank, 0), ch.e);
+                tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box(w, rank, 0), ch.e);
+              }
+              tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
+              tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
             }
-            tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
-            tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
           } else {
             const uint32_t bytes = C::LA_BYTES + nbh * C::LR_BOX_BYTES;
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * bytes);

@@ -43,10 +43,15 @@ struct WgradParams {
 
 template <int RP>
 struct WgradCfg {
-  static constexpr int BM = 128, BK = 64, STAGES = 8;
-  static constexpr int BIG_BYTES = BM * BK * 2;   // two 64-column boxes
+  // 128 rows per stage: 8 MMAs per wait and commit (the per-stage issue cost of the
+  // loader and MMA threads, not the bytes, bounded 64-row stages)
+  static constexpr int BM = 128, BK = 128;
+  static constexpr int BIG_BYTES = BM * BK * 2;   // two 64-column atoms of BK rows
   static constexpr int SMALL_BYTES = RP * BK * 2;
+  static constexpr int SMALL_NG = BK * 16;        // bytes between 8-column groups of Small
   static constexpr int STAGE_BYTES = BIG_BYTES + SMALL_BYTES;
+  static constexpr int STAGES_FIT = (232448 - 2048) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
   static constexpr int TMEM_COLS = 64;            // 2 x RP fp32 columns (RP <= 32)
 };
@@ -114,8 +119,8 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_2d(&tmBig, fb, sbig, d0, r0);
           tma_load_2d(&tmBig, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
         }
-        // Small tile [64 rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
-        // columns (128 B), row groups 128 B apart, column groups 1024 B apart.
+        // Small tile [BK rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
+        // columns (128 B), row groups 128 B apart, column groups SMALL_NG bytes apart.
         // Rows outside the chunk (and columns past r_small) are zero-filled.
         const uint32_t ssm = sbig + C::BIG_BYTES;
         constexpr int CG = RP / 8;
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(192, 1)
           const bool valid = row < ch.row_end && cg * 8 < p.r_small;
           const void* src = valid ? (const void*)(p.small + (size_t)row * p.ld_small + cg * 8)
                                   : (const void*)p.small;
-          cp_async_16(ssm + cg * 1024 + (rr & 7) * 16 + (rr >> 3) * 128, src, valid ? 16u : 0u);
+          cp_async_16(ssm + cg * C::SMALL_NG + (rr & 7) * 16 + (rr >> 3) * 128, src, valid ? 16u : 0u);
         }
         cp_async_mbar_arrive(fb);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -160,8 +165,8 @@ __global__ void __launch_bounds__(192, 1)
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             // Big^T: MN-major, 128-byte swizzle, 64-column atoms 8 KB apart, 8-row groups 1 KB apart
             const uint64_t ad = smem_desc(sbig + kk * 16 * 128, C::BIG_BYTES / 2, 1024, kSw128);
-            // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at 1024 B
-            const uint64_t bd = smem_desc(ssm + kk * 256, 128, 1024, kSwNone);
+            // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at SMALL_NG
+            const uint64_t bd = smem_desc(ssm + kk * 256, 128, C::SMALL_NG, kSwNone);
             umma_bf16(d, ad, bd, idesc, (ks | kk) ? 1u : 0u);
           }
           umma_commit(smem_u32(&empty[stage]));
