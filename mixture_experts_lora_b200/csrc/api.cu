@@ -73,7 +73,8 @@ struct Layout {
   int max_row_tiles, max_gchunks, max_chunks, chunk_rows, perm_chunks;
   size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
   size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
-  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial;
+  int max_dtiles;             // 128-column tiles of the widest adapter gradient
+  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial, partial2, counters;
   size_t total;
 };
 
@@ -111,6 +112,9 @@ Layout make_layout(const moe_dims_t& d) {
   L.lrc1 = take(P * rp * 2);
   L.lrc2 = take(P * rp * 2);
   L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
+  L.partial2 = take((size_t)L.max_chunks * dmax * rp * 4);
+  L.max_dtiles = (int)((dmax + 127) / 128);
+  L.counters = take((size_t)4 * E * L.max_dtiles * 4);   // one set per adapter gradient
   L.total = off;
   return L;
 }
@@ -139,7 +143,9 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
                               at<int>(ws, L.n_tiles), kGemmChunkRows, at<TileInfo>(ws, L.gchunks),
                               at<int>(ws, L.n_gchunks), L.chunk_rows,
                               with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
-                              at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start), s));
+                              at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start),
+                              with_chunks ? at<int>(ws, L.counters) : nullptr,
+                              with_chunks ? 4 * d.E * L.max_dtiles : 0, s));
   w->W_gu = W_gu;
   w->W_d = W_d;
   if (d.r != L.rp) {
@@ -333,23 +339,30 @@ moe_status_t moe_grouped_gemm_lora_bwd(
                               false, rows, t1, L.rp, L.rp, lrc1, s));
   // dH = dy W_d^T + (c T1) A_d^T
   MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
-  // dA_d = c H^T T1 ; dB_d = c HA^T dy
-  MOE_TRY(launch_lora_wgrad(g, save_H, d.n, t1, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
-                            partial, false, dA_d, s));
-  MOE_TRY(launch_lora_wgrad(g, rows, d.m, save_HA, d.r, chunks, n_chunks, L.max_chunks,
-                            chunk_start, partial, true, dB_d, s));
+  // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
+  float* partial2 = at<float>(ws, L.partial2);
+  int* counters = at<int>(ws, L.counters);
+  const size_t cstride = (size_t)d.E * L.max_dtiles;
+  {
+    const WgradJob jobs[2] = {
+        {save_H, d.n, t1, L.rp, false, dA_d, partial, counters},
+        {rows, d.m, save_HA, d.r, true, dB_d, partial2, counters + cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+  }
   // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
   MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
                               false, dgu, t2, L.rp, L.rp, lrc2, s));
   // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
-  // dB_gu = c XA^T dGU
-  MOE_TRY(launch_lora_wgrad(g, dgu, 2 * d.n, save_XA, d.r, chunks, n_chunks, L.max_chunks,
-                            chunk_start, partial, true, dB_gu, s));
-  // dA_gu = c X^T T2 (X re-gathered into the row buffer, dy no longer needed)
+  // X re-gathered into the row buffer (dy is no longer needed), then
+  // dB_gu = c XA^T dGU and dA_gu = c X^T T2, one launch
   MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
-  MOE_TRY(launch_lora_wgrad(g, rows, d.m, t2, L.rp, chunks, n_chunks, L.max_chunks, chunk_start,
-                            partial, false, dA_gu, s));
+  {
+    const WgradJob jobs[2] = {
+        {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
+        {rows, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+  }
   return MOE_OK;
 }
 

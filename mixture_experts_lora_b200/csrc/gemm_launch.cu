@@ -281,48 +281,50 @@ cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const
 }
 
 template <int RP>
-static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap& tm, const WgradParams& wp,
+static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const WgradParams& wp,
                             int max_chunks, cudaStream_t s) {
   using C = WgradCfg<RP>;
   auto kern = lora_wgrad_kernel<RP>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
-  const int64_t units = (int64_t)max_chunks * wp.n_dtiles;
-  if (units > 0) {
-    const int grid = (int)(units < g.num_sms ? units : g.num_sms);
-    ProfScope ps(K_WGRAD, s);
-    kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm, wp);
-    st = cudaGetLastError();
-    if (st != cudaSuccess) return st;
-  }
-  const int64_t total = (int64_t)g.E * wp.D;
-  ProfScope ps(K_WGRAD_REDUCE, s);
-  lora_wgrad_reduce_kernel<RP><<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-      wp.partial, wp.chunk_start, g.E, wp.D, g.r, g.scale, wp.transpose, wp.out);
+  int dtiles = wp.pr[0].n_dtiles + (wp.n_problems > 1 ? wp.pr[1].n_dtiles : 0);
+  const int64_t units = (int64_t)max_chunks * dtiles;
+  // at least one CTA per SM: the zero fill of experts without rows runs in every CTA
+  const int grid = (int)(units > 0 && units < g.num_sms ? units : g.num_sms);
+  ProfScope ps(K_WGRAD, s);
+  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm[0], tm[1], wp);
   return cudaGetLastError();
 }
 
-cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, const uint16_t* small,
-                              int ld_small, const TileInfo* chunks, const int* n_chunks,
-                              int max_chunks, const int32_t* chunk_start, float* partial,
-                              bool transpose, uint16_t* out, cudaStream_t s) {
-  CUtensorMap tm;
-  if (!encode2d(&tm, big, (uint64_t)(g.P > 0 ? g.P : 1), (uint64_t)D, WgradCfg<16>::BK, 64))
-    return cudaErrorInvalidValue;
+cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jobs,
+                              const TileInfo* chunks, const int* n_chunks, int max_chunks,
+                              const int32_t* chunk_start, cudaStream_t s) {
+  if (n_jobs < 1 || n_jobs > 2) return cudaErrorInvalidValue;
+  CUtensorMap tm[2];
   WgradParams wp{};
-  wp.small = reinterpret_cast<const __nv_bfloat16*>(small);
-  wp.ld_small = ld_small;
-  wp.r_small = ld_small;  // the caller's buffer has exactly ld_small columns
+  for (int j = 0; j < n_jobs; ++j) {
+    const WgradJob& jb = jobs[j];
+    if (!encode2d(&tm[j], jb.big, (uint64_t)(g.P > 0 ? g.P : 1), (uint64_t)jb.D, WgradCfg<16>::BK, 64))
+      return cudaErrorInvalidValue;
+    WgradProblem& q = wp.pr[j];
+    q.small = reinterpret_cast<const __nv_bfloat16*>(jb.small);
+    q.ld_small = jb.ld_small;
+    q.r_small = jb.ld_small;  // the caller's buffer has exactly ld_small columns
+    q.D = jb.D;
+    q.n_dtiles = (jb.D + 127) / 128;
+    q.transpose = jb.transpose;
+    q.out = reinterpret_cast<__nv_bfloat16*>(jb.out);
+    q.partial = jb.partial;
+    q.counters = jb.counters;
+  }
+  if (n_jobs == 1) tm[1] = tm[0];
+  wp.n_problems = n_jobs;
   wp.chunks = chunks;
   wp.n_chunks = n_chunks;
   wp.chunk_start = chunk_start;
-  wp.D = D;
-  wp.n_dtiles = (D + 127) / 128;
+  wp.E = g.E;
   wp.r = g.r;
   wp.scale = g.scale;
-  wp.transpose = transpose;
-  wp.out = reinterpret_cast<__nv_bfloat16*>(out);
-  wp.partial = partial;
   wp.err = g.err;
   if (g.rp == 16) return wgrad_rp<16>(g, tm, wp, max_chunks, s);
   return wgrad_rp<32>(g, tm, wp, max_chunks, s);

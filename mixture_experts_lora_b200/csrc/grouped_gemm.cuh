@@ -91,25 +91,6 @@ struct GemmCfg {
 // First feature of this CTA's 64-feature A box i for feature tile w (pair rank r).
 __device__ __forceinline__ int feat_box(int w, int r, int i) { return w * 256 + r * 128 + i * 64; }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// Barrier over `n` threads that also ORs a predicate across them, so that every
-// participating warp takes the same branch afterwards.
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
 template <class C>
 __global__ void __launch_bounds__(320, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmAct,

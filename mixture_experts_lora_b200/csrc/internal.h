@@ -16,7 +16,7 @@ struct TileInfo;
 enum KernelKind : int {
   K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
-  K_WGRAD_REDUCE, K_COMBINE, K_MEMSET, K_LOWRANK, K_ROWS_GATHER, K_ROWS_SWIGLU,
+  K_COMBINE, K_MEMSET, K_LOWRANK, K_ROWS_GATHER, K_ROWS_SWIGLU,
   K_ROWS_SWIGLU_BWD, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
@@ -51,7 +51,8 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
 cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
                                 int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
                                 int chunk_rows, TileInfo* chunks, int* n_chunks,
-                                int32_t* chunk_start, cudaStream_t s);
+                                int32_t* chunk_start, int* zero, int n_zero,
+                                cudaStream_t s);
 // out[q] = (w ? bf16(w[p] * src[p / k]) : src[p / k]),  p = sorted_pairs[q]
 cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
                                int64_t P, int k, int m, uint16_t* out, cudaStream_t s);
@@ -115,9 +116,20 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
                                 bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
                                 int r_save, uint16_t* outc, cudaStream_t s);
 // out = scale * sum_rows Big^T Small per expert, out [E, D, r] or (transpose) [E, r, D]
-cudaError_t launch_lora_wgrad(const GemmShape& g, const uint16_t* big, int D, const uint16_t* small,
-                              int ld_small, const TileInfo* chunks, const int* n_chunks,
-                              int max_chunks, const int32_t* chunk_start, float* partial,
-                              bool transpose, uint16_t* out, cudaStream_t s);
+// One adapter-gradient problem G_e = Big_e^T Small_e (see lora_wgrad.cuh).
+struct WgradJob {
+  const uint16_t* big;   // [P, D] sorted rows
+  int D;
+  const uint16_t* small; // [P, ld_small]
+  int ld_small;
+  bool transpose;        // out [E, r, D] instead of [E, D, r]
+  uint16_t* out;
+  float* partial;        // [max_chunks, D, rp] fp32 partials of multi-chunk experts
+  int* counters;         // [E, ceil(D / 128)], zero before the launch
+};
+// One launch for one or two problems.
+cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jobs,
+                              const TileInfo* chunks, const int* n_chunks, int max_chunks,
+                              const int32_t* chunk_start, cudaStream_t s);
 
 }  // namespace moe

@@ -8,36 +8,48 @@
 // Mixture-of-Experts Fine-Tuning", Mathematical Formulation section 2; Unsloth
 // docs "Implementation details": only the m*r + r*n adapter parameters train).
 //
-// Units are (row chunk of one expert, 128-wide D tile); a persistent CTA walks
-// its units with one continuous TMA/MMA pipeline:
+// One launch computes up to two such problems (the two gradients that become
+// computable at the same point of the backward).  Units are (problem, row chunk
+// of one expert, 128-wide D tile); a persistent CTA walks its units with one
+// continuous TMA/MMA pipeline:
 //   M = 128 columns of Big (MN-major A operand, TMA, 128-byte swizzle),
 //   N = RP (Small, MN-major, no swizzle, written by the producer warp with rows
 //       outside the chunk zeroed, so a ragged tail contributes nothing),
-//   K = rows of the chunk, 64 per stage.
+//   K = rows of the chunk, 128 per stage.
 // The accumulator is double buffered in TMEM.  A unit of an expert whose rows fit
-// in one chunk writes the final bf16 gradient (scaled, in its output orientation);
-// otherwise it writes an fp32 partial and a second kernel sums the expert's
-// partials in chunk order (deterministic, no atomics).
+// in one chunk writes the final bf16 gradient (scaled, in its output orientation).
+// Otherwise each unit writes an fp32 partial and counts itself in a per-(expert,
+// D tile) arrival counter; the unit that arrives last sums the expert's partials
+// in chunk order (deterministic, whatever the arrival order) and writes the
+// gradient.  Gradients of experts without rows are written as zeros by the same
+// launch.
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
-struct WgradParams {
+struct WgradProblem {
   const __nv_bfloat16* small;  // [P, ld_small]
   int ld_small;
   int r_small;                 // columns of `small` to read (rest zero)
-  const TileInfo* chunks;      // row chunks {e, row0, row_end}
-  const int* n_chunks;
-  const int32_t* chunk_start;  // [E+1]
   int D;
   int n_dtiles;
-  int r;                       // output rank
-  float scale;
   bool transpose;              // out [E, r, D] instead of [E, D, r]
   __nv_bfloat16* out;
   float* partial;              // [max_chunks, D, RP]
+  int* counters;               // [E, n_dtiles] arrival counters, zero on entry and exit
+};
+
+struct WgradParams {
+  WgradProblem pr[2];
+  int n_problems;
+  const TileInfo* chunks;      // row chunks {e, row0, row_end}
+  const int* n_chunks;
+  const int32_t* chunk_start;  // [E+1]
+  int E;
+  int r;                       // output rank
+  float scale;
   int* err;
 };
 
@@ -54,11 +66,52 @@ struct WgradCfg {
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
   static constexpr int TMEM_COLS = 64;            // 2 x RP fp32 columns (RP <= 32)
+  static constexpr int EPI_THREADS = 128;         // warps 2..5
 };
+
+// Unit t of the launch -> (problem, chunk, D tile).
+struct WgradUnit {
+  int prob, c, dt;
+};
+__device__ __forceinline__ WgradUnit wgrad_unit(const WgradParams& p, int nch, int t) {
+  WgradUnit u;
+  const int t0 = nch * p.pr[0].n_dtiles;
+  u.prob = t < t0 ? 0 : 1;
+  const int tt = u.prob == 0 ? t : t - t0;
+  const int nd = p.pr[u.prob].n_dtiles;
+  u.c = tt / nd;
+  u.dt = tt - u.c * nd;
+  return u;
+}
+
+// Scaled bf16 gradient row d of expert e from fp32 values v[0..RP).
+template <int RP>
+__device__ __forceinline__ void wgrad_store(const WgradProblem& q, int r, float scale, int e, int d,
+                                            const float (&v)[RP]) {
+  if (q.transpose) {
+#pragma unroll
+    for (int i = 0; i < RP; ++i)
+      if (i < r) q.out[((size_t)e * r + i) * q.D + d] = __float2bfloat16_rn(scale * v[i]);
+  } else {
+    __nv_bfloat16* dst = q.out + ((size_t)e * q.D + d) * r;
+#pragma unroll
+    for (int g = 0; g < RP / 8; ++g) {
+      if (g * 8 < r) {
+        uint4 o;
+        o.x = pack_bf16x2(scale * v[8 * g + 0], scale * v[8 * g + 1]);
+        o.y = pack_bf16x2(scale * v[8 * g + 2], scale * v[8 * g + 3]);
+        o.z = pack_bf16x2(scale * v[8 * g + 4], scale * v[8 * g + 5]);
+        o.w = pack_bf16x2(scale * v[8 * g + 6], scale * v[8 * g + 7]);
+        *reinterpret_cast<uint4*>(dst + 8 * g) = o;
+      }
+    }
+  }
+}
 
 template <int RP>
 __global__ void __launch_bounds__(192, 1)
-    lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig, const WgradParams p) {
+    lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig0,
+                      const __grid_constant__ CUtensorMap tmBig1, const WgradParams p) {
   using C = WgradCfg<RP>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -72,6 +125,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = acc_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_full + 6);
+  volatile int* last_flag = abort_flag + 1;
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -85,8 +139,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
+    *last_flag = 0;
     mbar_fence_init();
-    tma_prefetch_desc(&tmBig);
+    tma_prefetch_desc(&tmBig0);
+    if (p.n_problems > 1) tma_prefetch_desc(&tmBig1);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -96,7 +152,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int total = (*p.n_chunks) * p.n_dtiles;
+  const int nch = *p.n_chunks;
+  const int total = nch * (p.pr[0].n_dtiles + (p.n_problems > 1 ? p.pr[1].n_dtiles : 0));
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer (whole warp)
@@ -104,20 +161,23 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t phase = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const int c = t / p.n_dtiles, dt = t % p.n_dtiles;
-      const TileInfo ch = p.chunks[c];
-      const int d0 = dt * C::BM;
+      const WgradUnit u = wgrad_unit(p, nch, t);
+      const WgradProblem& q = p.pr[u.prob];
+      const CUtensorMap* tm = u.prob == 0 ? &tmBig0 : &tmBig1;
+      const TileInfo ch = p.chunks[u.c];
+      const int d0 = u.dt * C::BM;
       const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       for (int ks = 0; ks < nk; ++ks) {
-        bool w = !(*abort_flag) && mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
+        const bool w = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         const uint32_t fb = smem_u32(&full[stage]);
         const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
         const int r0 = ch.row0 + ks * C::BK;
         if (lane == 0) {
           mbar_arrive_expect_tx(fb, C::BIG_BYTES);
-          tma_load_2d(&tmBig, fb, sbig, d0, r0);
-          tma_load_2d(&tmBig, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
+          tma_load_2d(tm, fb, sbig, d0, r0);
+          tma_load_2d(tm, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
         }
         // Small tile [BK rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
         // columns (128 B), row groups 128 B apart, column groups SMALL_NG bytes apart.
@@ -128,16 +188,16 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = lane; i < C::BK * CG; i += 32) {
           const int rr = i / CG, cg = i % CG;
           const int row = r0 + rr;
-          const bool valid = row < ch.row_end && cg * 8 < p.r_small;
-          const void* src = valid ? (const void*)(p.small + (size_t)row * p.ld_small + cg * 8)
-                                  : (const void*)p.small;
+          const bool valid = row < ch.row_end && cg * 8 < q.r_small;
+          const void* src = valid ? (const void*)(q.small + (size_t)row * q.ld_small + cg * 8)
+                                  : (const void*)q.small;
           cp_async_16(ssm + cg * C::SMALL_NG + (rr & 7) * 16 + (rr >> 3) * 128, src, valid ? 16u : 0u);
         }
         cp_async_mbar_arrive(fb);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
-    if (!ok) *abort_flag = 1;
+    if (!ok && lane == 0) *abort_flag = 1;
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -147,15 +207,15 @@ __global__ void __launch_bounds__(192, 1)
       int it = 0;
       bool ok = true, issued_any = false;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const int c = t / p.n_dtiles;
-        const TileInfo ch = p.chunks[c];
+        const WgradUnit u = wgrad_unit(p, nch, t);
+        const TileInfo ch = p.chunks[u.c];
         const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
         const int b = it & 1;
         if (!mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + b * 32;
+        if (*abort_flag) { ok = false; break; }
         for (int ks = 0; ks < nk; ++ks) {
-          if (*abort_flag) { ok = false; break; }
           if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
           fence_proxy_async_smem();   // cp.async writes -> tcgen05 reads
           tc_fence_after();
@@ -163,7 +223,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t ssm = sbig + C::BIG_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
-            // Big^T: MN-major, 128-byte swizzle, 64-column atoms 8 KB apart, 8-row groups 1 KB apart
+            // Big^T: MN-major, 128-byte swizzle, 64-column atoms BIG_BYTES/2 apart, 8-row groups 1 KB apart
             const uint64_t ad = smem_desc(sbig + kk * 16 * 128, C::BIG_BYTES / 2, 1024, kSw128);
             // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at SMALL_NG
             const uint64_t bd = smem_desc(ssm + kk * 256, 128, C::SMALL_NG, kSwNone);
@@ -185,60 +245,91 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue (warps 2..5)
-    const int q = warp & 3;
+    const int q4 = warp & 3;                       // TMEM lane quarter of this warp
+    const int et = (warp - 2) * 32 + lane;         // 0..127
+    // gradients of experts without rows are zero
+    for (int prob = 0; prob < p.n_problems; ++prob) {
+      const WgradProblem& q = p.pr[prob];
+      const int64_t tot = (int64_t)p.E * q.D;
+      for (int64_t i = (int64_t)blockIdx.x * C::EPI_THREADS + et; i < tot;
+           i += (int64_t)gridDim.x * C::EPI_THREADS) {
+        const int e = (int)(i / q.D), d = (int)(i - (int64_t)e * q.D);
+        if (p.chunk_start[e + 1] == p.chunk_start[e]) {
+          float z[RP];
+#pragma unroll
+          for (int j = 0; j < RP; ++j) z[j] = 0.f;
+          wgrad_store<RP>(q, p.r, p.scale, e, d, z);
+        }
+      }
+    }
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const int c = t / p.n_dtiles, dt = t % p.n_dtiles;
-      const TileInfo ch = p.chunks[c];
+      const WgradUnit u = wgrad_unit(p, nch, t);
+      const WgradProblem& q = p.pr[u.prob];
+      const TileInfo ch = p.chunks[u.c];
       const int b = it & 1;
-      bool ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
-      if (!__all_sync(0xffffffffu, ok)) { *abort_flag = 1; break; }
+      const bool ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
+      // every epilogue warp takes the same branch (named barriers follow)
+      if (named_bar_or(1, C::EPI_THREADS, !ok || *abort_flag != 0)) { *abort_flag = 1; break; }
       tc_fence_after();
       float v[RP];
       if constexpr (RP == 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + b * 32, r);
+        uint32_t rr[16];
+        tmem_ld16(tmem + ((uint32_t)(q4 * 32) << 16) + b * 32, rr);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
       } else {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + b * 32, r);
+        uint32_t rr[32];
+        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + b * 32, rr);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
-      const int d = dt * C::BM + q * 32 + lane;
-      if (d < p.D) {
-        const bool single = p.chunk_start[ch.e + 1] - p.chunk_start[ch.e] == 1;
-        if (single) {
-          if (p.transpose) {
+      const int d = u.dt * C::BM + q4 * 32 + lane;
+      const int c0 = p.chunk_start[ch.e], c1 = p.chunk_start[ch.e + 1];
+      if (c1 - c0 == 1) {
+        if (d < q.D) wgrad_store<RP>(q, p.r, p.scale, ch.e, d, v);
+        continue;
+      }
+      // several chunks: fp32 partial, then the last arriving unit sums them in order
+      if (d < q.D) {
+        float4* dst = reinterpret_cast<float4*>(q.partial + ((size_t)u.c * q.D + d) * RP);
 #pragma unroll
-            for (int i = 0; i < RP; ++i)
-              if (i < p.r) p.out[((size_t)ch.e * p.r + i) * p.D + d] = __float2bfloat16_rn(p.scale * v[i]);
-          } else {
-            __nv_bfloat16* dst = p.out + ((size_t)ch.e * p.D + d) * p.r;
-#pragma unroll
-            for (int g = 0; g < RP / 8; ++g) {
-              if (g * 8 < p.r) {
-                uint4 o;
-                o.x = pack_bf16x2(p.scale * v[8 * g + 0], p.scale * v[8 * g + 1]);
-                o.y = pack_bf16x2(p.scale * v[8 * g + 2], p.scale * v[8 * g + 3]);
-                o.z = pack_bf16x2(p.scale * v[8 * g + 4], p.scale * v[8 * g + 5]);
-                o.w = pack_bf16x2(p.scale * v[8 * g + 6], p.scale * v[8 * g + 7]);
-                *reinterpret_cast<uint4*>(dst + 8 * g) = o;
-              }
-            }
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(p.partial + ((size_t)c * p.D + d) * RP);
-#pragma unroll
-          for (int i = 0; i < RP / 4; ++i)
-            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        for (int i = 0; i < RP / 4; ++i)
+          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      }
+      __threadfence();
+      named_bar(1, C::EPI_THREADS);
+      if (et == 0) {
+        int* cnt = q.counters + (size_t)ch.e * q.n_dtiles + u.dt;
+        const int last = atomicAdd(cnt, 1) == c1 - c0 - 1;
+        if (last) {
+          *cnt = 0;                                // ready for the next launch
+          __threadfence();
         }
+        *last_flag = last;
+      }
+      named_bar(1, C::EPI_THREADS);
+      if (*last_flag && d < q.D) {
+        float acc[RP];
+#pragma unroll
+        for (int i = 0; i < RP; ++i) acc[i] = 0.f;
+        for (int cc = c0; cc < c1; ++cc) {
+          const float4* src = reinterpret_cast<const float4*>(q.partial + ((size_t)cc * q.D + d) * RP);
+#pragma unroll
+          for (int i = 0; i < RP / 4; ++i) {
+            const float4 x = __ldcg(src + i);
+            acc[4 * i] += x.x;
+            acc[4 * i + 1] += x.y;
+            acc[4 * i + 2] += x.z;
+            acc[4 * i + 3] += x.w;
+          }
+        }
+        wgrad_store<RP>(q, p.r, p.scale, ch.e, d, acc);
       }
     }
   }
@@ -248,43 +339,6 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// Experts with 0 chunks get zeros; experts with 2+ chunks get
-// bf16(scale * sum of their partials in chunk order).  Single-chunk experts were
-// written by lora_wgrad_kernel.  transpose = false: out [E, D, r]; true: [E, r, D].
-template <int RP>
-__global__ void lora_wgrad_reduce_kernel(const float* __restrict__ partial,
-                                         const int* __restrict__ chunk_start, int E, int D, int r,
-                                         float scale, bool transpose,
-                                         __nv_bfloat16* __restrict__ out) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)E * D) return;
-  const int e = (int)(idx / D), d = (int)(idx % D);
-  const int c0 = chunk_start[e], c1 = chunk_start[e + 1];
-  if (c1 - c0 == 1) return;
-  float acc[RP];
-#pragma unroll
-  for (int i = 0; i < RP; ++i) acc[i] = 0.f;
-  for (int c = c0; c < c1; ++c) {
-    const float4* src = reinterpret_cast<const float4*>(partial + ((size_t)c * D + d) * RP);
-#pragma unroll
-    for (int i = 0; i < RP / 4; ++i) {
-      const float4 v = src[i];
-      acc[4 * i] += v.x;
-      acc[4 * i + 1] += v.y;
-      acc[4 * i + 2] += v.z;
-      acc[4 * i + 3] += v.w;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < RP; ++i) {
-    if (i < r) {
-      const __nv_bfloat16 o = __float2bfloat16_rn(scale * acc[i]);
-      if (transpose) out[((size_t)e * r + i) * D + d] = o;
-      else out[((size_t)e * D + d) * r + i] = o;
-    }
   }
 }
 

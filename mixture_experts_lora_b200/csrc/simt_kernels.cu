@@ -243,7 +243,9 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
                                     int gchunk_rows, TileInfo* __restrict__ gchunks,
                                     int* __restrict__ n_gchunks, int chunk_rows,
                                     TileInfo* __restrict__ chunks, int* __restrict__ n_chunks,
-                                    int32_t* __restrict__ chunk_start) {
+                                    int32_t* __restrict__ chunk_start, int* __restrict__ zero,
+                                    int n_zero) {
+  for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
   __shared__ int s_warp[33];
   const int e = threadIdx.x;
   int lo = 0, hi = 0;
@@ -292,10 +294,11 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
 cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
                                 int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
                                 int chunk_rows, TileInfo* chunks, int* n_chunks,
-                                int32_t* chunk_start, cudaStream_t s) {
+                                int32_t* chunk_start, int* zero, int n_zero, cudaStream_t s) {
   ProfScope ps(K_TABLES, s);
   build_tables_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_rows, tiles, n_tiles, gchunk_rows, gchunks,
-                                         n_gchunks, chunk_rows, chunks, n_chunks, chunk_start);
+                                         n_gchunks, chunk_rows, chunks, n_chunks, chunk_start,
+                                         zero, n_zero);
   return cudaGetLastError();
 }
 
