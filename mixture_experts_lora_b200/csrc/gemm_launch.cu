@@ -8,6 +8,7 @@
 #include "internal.h"
 #include "lora_wgrad.cuh"
 #include "lowrank.cuh"
+#include "rows_gather.cuh"
 #include "rows_lowrank.cuh"
 
 namespace moe {
@@ -194,6 +195,18 @@ static cudaError_t rows_rp(const GemmShape& g, const CUtensorMap* tl, const Rows
   return cudaGetLastError();
 }
 
+template <int RP, bool L_MN>
+static cudaError_t rows_gather_rp(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
+                                  cudaStream_t s) {
+  using C = RowsGatherCfg<RP>;
+  auto kern = rows_gather_kernel<RP, L_MN>;
+  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
+  if (st != cudaSuccess) return st;
+  ProfScope ps(K_ROWS_GATHER, s);
+  kern<<<g.max_row_tiles, RG_THREADS, C::SMEM_BYTES, s>>>(tl[0], rp_);
+  return cudaGetLastError();
+}
+
 template <int MODE, bool L_MN>
 static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
                              cudaStream_t s) {
@@ -239,8 +252,11 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
   p.r_save = r_save;
   p.outc = reinterpret_cast<__nv_bfloat16*>(outc);
   p.err = g.err;
-  if (mode == ROWS_GATHER)
-    return L_mn ? rows_mode<ROWS_GATHER, true>(g, tl, p, s) : rows_mode<ROWS_GATHER, false>(g, tl, p, s);
+  if (mode == ROWS_GATHER) {
+    if (g.rp == 16)
+      return L_mn ? rows_gather_rp<16, true>(g, tl, p, s) : rows_gather_rp<16, false>(g, tl, p, s);
+    return L_mn ? rows_gather_rp<32, true>(g, tl, p, s) : rows_gather_rp<32, false>(g, tl, p, s);
+  }
   if (mode == ROWS_SWIGLU) return rows_mode<ROWS_SWIGLU, true>(g, tl, p, s);
   return rows_mode<ROWS_SWIGLU_BWD, false>(g, tl, p, s);
 }
