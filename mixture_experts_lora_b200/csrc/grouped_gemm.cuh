@@ -74,13 +74,19 @@ struct GemmCfg {
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_BYTES = EPI_WARPS * BLK_BYTES;   // one transpose block per warp
   static constexpr int SMEM_LIMIT = 232448;
-  static constexpr int STAGES_FIT = (SMEM_LIMIT - EPI_BYTES - 2048) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 2048;
-  static constexpr int TMEM_COLS = 512;
   static constexpr int LA_BOX_BYTES = RP * 64 * 2;          // forward: 64 features x RP rows
   static constexpr int LA_BYTES = A_MN ? 2 * LA_BOX_BYTES : BM * RP * 2;
   static constexpr int LR_BOX_BYTES = BOXR * RP * 2;        // 64 token rows x RP
+  // LSIDE: the LoRA block's operands (LA: L_B^T, LR: c*LR rows) live in a double
+  // buffer of their own, loaded at the start of a tile, instead of taking a whole
+  // ring stage per tile (fits beside three stages for RP = 16)
+  static constexpr bool LSIDE = RP == 16;
+  static constexpr int LS_BYTES = LA_BYTES + NHALF * RP * 2;
+  static constexpr int LS_TOTAL = LSIDE ? 2 * LS_BYTES : 0;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - EPI_BYTES - LS_TOTAL - 2048) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LS_TOTAL + EPI_BYTES + 2048;
+  static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t LR_SWZ = RP == 16 ? kSw32 : kSw64;
   static constexpr uint32_t LR_SBO = RP == 16 ? 256 : 512;
   static_assert(RP == 16 || RP == 32, "RP");
@@ -100,7 +106,8 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  uint8_t* epi = smem + C::STAGES * C::STAGE_BYTES;
+  const uint32_t side_off = C::STAGES * C::STAGE_BYTES;   // LoRA side buffers (LSIDE)
+  uint8_t* epi = smem + C::STAGES * C::STAGE_BYTES + C::LS_TOTAL;
   uint64_t* bars = reinterpret_cast<uint64_t*>(epi + C::EPI_BYTES);
   uint64_t* full = bars;                       // [STAGES] (used in the leader)
   uint64_t* empty = bars + C::STAGES;          // [STAGES]
@@ -109,6 +116,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain = acc_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(acc_full + 6);
+  uint64_t* lfull = acc_full + 8;              // [2] LoRA side buffer loaded (leader)
+  uint64_t* lempty = acc_full + 10;            // [2] LoRA side buffer consumed
 
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
@@ -124,6 +133,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(smem_u32(&acc_empty[b]), 2 * C::EPI_WARPS);
     }
     mbar_init(smem_u32(drain), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&lfull[b]), 1);
+      mbar_init(smem_u32(&lempty[b]), 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmW);
@@ -149,14 +162,36 @@ __global__ void __launch_bounds__(320, 1)
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
-    for (int t = pair; t < total && ok; t += npairs) {
+    int it = 0;
+    for (int t = pair; t < total && ok; t += npairs, ++it) {
       const int c = t / p.n_ftiles, w = t % p.n_ftiles;
       const TileInfo ch = p.chunks[c];
       const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
       const int nbh = (half + C::BOXR - 1) / C::BOXR;
       const int r0 = ch.row0 + (int)rank * half;
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-      for (int ks = 0; ks <= p.nk; ++ks) {
+      if constexpr (C::LSIDE) {
+        // LoRA operands of this tile into side buffer it & 1
+        const int lb = it & 1;
+        const bool lok = mbar_wait(smem_u32(&lempty[lb]), ((it >> 1) & 1) ^ 1, p.err);
+        if (!__all_sync(0xffffffffu, lok)) { ok = false; break; }
+        if (lane == 0) {
+          const uint32_t lfb = mapa_smem(smem_u32(&lfull[lb]), 0);
+          const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
+          const uint32_t lr = la + C::LA_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&lfull[lb]), 2 * (C::LA_BYTES + nbh * C::LR_BOX_BYTES));
+          if constexpr (C::A_MN) {
+            tma_load_3d_pair(&tmLW, lfb, la, feat_box(w, rank, 0), 0, ch.e);
+            tma_load_3d_pair(&tmLW, lfb, la + C::LA_BOX_BYTES, feat_box(w, rank, 1), 0, ch.e);
+          } else {
+            tma_load_3d_pair(&tmLW, lfb, la, 0, feat_box(w, rank, 0), ch.e);
+          }
+          for (int j = 0; j < nbh; ++j)
+            tma_load_2d_pair(&tmLR, lfb, lr + j * C::LR_BOX_BYTES, 0, r0 + j * C::BOXR);
+        }
+        __syncwarp();
+      }
+      for (int ks = 0; ks < p.nk + (C::LSIDE ? 0 : 1); ++ks) {
         const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
         if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
         if (lane == 0) {
@@ -232,7 +267,27 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         const uint32_t d = tmem + b * C::NMAX;
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-        for (int ks = 0; ks <= p.nk; ++ks) {
+        if constexpr (C::LSIDE) {
+          // the LoRA block first (it starts the accumulation), from side buffer it & 1
+          const int lb = it & 1;
+          const bool lok = mbar_wait(smem_u32(&lfull[lb]), (it >> 1) & 1, p.err);
+          if (!__all_sync(0xffffffffu, lok)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
+            const uint32_t lr = la + C::LA_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < C::RP / 16; ++kk) {
+              const uint64_t ad = C::A_MN ? smem_desc(la + kk * 2048, C::LA_BOX_BYTES, 1024, kSw128)
+                                          : smem_desc(la + kk * 32, 16, C::LR_SBO, C::LR_SWZ);
+              umma_bf16_pair(d, ad, smem_desc(lr + kk * 32, 16, C::LR_SBO, C::LR_SWZ), idesc,
+                             kk ? 1u : 0u);
+            }
+            umma_commit_pair(smem_u32(&lempty[lb]), 0x3);
+          }
+          __syncwarp();
+        }
+        for (int ks = 0; ks < p.nk + (C::LSIDE ? 0 : 1); ++ks) {
           const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
           if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
           tc_fence_after();
@@ -247,7 +302,7 @@ __global__ void __launch_bounds__(320, 1)
                 const uint32_t ka = (uint32_t)((kk >> 2) * C::ATOM_A + (kk & 3) * 32) >> 4;
                 const uint32_t kb = (uint32_t)((kk >> 2) * C::ATOM_B + (kk & 3) * 32) >> 4;
                 umma_bf16_pair(d, a_desc0 + so + (C::A_MN ? kk * (2048 / 16) : ka), b_desc0 + so + kb,
-                               idesc, (ks | kk) ? 1u : 0u);
+                               idesc, (C::LSIDE || (ks | kk)) ? 1u : 0u);
               }
             } else {
 #pragma unroll
