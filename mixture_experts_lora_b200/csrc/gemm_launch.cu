@@ -9,6 +9,7 @@
 #include "lora_wgrad.cuh"
 #include "lowrank.cuh"
 #include "rows_gather.cuh"
+#include "rows_swiglu.cuh"
 #include "rows_lowrank.cuh"
 
 namespace moe {
@@ -207,6 +208,18 @@ static cudaError_t rows_gather_rp(const GemmShape& g, const CUtensorMap* tl, con
   return cudaGetLastError();
 }
 
+template <int MODE, int RP>
+static cudaError_t rows_swiglu_rp(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
+                                  cudaStream_t s) {
+  using C = RowsSwigluCfg<MODE, RP>;
+  auto kern = rows_swiglu_kernel<MODE, RP>;
+  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
+  if (st != cudaSuccess) return st;
+  ProfScope ps(MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD, s);
+  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
+  return cudaGetLastError();
+}
+
 template <int MODE, bool L_MN>
 static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
                              cudaStream_t s) {
@@ -257,8 +270,15 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
       return L_mn ? rows_gather_rp<16, true>(g, tl, p, s) : rows_gather_rp<16, false>(g, tl, p, s);
     return L_mn ? rows_gather_rp<32, true>(g, tl, p, s) : rows_gather_rp<32, false>(g, tl, p, s);
   }
-  if (mode == ROWS_SWIGLU) return rows_mode<ROWS_SWIGLU, true>(g, tl, p, s);
-  return rows_mode<ROWS_SWIGLU_BWD, false>(g, tl, p, s);
+  // SwiGLU modes: 128-row x 64-column input tiles, 128-byte swizzled (they become
+  // the MMA operand in place)
+  ok = encode2d(&tl[1], gu, P, 2 * n, 128, 64) &&
+       encode2d(&tl[2], dh != nullptr ? dh : gu, P, dh != nullptr ? n : 2 * n, 128, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  if (mode == ROWS_SWIGLU)
+    return g.rp == 16 ? rows_swiglu_rp<ROWS_SWIGLU, 16>(g, tl, p, s) : rows_swiglu_rp<ROWS_SWIGLU, 32>(g, tl, p, s);
+  return g.rp == 16 ? rows_swiglu_rp<ROWS_SWIGLU_BWD, 16>(g, tl, p, s)
+                    : rows_swiglu_rp<ROWS_SWIGLU_BWD, 32>(g, tl, p, s);
 }
 
 template <int RP, bool L_MN>
