@@ -7,10 +7,9 @@
 #include "grouped_gemm.cuh"
 #include "internal.h"
 #include "lora_wgrad.cuh"
-#include "lowrank.cuh"
 #include "rows_gather.cuh"
 #include "rows_swiglu.cuh"
-#include "rows_lowrank.cuh"
+#include "rows_common.cuh"
 
 namespace moe {
 
@@ -184,18 +183,6 @@ cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const
   return gemm_any(K_GEMM_GATEUP_BWD, g, w.W_gu, true, g.m, 2 * g.n, dGU, w.A_gu, T2c, dXp, s);
 }
 
-template <int MODE, int RP, bool L_MN>
-static cudaError_t rows_rp(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
-                           cudaStream_t s) {
-  using C = RowsCfg<MODE, RP, L_MN>;
-  auto kern = rows_lowrank_kernel<MODE, RP, L_MN>;
-  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
-  if (st != cudaSuccess) return st;
-  ProfScope ps(MODE == ROWS_GATHER ? K_ROWS_GATHER : (MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD), s);
-  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
-  return cudaGetLastError();
-}
-
 template <int RP, bool L_MN>
 static cudaError_t rows_gather_rp(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
                                   cudaStream_t s) {
@@ -218,13 +205,6 @@ static cudaError_t rows_swiglu_rp(const GemmShape& g, const CUtensorMap* tl, con
   ProfScope ps(MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD, s);
   kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
   return cudaGetLastError();
-}
-
-template <int MODE, bool L_MN>
-static cudaError_t rows_mode(const GemmShape& g, const CUtensorMap* tl, const RowsParams& rp_,
-                             cudaStream_t s) {
-  if (g.rp == 16) return rows_rp<MODE, 16, L_MN>(g, tl, rp_, s);
-  return rows_rp<MODE, 32, L_MN>(g, tl, rp_, s);
 }
 
 cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint16_t* src,
@@ -281,40 +261,6 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
                     : rows_swiglu_rp<ROWS_SWIGLU_BWD, 32>(g, tl, p, s);
 }
 
-template <int RP, bool L_MN>
-static cudaError_t lowrank_rp(const GemmShape& g, const CUtensorMap& ta, const CUtensorMap& tl,
-                              const LowrankParams& lp, cudaStream_t s) {
-  using C = LowrankCfg<RP, L_MN>;
-  auto kern = lowrank_kernel<RP, L_MN>;
-  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
-  if (st != cudaSuccess) return st;
-  ProfScope ps(K_LOWRANK, s);
-  kern<<<g.max_row_tiles, 128, C::SMEM_BYTES, s>>>(ta, tl, lp);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const uint16_t* L,
-                           bool L_mn, uint16_t* save, int ld_save, int r_save, uint16_t* outc,
-                           cudaStream_t s) {
-  CUtensorMap ta, tl;
-  const uint64_t E = g.E, rp = g.rp;
-  bool ok = encode2d(&ta, act, (uint64_t)g.P, (uint64_t)K, 128, 64);
-  ok = ok && (L_mn ? encode3d(&tl, L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
-                   : encode3d(&tl, L, E, rp, (uint64_t)K, (uint32_t)rp, 64));
-  if (!ok) return cudaErrorInvalidValue;
-  LowrankParams lp{};
-  lp.tiles = g.tiles;
-  lp.n_tiles = g.n_row_tiles;
-  lp.nk = (K + 63) / 64;
-  lp.scale = g.scale;
-  lp.save = reinterpret_cast<__nv_bfloat16*>(save);
-  lp.ld_save = ld_save;
-  lp.r_save = r_save;
-  lp.outc = reinterpret_cast<__nv_bfloat16*>(outc);
-  lp.err = g.err;
-  if (g.rp == 16) return L_mn ? lowrank_rp<16, true>(g, ta, tl, lp, s) : lowrank_rp<16, false>(g, ta, tl, lp, s);
-  return L_mn ? lowrank_rp<32, true>(g, ta, tl, lp, s) : lowrank_rp<32, false>(g, ta, tl, lp, s);
-}
 
 template <int RP>
 static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const WgradParams& wp,

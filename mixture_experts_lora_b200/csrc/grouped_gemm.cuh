@@ -12,7 +12,7 @@
 //
 // where Act is the expert-sorted activation matrix, Wt the weight oriented
 // feature-major and LRc = bf16(c * Act L_A[e]) the rank-r product from the
-// low-rank kernel; the second sum is one extra K-block of the same pipeline.
+// row kernel; the second sum is one extra K-block of the same pipeline.
 // This is Y = XW + (alpha/r)(XA)B of the Split-LoRA reordering ("Accelerating
 // Mixture-of-Experts Fine-Tuning", Mathematical Formulation section 2) with no
 // K x N adapter delta.

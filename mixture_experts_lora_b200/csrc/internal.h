@@ -16,7 +16,7 @@ struct TileInfo;
 enum KernelKind : int {
   K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
-  K_COMBINE, K_MEMSET, K_LOWRANK, K_ROWS_GATHER, K_ROWS_SWIGLU,
+  K_COMBINE, K_MEMSET, K_ROWS_GATHER, K_ROWS_SWIGLU,
   K_ROWS_SWIGLU_BWD, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
@@ -44,7 +44,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
                            int32_t* hist, int* err, cudaStream_t s);
 // From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
-// experts (low-rank kernel), token chunks of at most `gchunk_rows` rows split
+// experts (row kernels), token chunks of at most `gchunk_rows` rows split
 // evenly inside each expert (grouped GEMMs; all but the last chunk of an expert
 // are multiples of 16), and row chunks of `chunk_rows` rows (adapter gradients)
 // with chunk_start[e] = first chunk of expert e.
@@ -77,7 +77,7 @@ struct GemmShape {
   int64_t P;
   int m, n, E, r, rp;
   float scale;
-  int max_row_tiles;          // 128-row tiles (low-rank kernel)
+  int max_row_tiles;          // 128-row tiles (row kernels)
   const TileInfo* tiles;
   const int* n_row_tiles;
   int max_gchunks;            // token chunks of at most 256 rows (grouped GEMMs)
@@ -87,11 +87,6 @@ struct GemmShape {
   int num_sms;
 };
 
-// LR = Act L[e] per expert segment; save = LR (first r_save columns, ld_save),
-// outc = bf16(scale * LR) [P, rp].  L_mn: L stored [E, K, rp]; else [E, rp, K].
-cudaError_t launch_lowrank(const GemmShape& g, const uint16_t* act, int K, const uint16_t* L,
-                           bool L_mn, uint16_t* save, int ld_save, int r_save, uint16_t* outc,
-                           cudaStream_t s);
 // Grouped GEMMs (features on M, expert tokens on N, CTA pairs); each writes
 // out [P, F] in sorted token order.
 // GU = Xs W_gu + XAc B_gu             (XAc = bf16(c X A_gu))
@@ -106,7 +101,7 @@ cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const u
 // dXp = dGU W_gu^T + T2c A_gu^T
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
                                    const uint16_t* T2c, uint16_t* dXp, cudaStream_t s);
-// Row producer + rank-r product (rows_lowrank.cuh); mode: 0 gather (src rows by
+// Row producer + rank-r product (rows_gather.cuh, rows_swiglu.cuh); mode: 0 gather (src rows by
 // sorted pair, times w if given), 1 SwiGLU from gu, 2 SwiGLU backward from dh and gu.
 // Writes rows_out [P, K] (if not null), save = LR (first r_save columns, ld_save)
 // and outc = bf16(scale * LR) [P, rp].

@@ -17,7 +17,7 @@
 #pragma once
 
 #include "common.cuh"
-#include "rows_lowrank.cuh"
+#include "rows_common.cuh"
 
 namespace moe {
 
