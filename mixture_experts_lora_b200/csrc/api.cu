@@ -74,7 +74,8 @@ struct Layout {
   size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
   size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
   int max_dtiles;             // 128-column tiles of the widest adapter gradient
-  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial, partial2, counters;
+  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial, partial2, rows_partial;
+  size_t counters;           // [row kernels fwd 2][row kernels bwd 2][gradients 4] sets
   size_t total;
 };
 
@@ -114,7 +115,10 @@ Layout make_layout(const moe_dims_t& d) {
   L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
   L.partial2 = take((size_t)L.max_chunks * dmax * rp * 4);
   L.max_dtiles = (int)((dmax + 127) / 128);
-  L.counters = take((size_t)4 * E * L.max_dtiles * 4);   // one set per adapter gradient
+  L.rows_partial = take((size_t)kRowsMaxCtas * 2 * 128 * rp * 4);
+  // arrival counters: one set of max_row_tiles per row-kernel launch, then one set
+  // of E * max_dtiles per adapter gradient
+  L.counters = take(((size_t)4 * L.max_row_tiles + (size_t)4 * E * L.max_dtiles) * 4);
   L.total = off;
   return L;
 }
@@ -144,8 +148,10 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
                               at<int>(ws, L.n_gchunks), L.chunk_rows,
                               with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
                               at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start),
-                              with_chunks ? at<int>(ws, L.counters) : nullptr,
-                              with_chunks ? 4 * d.E * L.max_dtiles : 0, s));
+                              at<int>(ws, L.counters) + (with_chunks ? 2 * L.max_row_tiles : 0),
+                              with_chunks ? 2 * L.max_row_tiles + 4 * d.E * L.max_dtiles
+                                          : 2 * L.max_row_tiles,
+                              s));
   w->W_gu = W_gu;
   w->W_d = W_d;
   if (d.r != L.rp) {
@@ -276,14 +282,16 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   uint16_t* xs = at<uint16_t>(ws, L.rows);
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
+  float* rpart = at<float>(ws, L.rows_partial);
+  int* rcnt = at<int>(ws, L.counters);           // row-kernel sets 0 and 1 (zeroed above)
   // X rows in expert order, XA = X A_gu (saved) and bf16(c XA)
   MOE_TRY(launch_rows_lowrank(g, 0, d.m, X, sorted_pairs, nullptr, d.k, nullptr, nullptr, w.A_gu,
-                              true, xs, save_XA, d.r, d.r, xac, s));
+                              true, xs, save_XA, d.r, d.r, xac, rpart, rcnt, s));
   // GU = X W_gu + (c XA) B_gu
   MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, xac, save_GU, s));
   // H = silu(g) u, HA = H A_d (saved) and bf16(c HA)
   MOE_TRY(launch_rows_lowrank(g, 1, d.n, nullptr, nullptr, nullptr, d.k, save_GU, nullptr, w.A_d,
-                              true, save_H, save_HA, d.r, d.r, hac, s));
+                              true, save_H, save_HA, d.r, d.r, hac, rpart, rcnt + L.max_row_tiles, s));
   // Y = H W_d + (c HA) B_d
   MOE_TRY(launch_gemm_down_fwd(g, w, save_H, hac, Y_sorted, s));
   return MOE_OK;
@@ -334,14 +342,16 @@ moe_status_t moe_grouped_gemm_lora_bwd(
   uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
   uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
   uint16_t* dh = at<uint16_t>(ws, L.dh);
+  float* rpart = at<float>(ws, L.rows_partial);
+  int* rcnt = at<int>(ws, L.counters) + 2 * L.max_row_tiles;   // row-kernel sets 2 and 3
   // dy = w * dY[t] in expert order, T1 = dy B_d^T (kept for dA_d) and bf16(c T1)
   MOE_TRY(launch_rows_lowrank(g, 0, d.m, dY, sorted_pairs, topk_w, d.k, nullptr, nullptr, w.B_d,
-                              false, rows, t1, L.rp, L.rp, lrc1, s));
+                              false, rows, t1, L.rp, L.rp, lrc1, rpart, rcnt, s));
   // dH = dy W_d^T + (c T1) A_d^T
   MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
   // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
   float* partial2 = at<float>(ws, L.partial2);
-  int* counters = at<int>(ws, L.counters);
+  int* counters = at<int>(ws, L.counters) + 4 * L.max_row_tiles;   // gradient sets
   const size_t cstride = (size_t)d.E * L.max_dtiles;
   {
     const WgradJob jobs[2] = {
@@ -351,7 +361,7 @@ moe_status_t moe_grouped_gemm_lora_bwd(
   }
   // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
   MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
-                              false, dgu, t2, L.rp, L.rp, lrc2, s));
+                              false, dgu, t2, L.rp, L.rp, lrc2, rpart, rcnt + L.max_row_tiles, s));
   // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
   // X re-gathered into the row buffer (dy is no longer needed), then

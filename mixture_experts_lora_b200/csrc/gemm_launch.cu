@@ -202,8 +202,11 @@ static cudaError_t rows_swiglu_rp(const GemmShape& g, const CUtensorMap* tl, con
   auto kern = rows_swiglu_kernel<MODE, RP>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
+  // persistent: C::CTAS_PER_SM per SM (the kernel uses at most one CTA per unit)
+  int grid = g.num_sms * C::CTAS_PER_SM;
+  if (grid > kRowsMaxCtas) grid = kRowsMaxCtas;
   ProfScope ps(MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD, s);
-  kern<<<g.max_row_tiles, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
   return cudaGetLastError();
 }
 
@@ -211,7 +214,8 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
                                 const int32_t* sorted_pairs, const float* w, int k,
                                 const uint16_t* gu, const uint16_t* dh, const uint16_t* L,
                                 bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
-                                int r_save, uint16_t* outc, cudaStream_t s) {
+                                int r_save, uint16_t* outc, float* partial, int* counters,
+                                cudaStream_t s) {
   CUtensorMap tl[3];
   const uint64_t E = g.E, rp = g.rp, P = g.P, n = g.n;
   bool ok = L_mn ? encode3d(&tl[0], L, E, (uint64_t)K, rp, 64, (uint32_t)rp)
@@ -244,6 +248,8 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
   p.ld_save = ld_save;
   p.r_save = r_save;
   p.outc = reinterpret_cast<__nv_bfloat16*>(outc);
+  p.partial = partial;
+  p.counters = counters;
   p.err = g.err;
   if (mode == ROWS_GATHER) {
     if (g.rp == 16)

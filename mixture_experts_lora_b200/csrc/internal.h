@@ -38,6 +38,8 @@ int* moe_status_word();
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
+// persistent row kernels run at most this many CTAs (sizes their partial buffer)
+constexpr int kRowsMaxCtas = 1024;
 // one block per chunk of kPermuteChunk pairs; hist holds n_chunks * E ints
 constexpr int kPermuteChunk = 512;
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
@@ -109,7 +111,8 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
                                 const int32_t* sorted_pairs, const float* w, int k,
                                 const uint16_t* gu, const uint16_t* dh, const uint16_t* L,
                                 bool L_mn, uint16_t* rows_out, uint16_t* save, int ld_save,
-                                int r_save, uint16_t* outc, cudaStream_t s);
+                                int r_save, uint16_t* outc, float* partial, int* counters,
+                                cudaStream_t s);
 // out = scale * sum_rows Big^T Small per expert, out [E, D, r] or (transpose) [E, r, D]
 // One adapter-gradient problem G_e = Big_e^T Small_e (see lora_wgrad.cuh).
 struct WgradJob {
