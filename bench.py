@@ -44,11 +44,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="qwen3_30b_a3b", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel from the host in the timed steps instead of replaying "
+                         "one captured CUDA graph per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="tokens per oracle sample (0: sized for ~15 s)")
@@ -72,7 +75,7 @@ def workload_name(cfg):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """nvidia-smi samples every 100 ms while the timed region runs."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -86,7 +89,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -267,7 +270,9 @@ def run_reference(args, cfg):
         return
     cpu = generate(cfg, seed=0, device="cpu")
     W64 = oracle_setup(cfg, cpu)
-    ntok = pick_sample_tokens(cfg, cpu, W64, 2.0, args.cpu_sample_tokens)
+    # each step a bounded sample: about two minutes for the whole run
+    per_step_s = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    ntok = pick_sample_tokens(cfg, cpu, W64, per_step_s, args.cpu_sample_tokens)
     for s in range(args.warmup):
         time_oracle_sample(cfg, cpu, W64, (s * ntok) % max(1, cfg.T - ntok), ntok)
     times = []
@@ -339,28 +344,55 @@ def run_ours(args, cfg):
     top = max(prof_all, key=lambda k: prof_all[k][1]) if prof_all else None
 
     # ---- timed region (device time, CUDA events per step, L2 flushed before each
-    # step); only the dominant kernel kind is traced, so its events add two
-    # records per launch and nothing to the other kernels
+    # step outside the events); only the dominant kernel kind is traced, so its
+    # events add two records per launch and nothing to the other kernels.  By
+    # default each timed step replays its own CUDA graph of the layer's launches
+    # (captured here, with the dominant kernel's trace events as graph nodes), so
+    # the step carries no host launch gaps; the gradient all-reduce (N > 1) runs
+    # after the replay, inside the step's events.
+    if top is not None:
+        ml.moe_profile_select(top)
+        ml.moe_profile_enable(True)
+    graphs = []
+    if not args.no_graph:
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                ml.layer_step(inp, cfg.k, cfg.scale, buf)
+            graphs.append(gph)
+        ml.moe_profile_enable(False)
+        for gph in graphs:                 # upload; the trace records are read after the timed replays
+            gph.replay()
+        torch.cuda.synchronize()
+
+    def timed_step(i):
+        if graphs:
+            graphs[i].replay()
+            dp.allreduce_adapter_grads(grads)
+        else:
+            step()
+
     clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
+    time.sleep(1.0)                       # nvidia-smi's first sample precedes the timed steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    if top is not None:
-        ml.moe_profile_select(top)
+    if top is not None and not graphs:
         ml.moe_profile_enable(True)
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
-        step()
+        timed_step(i)
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     ml.moe_profile_enable(False)
     prof_top = ml.moe_profile_read()
     ml.moe_profile_select(None)
+    del graphs
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -471,6 +503,7 @@ def run_ours(args, cfg):
         "roofline": roof,
         "kernels": kernels,
         "kernels_source": "separate traced pass of the same steps (every launch bracketed by CUDA events)",
+        "launch": "host launches" if args.no_graph else "one CUDA graph replay per timed step",
         "gpu_launches": launches_total,
         "step_ms_min_max": [min(step_ms), max(step_ms)],
         "step_ms_median": median_ms,

@@ -198,7 +198,10 @@ const char* moe_status_string(moe_status_t status);
 /* Kernel timing, a tracing aid (no counterpart on the pages).  While enabled,
  * every kernel the library launches is bracketed by two CUDA events recorded
  * on its stream (a few hundred nanoseconds of device time each); events come
- * from a host-side pool, no device memory is allocated.  Off by default. */
+ * from a host-side pool, no device memory is allocated.  Off by default.
+ * Launches made while the stream is captured into a CUDA graph get event-record
+ * nodes instead; moe_profile_read then reports the times of the graph's most
+ * recent launch, so read after launching it (each capture holds its own events). */
 void moe_profile_enable(int on);
 
 /* Restricts the tracing to the kernel kinds named in `kinds`, a comma-separated

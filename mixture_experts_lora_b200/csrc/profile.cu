@@ -1,6 +1,7 @@
 // Kernel timing for the benchmark and for tracing: while enabled, every launch
 // the library makes is bracketed by a pair of CUDA events recorded on the
-// launch stream.  moe_profile_read() waits for the events and reports, per
+// launch stream (as event-record nodes when the stream is being captured into a
+// CUDA graph, so that a captured step is timed at each of its launches).  moe_profile_read() waits for the events and reports, per
 // kernel kind, the number of launches and their summed device time.  Events
 // come from a pool that grows on demand and is reused; no device memory is
 // allocated.
@@ -47,18 +48,27 @@ bool prof_enabled() { return g_on.load(); }
 
 bool prof_traced(int kind) { return g_on.load() && ((g_kinds.load() >> kind) & 1u); }
 
+// While `s` is being captured into a CUDA graph the records become event-record
+// nodes of the graph (timed when the graph is launched).
+cudaError_t record(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  return cudaEventRecord(e, s);
+}
+
 void* prof_begin(int kind, cudaStream_t s) {
   std::lock_guard<std::mutex> lk(g_mu);
   Rec* r = new Rec{kind, take_event(), take_event(), false};
   if (r->a == nullptr || r->b == nullptr) { delete r; return nullptr; }
-  cudaEventRecord(r->a, s);
+  record(r->a, s);
   g_recs.push_back(r);
   return r;
 }
 
 void prof_end(void* token, cudaStream_t s) {
   Rec* r = static_cast<Rec*>(token);
-  cudaEventRecord(r->b, s);
+  record(r->b, s);
   std::lock_guard<std::mutex> lk(g_mu);
   r->closed = true;
 }
