@@ -22,6 +22,7 @@
 namespace moe {
 
 constexpr int RG_STAGES = 4;
+constexpr int RG_LOOK = 2;      // stages of copies in flight ahead of the one being consumed
 constexpr int RG_WORKERS = 256;
 constexpr int RG_THREADS = RG_WORKERS + 32;   // + the control warp
 
@@ -105,14 +106,15 @@ __global__ void __launch_bounds__(RG_THREADS)
                     v ? (const void*)(srow[j] + col) : (const void*)p.src, v ? 16u : 0u);
       }
     };
-    // two stages ahead: the stage refilled at iteration it was last read by the
-    // MMAs of iteration it - 2, which have had a whole iteration to complete
-    issue(0);
-    cp_async_commit();
-    if (n_it > 1) issue(1);
-    cp_async_commit();
+    // RG_LOOK stages ahead: the stage refilled at iteration it was last read by the
+    // MMAs of iteration it + RG_LOOK - RG_STAGES, which have had time to complete
+#pragma unroll
+    for (int j = 0; j < RG_LOOK; ++j) {
+      if (j < n_it) issue(j);
+      cp_async_commit();
+    }
     for (int it = 0; it < n_it; ++it) {
-      const int nx = it + 2;
+      const int nx = it + RG_LOOK;
       if (nx < n_it) {
         // after a failed wait the tile's results are discarded: stop waiting
         if (ok && nx >= RG_STAGES)
@@ -120,7 +122,7 @@ __global__ void __launch_bounds__(RG_THREADS)
         issue(nx);
       }
       cp_async_commit();
-      cp_async_wait<2>();                        // this thread's pieces of stage it landed
+      cp_async_wait<RG_LOOK>();                  // this thread's pieces of stage it landed
       uint8_t* st = smem + (it % RG_STAGES) * C::TILE_BYTES;
       const int col = it * C::BK + cv * 8;
 #pragma unroll

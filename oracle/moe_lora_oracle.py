@@ -23,6 +23,9 @@ with gate = first n columns; renormalised top-k softmax with ties broken
 toward the lower expert index; stable (ascending pair index) order inside an
 expert segment; the router is frozen and its logits are an input.
 
+Beyond the path, router_backward gives the gradient into the router logits
+(for when the logits come from x W_r inside a model).
+
 Pins (tests/test_oracle_pins.py): Split-LoRA equals the materialised
 X(W + c A B); B = 0 gives the base MoE exactly; k = E with equal logits gives
 the plain average of all experts; gradients match central finite differences
@@ -37,7 +40,7 @@ __all__ = [
     "to64", "route_topk", "permute", "silu", "sigmoid",
     "expert_forward", "expert_forward_merged", "expert_backward",
     "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
-    "token_forward", "token_backward_dx", "expert_lora_grads",
+    "token_forward", "token_backward_dx", "expert_lora_grads", "router_backward",
 ]
 
 
@@ -362,3 +365,30 @@ def expert_lora_grads(inp, e: int, k: int, c: float, ids=None, w=None, W=None):
     f = expert_forward(x, *args)
     b = expert_backward(x, f, dy, *args)
     return b["dA_gu"], b["dB_gu"], b["dA_d"], b["dB_d"]
+
+
+# --------------------------------------------------------------------------
+# Router backward: the step before the path once the logits come from x W_r
+# inside a model ([Cookbook] "The Dynamic Dispatch Bottleneck in
+# Mixture-of-Experts Architectures", router equation; [MoE12x] "Implementation
+# details": the router weights stay frozen, a gradient still flows into x).
+# Y[t] = sum_j w[t,j] y_(t,j), so dL/dw[t,j] = <dY[t], y_(t,j)>.  The weights are
+# a softmax over the k picked logits, so
+#     dL/dl[t, ids[t,j]] = w[t,j] (dw[t,j] - sum_i w[t,i] dw[t,i]),
+# and logits that were not picked get zero (the selection is piecewise constant).
+# --------------------------------------------------------------------------
+def router_backward(dY, yp, ids, w, pair_pos, E: int):
+    """Return (dlogits fp64 [T, E], dw fp64 [T, k]); yp = expert outputs in sorted order."""
+    dY = to64(dY)
+    yp = to64(yp)
+    ids = np.asarray(ids, dtype=np.int64)
+    w = np.asarray(w, dtype=np.float64)
+    T, k = ids.shape
+    pos = np.asarray(pair_pos, dtype=np.int64).reshape(T, k)
+    dw = np.zeros((T, k))
+    for j in range(k):
+        dw[:, j] = np.sum(dY * yp[pos[:, j]], axis=1)
+    s = np.sum(w * dw, axis=1, keepdims=True)
+    dlogits = np.zeros((T, E))
+    np.put_along_axis(dlogits, ids, w * (dw - s), axis=1)
+    return dlogits, dw

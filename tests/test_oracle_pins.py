@@ -313,3 +313,75 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "route_topk", bad_route)
     assert not check_route()
     monkeypatch.setattr(O, "route_topk", good_route)
+
+
+# ---------------------------------------------------------------- router backward
+def _router_loss(logits64, ids, yp, pos, dY):
+    """L = sum_t <dY[t], sum_j w[t,j] y_(t,j)> with w = softmax over the fixed picks."""
+    T, k = ids.shape
+    sel = np.take_along_axis(logits64, ids, axis=1)
+    z = np.exp(sel - sel.max(axis=1, keepdims=True))
+    w = z / z.sum(axis=1, keepdims=True)
+    Y = np.zeros_like(dY)
+    for j in range(k):
+        Y += w[:, j:j + 1] * yp[pos.reshape(T, k)[:, j]]
+    return float(np.sum(Y * dY))
+
+
+def _router_case(seed=3):
+    cfg = small_config(T=40, m=32, n=16, E=7, k=3, r=8, alpha=16.0)
+    inp = _inp64(cfg, seed=seed)
+    Y, aux = O.moe_forward(inp, cfg.k, cfg.scale)
+    return cfg, inp, Y, aux
+
+
+def check_router_fd(h=1e-6):
+    cfg, inp, Y, aux = _router_case()
+    dl, _ = O.router_backward(inp["dY"], aux["yp"], aux["ids"], aux["w"], aux["pair_pos"], cfg.E)
+    lg = inp["logits"].astype(np.float64)
+    worst, scale = 0.0, max(np.max(np.abs(dl)), 1e-12)
+    for t in range(0, cfg.T, 3):
+        for e in range(cfg.E):            # picked and unpicked logits alike
+            lp, lm = lg.copy(), lg.copy()
+            lp[t, e] += h
+            lm[t, e] -= h
+            fd = (_router_loss(lp, aux["ids"], aux["yp"], aux["pair_pos"], inp["dY"]) -
+                  _router_loss(lm, aux["ids"], aux["yp"], aux["pair_pos"], inp["dY"])) / (2 * h)
+            worst = max(worst, abs(fd - dl[t, e]) / scale)
+    return worst
+
+
+def test_router_backward_matches_finite_differences():
+    assert check_router_fd() < 1e-6
+
+
+def test_router_backward_matches_autograd_and_sums_to_zero():
+    cfg, inp, Y, aux = _router_case(seed=5)
+    dl, dw = O.router_backward(inp["dY"], aux["yp"], aux["ids"], aux["w"], aux["pair_pos"], cfg.E)
+    # autograd through a differently written renormalisation: full softmax over E,
+    # pick, divide by the picked sum (equal to a softmax over the picked logits)
+    lt = torch.tensor(inp["logits"].astype(np.float64), requires_grad=True)
+    probs = torch.softmax(lt, dim=-1)
+    ids = torch.tensor(aux["ids"])
+    pv = torch.gather(probs, 1, ids)
+    pv = pv / pv.sum(-1, keepdim=True)
+    yp = torch.tensor(aux["yp"])
+    pos = torch.tensor(aux["pair_pos"]).reshape(cfg.T, cfg.k)
+    Yt = sum(pv[:, j:j + 1] * yp[pos[:, j]] for j in range(cfg.k))
+    assert _rel(Y, Yt.detach().numpy()) < 1e-12
+    (Yt * torch.tensor(inp["dY"])).sum().backward()
+    assert _rel(dl, lt.grad.numpy()) < 1e-11
+    # the softmax Jacobian annihilates constants: every row sums to zero
+    assert np.max(np.abs(dl.sum(axis=1))) < 1e-12 * max(1.0, np.max(np.abs(dl)))
+
+
+def test_router_pin_catches_planted_mistake(monkeypatch):
+    good = O.router_backward
+
+    def bad(dY, yp, ids, w, pair_pos, E):       # forgets the - sum_i w_i dw_i term
+        dl, dw = good(dY, yp, ids, w, pair_pos, E)
+        out = np.zeros_like(dl)
+        np.put_along_axis(out, np.asarray(ids), np.asarray(w) * dw, axis=1)
+        return out, dw
+    monkeypatch.setattr(O, "router_backward", bad)
+    assert check_router_fd() > 1e-3
