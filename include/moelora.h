@@ -188,6 +188,25 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* Y_sorted, const float* topk
                                    const int32_t* pair_pos, int64_t T, int32_t k,
                                    int32_t m, moe_bf16_t* Y, void* stream);
 
+/* Router backward, the step before the path once the logits come from x W_r
+ * inside a model ("Accelerating Mixture-of-Experts Fine-Tuning", section "The
+ * Dynamic Dispatch Bottleneck in Mixture-of-Experts Architectures": router
+ * equation; Unsloth faster-moe docs, "Implementation details": the router stays
+ * frozen but a gradient still flows into its input).  With Y[t] = sum_j
+ * w[t,j] y_(t,j) and w the softmax over the k picked logits:
+ *   dw[t,j]                = <dY[t], Y_sorted[pair_pos[t*k + j]]>   (fp32)
+ *   dlogits[t, ids[t,j]]   = w[t,j] (dw[t,j] - sum_i w[t,i] dw[t,i])
+ *   dlogits[t, e]          = 0 for every expert e not picked for token t.
+ * Inputs (device, read): dY bf16 [T, m]; Y_sorted bf16 [P, m] (the expert outputs
+ *   of moe_grouped_gemm_lora_fwd); topk_ids int32 [T, k]; topk_w fp32 [T, k];
+ *   pair_pos int32 [P].  Output (device, written): dlogits fp32 [T, E], every entry.
+ * Supported: 1 <= k <= 32, k <= E <= 1024, m % 8 == 0; dY and Y_sorted 16-byte
+ * aligned.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+moe_status_t moe_router_backward(const moe_bf16_t* dY, const moe_bf16_t* Y_sorted,
+                                 const int32_t* topk_ids, const float* topk_w,
+                                 const int32_t* pair_pos, int64_t T, int32_t k, int32_t E,
+                                 int32_t m, float* dlogits, void* stream);
+
 /* Synchronises `stream`, returns the device error word of the current device
  * (MOE_OK if no kernel reported a problem) and clears it. */
 moe_status_t moe_get_device_error(void* stream);

@@ -31,7 +31,7 @@ EXPORTED = (
     "moe_workspace_bytes", "moe_route_topk", "moe_permute", "moe_grouped_gemm_lora_fwd",
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
     "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
-    "moe_permute_noalloc",
+    "moe_permute_noalloc", "moe_router_backward",
 )
 
 
@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
         h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 15 + [SZ, P]
         h.moe_grouped_gemm_lora_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
         h.moe_unpermute_combine.argtypes = [P, P, P, I64, I32, I32, P, P]
+        h.moe_router_backward.argtypes = [P, P, P, P, P, I64, I32, I32, I32, P, P]
         h.moe_get_device_error.argtypes = [P]
         h.moe_status_string.argtypes = [ctypes.c_int]
         h.moe_status_string.restype = ctypes.c_char_p
@@ -156,6 +157,15 @@ def moe_unpermute_combine(Y_sorted, topk_w, pair_pos, T, k, m, Y, stream=None):
     _check("moe_unpermute_combine", lib().moe_unpermute_combine(
         _ptr(Y_sorted), _ptr(topk_w), _ptr(pair_pos), int(T), int(k), int(m), _ptr(Y),
         _stream(stream)))
+
+
+def moe_router_backward(dY, Y_sorted, topk_ids, topk_w, pair_pos, E: int, dlogits, stream=None):
+    """dlogits [T, E] fp32: gradient into the router logits (see include/moelora.h)."""
+    T, m = dY.shape
+    k = topk_ids.shape[1]
+    _check("moe_router_backward", lib().moe_router_backward(
+        _ptr(dY), _ptr(Y_sorted), _ptr(topk_ids), _ptr(topk_w), _ptr(pair_pos), int(T), int(k),
+        int(E), int(m), _ptr(dlogits), _stream(stream)))
 
 
 def moe_get_device_error(stream=None) -> int:

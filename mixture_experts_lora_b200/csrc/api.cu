@@ -376,6 +376,21 @@ moe_status_t moe_grouped_gemm_lora_bwd(
   return MOE_OK;
 }
 
+moe_status_t moe_router_backward(const moe_bf16_t* dY, const moe_bf16_t* Y_sorted,
+                                 const int32_t* topk_ids, const float* topk_w,
+                                 const int32_t* pair_pos, int64_t T, int32_t k, int32_t E,
+                                 int32_t m, float* dlogits, void* stream) {
+  if (T < 0 || m < 8) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > 32 || E < k || E > 1024 || m % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!aligned16(dY) || !aligned16(Y_sorted) || topk_ids == nullptr || topk_w == nullptr ||
+      pair_pos == nullptr || dlogits == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_router_backward(dY, Y_sorted, topk_ids, topk_w, pair_pos, T, k, E, m,
+                                            dlogits, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_unpermute_combine(const moe_bf16_t* Y_sorted, const float* topk_w,
                                    const int32_t* pair_pos, int64_t T, int32_t k, int32_t m,
                                    moe_bf16_t* Y, void* stream) {

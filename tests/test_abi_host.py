@@ -110,6 +110,23 @@ def test_host_validation_returns_before_launch(L):
     assert L.moe_unpermute_combine(fake, null, fake, 0, 2, 16, fake, null) == ml.MOE_OK
 
 
+def test_router_backward_host_validation(L):
+    null = None
+    fake = ctypes.c_void_p(256)       # 16-byte aligned, never dereferenced
+    odd = ctypes.c_void_p(258)
+    args = lambda **kw: [kw.get("dY", fake), kw.get("ys", fake), fake, fake, fake, kw.get("T", 4),
+                         kw.get("k", 2), kw.get("E", 8), kw.get("m", 64), kw.get("out", fake), null]
+    assert L.moe_router_backward(*args(k=0)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_backward(*args(k=33, E=64)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_backward(*args(E=1)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_backward(*args(m=12)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_backward(*args(m=4)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(*args(T=-1)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(*args(dY=odd)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(*args(out=null)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(*args(T=0, out=null)) == ml.MOE_OK   # empty input
+
+
 def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ml, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(ml, "_lib_handle", None)
