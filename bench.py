@@ -408,6 +408,32 @@ def run_ours(args, cfg):
         raise SystemExit(f"device error in timed region: {ml.status_string(st)}")
     active_experts = int((buf.counts > 0).sum().item())
 
+    # ---- rows beyond the step, timed on their own (not part of the step's value):
+    # the router backward (gradient into the logits), inputs from the last step
+    extras = {}
+    dlog = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device=dev)
+
+    def router_bwd():
+        ml.moe_router_backward(inp["dY"], buf.Y_sorted, buf.ids, buf.w, buf.pair_pos, cfg.E, dlog)
+
+    for _ in range(3):
+        router_bwd()
+    rb_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(min(args.steps, 50))]
+    for a, b in rb_evs:
+        flush.zero_()
+        a.record(stream)
+        router_bwd()
+        b.record(stream)
+    torch.cuda.synchronize()
+    rb_ms = statistics.mean(a.elapsed_time(b) for a, b in rb_evs)
+    P = cfg.T * cfg.k
+    rb_bytes = P * cfg.m * 2 + cfg.T * cfg.m * 2 + cfg.T * cfg.E * 4 + P * 12
+    extras["router_backward"] = {
+        "what": "dlogits [T, E] from dY and the expert outputs (NEXT-1 row; not part of the step)",
+        "ms_per_launch": rb_ms, "algorithmic_bytes": rb_bytes,
+        "achieved": rb_bytes / (rb_ms / 1e3) / 1e9, "unit": "GB/s"}
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -454,6 +480,9 @@ def run_ours(args, cfg):
 
     # ---- report
     peaks, peak_src = load_peaks()
+    for ex in extras.values():
+        ex["peak"] = peaks["hbm_gbs"]
+        ex["frac"] = ex["achieved"] / peaks["hbm_gbs"]
     flops = acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r)
     tflops = flops / (mean_ms / 1e3) / 1e12
     work = kernel_work(cfg, active_experts)
@@ -511,6 +540,7 @@ def run_ours(args, cfg):
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "extras": extras,
     }
     print(json.dumps(line), flush=True)
 

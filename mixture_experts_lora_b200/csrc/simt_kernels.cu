@@ -400,64 +400,64 @@ cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_
 // Beyond the path: the gradient into the router logits (for logits computed as
 // x W_r inside a model; router equation of "Accelerating Mixture-of-Experts
 // Fine-Tuning", section "The Dynamic Dispatch Bottleneck in Mixture-of-Experts
-// Architectures").  One warp per token:
-//   dw[j] = <dY[t], y_(t,j)>   (fp32 over 16-byte column pieces, y in sorted order)
-//   dlogits[t, ids[t,j]] = w[t,j] (dw[j] - sum_i w[t,i] dw[i]),  0 for the others.
+// Architectures").  A block of 8 warps owns TPB = max(1, 8 / k) whole tokens;
+// each warp takes pairs (t, j) of the block in turn:
+//   dw[t,j] = <dY[t], y_(t,j)>   (fp32 over 16-byte column pieces, y in sorted order;
+//                                  the block's warps share dY[t] through L1)
+// and one warp per token then writes the row
+//   dlogits[t, ids[t,j]] = w[t,j] (dw[t,j] - sum_i w[t,i] dw[t,i]),  0 for the others.
 __device__ __forceinline__ float warp_allsum(float v) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
 }
 
-__global__ void router_backward_kernel(const uint4* __restrict__ dY, const uint4* __restrict__ ys,
-                                       const int32_t* __restrict__ ids, const float* __restrict__ w,
-                                       const int32_t* __restrict__ pos, int64_t T, int k, int E,
-                                       int vpr, float* __restrict__ dlogits) {
+__global__ void __launch_bounds__(256)
+    router_backward_kernel(const uint4* __restrict__ dY, const uint4* __restrict__ ys,
+                           const int32_t* __restrict__ ids, const float* __restrict__ w,
+                           const int32_t* __restrict__ pos, int64_t T, int k, int E, int vpr,
+                           float* __restrict__ dlogits) {
+  __shared__ float s_dw[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-  if (t >= T) return;
-  const int my_pos = lane < k ? pos[t * k + lane] : 0;
-  int q[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) q[j] = __shfl_sync(0xffffffffu, my_pos, j);
-  float acc[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-  for (int v = lane; v < vpr; v += 32) {
-    const uint4 a = dY[t * vpr + v];
-    const float d0 = bf16_lo(a.x), d1 = bf16_hi(a.x), d2 = bf16_lo(a.y), d3 = bf16_hi(a.y);
-    const float d4 = bf16_lo(a.z), d5 = bf16_hi(a.z), d6 = bf16_lo(a.w), d7 = bf16_hi(a.w);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < k) {
-        const uint4 b = ys[(int64_t)q[j] * vpr + v];
-        acc[j] += d0 * bf16_lo(b.x) + d1 * bf16_hi(b.x) + d2 * bf16_lo(b.y) + d3 * bf16_hi(b.y) +
-                  d4 * bf16_lo(b.z) + d5 * bf16_hi(b.z) + d6 * bf16_lo(b.w) + d7 * bf16_hi(b.w);
-      }
+  const int tpb = k >= 8 ? 1 : 8 / k;                 // tokens per block
+  const int64_t t0 = (int64_t)blockIdx.x * tpb;
+  const int npairs = (int)((t0 + tpb <= T ? tpb : T - t0) * k);
+  for (int i = warp; i < npairs; i += 8) {
+    const int64_t t = t0 + i / k;
+    const int64_t q = pos[t0 * k + i];
+    const uint4* a = dY + t * vpr;
+    const uint4* b = ys + q * vpr;
+    float acc = 0.f;
+    for (int v = lane; v < vpr; v += 32) {
+      const uint4 x = a[v], y = b[v];
+      acc += bf16_lo(x.x) * bf16_lo(y.x) + bf16_hi(x.x) * bf16_hi(y.x) +
+             bf16_lo(x.y) * bf16_lo(y.y) + bf16_hi(x.y) * bf16_hi(y.y) +
+             bf16_lo(x.z) * bf16_lo(y.z) + bf16_hi(x.z) * bf16_hi(y.z) +
+             bf16_lo(x.w) * bf16_lo(y.w) + bf16_hi(x.w) * bf16_hi(y.w);
     }
+    acc = warp_allsum(acc);
+    if (lane == 0) s_dw[i] = acc;
   }
-  float my_dw = 0.f;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (j < k) {
-      const float s = warp_allsum(acc[j]);
-      if (lane == j) my_dw = s;
-    }
+  __syncthreads();
+  const int ntok = npairs / k;
+  if (warp < ntok) {
+    const int64_t t = t0 + warp;
+    const float my_dw = lane < k ? s_dw[warp * k + lane] : 0.f;
+    const float my_w = lane < k ? w[t * k + lane] : 0.f;
+    const float mean = warp_allsum(my_w * my_dw);
+    for (int e = lane; e < E; e += 32) dlogits[t * E + e] = 0.f;
+    __syncwarp();
+    if (lane < k) dlogits[t * E + ids[t * k + lane]] = my_w * (my_dw - mean);
   }
-  const float my_w = lane < k ? w[t * k + lane] : 0.f;
-  const float mean = warp_allsum(my_w * my_dw);
-  for (int e = lane; e < E; e += 32) dlogits[t * E + e] = 0.f;
-  __syncwarp();
-  if (lane < k) dlogits[t * E + ids[t * k + lane]] = my_w * (my_dw - mean);
 }
 
 cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const int32_t* ids,
                                    const float* w, const int32_t* pos, int64_t T, int k, int E,
                                    int m, float* dlogits, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
-  const int warps = 8;
+  const int tpb = k >= 8 ? 1 : 8 / k;
   ProfScope ps(K_ROUTER_BWD, s);
-  router_backward_kernel<<<(unsigned)((T + warps - 1) / warps), warps * 32, 0, s>>>(
+  router_backward_kernel<<<(unsigned)((T + tpb - 1) / tpb), 256, 0, s>>>(
       reinterpret_cast<const uint4*>(dY), reinterpret_cast<const uint4*>(ys), ids, w, pos, T, k, E,
       m / 8, dlogits);
   return cudaGetLastError();
