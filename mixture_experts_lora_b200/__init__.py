@@ -278,3 +278,15 @@ def layer_step(inp: dict, k: int, scale: float, buf: LayerBuffers, stream=None):
     layer_forward(inp, k, scale, buf, stream)
     layer_backward(inp, inp["dY"], k, scale, buf, stream)
     return buf
+
+
+def shared_expert_step(inp: dict, scale: float, buf: LayerBuffers, stream=None):
+    """Shared expert: a dense SwiGLU MLP with LoRA applied to every token, whose output
+    the caller adds to the routed experts' Y (and its dX to theirs).  It is this layer
+    with one expert, k = 1 and routing weight 1: `inp` holds X, dY and the six weight
+    tensors with a leading expert dimension of 1, plus logits [T, 1] (any values; the
+    softmax over one picked logit is 1).  Outputs land in buf.Y, buf.dX and the
+    adapter gradients like layer_step; `buf` comes from alloc_buffers(T, m, n, 1, 1, r, scale)."""
+    if inp["W_gu"].shape[0] != 1 or inp["logits"].shape[1] != 1:
+        raise ValueError("a shared expert has exactly one expert and logits of width 1")
+    return layer_step(inp, 1, scale, buf, stream)

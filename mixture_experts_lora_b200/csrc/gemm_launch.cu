@@ -71,13 +71,15 @@ bool encode3d(CUtensorMap* m, const void* base, uint64_t E, uint64_t rows, uint6
 
 // [E, R, C] row-major (C % 64 == 0) seen as [E][C/64 atoms][R][64]: a box of
 // `box_atoms` 64-wide atoms of `box_r` rows lands as atom-major 128-byte-swizzled
-// tiles, so one copy fills a whole operand tile.  E = 1 for a 2-D tensor.
-bool encode_atoms(CUtensorMap* m, const void* base, uint64_t E, uint64_t R, uint64_t C,
-                  uint32_t box_r, uint32_t box_atoms) {
+// tiles, so one copy fills a whole operand tile.  per_expert = false: a 2-D tensor
+// [R, C] (3-D view, E ignored); true: always the 4-D view, even for E = 1, since the
+// kernels address it with four coordinates.
+bool encode_atoms(CUtensorMap* m, const void* base, bool per_expert, uint64_t E, uint64_t R,
+                  uint64_t C, uint32_t box_r, uint32_t box_atoms) {
   const uint64_t dims[4] = {64, R, C / 64, E};
   const uint64_t str[3] = {C * 2, 128, R * C * 2};
   const uint32_t box[4] = {64, box_r, box_atoms, 1};
-  return encode(m, base, E > 1 ? 4 : 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode(m, base, per_expert ? 4 : 3, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 template <class Kern>
@@ -124,15 +126,15 @@ cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk,
   // atom views (one copy per operand and stage) when the K (and MN-major F) extents
   // are whole 64-wide atoms
   const bool v = K % 64 == 0 && (w_fk || F % 64 == 0);
-  bool ok = (v ? encode_atoms(&mp[1], act, 1, P, (uint64_t)K, C0::NHALF, C0::BK / 64)
+  bool ok = (v ? encode_atoms(&mp[1], act, false, 1, P, (uint64_t)K, C0::NHALF, C0::BK / 64)
                : encode2d(&mp[1], act, P, (uint64_t)K, C0::NHALF, C0::KA)) &&
             encode2d(&mp[3], lrc, P, rp, C0::BOXR, (uint32_t)rp);
   if (w_fk) {
-    ok = ok && (v ? encode_atoms(&mp[0], W, E, (uint64_t)F, (uint64_t)K, C0::BM, C0::BK / 64)
+    ok = ok && (v ? encode_atoms(&mp[0], W, true, E, (uint64_t)F, (uint64_t)K, C0::BM, C0::BK / 64)
                   : encode3d(&mp[0], W, E, (uint64_t)F, (uint64_t)K, 128, 64)) &&
          encode3d(&mp[2], lw, E, (uint64_t)F, rp, 128, (uint32_t)rp);
   } else {
-    ok = ok && (v ? encode_atoms(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 2)
+    ok = ok && (v ? encode_atoms(&mp[0], W, true, E, (uint64_t)K, (uint64_t)F, C0::BK, 2)
                   : encode3d(&mp[0], W, E, (uint64_t)K, (uint64_t)F, C0::BK, 64)) &&
          encode3d(&mp[2], lw, E, rp, (uint64_t)F, (uint32_t)rp, 64);
   }
