@@ -434,6 +434,32 @@ def run_ours(args, cfg):
         "ms_per_launch": rb_ms, "algorithmic_bytes": rb_bytes,
         "achieved": rb_bytes / (rb_ms / 1e3) / 1e9, "unit": "GB/s"}
 
+    # the shared expert (dense MLP + LoRA on every token, NEXT-4): the layer with one
+    # expert at the same token count and dimensions
+    from moe_inputs import LayerConfig
+    scfg = LayerConfig("shared_expert", T=cfg.T, m=cfg.m, n=cfg.n, E=1, k=1, r=cfg.r, alpha=cfg.alpha)
+    sinp = generate(scfg, seed=7, device=dev)
+    sbuf = ml.alloc_buffers(scfg.T, scfg.m, scfg.n, 1, 1, scfg.r, scfg.scale, device=dev)
+    for _ in range(3):
+        ml.shared_expert_step(sinp, scfg.scale, sbuf)
+    se_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(min(args.steps, 50))]
+    for a, b in se_evs:
+        flush.zero_()
+        a.record(stream)
+        ml.shared_expert_step(sinp, scfg.scale, sbuf)
+        b.record(stream)
+    torch.cuda.synchronize()
+    if ml.moe_get_device_error() != ml.MOE_OK:
+        raise SystemExit("device error in the shared-expert timing")
+    se_ms = statistics.mean(a.elapsed_time(b) for a, b in se_evs)
+    se_flops = acc.flops_step(scfg.T, scfg.m, scfg.n, 1, scfg.r)
+    extras["shared_expert"] = {
+        "what": f"dense SwiGLU MLP + LoRA on all {scfg.T} tokens, fwd+bwd (NEXT-4 row; not part of the step)",
+        "ms_per_step": se_ms, "tokens_per_s": scfg.T / (se_ms / 1e3),
+        "tflops": se_flops / (se_ms / 1e3) / 1e12}
+    del sinp, sbuf
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
@@ -481,8 +507,11 @@ def run_ours(args, cfg):
     # ---- report
     peaks, peak_src = load_peaks()
     for ex in extras.values():
-        ex["peak"] = peaks["hbm_gbs"]
-        ex["frac"] = ex["achieved"] / peaks["hbm_gbs"]
+        if "achieved" in ex:
+            ex["peak"] = peaks["hbm_gbs"]
+            ex["frac"] = ex["achieved"] / peaks["hbm_gbs"]
+        if "tflops" in ex:
+            ex["frac_bf16_sustained"] = ex["tflops"] / peaks["bf16_tflops_sustained"]
     flops = acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r)
     tflops = flops / (mean_ms / 1e3) / 1e12
     work = kernel_work(cfg, active_experts)
