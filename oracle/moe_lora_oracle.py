@@ -24,7 +24,8 @@ toward the lower expert index; stable (ascending pair index) order inside an
 expert segment; the router is frozen and its logits are an input.
 
 Beyond the path, router_backward gives the gradient into the router logits
-(for when the logits come from x W_r inside a model).
+(for when the logits come from x W_r inside a model), and layer_split_gate_up
+the layer with separate gate and up adapters.
 
 Pins (tests/test_oracle_pins.py): Split-LoRA equals the materialised
 X(W + c A B); B = 0 gives the base MoE exactly; k = E with equal logits gives
@@ -41,6 +42,7 @@ __all__ = [
     "expert_forward", "expert_forward_merged", "expert_backward",
     "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
     "token_forward", "token_backward_dx", "expert_lora_grads", "router_backward",
+    "layer_split_gate_up",
 ]
 
 
@@ -392,3 +394,71 @@ def router_backward(dY, yp, ids, w, pair_pos, E: int):
     dlogits = np.zeros((T, E))
     np.put_along_axis(dlogits, ids, w * (dw - s), axis=1)
     return dlogits, dw
+
+
+# --------------------------------------------------------------------------
+# Adapter variant: separate gate and up adapters ([MoE12x] "MoE LoRA changes
+# things": LoRA targets gate, up and down projections; the fused gate_up weight
+# then carries two adapters).  Per expert
+#     g = x W_g + c (x A_g) B_g,   u = x W_u + c (x A_u) B_u,   W_gu = [W_g | W_u],
+# the SwiGLU and the down projection as above.  Written out on its own (not via
+# the fused adapter) so that it pins the rank-2r block packing the library uses.
+# --------------------------------------------------------------------------
+def layer_split_gate_up(inp, k: int, c: float):
+    """Forward and backward of the layer with separate gate/up adapters.
+
+    inp holds X, logits, dY, W_gu, W_d, A_d, B_d and A_g, B_g, A_u, B_u
+    ([E, m, r], [E, r, n] each).  Returns (Y [T, m], grads: dX, dA_g, dB_g, dA_u,
+    dB_u, dA_d, dB_d).
+    """
+    X = to64(inp["X"])
+    dY = to64(inp["dY"])
+    T, m = X.shape
+    Wgu, Wd = to64(inp["W_gu"]), to64(inp["W_d"])
+    Ag, Bg, Au, Bu = (to64(inp[name]) for name in ("A_g", "B_g", "A_u", "B_u"))
+    Ad, Bd = to64(inp["A_d"]), to64(inp["B_d"])
+    E = Wgu.shape[0]
+    n = Wgu.shape[2] // 2
+    r = Ag.shape[2]
+    ids, w, counts, offsets, sorted_pairs, pair_pos = _route_and_permute(inp, k)
+    P = T * k
+    yp = np.zeros((P, m))
+    dxp = np.zeros((P, m))
+    gr = {"dA_g": np.zeros((E, m, r)), "dB_g": np.zeros((E, r, n)),
+          "dA_u": np.zeros((E, m, r)), "dB_u": np.zeros((E, r, n)),
+          "dA_d": np.zeros((E, n, r)), "dB_d": np.zeros((E, r, m))}
+    wflat = w.reshape(-1)
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        pairs = sorted_pairs[lo:hi]
+        x = X[pairs // k]
+        xg, xu = x @ Ag[e], x @ Au[e]
+        g = x @ Wgu[e][:, :n] + c * (xg @ Bg[e])
+        u = x @ Wgu[e][:, n:] + c * (xu @ Bu[e])
+        h = silu(g) * u
+        ha = h @ Ad[e]
+        yp[lo:hi] = h @ Wd[e] + c * (ha @ Bd[e])
+        dy = wflat[pairs][:, None] * dY[pairs // k]
+        t1 = dy @ Bd[e].T
+        dh = dy @ Wd[e].T + c * (t1 @ Ad[e].T)
+        gr["dA_d"][e] = c * (h.T @ t1)
+        gr["dB_d"][e] = c * (ha.T @ dy)
+        s = sigmoid(g)
+        dg = dh * u * s * (1.0 + g * (1.0 - s))
+        du = dh * g * s
+        tg, tu = dg @ Bg[e].T, du @ Bu[e].T
+        dxp[lo:hi] = dg @ Wgu[e][:, :n].T + du @ Wgu[e][:, n:].T + c * (tg @ Ag[e].T + tu @ Au[e].T)
+        gr["dA_g"][e] = c * (x.T @ tg)
+        gr["dB_g"][e] = c * (xg.T @ dg)
+        gr["dA_u"][e] = c * (x.T @ tu)
+        gr["dB_u"][e] = c * (xu.T @ du)
+    Y = np.zeros((T, m))
+    dX = np.zeros((T, m))
+    for j in range(k):
+        sel = pair_pos[np.arange(T) * k + j]
+        Y += w[:, j:j + 1] * yp[sel]
+        dX += dxp[sel]
+    gr["dX"] = dX
+    return Y, gr

@@ -385,3 +385,98 @@ def test_router_pin_catches_planted_mistake(monkeypatch):
         return out, dw
     monkeypatch.setattr(O, "router_backward", bad)
     assert check_router_fd() > 1e-3
+
+
+# ---------------------------------------------------------------- separate gate/up adapters
+def _split_inputs(cfg, seed=7, b_std=0.5):
+    inp = _inp64(cfg, seed=seed)
+    rng = np.random.default_rng(seed)
+    E, m, n, r = cfg.E, cfg.m, cfg.n, cfg.r
+    inp["A_g"] = rng.normal(0, 1 / math.sqrt(m), (E, m, r))
+    inp["A_u"] = rng.normal(0, 1 / math.sqrt(m), (E, m, r))
+    inp["B_g"] = rng.normal(0, b_std, (E, r, n))
+    inp["B_u"] = rng.normal(0, b_std, (E, r, n))
+    return inp
+
+
+def _packed(inp):
+    """Rank-2r fused adapter A = [A_g | A_u], B = [[B_g, 0], [0, B_u]]; the down
+    adapter is padded to rank 2r with zeros (one rank for both projections)."""
+    E, r, n = inp["B_g"].shape
+    A = np.concatenate([inp["A_g"], inp["A_u"]], axis=2)
+    B = np.zeros((E, 2 * r, 2 * n))
+    B[:, :r, :n] = inp["B_g"]
+    B[:, r:, n:] = inp["B_u"]
+    Ad = np.concatenate([inp["A_d"], np.zeros_like(inp["A_d"])], axis=2)
+    Bd = np.concatenate([inp["B_d"], np.zeros_like(inp["B_d"])], axis=1)
+    return A, B, Ad, Bd
+
+
+CFG_SPLIT = small_config(T=40, m=32, n=16, E=5, k=2, r=4, alpha=8.0)
+
+
+def test_split_gate_up_equals_block_packed_fused_adapter():
+    cfg = CFG_SPLIT
+    inp = _split_inputs(cfg)
+    Y, g = O.layer_split_gate_up(inp, cfg.k, cfg.scale)
+    packed = dict(inp)
+    packed["A_gu"], packed["B_gu"], packed["A_d"], packed["B_d"] = _packed(inp)
+    Yp, aux = O.moe_forward(packed, cfg.k, cfg.scale)
+    gp = O.moe_backward(packed, aux, packed["dY"], cfg.k, cfg.scale)
+    r, n = cfg.r, cfg.n
+    assert _rel(Y, Yp) < 1e-12
+    assert _rel(g["dX"], gp["dX"]) < 1e-12
+    assert _rel(g["dA_g"], gp["dA_gu"][:, :, :r]) < 1e-12
+    assert _rel(g["dA_u"], gp["dA_gu"][:, :, r:]) < 1e-12
+    assert _rel(g["dB_g"], gp["dB_gu"][:, :r, :n]) < 1e-12
+    assert _rel(g["dB_u"], gp["dB_gu"][:, r:, n:]) < 1e-12
+    assert _rel(g["dA_d"], gp["dA_d"][:, :, :r]) < 1e-12 and _rel(g["dB_d"], gp["dB_d"][:, :r]) < 1e-12
+    assert np.all(gp["dA_d"][:, :, r:] == 0) and np.all(gp["dB_d"][:, r:] == 0)   # padding stays zero
+
+
+def test_split_gate_up_zero_b_is_base_moe():
+    cfg = CFG_SPLIT
+    inp = _split_inputs(cfg)
+    inp["B_g"][:] = 0.0
+    inp["B_u"][:] = 0.0
+    inp["B_d"][:] = 0.0
+    Y, _ = O.layer_split_gate_up(inp, cfg.k, cfg.scale)
+    assert _rel(Y, O.moe_forward_base(inp, cfg.k)) < 1e-13
+
+
+def check_split_fd(h=1e-6, n_coords=24, seed=2):
+    cfg = CFG_SPLIT
+    inp = _split_inputs(cfg)
+    _, g = O.layer_split_gate_up(inp, cfg.k, cfg.scale)
+    dY = inp["dY"]
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for name, key in (("X", "dX"), ("A_g", "dA_g"), ("B_g", "dB_g"), ("A_u", "dA_u"), ("B_u", "dB_u")):
+        base = inp[name]
+        G = g[key]
+        scale = max(np.max(np.abs(G)), 1e-12)
+        for fi in rng.choice(base.size, size=n_coords, replace=False):
+            idx = np.unravel_index(fi, base.shape)
+            orig = base[idx]
+            base[idx] = orig + h
+            lp = float(np.sum(O.layer_split_gate_up(inp, cfg.k, cfg.scale)[0] * dY))
+            base[idx] = orig - h
+            lm = float(np.sum(O.layer_split_gate_up(inp, cfg.k, cfg.scale)[0] * dY))
+            base[idx] = orig
+            worst = max(worst, abs((lp - lm) / (2 * h) - G[idx]) / scale)
+    return worst
+
+
+def test_split_gate_up_gradients_match_finite_differences():
+    assert check_split_fd() < 1e-6
+
+
+def test_split_pin_catches_planted_mistake(monkeypatch):
+    good = O.layer_split_gate_up
+
+    def bad(inp, k, c):                     # gate adapter gradient scaled twice
+        Y, g = good(inp, k, c)
+        g["dA_g"] = g["dA_g"] * c
+        return Y, g
+    monkeypatch.setattr(O, "layer_split_gate_up", bad)
+    assert check_split_fd(n_coords=6) > 1e-3
