@@ -290,3 +290,43 @@ def shared_expert_step(inp: dict, scale: float, buf: LayerBuffers, stream=None):
     if inp["W_gu"].shape[0] != 1 or inp["logits"].shape[1] != 1:
         raise ValueError("a shared expert has exactly one expert and logits of width 1")
     return layer_step(inp, 1, scale, buf, stream)
+
+
+# ---------------------------------------------------------------- adapter variants
+class SplitGateUpAdapters:
+    """Separate gate and up adapters (rank r each) held in the library's fused layout.
+
+    gate_up carries one adapter of rank 2r with A_gu = [A_g | A_u] and
+    B_gu = [[B_g, 0], [0, B_u]]; the down adapter is zero-padded to the same rank
+    (the library uses one rank for both projections).  The result is exactly the
+    layer with separate adapters.  The attributes A_g, B_g, A_u, B_u, A_d, B_d are
+    views into the packed tensors: write them, or let an optimizer update them, in
+    place.  Nothing ever writes the off-diagonal blocks or the padding, so those
+    stay zero.  Pass A_gu, B_gu, A_d_packed and B_d_packed to the layer with rank 2r
+    and the scale of one adapter (alpha / r, or alpha / sqrt(r) for rsLoRA)."""
+
+    def __init__(self, E: int, m: int, n: int, r: int, device="cuda"):
+        if 2 * r > 32:
+            raise ValueError("separate gate/up adapters need 2r <= 32")
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.r, self.n = r, n
+        self.A_gu = torch.zeros(E, m, 2 * r, **bf)
+        self.B_gu = torch.zeros(E, 2 * r, 2 * n, **bf)
+        self.A_d_packed = torch.zeros(E, n, 2 * r, **bf)
+        self.B_d_packed = torch.zeros(E, 2 * r, m, **bf)
+        self.A_g, self.A_u = self.A_gu[:, :, :r], self.A_gu[:, :, r:]
+        self.B_g, self.B_u = self.B_gu[:, :r, :n], self.B_gu[:, r:, n:]
+        self.A_d, self.B_d = self.A_d_packed[:, :, :r], self.B_d_packed[:, :r, :]
+
+    def layer_inputs(self, inp: dict) -> dict:
+        """inp (X, logits, dY, W_gu, W_d) completed with the packed adapters."""
+        out = dict(inp)
+        out.update(A_gu=self.A_gu, B_gu=self.B_gu, A_d=self.A_d_packed, B_d=self.B_d_packed)
+        return out
+
+    def grads(self, buf: LayerBuffers) -> dict:
+        """Views of the separate adapters' gradients in a rank-2r LayerBuffers."""
+        r, n = self.r, self.n
+        return {"dA_g": buf.dA_gu[:, :, :r], "dA_u": buf.dA_gu[:, :, r:],
+                "dB_g": buf.dB_gu[:, :r, :n], "dB_u": buf.dB_gu[:, r:, n:],
+                "dA_d": buf.dA_d[:, :, :r], "dB_d": buf.dB_d[:, :r, :]}
