@@ -460,6 +460,39 @@ def run_ours(args, cfg):
         "tflops": se_flops / (se_ms / 1e3) / 1e12}
     del sinp, sbuf
 
+    # separate gate/up adapters of rank r (NEXT-2): the same workload run as the fused
+    # rank-2r adapter (skipped when 2r > 32)
+    if 2 * cfg.r <= 32:
+        ad = ml.SplitGateUpAdapters(cfg.E, cfg.m, cfg.n, cfg.r, device=dev)
+        gsp = torch.Generator(device=dev).manual_seed(5)
+        for name in ("A_g", "A_u"):
+            getattr(ad, name).copy_(torch.randn(getattr(ad, name).shape, generator=gsp, device=dev)
+                                    / cfg.m ** 0.5)
+        for name in ("B_g", "B_u"):
+            getattr(ad, name).copy_(torch.randn(getattr(ad, name).shape, generator=gsp, device=dev) * 0.02)
+        ad.A_d.copy_(inp["A_d"])
+        ad.B_d.copy_(inp["B_d"])
+        sp_inp = ad.layer_inputs(inp)
+        sp_buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, 2 * cfg.r, cfg.scale, device=dev)
+        for _ in range(3):
+            ml.layer_step(sp_inp, cfg.k, cfg.scale, sp_buf)
+        sp_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(min(args.steps, 50))]
+        for a, b in sp_evs:
+            flush.zero_()
+            a.record(stream)
+            ml.layer_step(sp_inp, cfg.k, cfg.scale, sp_buf)
+            b.record(stream)
+        torch.cuda.synchronize()
+        if ml.moe_get_device_error() != ml.MOE_OK:
+            raise SystemExit("device error in the separate-adapter timing")
+        sp_ms = statistics.mean(a.elapsed_time(b) for a, b in sp_evs)
+        extras["separate_gate_up_adapters"] = {
+            "what": f"the step with separate gate and up adapters of rank {cfg.r} (fused rank {2 * cfg.r}, "
+                    "host launches; NEXT-2 row)",
+            "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
+        del sp_buf, sp_inp, ad
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
