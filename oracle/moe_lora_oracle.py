@@ -15,6 +15,8 @@ Sources (web pages on the method):
              and French editions).
   [Cookbook] "Accelerating Mixture-of-Experts Fine-Tuning: Unsloth Faster MoE,
              Split LoRA, and Grouped GEMM" (ailinkdeeptech.com cookbook).
+  [Terra]    "GPT-5.6-Terraに触れてみたよ" (bluecore.net blog post on Unsloth's
+             training modes).
 
 Readings taken where the pages are silent or inconsistent (each is listed in
 the design notes): adapters A:[K,r], B:[r,N] with delta W = A B and scale
@@ -24,8 +26,9 @@ toward the lower expert index; stable (ascending pair index) order inside an
 expert segment; the router is frozen and its logits are an input.
 
 Beyond the path, router_backward gives the gradient into the router logits
-(for when the logits come from x W_r inside a model), and layer_split_gate_up
-the layer with separate gate and up adapters.
+(for when the logits come from x W_r inside a model), layer_split_gate_up
+the layer with separate gate and up adapters, and moe_weight_grads the
+gradients of the expert weights themselves (full fine-tuning).
 
 Pins (tests/test_oracle_pins.py): Split-LoRA equals the materialised
 X(W + c A B); B = 0 gives the base MoE exactly; k = E with equal logits gives
@@ -42,7 +45,7 @@ __all__ = [
     "expert_forward", "expert_forward_merged", "expert_backward",
     "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
     "token_forward", "token_backward_dx", "expert_lora_grads", "router_backward",
-    "layer_split_gate_up",
+    "layer_split_gate_up", "moe_weight_grads",
 ]
 
 
@@ -462,3 +465,35 @@ def layer_split_gate_up(inp, k: int, c: float):
         dX += dxp[sel]
     gr["dX"] = dX
     return Y, gr
+
+
+# --------------------------------------------------------------------------
+# Full fine-tuning: gradients of the expert weights themselves.  [Terra],
+# section "フルファインチューニングもできるが、別物として考える" (full fine-tuning
+# is possible but a different thing): it trains the base weights W0 instead of
+# freezing them as LoRA does; [MoE12x] opening list: the kernels serve full
+# fine-tuning as well as LoRA.  The loss sees W_gu only through x W_gu and W_d
+# only through h W_d, so for expert e over its rows (any number, zero included)
+#     dW_gu[e] = X_e^T dGU_e        [m, 2n]
+#     dW_d[e]  = H_e^T dy_e         [n, m],   dy = w * dY[t]
+# with dGU the SwiGLU-backward rows of moe_backward and H the forward's.
+def moe_weight_grads(inp, aux, bwd, dY, k: int):
+    """(dW_gu [E, m, 2n], dW_d [E, n, m]) from the forward's aux (keep=True) and
+    moe_backward's output; experts with no rows get zeros."""
+    X = to64(inp["X"])
+    dY = to64(dY)
+    E, m, n2 = inp["W_gu"].shape
+    n = n2 // 2
+    offsets, sorted_pairs = aux["offsets"], aux["sorted_pairs"]
+    wflat = aux["w"].reshape(-1)
+    dW_gu = np.zeros((E, m, n2))
+    dW_d = np.zeros((E, n, m))
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        pairs = sorted_pairs[lo:hi]
+        tok = pairs // k
+        dW_gu[e] = X[tok].T @ bwd["dgu"][lo:hi]
+        dW_d[e] = aux["h"][lo:hi].T @ (wflat[pairs][:, None] * dY[tok])
+    return dW_gu, dW_d

@@ -4,6 +4,8 @@
 - B = 0 reduces exactly to the base MoE with no adapters
 - k = E with equal logits is the plain average of all experts
 - gradients match central finite differences and torch.autograd (fp64)
+- full fine-tuning: the expert-weight gradients match finite differences and
+  autograd, and chain to the adapter gradients through W' = W + c A B
 - routing and permutation match brute force, ties included
 - a single expert with k = 1 and no adapters is the textbook SwiGLU MLP
 - the accounting helpers match the worked numbers the pages print
@@ -132,7 +134,10 @@ def test_gradients_match_torch_autograd():
     Y, aux = O.moe_forward(inp, cfg.k, cfg.scale)
     g = O.moe_backward(inp, aux, inp["dY"], cfg.k, cfg.scale)
 
-    T = {k: torch.tensor(v, dtype=torch.float64, requires_grad=k in ("X", "A_gu", "B_gu", "A_d", "B_d"))
+    dW_gu, dW_d = O.moe_weight_grads(inp, aux, g, inp["dY"], cfg.k)
+    g["dW_gu"], g["dW_d"] = dW_gu, dW_d
+    T = {k: torch.tensor(v, dtype=torch.float64,
+                         requires_grad=k in ("X", "A_gu", "B_gu", "A_d", "B_d", "W_gu", "W_d"))
          for k, v in inp.items() if k != "logits"}
     # routing written differently from the oracle: softmax over all experts, then
     # torch.topk, then renormalise (no ties at these random logits)
@@ -154,7 +159,8 @@ def test_gradients_match_torch_autograd():
     Yt = torch.stack(rows)
     assert _rel(Y, Yt.detach().numpy()) < 1e-12
     (Yt * T["dY"]).sum().backward()
-    for name, key in (("X", "dX"), ("A_gu", "dA_gu"), ("B_gu", "dB_gu"), ("A_d", "dA_d"), ("B_d", "dB_d")):
+    for name, key in (("X", "dX"), ("A_gu", "dA_gu"), ("B_gu", "dB_gu"), ("A_d", "dA_d"), ("B_d", "dB_d"),
+                      ("W_gu", "dW_gu"), ("W_d", "dW_d")):
         assert _rel(g[key], T[name].grad.numpy()) < 1e-11, name
 
 
@@ -221,10 +227,12 @@ def test_empty_experts_have_zero_grads():
     inp["logits"][:, 1] = 5.0           # every token picks expert 1
     Y, aux = O.moe_forward(inp, cfg.k, cfg.scale)
     g = O.moe_backward(inp, aux, inp["dY"], cfg.k, cfg.scale)
+    g["dW_gu"], g["dW_d"] = O.moe_weight_grads(inp, aux, g, inp["dY"], cfg.k)
     assert aux["counts"][1] == cfg.T
     for e in (0, 2, 3, 4, 5):
-        for key in ("dA_gu", "dB_gu", "dA_d", "dB_d"):
+        for key in ("dA_gu", "dB_gu", "dA_d", "dB_d", "dW_gu", "dW_d"):
             assert not np.any(g[key][e])
+    assert np.any(g["dW_gu"][1]) and np.any(g["dW_d"][1])
 
 
 def test_sampled_helpers_agree_with_full_layer():
@@ -264,6 +272,75 @@ def test_flop_formula_matches_qwen_figure():
     parts = (acc.flops_gemm_gate_up_fwd, acc.flops_gemm_down_fwd, acc.flops_gemm_down_bwd,
              acc.flops_gemm_gate_up_bwd, acc.flops_lora_wgrad)
     assert sum(f(c.T, c.m, c.n, c.k, c.r) for f in parts) == total
+
+
+# ---------------------------------------------------------------- full fine-tuning
+CFG_W = small_config(T=24, m=32, n=16, E=4, k=2, r=4, alpha=8.0)
+
+
+def _weight_case(cfg=CFG_W):
+    inp = _inp64(cfg)
+    Y, aux = O.moe_forward(inp, cfg.k, cfg.scale)
+    g = O.moe_backward(inp, aux, inp["dY"], cfg.k, cfg.scale)
+    dW_gu, dW_d = O.moe_weight_grads(inp, aux, g, inp["dY"], cfg.k)
+    return inp, g, dW_gu, dW_d
+
+
+def check_weight_fd(n_coords=40, seed=4, h=1e-6):
+    """Max relative error of dW_gu, dW_d against central differences of <dY, Y>."""
+    cfg = CFG_W
+    inp, _, dW_gu, dW_d = _weight_case(cfg)
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for name, G in (("W_gu", dW_gu), ("W_d", dW_d)):
+        base = inp[name]
+        scale = max(np.max(np.abs(G)), 1e-12)
+        for fi in rng.choice(base.size, size=n_coords, replace=False):
+            idx = np.unravel_index(fi, base.shape)
+            orig = base[idx]
+            base[idx] = orig + h
+            lp = _loss(inp, inp["dY"], cfg)
+            base[idx] = orig - h
+            lm = _loss(inp, inp["dY"], cfg)
+            base[idx] = orig
+            worst = max(worst, abs((lp - lm) / (2 * h) - G[idx]) / scale)
+    return worst
+
+
+def test_weight_grads_match_finite_differences():
+    assert check_weight_fd() < 1e-6
+
+
+def test_weight_grads_chain_to_adapter_grads():
+    # the layer sees W and the adapters only through W' = W + c A B, so
+    # dL/dA = c dL/dW' B^T and dL/dB = c A^T dL/dW' (the adapter gradients are
+    # pinned on their own by finite differences and autograd)
+    cfg = CFG_S
+    inp, g, dW_gu, dW_d = _weight_case(cfg)
+    c = cfg.scale
+    for e in range(cfg.E):
+        assert _rel(c * dW_gu[e] @ inp["B_gu"][e].T, g["dA_gu"][e]) < 1e-12
+        assert _rel(c * inp["A_gu"][e].T @ dW_gu[e], g["dB_gu"][e]) < 1e-12
+        assert _rel(c * dW_d[e] @ inp["B_d"][e].T, g["dA_d"][e]) < 1e-12
+        assert _rel(c * inp["A_d"][e].T @ dW_d[e], g["dB_d"][e]) < 1e-12
+
+
+def test_weight_pin_catches_planted_mistakes(monkeypatch):
+    good = O.moe_weight_grads
+
+    def unweighted(inp, aux, bwd, dY, k):       # dW_d from dY without the routing weight
+        a = dict(aux)
+        a["w"] = np.ones_like(aux["w"])
+        return good(inp, a, bwd, dY, k)
+    monkeypatch.setattr(O, "moe_weight_grads", unweighted)
+    assert check_weight_fd(n_coords=8) > 1e-3
+
+    def scaled(inp, aux, bwd, dY, k):           # the LoRA scale applied to dW_gu
+        gu, d = good(inp, aux, bwd, dY, k)
+        return CFG_W.scale * gu, d
+    monkeypatch.setattr(O, "moe_weight_grads", scaled)
+    assert check_weight_fd(n_coords=8) > 1e-3
+    monkeypatch.setattr(O, "moe_weight_grads", good)
 
 
 # ---------------------------------------------------------------- planted mistakes
