@@ -157,6 +157,10 @@ def kernel_work(cfg, active_experts=None):
         "rows_swiglu_bwd": {"byte": P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + lr_out},
         "gather_rows": {"byte": acc.bytes_gather(T, m, k)},       # X again for dA_gu
         "unpermute_combine": {"byte": 2 * acc.bytes_combine(T, m, k)},  # Y and dX
+        # full fine-tuning only: expert-weight gradients (sorted operands read once,
+        # every expert's gradient written once)
+        "gemm_dw_gu": {"flop": 4 * P * m * n, "byte": P * m * 2 + P * 2 * n * 2 + E * m * 2 * n * 2},
+        "gemm_dw_d": {"flop": 2 * P * n * m, "byte": P * n * 2 + P * m * 2 + E * n * m * 2},
     }
 
 
@@ -492,6 +496,53 @@ def run_ours(args, cfg):
                     "host launches; NEXT-2 row)",
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
+
+    # full fine-tuning (NEXT-3): forward, then the backward with the expert-weight
+    # gradients dW_gu, dW_d and no adapter gradients
+    dWg = torch.empty(cfg.E, cfg.m, 2 * cfg.n, dtype=torch.bfloat16, device=dev)
+    dWd = torch.empty(cfg.E, cfg.n, cfg.m, dtype=torch.bfloat16, device=dev)
+
+    def fft_step():
+        ml.layer_forward(inp, cfg.k, cfg.scale, buf)
+        ml.layer_backward_full(inp, inp["dY"], cfg.k, cfg.scale, buf, dWg, dWd, adapters=False)
+
+    for _ in range(3):
+        fft_step()
+    ft_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(min(args.steps, 50))]
+    for a, b in ft_evs:
+        flush.zero_()
+        a.record(stream)
+        fft_step()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ft_ms = statistics.mean(a.elapsed_time(b) for a, b in ft_evs)
+    # the two weight-gradient kernels, timed on their own launches in a few more steps
+    ml.moe_profile_select(["gemm_dw_gu", "gemm_dw_d"])
+    ml.moe_profile_enable(True)
+    for _ in range(10):
+        flush.zero_()
+        fft_step()
+    ml.moe_profile_enable(False)
+    ft_prof = ml.moe_profile_read()
+    ml.moe_profile_select(None)
+    if ml.moe_get_device_error() != ml.MOE_OK:
+        raise SystemExit("device error in the full fine-tuning timing")
+    ft_flops = (acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r)
+                - acc.flops_lora_wgrad(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r) + 6 * P * cfg.m * cfg.n)
+    ft_kern = {}
+    ft_work, (ft_peaks, _) = kernel_work(cfg, active_experts), load_peaks()
+    for name in ("gemm_dw_gu", "gemm_dw_d"):
+        if name in ft_prof and ft_prof[name][0] > 0:
+            launches, tot = ft_prof[name]
+            ft_kern[name] = {"ms_per_launch": tot / launches,
+                             **roof_entry(ft_work[name], tot / launches, 1, ft_peaks)}
+    extras["full_fine_tuning"] = {
+        "what": "forward + backward with the expert-weight gradients dW_gu, dW_d (no adapter "
+                "gradients; NEXT-3 row; not part of the step)",
+        "ms_per_step": ft_ms, "tokens_per_s": world * cfg.T / (ft_ms / 1e3),
+        "tflops": ft_flops / (ft_ms / 1e3) / 1e12, "kernels": ft_kern}
+    del dWg, dWd
 
     # ---- end to end through the public API with host buffers
     e2e = None

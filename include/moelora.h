@@ -160,6 +160,30 @@ moe_status_t moe_grouped_gemm_lora_bwd(
     moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream);
 
+/* Backward for full fine-tuning: everything moe_grouped_gemm_lora_bwd() computes,
+ * plus the gradients of the expert weights themselves ("GPT-5.6-Terraに触れてみたよ",
+ * section on full fine-tuning: the base weights W0 are trained instead of frozen;
+ * "Fine-tune MoE models 12x faster with Unsloth", opening list: the kernels serve
+ * full fine-tuning as well as LoRA):
+ *   dW_gu[e] = X_e^T dGU_e     bf16 [E, m, 2n]
+ *   dW_d[e]  = H_e^T dy_e      bf16 [E, n, m]
+ * summed in fp32 over the rows of expert e (a contraction of P_e rows, P_e >= 0;
+ * experts with no rows get zeros), rounded once.  dW_gu and dW_d are required.
+ * dA_gu, dB_gu, dA_d, dB_d: all four given (computed as in the LoRA backward) or
+ * all four NULL (adapter gradients skipped; pass B_gu = B_d = 0 for a layer
+ * without adapters, whose rank-r terms then add exact zeros).  Other arguments,
+ * outputs and errors as moe_grouped_gemm_lora_bwd(); each weight-gradient tile
+ * sums its rows in one fixed order (deterministic). */
+moe_status_t moe_grouped_gemm_full_bwd(
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_bf16_t* X, const int32_t* sorted_pairs, const int32_t* offsets,
+    const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
+    const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
+    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
+    const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dW_gu,
+    moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
+    moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream);
+
 /* The same permutation as moe_permute(), for callers that cannot allocate device
  * memory: plug-ins hosted inside another framework that owns all device memory
  * and hands them no allocator, or code that must run with a fixed device-memory

@@ -31,7 +31,7 @@ EXPORTED = (
     "moe_workspace_bytes", "moe_route_topk", "moe_permute", "moe_grouped_gemm_lora_fwd",
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
     "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
-    "moe_permute_noalloc", "moe_router_backward",
+    "moe_permute_noalloc", "moe_router_backward", "moe_grouped_gemm_full_bwd",
 )
 
 
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
         h.moe_permute_noalloc.argtypes = [P, I64, I32, I32, P, P, P, P, P]
         h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 15 + [SZ, P]
         h.moe_grouped_gemm_lora_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
+        h.moe_grouped_gemm_full_bwd.argtypes = [D] + [P] * 23 + [SZ, P]
         h.moe_unpermute_combine.argtypes = [P, P, P, I64, I32, I32, P, P]
         h.moe_router_backward.argtypes = [P, P, P, P, P, I64, I32, I32, I32, P, P]
         h.moe_get_device_error.argtypes = [P]
@@ -149,6 +150,20 @@ def moe_grouped_gemm_lora_bwd(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, 
     args = [dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU,
             save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, ws]
     _check("moe_grouped_gemm_lora_bwd", lib().moe_grouped_gemm_lora_bwd(
+        ctypes.byref(dims), *[_ptr(a) for a in args], ws.numel() * ws.element_size(),
+        _stream(stream)))
+
+
+def moe_grouped_gemm_full_bwd(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu,
+                              A_d, B_d, save_GU, save_H, save_XA, save_HA, dX_sorted, dW_gu, dW_d,
+                              dA_gu=None, dB_gu=None, dA_d=None, dB_d=None, ws=None, stream=None):
+    """Backward with the expert-weight gradients dW_gu [E, m, 2n] and dW_d [E, n, m]
+    (full fine-tuning); the adapter gradients are computed when all four are given."""
+    if ws is None:
+        raise ValueError("moe_grouped_gemm_full_bwd needs the workspace")
+    args = [dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU,
+            save_H, save_XA, save_HA, dX_sorted, dW_gu, dW_d, dA_gu, dB_gu, dA_d, dB_d, ws]
+    _check("moe_grouped_gemm_full_bwd", lib().moe_grouped_gemm_full_bwd(
         ctypes.byref(dims), *[_ptr(a) for a in args], ws.numel() * ws.element_size(),
         _stream(stream)))
 
@@ -269,6 +284,23 @@ def layer_backward(inp: dict, dY, k: int, scale: float, buf: LayerBuffers, strea
                               inp["B_d"], buf.save_GU, buf.save_H, buf.save_XA, buf.save_HA,
                               buf.dX_sorted, buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d, buf.ws,
                               stream)
+    moe_unpermute_combine(buf.dX_sorted, None, buf.pair_pos, T, k, m, buf.dX, stream)
+    return buf.dX
+
+
+def layer_backward_full(inp: dict, dY, k: int, scale: float, buf: LayerBuffers, dW_gu, dW_d,
+                        adapters: bool = True, stream=None):
+    """layer_backward plus the expert-weight gradients (full fine-tuning) into dW_gu
+    [E, m, 2n] and dW_d [E, n, m]; adapters=False skips the adapter gradients."""
+    T, m = inp["X"].shape
+    E, _, n2 = inp["W_gu"].shape
+    r = inp["A_gu"].shape[2]
+    dims = make_dims(T, m, n2 // 2, E, k, r, scale)
+    lora = (buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d) if adapters else (None,) * 4
+    moe_grouped_gemm_full_bwd(dims, dY, buf.w, inp["X"], buf.sorted_pairs, buf.offsets,
+                              inp["W_gu"], inp["W_d"], inp["A_gu"], inp["B_gu"], inp["A_d"],
+                              inp["B_d"], buf.save_GU, buf.save_H, buf.save_XA, buf.save_HA,
+                              buf.dX_sorted, dW_gu, dW_d, *lora, ws=buf.ws, stream=stream)
     moe_unpermute_combine(buf.dX_sorted, None, buf.pair_pos, T, k, m, buf.dX, stream)
     return buf.dX
 

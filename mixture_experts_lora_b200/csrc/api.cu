@@ -185,6 +185,100 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
   return MOE_OK;
 }
 
+// The backward pass.  Adapter gradients when dA_gu.. are given (all four or none),
+// expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given; each weight
+// gradient runs while its sorted operands are in the row buffer (dy after the
+// down backward, X after its re-gather).
+moe_status_t backward(
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
+    const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
+    moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, moe_bf16_t* dW_gu,
+    moe_bf16_t* dW_d, void* ws, size_t ws_bytes, void* stream) {
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t d = *dims;
+  const bool lora = dA_gu != nullptr, full = dW_gu != nullptr;
+  const void* outs[] = {dA_gu, dB_gu, dA_d, dB_d, dW_gu, dW_d};
+  for (const void* p : outs)
+    if (p != nullptr && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t E = d.E, m = d.m, n = d.n, r = d.r;
+  if (d.T == 0) {
+    if (lora) {
+      MOE_TRY(launch_zero(dA_gu, E * m * r * 2, s));
+      MOE_TRY(launch_zero(dB_gu, E * r * 2 * n * 2, s));
+      MOE_TRY(launch_zero(dA_d, E * n * r * 2, s));
+      MOE_TRY(launch_zero(dB_d, E * r * m * 2, s));
+    }
+    if (full) {
+      MOE_TRY(launch_zero(dW_gu, E * m * 2 * n * 2, s));
+      MOE_TRY(launch_zero(dW_d, E * n * m * 2, s));
+    }
+    return MOE_OK;
+  }
+  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA, save_HA,
+                       dX_sorted, ws};
+  for (const void* p : ins)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (topk_w == nullptr || sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(d);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  GemmShape g;
+  LayerPtrs w;
+  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, s, &g, &w);
+  if (st != MOE_OK) return st;
+  uint16_t* rows = at<uint16_t>(ws, L.rows);
+  uint16_t* dgu = at<uint16_t>(ws, L.dgu);
+  uint16_t* t1 = at<uint16_t>(ws, L.t1);
+  uint16_t* t2 = at<uint16_t>(ws, L.t2);
+  float* partial = at<float>(ws, L.partial);
+  const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
+  const int* n_chunks = at<int>(ws, L.n_chunks);
+  const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
+  uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
+  uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
+  uint16_t* dh = at<uint16_t>(ws, L.dh);
+  float* rpart = at<float>(ws, L.rows_partial);
+  int* rcnt = at<int>(ws, L.counters) + 2 * L.max_row_tiles;   // row-kernel sets 2 and 3
+  // dy = w * dY[t] in expert order, T1 = dy B_d^T (kept for dA_d) and bf16(c T1)
+  MOE_TRY(launch_rows_lowrank(g, 0, d.m, dY, sorted_pairs, topk_w, d.k, nullptr, nullptr, w.B_d,
+                              false, rows, t1, L.rp, L.rp, lrc1, rpart, rcnt, s));
+  // dH = dy W_d^T + (c T1) A_d^T
+  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
+  // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
+  float* partial2 = at<float>(ws, L.partial2);
+  int* counters = at<int>(ws, L.counters) + 4 * L.max_row_tiles;   // gradient sets
+  const size_t cstride = (size_t)d.E * L.max_dtiles;
+  if (lora) {
+    const WgradJob jobs[2] = {
+        {save_H, d.n, t1, L.rp, false, dA_d, partial, counters},
+        {rows, d.m, save_HA, d.r, true, dB_d, partial2, counters + cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+  }
+  // dW_d = H^T dy per expert
+  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_D, g, offsets, save_H, d.n, rows, d.m, dW_d, s));
+  // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
+  MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
+                              false, dgu, t2, L.rp, L.rp, lrc2, rpart, rcnt + L.max_row_tiles, s));
+  // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
+  MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
+  // X re-gathered into the row buffer (dy is no longer needed), then
+  // dB_gu = c XA^T dGU and dA_gu = c X^T T2, one launch
+  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
+  if (lora) {
+    const WgradJob jobs[2] = {
+        {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
+        {rows, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+  }
+  // dW_gu = X^T dGU per expert
+  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, rows, d.m, dgu, 2 * d.n, dW_gu, s));
+  return MOE_OK;
+}
+
 }  // namespace
 
 int* moe_status_word() { return status_ptr(); }
@@ -305,75 +399,27 @@ moe_status_t moe_grouped_gemm_lora_bwd(
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream) {
-  moe_status_t st = check_dims(dims);
-  if (st != MOE_OK) return st;
-  const moe_dims_t d = *dims;
-  const void* outs[] = {dA_gu, dB_gu, dA_d, dB_d};
-  for (const void* p : outs)
-    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t E = d.E, m = d.m, n = d.n, r = d.r;
-  if (d.T == 0) {
-    MOE_TRY(launch_zero(dA_gu, E * m * r * 2, s));
-    MOE_TRY(launch_zero(dB_gu, E * r * 2 * n * 2, s));
-    MOE_TRY(launch_zero(dA_d, E * n * r * 2, s));
-    MOE_TRY(launch_zero(dB_d, E * r * m * 2, s));
-    return MOE_OK;
-  }
-  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA, save_HA,
-                       dX_sorted, ws};
-  for (const void* p : ins)
-    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (topk_w == nullptr || sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
-  const Layout L = make_layout(d);
-  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  GemmShape g;
-  LayerPtrs w;
-  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, s, &g, &w);
-  if (st != MOE_OK) return st;
-  uint16_t* rows = at<uint16_t>(ws, L.rows);
-  uint16_t* dgu = at<uint16_t>(ws, L.dgu);
-  uint16_t* t1 = at<uint16_t>(ws, L.t1);
-  uint16_t* t2 = at<uint16_t>(ws, L.t2);
-  float* partial = at<float>(ws, L.partial);
-  const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
-  const int* n_chunks = at<int>(ws, L.n_chunks);
-  const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
-  uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
-  uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
-  uint16_t* dh = at<uint16_t>(ws, L.dh);
-  float* rpart = at<float>(ws, L.rows_partial);
-  int* rcnt = at<int>(ws, L.counters) + 2 * L.max_row_tiles;   // row-kernel sets 2 and 3
-  // dy = w * dY[t] in expert order, T1 = dy B_d^T (kept for dA_d) and bf16(c T1)
-  MOE_TRY(launch_rows_lowrank(g, 0, d.m, dY, sorted_pairs, topk_w, d.k, nullptr, nullptr, w.B_d,
-                              false, rows, t1, L.rp, L.rp, lrc1, rpart, rcnt, s));
-  // dH = dy W_d^T + (c T1) A_d^T
-  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
-  // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
-  float* partial2 = at<float>(ws, L.partial2);
-  int* counters = at<int>(ws, L.counters) + 4 * L.max_row_tiles;   // gradient sets
-  const size_t cstride = (size_t)d.E * L.max_dtiles;
-  {
-    const WgradJob jobs[2] = {
-        {save_H, d.n, t1, L.rp, false, dA_d, partial, counters},
-        {rows, d.m, save_HA, d.r, true, dB_d, partial2, counters + cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
-  }
-  // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
-  MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
-                              false, dgu, t2, L.rp, L.rp, lrc2, rpart, rcnt + L.max_row_tiles, s));
-  // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
-  MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
-  // X re-gathered into the row buffer (dy is no longer needed), then
-  // dB_gu = c XA^T dGU and dA_gu = c X^T T2, one launch
-  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
-  {
-    const WgradJob jobs[2] = {
-        {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
-        {rows, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
-  }
-  return MOE_OK;
+  if (dA_gu == nullptr || dB_gu == nullptr || dA_d == nullptr || dB_d == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
+                  nullptr, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_grouped_gemm_full_bwd(
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
+    const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
+    moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
+    moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream) {
+  if (dW_gu == nullptr || dW_d == nullptr) return MOE_ERR_INVALID_ARG;
+  const int given = (dA_gu != nullptr) + (dB_gu != nullptr) + (dA_d != nullptr) + (dB_d != nullptr);
+  if (given != 0 && given != 4) return MOE_ERR_INVALID_ARG;
+  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
+                  dW_d, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_router_backward(const moe_bf16_t* dY, const moe_bf16_t* Y_sorted,

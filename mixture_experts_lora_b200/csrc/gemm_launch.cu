@@ -4,6 +4,7 @@
 
 #include <mutex>
 
+#include "expert_dw.cuh"
 #include "grouped_gemm.cuh"
 #include "internal.h"
 #include "lora_wgrad.cuh"
@@ -318,6 +319,43 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
   wp.err = g.err;
   if (g.rp == 16) return wgrad_rp<16>(g, tm, wp, max_chunks, s);
   return wgrad_rp<32>(g, tm, wp, max_chunks, s);
+}
+
+template <class C>
+static cudaError_t expert_dw_launch(int kind, const CUtensorMap* tm, const DwParams& p, int num_sms,
+                                    cudaStream_t s) {
+  auto kern = moe_dw_kernel<C>;
+  cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
+  if (st != cudaSuccess) return st;
+  const int64_t total = (int64_t)p.E * p.n_mt * p.n_nt;
+  const int grid = (int)(total < num_sms ? total : num_sms);
+  ProfScope ps(kind, s);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tm[0], tm[1], p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_expert_dw(int kind, const GemmShape& g, const int32_t* offsets, const uint16_t* Lm,
+                             int Mdim, const uint16_t* Rm, int Ndim, uint16_t* out, cudaStream_t s) {
+  using C = DwCfg<true>;
+  CUtensorMap tm[2];
+  const uint64_t P = (uint64_t)g.P;
+  const bool v = Mdim % 64 == 0 && Ndim % 64 == 0;
+  const bool ok = v ? encode_atoms(&tm[0], Lm, false, 1, P, (uint64_t)Mdim, C::BK, 2) &&
+                          encode_atoms(&tm[1], Rm, false, 1, P, (uint64_t)Ndim, C::BK, 4)
+                    : encode2d(&tm[0], Lm, P, (uint64_t)Mdim, C::BK, 64) &&
+                          encode2d(&tm[1], Rm, P, (uint64_t)Ndim, C::BK, 64);
+  if (!ok) return cudaErrorInvalidValue;
+  DwParams p{};
+  p.offsets = offsets;
+  p.E = g.E;
+  p.Mdim = Mdim;
+  p.Ndim = Ndim;
+  p.n_mt = (Mdim + C::BM - 1) / C::BM;
+  p.n_nt = (Ndim + C::BN - 1) / C::BN;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.err = g.err;
+  return v ? expert_dw_launch<DwCfg<true>>(kind, tm, p, g.num_sms, s)
+           : expert_dw_launch<DwCfg<false>>(kind, tm, p, g.num_sms, s);
 }
 
 }  // namespace moe

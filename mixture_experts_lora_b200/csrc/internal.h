@@ -17,7 +17,7 @@ enum KernelKind : int {
   K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
   K_COMBINE, K_MEMSET, K_ROWS_GATHER, K_ROWS_SWIGLU,
-  K_ROWS_SWIGLU_BWD, K_ROUTER_BWD, K_NUM_KINDS
+  K_ROWS_SWIGLU_BWD, K_ROUTER_BWD, K_GEMM_DW_GU, K_GEMM_DW_D, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
 bool prof_enabled();
@@ -133,5 +133,10 @@ struct WgradJob {
 cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jobs,
                               const TileInfo* chunks, const int* n_chunks, int max_chunks,
                               const int32_t* chunk_start, cudaStream_t s);
+
+// Expert-weight gradients (expert_dw.cuh): out[e] = Lm_e^T Rm_e over the rows of expert
+// e (offsets), Lm [P, Mdim], Rm [P, Ndim] sorted rows, out [E, Mdim, Ndim] bf16.
+cudaError_t launch_expert_dw(int kind, const GemmShape& g, const int32_t* offsets, const uint16_t* Lm,
+                             int Mdim, const uint16_t* Rm, int Ndim, uint16_t* out, cudaStream_t s);
 
 }  // namespace moe

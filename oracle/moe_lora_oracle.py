@@ -45,7 +45,7 @@ __all__ = [
     "expert_forward", "expert_forward_merged", "expert_backward",
     "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
     "token_forward", "token_backward_dx", "expert_lora_grads", "router_backward",
-    "layer_split_gate_up", "moe_weight_grads",
+    "layer_split_gate_up", "moe_weight_grads", "expert_weight_grads",
 ]
 
 
@@ -497,3 +497,22 @@ def moe_weight_grads(inp, aux, bwd, dY, k: int):
         dW_gu[e] = X[tok].T @ bwd["dgu"][lo:hi]
         dW_d[e] = aux["h"][lo:hi].T @ (wflat[pairs][:, None] * dY[tok])
     return dW_gu, dW_d
+
+
+def expert_weight_grads(inp, e: int, k: int, c: float, ids=None, w=None, W=None):
+    """(dW_gu[e], dW_d[e]) of expert e alone, from its rows' forward and backward."""
+    W = W if W is not None else _weights64(inp)
+    if ids is None:
+        ids, w = route_topk(to64(inp["logits"]).astype(np.float32), k)
+    pairs = np.nonzero(ids.reshape(-1) == e)[0]            # ascending pair index
+    m = W["W_gu"].shape[1]
+    n = W["W_gu"].shape[2] // 2
+    if pairs.size == 0:
+        return np.zeros((m, 2 * n)), np.zeros((n, m))
+    tok = pairs // k
+    x = to64(inp["X"][tok])
+    dy = w.reshape(-1)[pairs][:, None] * to64(inp["dY"][tok])
+    args = (W["W_gu"][e], W["A_gu"][e], W["B_gu"][e], W["W_d"][e], W["A_d"][e], W["B_d"][e], c)
+    f = expert_forward(x, *args)
+    b = expert_backward(x, f, dy, *args)
+    return x.T @ b["dgu"], f["h"].T @ dy

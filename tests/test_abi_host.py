@@ -110,6 +110,33 @@ def test_host_validation_returns_before_launch(L):
     assert L.moe_unpermute_combine(fake, null, fake, 0, 2, 16, fake, null) == ml.MOE_OK
 
 
+def test_full_backward_host_validation(L):
+    P = ctypes.c_void_p
+    d = dims()
+    ptrs = [P(4096)] * 23         # ... dX_sorted, dW_gu (16), dW_d (17), dA_gu .. dB_d (18-21), ws
+
+    def call(p, ws_bytes=1 << 30):
+        return L.moe_grouped_gemm_full_bwd(ctypes.byref(d), *p, ws_bytes, None)
+    bad = list(ptrs)
+    bad[16] = None                # the expert-weight gradients are required
+    assert call(bad) == ml.MOE_ERR_INVALID_ARG
+    bad = list(ptrs)
+    bad[19] = None                # adapter gradients: all four or none
+    assert call(bad) == ml.MOE_ERR_INVALID_ARG
+    bad = list(ptrs)
+    bad[17] = P(4100)             # misaligned dW_d
+    assert call(bad) == ml.MOE_ERR_INVALID_ARG
+    assert call(ptrs, 16) == ml.MOE_ERR_WORKSPACE
+    no_adapters = list(ptrs)
+    no_adapters[18:22] = [None] * 4
+    assert call(no_adapters, 16) == ml.MOE_ERR_WORKSPACE
+    assert L.moe_grouped_gemm_full_bwd(ctypes.byref(dims(m=100)), *ptrs, 1 << 30, None) == ml.MOE_ERR_UNSUPPORTED
+    # the LoRA backward keeps requiring its adapter gradients
+    lb = [P(4096)] * 21
+    lb[18] = None
+    assert L.moe_grouped_gemm_lora_bwd(ctypes.byref(d), *lb, 1 << 30, None) == ml.MOE_ERR_INVALID_ARG
+
+
 def test_router_backward_host_validation(L):
     null = None
     fake = ctypes.c_void_p(256)       # 16-byte aligned, never dereferenced

@@ -242,10 +242,13 @@ def test_sampled_helpers_agree_with_full_layer():
     for t in (0, 7, CFG_S.T - 1):
         assert _rel(O.token_forward(inp, t, CFG_S.k, CFG_S.scale), Y[t]) < 1e-13
         assert _rel(O.token_backward_dx(inp, t, CFG_S.k, CFG_S.scale), g["dX"][t]) < 1e-13
+    dW_gu, dW_d = O.moe_weight_grads(inp, aux, g, inp["dY"], CFG_S.k)
     for e in (0, 3):
         gs = O.expert_lora_grads(inp, e, CFG_S.k, CFG_S.scale)
         for got, key in zip(gs, ("dA_gu", "dB_gu", "dA_d", "dB_d")):
             assert _rel(got, g[key][e]) < 1e-13
+        wg, wd = O.expert_weight_grads(inp, e, CFG_S.k, CFG_S.scale)
+        assert _rel(wg, dW_gu[e]) < 1e-13 and _rel(wd, dW_d[e]) < 1e-13
 
 
 # ---------------------------------------------------------------- worked numbers
