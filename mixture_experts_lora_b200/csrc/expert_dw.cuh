@@ -24,8 +24,10 @@
 //
 // Roles (320 threads): warp 0 issues the TMA copies, warp 1 owns TMEM, zeroes tails
 // and issues the MMAs, warps 2-9 drain TMEM (two warps per lane quarter, alternate
-// 32-column chunks) into 16-byte bf16 stores along the output rows.  TMEM holds two
-// 256-column accumulators, so a tile's epilogue overlaps the next tile's MMAs.
+// 32-column chunks): each 32 x 32 block goes to bf16 in a 64-byte-swizzled staging
+// buffer of the warp (two per warp, alternating) and out with one TMA tensor store,
+// which writes whole row segments and clips rows and columns past the matrix.  TMEM
+// holds two 256-column accumulators, so a tile's epilogue overlaps the next tile's MMAs.
 #pragma once
 
 #include "common.cuh"
@@ -53,7 +55,9 @@ struct DwCfg {
   static constexpr int STAGES = 4;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int STG_BYTES = 32 * 32 * 2;         // one 32 x 32 bf16 output block
+  static constexpr int STG_TOTAL = EPI_WARPS * 2 * STG_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_TOTAL + 256 + 1024;
   static constexpr int TMEM_COLS = 2 * BN;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -61,12 +65,13 @@ struct DwCfg {
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     moe_dw_kernel(const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmR,
-                  const DwParams p) {
+                  const __grid_constant__ CUtensorMap tmO, const DwParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stg_all = smem + C::STAGES * C::STAGE_BYTES;   // epilogue staging blocks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stg_all + C::STG_TOTAL);
   uint64_t* full = bars;                       // [STAGES]
   uint64_t* empty = bars + C::STAGES;          // [STAGES]
   uint64_t* acc_full = bars + 2 * C::STAGES;   // [2]
@@ -90,6 +95,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_fence_init();
     tma_prefetch_desc(&tmL);
     tma_prefetch_desc(&tmR);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -203,6 +209,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int q = warp & 3;                         // TMEM lane quarter of this warp
     const int hsel = (warp - 2) >> 2;               // which alternate 32-column chunks
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+    uint8_t* stg = stg_all + (warp - 2) * 2 * C::STG_BYTES;
+    int sel = 0;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const int e = t / per_e, rem = t % per_e;
@@ -234,19 +242,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (; c0 < C::BN; c0 += 64) {
         const bool more = c0 + 64 < C::BN;
         if (more) tmem_ld32(acc + c0 + 64, vn);     // next chunk, in flight meanwhile
-        if (row < p.Mdim) {
+        if (col0 + c0 < p.Ndim) {
+          // staging buffer `sel` was last handed to a store two blocks ago: wait
+          // until that store has read it
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          uint8_t* blk = stg + sel * C::STG_BYTES;
+          // row `lane` of the block: four 16-byte chunks, 64-byte swizzle (chunk j of
+          // row r sits at chunk j ^ ((r >> 1) & 3)), conflict-free for the warp
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const int col = col0 + c0 + 8 * g;
-            if (col < p.Ndim) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
-              o.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
-              o.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
-              o.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
-              *reinterpret_cast<uint4*>(orow + col) = o;
-            }
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
+            o.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
+            o.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
+            o.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
+            *reinterpret_cast<uint4*>(blk + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = o;
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmO, smem_u32(blk), col0 + c0, mt * C::BM + q * 32, e);
+            bulk_commit_group();
+          }
+          sel ^= 1;
         }
         if (more) {
           tmem_wait_ld();
@@ -259,6 +278,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
       ++it;
     }
+    if (lane == 0) bulk_wait<0>();                // every store of this warp complete
+    __syncwarp();
   }
 
   tc_fence_before();

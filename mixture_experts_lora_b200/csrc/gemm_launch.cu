@@ -330,21 +330,26 @@ static cudaError_t expert_dw_launch(int kind, const CUtensorMap* tm, const DwPar
   const int64_t total = (int64_t)p.E * p.n_mt * p.n_nt;
   const int grid = (int)(total < num_sms ? total : num_sms);
   ProfScope ps(kind, s);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tm[0], tm[1], p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tm[0], tm[1], tm[2], p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_expert_dw(int kind, const GemmShape& g, const int32_t* offsets, const uint16_t* Lm,
                              int Mdim, const uint16_t* Rm, int Ndim, uint16_t* out, cudaStream_t s) {
   using C = DwCfg<true>;
-  CUtensorMap tm[2];
+  CUtensorMap tm[3];
   const uint64_t P = (uint64_t)g.P;
   const bool v = Mdim % 64 == 0 && Ndim % 64 == 0;
   const bool ok = v ? encode_atoms(&tm[0], Lm, false, 1, P, (uint64_t)Mdim, C::BK, 2) &&
                           encode_atoms(&tm[1], Rm, false, 1, P, (uint64_t)Ndim, C::BK, 4)
                     : encode2d(&tm[0], Lm, P, (uint64_t)Mdim, C::BK, 64) &&
                           encode2d(&tm[1], Rm, P, (uint64_t)Ndim, C::BK, 64);
-  if (!ok) return cudaErrorInvalidValue;
+  // output [E, Mdim, Ndim] in 32 x 32 blocks, 64-byte swizzle (the staging layout)
+  const uint64_t odims[3] = {(uint64_t)Ndim, (uint64_t)Mdim, (uint64_t)g.E};
+  const uint64_t ostr[2] = {(uint64_t)Ndim * 2, (uint64_t)Mdim * Ndim * 2};
+  const uint32_t obox[3] = {32, 32, 1};
+  if (!ok || !encode(&tm[2], out, 3, odims, ostr, obox, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   DwParams p{};
   p.offsets = offsets;
   p.E = g.E;
