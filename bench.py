@@ -155,7 +155,6 @@ def kernel_work(cfg, active_experts=None):
         "rows_gather": {"byte": 2 * (acc.bytes_gather(T, m, k) + P * 4 + lr_out)},
         "rows_swiglu": {"byte": P * 2 * n * 2 + P * n * 2 + lr_out},
         "rows_swiglu_bwd": {"byte": P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + lr_out},
-        "gather_rows": {"byte": acc.bytes_gather(T, m, k)},       # X again for dA_gu
         "unpermute_combine": {"byte": 2 * acc.bytes_combine(T, m, k)},  # Y and dX
         # full fine-tuning only: expert-weight gradients (sorted operands read once,
         # every expert's gradient written once)

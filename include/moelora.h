@@ -122,9 +122,11 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
  * Inputs (device, read): X bf16 [T, m]; sorted_pairs [P]; offsets [E+1]; the six
  *   weight tensors in the layouts above.
  * Outputs (device, written, bf16, sorted order):
- *   Y_sorted [P, m]; save_GU [P, 2n]; save_H [P, n]; save_XA [P, r] = X A_gu
- *   (unscaled); save_HA [P, r] = H A_d (unscaled).  The save_* tensors are what
- *   moe_grouped_gemm_lora_bwd() needs.
+ *   Y_sorted [P, m]; save_Xs [P, m] = X[sorted_pairs / k] (the expert-sorted input
+ *   rows, the grouped GEMM's operand, kept for the backward as an autograd
+ *   implementation keeps the permuted input); save_GU [P, 2n]; save_H [P, n];
+ *   save_XA [P, r] = X A_gu (unscaled); save_HA [P, r] = H A_d (unscaled).  The
+ *   save_* tensors are what moe_grouped_gemm_lora_bwd() needs.
  * Accumulation is fp32; every stored value is rounded once to bf16.  The LoRA
  * term multiplies bf16(c * X A) by B.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
@@ -132,7 +134,7 @@ moe_status_t moe_grouped_gemm_lora_fwd(
     const moe_dims_t* dims, const moe_bf16_t* X, const int32_t* sorted_pairs,
     const int32_t* offsets, const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
     const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_GU,
+    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs, moe_bf16_t* save_GU,
     moe_bf16_t* save_H, moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws,
     size_t ws_bytes, void* stream);
 
@@ -143,8 +145,9 @@ moe_status_t moe_grouped_gemm_lora_fwd(
  *   T2       = dGU B_gu^T, dX_sorted = dGU W_gu^T + c T2 A_gu^T
  *   dA_d[e]  = c H_e^T T1_e,   dB_d[e]  = c HA_e^T dy_e
  *   dA_gu[e] = c X_e^T T2_e,   dB_gu[e] = c XA_e^T dGU_e
- * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; X; sorted_pairs;
- *   offsets; the six weights; save_GU, save_H, save_XA, save_HA from the forward.
+ * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; sorted_pairs;
+ *   offsets; the six weights; save_Xs, save_GU, save_H, save_XA, save_HA from the
+ *   forward.
  * Outputs (device, written, bf16): dX_sorted [P, m] (sorted order; reduce with
  *   moe_unpermute_combine(topk_w = NULL)); dA_gu [E, m, r]; dB_gu [E, r, 2n];
  *   dA_d [E, n, r]; dB_d [E, r, m].  Experts with no rows get zero gradients.
@@ -152,10 +155,11 @@ moe_status_t moe_grouped_gemm_lora_fwd(
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 moe_status_t moe_grouped_gemm_lora_bwd(
     const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
-    const moe_bf16_t* X, const int32_t* sorted_pairs, const int32_t* offsets,
+    const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
+    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA,
     const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dA_gu,
     moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream);
@@ -176,10 +180,11 @@ moe_status_t moe_grouped_gemm_lora_bwd(
  * sums its rows in one fixed order (deterministic). */
 moe_status_t moe_grouped_gemm_full_bwd(
     const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
-    const moe_bf16_t* X, const int32_t* sorted_pairs, const int32_t* offsets,
+    const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
+    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA,
     const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dW_gu,
     moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
     moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream);

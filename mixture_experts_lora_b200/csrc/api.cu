@@ -187,13 +187,13 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
 
 // The backward pass.  Adapter gradients when dA_gu.. are given (all four or none),
 // expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given; each weight
-// gradient runs while its sorted operands are in the row buffer (dy after the
-// down backward, X after its re-gather).
+// gradient runs while its sorted operands are at hand (dy in the row buffer after
+// the down backward; X sorted saved by the forward).
 moe_status_t backward(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, moe_bf16_t* dW_gu,
     moe_bf16_t* dW_d, void* ws, size_t ws_bytes, void* stream) {
@@ -219,8 +219,8 @@ moe_status_t backward(
     }
     return MOE_OK;
   }
-  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA, save_HA,
-                       dX_sorted, ws};
+  const void* ins[] = {dY, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_Xs, save_GU, save_H, save_XA,
+                       save_HA, dX_sorted, ws};
   for (const void* p : ins)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (topk_w == nullptr || sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
@@ -265,17 +265,15 @@ moe_status_t backward(
                               false, dgu, t2, L.rp, L.rp, lrc2, rpart, rcnt + L.max_row_tiles, s));
   // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
-  // X re-gathered into the row buffer (dy is no longer needed), then
-  // dB_gu = c XA^T dGU and dA_gu = c X^T T2, one launch
-  MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
+  // dB_gu = c XA^T dGU and dA_gu = c X^T T2 (X in expert order from the forward), one launch
   if (lora) {
     const WgradJob jobs[2] = {
         {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
-        {rows, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
+        {save_Xs, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
     MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
   }
   // dW_gu = X^T dGU per expert
-  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, rows, d.m, dgu, 2 * d.n, dW_gu, s));
+  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, save_Xs, d.m, dgu, 2 * d.n, dW_gu, s));
   return MOE_OK;
 }
 
@@ -353,7 +351,8 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
                                        const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
                                        const moe_bf16_t* A_gu, const moe_bf16_t* B_gu,
                                        const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_GU,
+                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs,
+                                       moe_bf16_t* save_GU,
                                        moe_bf16_t* save_H, moe_bf16_t* save_XA,
                                        moe_bf16_t* save_HA, void* ws, size_t ws_bytes,
                                        void* stream) {
@@ -361,8 +360,8 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   if (st != MOE_OK) return st;
   const moe_dims_t d = *dims;
   if (d.T == 0) return MOE_OK;
-  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_GU, save_H, save_XA,
-                        save_HA, ws};
+  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_Xs, save_GU, save_H,
+                        save_XA, save_HA, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (sorted_pairs == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
@@ -373,7 +372,7 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   LayerPtrs w;
   st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, s, &g, &w);
   if (st != MOE_OK) return st;
-  uint16_t* xs = at<uint16_t>(ws, L.rows);
+  uint16_t* xs = save_Xs;
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
   float* rpart = at<float>(ws, L.rows_partial);
@@ -392,33 +391,33 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
 }
 
 moe_status_t moe_grouped_gemm_lora_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream) {
   if (dA_gu == nullptr || dB_gu == nullptr || dA_d == nullptr || dB_d == nullptr)
     return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
+  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
                   nullptr, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_grouped_gemm_full_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
     moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream) {
   if (dW_gu == nullptr || dW_d == nullptr) return MOE_ERR_INVALID_ARG;
   const int given = (dA_gu != nullptr) + (dB_gu != nullptr) + (dA_d != nullptr) + (dB_d != nullptr);
   if (given != 0 && given != 4) return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
+  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
                   dW_d, ws, ws_bytes, stream);
 }
 

@@ -14,7 +14,7 @@ struct TileInfo;
 // ---- kernel timing (profile.cu): while enabled, each launch is bracketed by
 // CUDA events on its stream and attributed to one of these kinds.
 enum KernelKind : int {
-  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD, K_GATHER,
+  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES, K_PAD,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
   K_COMBINE, K_MEMSET, K_ROWS_GATHER, K_ROWS_SWIGLU,
   K_ROWS_SWIGLU_BWD, K_ROUTER_BWD, K_GEMM_DW_GU, K_GEMM_DW_D, K_NUM_KINDS
@@ -55,13 +55,10 @@ cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, Ti
                                 int chunk_rows, TileInfo* chunks, int* n_chunks,
                                 int32_t* chunk_start, int* zero, int n_zero,
                                 cudaStream_t s);
-// out[q] = (w ? bf16(w[p] * src[p / k]) : src[p / k]),  p = sorted_pairs[q]
 // dlogits [T, E] fp32 = router backward (see simt_kernels.cu); m % 8 == 0
 cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const int32_t* ids,
                                    const float* w, const int32_t* pos, int64_t T, int k, int E,
                                    int m, float* dlogits, cudaStream_t s);
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
-                               int64_t P, int k, int m, uint16_t* out, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_t* pair_pos,
                            int64_t T, int k, int m, uint16_t* y, cudaStream_t s);
 // out [E, Ro, Co] = in [E, Ri, Ci] zero-padded (Ro >= Ri, Co >= Ci)

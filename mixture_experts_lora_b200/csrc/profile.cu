@@ -16,7 +16,7 @@ namespace moe {
 
 const char* const kKernelNames[K_NUM_KINDS] = {
     "route_topk",        "permute_hist",      "permute_scan",     "permute_scatter",
-    "build_tables",      "pad_lora",          "gather_rows",      "gemm_gateup_fwd",
+    "build_tables",      "pad_lora",          "gemm_gateup_fwd",
     "gemm_down_fwd",     "gemm_down_bwd",     "gemm_gateup_bwd",  "lora_wgrad",
     "unpermute_combine", "memset",            "rows_gather",       "rows_swiglu",       "rows_swiglu_bwd",
     "router_backward",   "gemm_dw_gu",        "gemm_dw_d"};

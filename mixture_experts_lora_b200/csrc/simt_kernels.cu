@@ -302,30 +302,6 @@ cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, Ti
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ gather
-// out[q, :] = src[p / k, :] (optionally scaled by w[p] before the bf16 rounding),
-// p = sorted_pairs[q].  One thread per 16-byte vector.
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ sp,
-                                   const float* __restrict__ w, int64_t P, int k, int vpr,
-                                   uint4* __restrict__ out) {
-  const int64_t total = P * vpr;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t q = i / vpr;
-    const int v = (int)(i - q * vpr);
-    const int p = sp[q];
-    uint4 x = src[(int64_t)(p / k) * vpr + v];
-    if (w != nullptr) {
-      const float s = w[p];
-      x.x = pack_bf16x2(s * bf16_lo(x.x), s * bf16_hi(x.x));
-      x.y = pack_bf16x2(s * bf16_lo(x.y), s * bf16_hi(x.y));
-      x.z = pack_bf16x2(s * bf16_lo(x.z), s * bf16_hi(x.z));
-      x.w = pack_bf16x2(s * bf16_lo(x.w), s * bf16_hi(x.w));
-    }
-    out[i] = x;
-  }
-}
-
 static int g_num_sms_cache = 0;
 static int num_sms() {
   if (g_num_sms_cache == 0) {
@@ -341,16 +317,6 @@ static unsigned grid_for(int64_t work, int threads) {
   const int64_t want = (work + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms() * 16;
   return (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
-}
-
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
-                               int64_t P, int k, int m, uint16_t* out, cudaStream_t s) {
-  if (P == 0) return cudaSuccess;
-  const int vpr = m / 8;
-  ProfScope ps(K_GATHER, s);
-  gather_rows_kernel<<<grid_for(P * vpr, 256), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(src), sorted_pairs, w, P, k, vpr, reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ combine

@@ -85,7 +85,7 @@ def test_host_validation_returns_before_launch(L):
     assert L.moe_permute(fake, 4, 2, 8, fake, fake, fake, fake, fake, 8, null) == ml.MOE_ERR_WORKSPACE
     # forward: bad dims, NULL / misaligned pointers, small workspace
     d = dims()
-    ptrs = [P(4096)] * 15
+    ptrs = [P(4096)] * 16
     assert L.moe_grouped_gemm_lora_fwd(ctypes.byref(dims(m=100)), *ptrs, 1 << 30, null) == ml.MOE_ERR_UNSUPPORTED
     assert L.moe_grouped_gemm_lora_fwd(None, *ptrs, 1 << 30, null) == ml.MOE_ERR_INVALID_ARG
     bad = list(ptrs)
