@@ -271,11 +271,11 @@ cudaError_t launch_rows_lowrank(const GemmShape& g, int mode, int K, const uint1
 }
 
 
-template <int RP>
+template <int RP, bool V>
 static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const WgradParams& wp,
                             int max_chunks, cudaStream_t s) {
-  using C = WgradCfg<RP>;
-  auto kern = lora_wgrad_kernel<RP>;
+  using C = WgradCfg<RP, V>;
+  auto kern = lora_wgrad_kernel<RP, V>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
   int dtiles = wp.pr[0].n_dtiles + (wp.n_problems > 1 ? wp.pr[1].n_dtiles : 0);
@@ -283,7 +283,7 @@ static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const Wgr
   // at least one CTA per SM: the zero fill of experts without rows runs in every CTA
   const int grid = (int)(units > 0 && units < g.num_sms ? units : g.num_sms);
   ProfScope ps(K_WGRAD, s);
-  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm[0], tm[1], wp);
+  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm[0], tm[1], tm[2], tm[3], wp);
   return cudaGetLastError();
 }
 
@@ -291,11 +291,23 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
                               const TileInfo* chunks, const int* n_chunks, int max_chunks,
                               const int32_t* chunk_start, cudaStream_t s) {
   if (n_jobs < 1 || n_jobs > 2) return cudaErrorInvalidValue;
-  CUtensorMap tm[2];
+  using C0 = WgradCfg<16>;
+  CUtensorMap tm[4];      // Big of each problem, then Small of each problem
   WgradParams wp{};
+  const uint64_t P = (uint64_t)(g.P > 0 ? g.P : 1);
+  bool v = true;
+  for (int j = 0; j < n_jobs; ++j) v = v && jobs[j].D % 64 == 0;
   for (int j = 0; j < n_jobs; ++j) {
     const WgradJob& jb = jobs[j];
-    if (!encode2d(&tm[j], jb.big, (uint64_t)(g.P > 0 ? g.P : 1), (uint64_t)jb.D, WgradCfg<16>::BK, 64))
+    // Big [P, D]: BK rows x 128 columns per stage
+    const bool okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, 2)
+                       : encode2d(&tm[j], jb.big, P, (uint64_t)jb.D, C0::BK, 64);
+    // Small [P, ld_small] seen as [ld_small / 8 groups][P rows][8 columns]: a box of
+    // BK rows x all groups lands group-major (groups past ld_small read as zero)
+    const uint64_t sd[3] = {8, P, (uint64_t)jb.ld_small / 8};
+    const uint64_t ss[2] = {(uint64_t)jb.ld_small * 2, 16};
+    const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)g.rp / 8};
+    if (!okb || !encode(&tm[2 + j], jb.small, 3, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     WgradProblem& q = wp.pr[j];
     q.small = reinterpret_cast<const __nv_bfloat16*>(jb.small);
@@ -308,7 +320,10 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
     q.partial = jb.partial;
     q.counters = jb.counters;
   }
-  if (n_jobs == 1) tm[1] = tm[0];
+  if (n_jobs == 1) {
+    tm[1] = tm[0];
+    tm[3] = tm[2];
+  }
   wp.n_problems = n_jobs;
   wp.chunks = chunks;
   wp.n_chunks = n_chunks;
@@ -317,8 +332,8 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
   wp.r = g.r;
   wp.scale = g.scale;
   wp.err = g.err;
-  if (g.rp == 16) return wgrad_rp<16>(g, tm, wp, max_chunks, s);
-  return wgrad_rp<32>(g, tm, wp, max_chunks, s);
+  if (g.rp == 16) return v ? wgrad_rp<16, true>(g, tm, wp, max_chunks, s) : wgrad_rp<16, false>(g, tm, wp, max_chunks, s);
+  return v ? wgrad_rp<32, true>(g, tm, wp, max_chunks, s) : wgrad_rp<32, false>(g, tm, wp, max_chunks, s);
 }
 
 template <class C>

@@ -12,10 +12,17 @@
 // computable at the same point of the backward).  Units are (problem, row chunk
 // of one expert, 128-wide D tile); a persistent CTA walks its units with one
 // continuous TMA/MMA pipeline:
-//   M = 128 columns of Big (MN-major A operand, TMA, 128-byte swizzle),
-//   N = RP (Small, MN-major, no swizzle, written by the producer warp with rows
-//       outside the chunk zeroed, so a ragged tail contributes nothing),
-//   K = rows of the chunk, 128 per stage.
+//   M = 128 columns of Big (MN-major A operand, 128-byte swizzle),
+//   N = RP (Small, MN-major, no swizzle),
+//   K = rows of the chunk, 128 per stage,
+// with one TMA copy per operand and stage (Big through a view of 64-column atoms
+// when D % 64 == 0, Small through a view of 8-column groups that lands in the
+// core-matrix layout).  Every copy is full-size from the chunk's first row, so the
+// stage that crosses the chunk's end also holds rows of the next chunk: the MMA
+// warp issues only the 16-row K steps that reach into the chunk and zeroes Small's
+// rows past its end in the last of them, so a ragged tail contributes nothing.
+// The loader and MMA threads each spend a fixed number of instructions per stage
+// (two copies; precomputed descriptors advanced by offsets).
 // The accumulator is double buffered in TMEM.  A unit of an expert whose rows fit
 // in one chunk writes the final bf16 gradient (scaled, in its output orientation).
 // Otherwise each unit writes an fp32 partial and counts itself in a per-(expert,
@@ -53,8 +60,9 @@ struct WgradParams {
   int* err;
 };
 
-template <int RP>
+template <int RP, bool V_ = true>
 struct WgradCfg {
+  static constexpr bool V = V_;             // Big through the atom view (D % 64 == 0)
   // 128 rows per stage: 8 MMAs per wait and commit (the per-stage issue cost of the
   // loader and MMA threads, not the bytes, bounded 64-row stages)
   static constexpr int BM = 128, BK = 128;
@@ -108,11 +116,13 @@ __device__ __forceinline__ void wgrad_store(const WgradProblem& q, int r, float 
   }
 }
 
-template <int RP>
+template <int RP, bool V>
 __global__ void __launch_bounds__(192, 1)
     lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig0,
-                      const __grid_constant__ CUtensorMap tmBig1, const WgradParams p) {
-  using C = WgradCfg<RP>;
+                      const __grid_constant__ CUtensorMap tmBig1,
+                      const __grid_constant__ CUtensorMap tmSmall0,
+                      const __grid_constant__ CUtensorMap tmSmall1, const WgradParams p) {
+  using C = WgradCfg<RP, V>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -130,7 +140,7 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 33);   // TMA expect_tx arrive + 32 cp.async arrivals
+      mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -142,7 +152,11 @@ __global__ void __launch_bounds__(192, 1)
     *last_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmBig0);
-    if (p.n_problems > 1) tma_prefetch_desc(&tmBig1);
+    tma_prefetch_desc(&tmSmall0);
+    if (p.n_problems > 1) {
+      tma_prefetch_desc(&tmBig1);
+      tma_prefetch_desc(&tmSmall1);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -162,8 +176,8 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const WgradUnit u = wgrad_unit(p, nch, t);
-      const WgradProblem& q = p.pr[u.prob];
-      const CUtensorMap* tm = u.prob == 0 ? &tmBig0 : &tmBig1;
+      const CUtensorMap* tb = u.prob == 0 ? &tmBig0 : &tmBig1;
+      const CUtensorMap* ts = u.prob == 0 ? &tmSmall0 : &tmSmall1;
       const TileInfo ch = p.chunks[u.c];
       const int d0 = u.dt * C::BM;
       const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
@@ -171,97 +185,91 @@ __global__ void __launch_bounds__(192, 1)
       for (int ks = 0; ks < nk; ++ks) {
         const bool w = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
-        const uint32_t fb = smem_u32(&full[stage]);
-        const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
-        const int r0 = ch.row0 + ks * C::BK;
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, C::BIG_BYTES);
-          tma_load_2d(tm, fb, sbig, d0, r0);
-          tma_load_2d(tm, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
+          const uint32_t fb = smem_u32(&full[stage]);
+          const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
+          const int r0 = ch.row0 + ks * C::BK;
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          if constexpr (C::V) {
+            tma_load_3d(tb, fb, sbig, 0, r0, d0 / 64);
+          } else {
+            tma_load_2d(tb, fb, sbig, d0, r0);
+            tma_load_2d(tb, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
+          }
+          // Small [BK rows][RP]: groups of 8 columns, each BK rows x 16 bytes
+          // (MN-major, no swizzle: core matrices of 8 rows x 8 columns)
+          tma_load_3d(ts, fb, sbig + C::BIG_BYTES, 0, r0, 0);
         }
-        // Small tile [BK rows][RP]: MN-major, no swizzle; core matrix = 8 rows x 8
-        // columns (128 B), row groups 128 B apart, column groups SMALL_NG bytes apart.
-        // Rows outside the chunk (and columns past r_small) are zero-filled.
-        const uint32_t ssm = sbig + C::BIG_BYTES;
-        constexpr int CG = RP / 8;
-#pragma unroll
-        for (int i = lane; i < C::BK * CG; i += 32) {
-          const int rr = i / CG, cg = i % CG;
-          const int row = r0 + rr;
-          const bool valid = row < ch.row_end && cg * 8 < q.r_small;
-          const void* src = valid ? (const void*)(q.small + (size_t)row * q.ld_small + cg * 8)
-                                  : (const void*)q.small;
-          cp_async_16(ssm + cg * C::SMALL_NG + (rr & 7) * 16 + (rr >> 3) * 128, src, valid ? 16u : 0u);
-        }
-        cp_async_mbar_arrive(fb);
+        __syncwarp();
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
     if (!ok && lane == 0) *abort_flag = 1;
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, RP, 1, 1);
-      int stage = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      bool ok = true, issued_any = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const WgradUnit u = wgrad_unit(p, nch, t);
-        const TileInfo ch = p.chunks[u.c];
-        const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
-        const int b = it & 1;
-        if (!mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d = tmem + b * 32;
-        if (*abort_flag) { ok = false; break; }
-        for (int ks = 0; ks < nk; ++ks) {
-          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
-          fence_proxy_async_smem();   // cp.async writes -> tcgen05 reads
-          tc_fence_after();
-          const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
-          const uint32_t ssm = sbig + C::BIG_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk) {
-            // Big^T: MN-major, 128-byte swizzle, 64-column atoms BIG_BYTES/2 apart, 8-row groups 1 KB apart
-            const uint64_t ad = smem_desc(sbig + kk * 16 * 128, C::BIG_BYTES / 2, 1024, kSw128);
-            // Small: MN-major, no swizzle; K (row) groups at 128 B, N (column) groups at SMALL_NG
-            const uint64_t bd = smem_desc(ssm + kk * 256, 128, C::SMALL_NG, kSwNone);
-            umma_bf16(d, ad, bd, idesc, (ks | kk) ? 1u : 0u);
+    // ---------------------------------------------------------- MMA issuer (whole warp)
+    // Big^T: MN-major, 128-byte swizzle, 64-column atoms BIG_BYTES/2 apart, 8-row
+    // groups 1 KB apart (a 16-row K step advances 2 KB).  Small: MN-major, no swizzle,
+    // 8-row groups 128 bytes apart, 8-column groups SMALL_NG apart (a K step: 256 B).
+    const uint32_t idesc = idesc_bf16(128, RP, 1, 1);
+    const uint64_t a_desc0 = smem_desc(s_base, C::BIG_BYTES / 2, 1024, kSw128);
+    const uint64_t b_desc0 = smem_desc(s_base + C::BIG_BYTES, 128, C::SMALL_NG, kSwNone);
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true, issued_any = false;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+      const WgradUnit u = wgrad_unit(p, nch, t);
+      const TileInfo ch = p.chunks[u.c];
+      const int rows = ch.row_end - ch.row0;
+      const int nk = (rows + C::BK - 1) / C::BK;
+      const int b = it & 1;
+      const bool aok = mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err);
+      if (!__all_sync(0xffffffffu, aok) || *abort_flag) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d = tmem + b * 32;
+      for (int ks = 0; ks < nk; ++ks) {
+        const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
+        if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
+        const int kv = rows - ks * C::BK < C::BK ? rows - ks * C::BK : C::BK;   // rows of the chunk
+        const int nsteps = (kv + 15) >> 4;
+        const int z = nsteps * 16 - kv;                                          // rows past its end
+        if (z > 0) {
+          // zero Small rows kv .. 16 nsteps - 1 in every 8-column group
+          uint8_t* zs = smem + stage * C::STAGE_BYTES + C::BIG_BYTES + kv * 16;
+          for (int i = lane; i < z * (RP / 8); i += 32) {
+            const int g = i / z, rr = i - g * z;
+            *reinterpret_cast<uint4*>(zs + g * C::SMALL_NG + rr * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
-          umma_commit(smem_u32(&empty[stage]));
-          issued_any = true;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        if (!ok) break;
-        umma_commit(smem_u32(&acc_full[b]));
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t so = (uint32_t)(stage * C::STAGE_BYTES) >> 4;
+          for (int kk = 0; kk < nsteps; ++kk)
+            umma_bf16(d, a_desc0 + so + kk * (2048 / 16), b_desc0 + so + kk * (256 / 16), idesc,
+                      (ks | kk) ? 1u : 0u);
+          umma_commit(smem_u32(&empty[stage]));
+        }
+        __syncwarp();
+        issued_any = true;
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
-      if (!ok) *abort_flag = 1;
-      if (issued_any) {
-        umma_commit(smem_u32(drain));
-        mbar_wait(smem_u32(drain), 0, p.err);
-      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&acc_full[b]));
+      __syncwarp();
+    }
+    if (!ok && lane == 0) *abort_flag = 1;
+    if (issued_any) {
+      if (lane == 0) umma_commit(smem_u32(drain));
+      __syncwarp();
+      mbar_wait(smem_u32(drain), 0, p.err);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue (warps 2..5)
     const int q4 = warp & 3;                       // TMEM lane quarter of this warp
     const int et = (warp - 2) * 32 + lane;         // 0..127
-    // gradients of experts without rows are zero
-    for (int prob = 0; prob < p.n_problems; ++prob) {
-      const WgradProblem& q = p.pr[prob];
-      const int64_t tot = (int64_t)p.E * q.D;
-      for (int64_t i = (int64_t)blockIdx.x * C::EPI_THREADS + et; i < tot;
-           i += (int64_t)gridDim.x * C::EPI_THREADS) {
-        const int e = (int)(i / q.D), d = (int)(i - (int64_t)e * q.D);
-        if (p.chunk_start[e + 1] == p.chunk_start[e]) {
-          float z[RP];
-#pragma unroll
-          for (int j = 0; j < RP; ++j) z[j] = 0.f;
-          wgrad_store<RP>(q, p.r, p.scale, e, d, z);
-        }
-      }
-    }
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const WgradUnit u = wgrad_unit(p, nch, t);
@@ -330,6 +338,18 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         wgrad_store<RP>(q, p.r, p.scale, ch.e, d, acc);
+      }
+    }
+    // gradients of experts without rows are zero: after the units, so the scan never
+    // holds up the accumulators; CTA b takes experts b, b + grid, ...
+    for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
+      if (p.chunk_start[e + 1] != p.chunk_start[e]) continue;
+      for (int prob = 0; prob < p.n_problems; ++prob) {
+        const WgradProblem& q = p.pr[prob];
+        float z[RP];
+#pragma unroll
+        for (int j = 0; j < RP; ++j) z[j] = 0.f;
+        for (int d = et; d < q.D; d += C::EPI_THREADS) wgrad_store<RP>(q, p.r, p.scale, e, d, z);
       }
     }
   }
