@@ -299,14 +299,15 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
   for (int j = 0; j < n_jobs; ++j) v = v && jobs[j].D % 64 == 0;
   for (int j = 0; j < n_jobs; ++j) {
     const WgradJob& jb = jobs[j];
-    // Big [P, D]: BK rows x 128 columns per stage
-    const bool okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, 2)
+    // Big [P, D]: BK rows x 256 columns per stage (four 64-column atoms)
+    const bool okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, C0::BN / 64)
                        : encode2d(&tm[j], jb.big, P, (uint64_t)jb.D, C0::BK, 64);
     // Small [P, ld_small] seen as [ld_small / 8 groups][P rows][8 columns]: a box of
-    // BK rows x all groups lands group-major (groups past ld_small read as zero)
+    // BK rows x 16 groups (the MMA's 128 rank rows) lands group-major, groups past
+    // ld_small reading as zero
     const uint64_t sd[3] = {8, P, (uint64_t)jb.ld_small / 8};
     const uint64_t ss[2] = {(uint64_t)jb.ld_small * 2, 16};
-    const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)g.rp / 8};
+    const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)C0::BM / 8};
     if (!okb || !encode(&tm[2 + j], jb.small, 3, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     WgradProblem& q = wp.pr[j];
@@ -314,7 +315,7 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
     q.ld_small = jb.ld_small;
     q.r_small = jb.ld_small;  // the caller's buffer has exactly ld_small columns
     q.D = jb.D;
-    q.n_dtiles = (jb.D + 127) / 128;
+    q.n_dtiles = (jb.D + C0::BN - 1) / C0::BN;
     q.transpose = jb.transpose;
     q.out = reinterpret_cast<__nv_bfloat16*>(jb.out);
     q.partial = jb.partial;

@@ -10,26 +10,28 @@
 //
 // One launch computes up to two such problems (the two gradients that become
 // computable at the same point of the backward).  Units are (problem, row chunk
-// of one expert, 128-wide D tile); a persistent CTA walks its units with one
-// continuous TMA/MMA pipeline:
-//   M = 128 columns of Big (MN-major A operand, 128-byte swizzle),
-//   N = RP (Small, MN-major, no swizzle),
-//   K = rows of the chunk, 128 per stage,
-// with one TMA copy per operand and stage (Big through a view of 64-column atoms
-// when D % 64 == 0, Small through a view of 8-column groups that lands in the
-// core-matrix layout).  Every copy is full-size from the chunk's first row, so the
-// stage that crosses the chunk's end also holds rows of the next chunk: the MMA
-// warp issues only the 16-row K steps that reach into the chunk and zeroes Small's
-// rows past its end in the last of them, so a ragged tail contributes nothing.
-// The loader and MMA threads each spend a fixed number of instructions per stage
-// (two copies; precomputed descriptors advanced by offsets).
-// The accumulator is double buffered in TMEM.  A unit of an expert whose rows fit
-// in one chunk writes the final bf16 gradient (scaled, in its output orientation).
-// Otherwise each unit writes an fp32 partial and counts itself in a per-(expert,
-// D tile) arrival counter; the unit that arrives last sums the expert's partials
-// in chunk order (deterministic, whatever the arrival order) and writes the
-// gradient.  Gradients of experts without rows are written as zeros by the same
-// launch.
+// of one expert, 256-wide column tile of Big); a persistent CTA walks its units
+// with one continuous TMA/MMA pipeline computing G^T for the tile:
+//   M = 128 rank rows (Small^T, MN-major, no swizzle: groups of 8 rank columns;
+//       the TMA view has 16 groups, those past Small's width read as zero),
+//   N = 256 columns of Big (MN-major, 128-byte swizzle, four 64-column atoms),
+//   K = rows of the chunk, 64 per stage,
+// one TMA copy per operand and stage.  A rank of at most 32 uses a quarter of M,
+// but each MMA then moves 256 columns of Big: a thin N = r MMA costs the tensor
+// pipe about as long as a full one and would bound the kernel instead of HBM.
+// Every copy is full-size from the chunk's first row, so the stage that crosses the
+// chunk's end also holds rows of the next chunk: the MMA warp issues only the
+// 16-row K steps that reach into the chunk and zeroes Small's rows past its end in
+// the last of them.
+// The accumulator (128 lanes x 256 fp32 columns) is double buffered in TMEM.  The
+// warp that owns TMEM lanes 0-31 (the rank rows) copies them to shared memory; all
+// four epilogue warps then write the gradient with 16-byte stores in its output
+// orientation.  A unit of an expert whose rows fit in one chunk writes the final
+// bf16 gradient (scaled).  Otherwise each unit writes an fp32 partial and counts
+// itself in a per-(expert, column tile) arrival counter; the unit that arrives
+// last sums the expert's partials in chunk order (deterministic, whatever the
+// arrival order) and writes the gradient.  Gradients of experts without rows are
+// written as zeros by the same launch.
 #pragma once
 
 #include "common.cuh"
@@ -41,7 +43,7 @@ struct WgradProblem {
   int ld_small;
   int r_small;                 // columns of `small` to read (rest zero)
   int D;
-  int n_dtiles;
+  int n_dtiles;                // 256-column tiles of Big
   bool transpose;              // out [E, r, D] instead of [E, D, r]
   __nv_bfloat16* out;
   float* partial;              // [max_chunks, D, RP]
@@ -63,21 +65,24 @@ struct WgradParams {
 template <int RP, bool V_ = true>
 struct WgradCfg {
   static constexpr bool V = V_;             // Big through the atom view (D % 64 == 0)
-  // 128 rows per stage: 8 MMAs per wait and commit (the per-stage issue cost of the
-  // loader and MMA threads, not the bytes, bounded 64-row stages)
-  static constexpr int BM = 128, BK = 128;
-  static constexpr int BIG_BYTES = BM * BK * 2;   // two 64-column atoms of BK rows
-  static constexpr int SMALL_BYTES = RP * BK * 2;
-  static constexpr int SMALL_NG = BK * 16;        // bytes between 8-column groups of Small
-  static constexpr int STAGE_BYTES = BIG_BYTES + SMALL_BYTES;
-  static constexpr int STAGES_FIT = (232448 - 2048) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
-  static constexpr int TMEM_COLS = 64;            // 2 x RP fp32 columns (RP <= 32)
-  static constexpr int EPI_THREADS = 128;         // warps 2..5
+  static constexpr int BM = 128;            // rank rows on M (RP of them are used)
+  static constexpr int BN = 256;            // Big columns per unit
+  static constexpr int BK = 64;             // rows per stage
+  static constexpr int SMALL_NG = BK * 16;  // bytes between 8-column groups of Small
+  static constexpr int A_BYTES = (BM / 8) * SMALL_NG;     // 16 KB: 16 groups of 8 rank columns
+  static constexpr int ATOM = BK * 128;                   // 8 KB: 64 Big columns x BK rows
+  static constexpr int B_BYTES = (BN / 64) * ATOM;        // 32 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 4;
+  static constexpr int ST_LD = BN + 4;                    // fp32 staging row (rank j), padded
+  static constexpr int STG_BYTES = RP * ST_LD * 4;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 512 + 1024;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int EPI_THREADS = 128;                 // warps 2..5
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-// Unit t of the launch -> (problem, chunk, D tile).
+// Unit t of the launch -> (problem, chunk, column tile).
 struct WgradUnit {
   int prob, c, dt;
 };
@@ -92,28 +97,14 @@ __device__ __forceinline__ WgradUnit wgrad_unit(const WgradParams& p, int nch, i
   return u;
 }
 
-// Scaled bf16 gradient row d of expert e from fp32 values v[0..RP).
-template <int RP>
-__device__ __forceinline__ void wgrad_store(const WgradProblem& q, int r, float scale, int e, int d,
-                                            const float (&v)[RP]) {
-  if (q.transpose) {
-#pragma unroll
-    for (int i = 0; i < RP; ++i)
-      if (i < r) q.out[((size_t)e * r + i) * q.D + d] = __float2bfloat16_rn(scale * v[i]);
-  } else {
-    __nv_bfloat16* dst = q.out + ((size_t)e * q.D + d) * r;
-#pragma unroll
-    for (int g = 0; g < RP / 8; ++g) {
-      if (g * 8 < r) {
-        uint4 o;
-        o.x = pack_bf16x2(scale * v[8 * g + 0], scale * v[8 * g + 1]);
-        o.y = pack_bf16x2(scale * v[8 * g + 2], scale * v[8 * g + 3]);
-        o.z = pack_bf16x2(scale * v[8 * g + 4], scale * v[8 * g + 5]);
-        o.w = pack_bf16x2(scale * v[8 * g + 6], scale * v[8 * g + 7]);
-        *reinterpret_cast<uint4*>(dst + 8 * g) = o;
-      }
-    }
-  }
+// 8 consecutive output values as one 16-byte bf16 store (scaled).
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, float s, const float (&v)[8]) {
+  uint4 o;
+  o.x = pack_bf16x2(s * v[0], s * v[1]);
+  o.y = pack_bf16x2(s * v[2], s * v[3]);
+  o.z = pack_bf16x2(s * v[4], s * v[5]);
+  o.w = pack_bf16x2(s * v[6], s * v[7]);
+  *reinterpret_cast<uint4*>(dst) = o;
 }
 
 template <int RP, bool V>
@@ -127,8 +118,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* full = bars;                     // [STAGES]: TMA bytes + producer stores
+  float* stg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);   // [RP][ST_LD]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::STG_BYTES);
+  uint64_t* full = bars;                     // [STAGES]
   uint64_t* empty = bars + C::STAGES;        // [STAGES]
   uint64_t* acc_full = bars + 2 * C::STAGES; // [2]
   uint64_t* acc_empty = acc_full + 2;        // [2]
@@ -145,7 +137,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 4);
+      mbar_init(smem_u32(&acc_empty[b]), 1);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
@@ -179,7 +171,7 @@ __global__ void __launch_bounds__(192, 1)
       const CUtensorMap* tb = u.prob == 0 ? &tmBig0 : &tmBig1;
       const CUtensorMap* ts = u.prob == 0 ? &tmSmall0 : &tmSmall1;
       const TileInfo ch = p.chunks[u.c];
-      const int d0 = u.dt * C::BM;
+      const int d0 = u.dt * C::BN;
       const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       for (int ks = 0; ks < nk; ++ks) {
@@ -187,18 +179,19 @@ __global__ void __launch_bounds__(192, 1)
         if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
         if (lane == 0) {
           const uint32_t fb = smem_u32(&full[stage]);
-          const uint32_t sbig = s_base + stage * C::STAGE_BYTES;
+          const uint32_t sa = s_base + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
           const int r0 = ch.row0 + ks * C::BK;
           mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          // Small [BK rows][128 rank columns as 16 groups of 8]: groups past its width
+          // read as zero (MN-major, no swizzle: core matrices of 8 rows x 8 columns)
+          tma_load_3d(ts, fb, sa, 0, r0, 0);
           if constexpr (C::V) {
-            tma_load_3d(tb, fb, sbig, 0, r0, d0 / 64);
+            tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
           } else {
-            tma_load_2d(tb, fb, sbig, d0, r0);
-            tma_load_2d(tb, fb, sbig + C::BIG_BYTES / 2, d0 + 64, r0);
+#pragma unroll
+            for (int a = 0; a < C::BN / 64; ++a) tma_load_2d(tb, fb, sb + a * C::ATOM, d0 + a * 64, r0);
           }
-          // Small [BK rows][RP]: groups of 8 columns, each BK rows x 16 bytes
-          // (MN-major, no swizzle: core matrices of 8 rows x 8 columns)
-          tma_load_3d(ts, fb, sbig + C::BIG_BYTES, 0, r0, 0);
         }
         __syncwarp();
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -207,12 +200,12 @@ __global__ void __launch_bounds__(192, 1)
     if (!ok && lane == 0) *abort_flag = 1;
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer (whole warp)
-    // Big^T: MN-major, 128-byte swizzle, 64-column atoms BIG_BYTES/2 apart, 8-row
-    // groups 1 KB apart (a 16-row K step advances 2 KB).  Small: MN-major, no swizzle,
-    // 8-row groups 128 bytes apart, 8-column groups SMALL_NG apart (a K step: 256 B).
-    const uint32_t idesc = idesc_bf16(128, RP, 1, 1);
-    const uint64_t a_desc0 = smem_desc(s_base, C::BIG_BYTES / 2, 1024, kSw128);
-    const uint64_t b_desc0 = smem_desc(s_base + C::BIG_BYTES, 128, C::SMALL_NG, kSwNone);
+    // A = Small^T: MN-major, no swizzle, 8-row K groups 128 B apart, 8-column M groups
+    // SMALL_NG apart (a 16-row K step advances 256 B).  B = Big: MN-major, 128-byte
+    // swizzle, 64-column atoms ATOM apart, 8-row K groups 1 KB apart (a K step: 2 KB).
+    const uint32_t idesc = idesc_bf16(C::BM, C::BN, 1, 1);
+    const uint64_t a_desc0 = smem_desc(s_base, 128, C::SMALL_NG, kSwNone);
+    const uint64_t b_desc0 = smem_desc(s_base + C::A_BYTES, C::ATOM, 1024, kSw128);
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
@@ -226,7 +219,7 @@ __global__ void __launch_bounds__(192, 1)
       const bool aok = mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err);
       if (!__all_sync(0xffffffffu, aok) || *abort_flag) { ok = false; break; }
       tc_fence_after();
-      const uint32_t d = tmem + b * 32;
+      const uint32_t d = tmem + b * C::BN;
       for (int ks = 0; ks < nk; ++ks) {
         const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
         if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
@@ -234,8 +227,8 @@ __global__ void __launch_bounds__(192, 1)
         const int nsteps = (kv + 15) >> 4;
         const int z = nsteps * 16 - kv;                                          // rows past its end
         if (z > 0) {
-          // zero Small rows kv .. 16 nsteps - 1 in every 8-column group
-          uint8_t* zs = smem + stage * C::STAGE_BYTES + C::BIG_BYTES + kv * 16;
+          // zero Small rows kv .. 16 nsteps - 1 in the groups that hold rank columns
+          uint8_t* zs = smem + stage * C::STAGE_BYTES + kv * 16;
           for (int i = lane; i < z * (RP / 8); i += 32) {
             const int g = i / z, rr = i - g * z;
             *reinterpret_cast<uint4*>(zs + g * C::SMALL_NG + rr * 16) = make_uint4(0u, 0u, 0u, 0u);
@@ -247,7 +240,7 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
           const uint32_t so = (uint32_t)(stage * C::STAGE_BYTES) >> 4;
           for (int kk = 0; kk < nsteps; ++kk)
-            umma_bf16(d, a_desc0 + so + kk * (2048 / 16), b_desc0 + so + kk * (256 / 16), idesc,
+            umma_bf16(d, a_desc0 + so + kk * (256 / 16), b_desc0 + so + kk * (2048 / 16), idesc,
                       (ks | kk) ? 1u : 0u);
           umma_commit(smem_u32(&empty[stage]));
         }
@@ -268,47 +261,77 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- epilogue (warps 2..5)
-    const int q4 = warp & 3;                       // TMEM lane quarter of this warp
     const int et = (warp - 2) * 32 + lane;         // 0..127
+    const bool owner = (warp & 3) == 0;            // the warp of TMEM lanes 0-31 (rank rows)
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const WgradUnit u = wgrad_unit(p, nch, t);
       const WgradProblem& q = p.pr[u.prob];
       const TileInfo ch = p.chunks[u.c];
       const int b = it & 1;
-      const bool ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
+      bool ok = true;
+      if (owner) {
+        ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
+        if (ok) {
+          // rank row `lane` of the accumulator -> staging row lane (fp32)
+          tc_fence_after();
+          const uint32_t acc = tmem + b * C::BN;
+#pragma unroll 1
+          for (int c0 = 0; c0 < C::BN; c0 += 32) {
+            uint32_t v[32];
+            tmem_ld32(acc + c0, v);
+            tmem_wait_ld();
+            if (lane < RP) {
+              float4* dst = reinterpret_cast<float4*>(stg + lane * C::ST_LD + c0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+          }
+          tc_fence_before();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+      }
       // every epilogue warp takes the same branch (named barriers follow)
       if (named_bar_or(1, C::EPI_THREADS, !ok || *abort_flag != 0)) { *abort_flag = 1; break; }
-      tc_fence_after();
-      float v[RP];
-      if constexpr (RP == 16) {
-        uint32_t rr[16];
-        tmem_ld16(tmem + ((uint32_t)(q4 * 32) << 16) + b * 32, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(rr[i]);
-      } else {
-        uint32_t rr[32];
-        tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + b * 32, rr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
-      const int d = u.dt * C::BM + q4 * 32 + lane;
+      const int d0 = u.dt * C::BN;
       const int c0 = p.chunk_start[ch.e], c1 = p.chunk_start[ch.e + 1];
       if (c1 - c0 == 1) {
-        if (d < q.D) wgrad_store<RP>(q, p.r, p.scale, ch.e, d, v);
+        if (q.transpose) {
+          // out [E][r][D]: row j, 8 consecutive columns per store
+          for (int i = et; i < p.r * (C::BN / 8); i += C::EPI_THREADS) {
+            const int j = i / (C::BN / 8), cc = (i - j * (C::BN / 8)) * 8;
+            if (d0 + cc >= q.D) continue;
+            float v[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) v[x] = stg[j * C::ST_LD + cc + x];
+            store_bf16x8(q.out + ((size_t)ch.e * p.r + j) * q.D + d0 + cc, p.scale, v);
+          }
+        } else {
+          // out [E][D][r]: column d, 8 consecutive rank entries per store
+          for (int i = et; i < C::BN * (p.r / 8); i += C::EPI_THREADS) {
+            const int dd = i / (p.r / 8), g = i - dd * (p.r / 8);
+            if (d0 + dd >= q.D) continue;
+            float v[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) v[x] = stg[(g * 8 + x) * C::ST_LD + dd];
+            store_bf16x8(q.out + ((size_t)ch.e * q.D + d0 + dd) * p.r + g * 8, p.scale, v);
+          }
+        }
+        named_bar(1, C::EPI_THREADS);             // staging is rewritten by the next unit
         continue;
       }
-      // several chunks: fp32 partial, then the last arriving unit sums them in order
-      if (d < q.D) {
-        float4* dst = reinterpret_cast<float4*>(q.partial + ((size_t)u.c * q.D + d) * RP);
+      // several chunks: fp32 partial [chunk][d][RP], then the last arriving unit sums
+      // the expert's partials in chunk order and writes the gradient
+      for (int dd = et; dd < C::BN; dd += C::EPI_THREADS) {
+        if (d0 + dd >= q.D) continue;
+        float4* dst = reinterpret_cast<float4*>(q.partial + ((size_t)u.c * q.D + d0 + dd) * RP);
 #pragma unroll
         for (int i = 0; i < RP / 4; ++i)
-          dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          dst[i] = make_float4(stg[(4 * i) * C::ST_LD + dd], stg[(4 * i + 1) * C::ST_LD + dd],
+                               stg[(4 * i + 2) * C::ST_LD + dd], stg[(4 * i + 3) * C::ST_LD + dd]);
       }
       __threadfence();
       named_bar(1, C::EPI_THREADS);
@@ -322,34 +345,53 @@ __global__ void __launch_bounds__(192, 1)
         *last_flag = last;
       }
       named_bar(1, C::EPI_THREADS);
-      if (*last_flag && d < q.D) {
-        float acc[RP];
+      if (*last_flag) {
+        for (int dd = et; dd < C::BN; dd += C::EPI_THREADS) {
+          const int dg = d0 + dd;
+          if (dg >= q.D) continue;
+          float acc[RP];
 #pragma unroll
-        for (int i = 0; i < RP; ++i) acc[i] = 0.f;
-        for (int cc = c0; cc < c1; ++cc) {
-          const float4* src = reinterpret_cast<const float4*>(q.partial + ((size_t)cc * q.D + d) * RP);
+          for (int i = 0; i < RP; ++i) acc[i] = 0.f;
+          for (int cc = c0; cc < c1; ++cc) {
+            const float4* src = reinterpret_cast<const float4*>(q.partial + ((size_t)cc * q.D + dg) * RP);
 #pragma unroll
-          for (int i = 0; i < RP / 4; ++i) {
-            const float4 x = __ldcg(src + i);
-            acc[4 * i] += x.x;
-            acc[4 * i + 1] += x.y;
-            acc[4 * i + 2] += x.z;
-            acc[4 * i + 3] += x.w;
+            for (int i = 0; i < RP / 4; ++i) {
+              const float4 x = __ldcg(src + i);
+              acc[4 * i] += x.x;
+              acc[4 * i + 1] += x.y;
+              acc[4 * i + 2] += x.z;
+              acc[4 * i + 3] += x.w;
+            }
+          }
+          if (q.transpose) {
+#pragma unroll
+            for (int i = 0; i < RP; ++i)
+              if (i < p.r) q.out[((size_t)ch.e * p.r + i) * q.D + dg] = __float2bfloat16_rn(p.scale * acc[i]);
+          } else {
+#pragma unroll
+            for (int g = 0; g < RP / 8; ++g)
+              if (g * 8 < p.r) {
+                float v[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) v[x] = acc[8 * g + x];
+                store_bf16x8(q.out + ((size_t)ch.e * q.D + dg) * p.r + 8 * g, p.scale, v);
+              }
           }
         }
-        wgrad_store<RP>(q, p.r, p.scale, ch.e, d, acc);
       }
+      named_bar(1, C::EPI_THREADS);                 // the flag and staging are rewritten next
     }
-    // gradients of experts without rows are zero: after the units, so the scan never
-    // holds up the accumulators; CTA b takes experts b, b + grid, ...
+    // gradients of experts without rows are zero (D * r contiguous values in either
+    // orientation): after the units, so the scan never holds up the accumulators;
+    // CTA b takes experts b, b + grid, ...
     for (int e = blockIdx.x; e < p.E; e += gridDim.x) {
       if (p.chunk_start[e + 1] != p.chunk_start[e]) continue;
+      const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int prob = 0; prob < p.n_problems; ++prob) {
         const WgradProblem& q = p.pr[prob];
-        float z[RP];
-#pragma unroll
-        for (int j = 0; j < RP; ++j) z[j] = 0.f;
-        for (int d = et; d < q.D; d += C::EPI_THREADS) wgrad_store<RP>(q, p.r, p.scale, e, d, z);
+        const int64_t n8 = (int64_t)q.D * p.r / 8;
+        for (int64_t i = et; i < n8; i += C::EPI_THREADS)
+          store_bf16x8(q.out + (size_t)e * q.D * p.r + i * 8, 0.f, z);
       }
     }
   }
