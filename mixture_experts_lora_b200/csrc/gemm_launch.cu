@@ -303,11 +303,10 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
     const bool okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, C0::BN / 64)
                        : encode2d(&tm[j], jb.big, P, (uint64_t)jb.D, C0::BK, 64);
     // Small [P, ld_small] seen as [ld_small / 8 groups][P rows][8 columns]: a box of
-    // BK rows x 16 groups (the MMA's 128 rank rows) lands group-major, groups past
-    // ld_small reading as zero
+    // BK rows x rp / 8 groups lands group-major, groups past ld_small reading as zero
     const uint64_t sd[3] = {8, P, (uint64_t)jb.ld_small / 8};
     const uint64_t ss[2] = {(uint64_t)jb.ld_small * 2, 16};
-    const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)C0::BM / 8};
+    const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)g.rp / 8};
     if (!okb || !encode(&tm[2 + j], jb.small, 3, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     WgradProblem& q = wp.pr[j];

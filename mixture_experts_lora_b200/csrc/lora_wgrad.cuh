@@ -12,8 +12,9 @@
 // computable at the same point of the backward).  Units are (problem, row chunk
 // of one expert, 256-wide column tile of Big); a persistent CTA walks its units
 // with one continuous TMA/MMA pipeline computing G^T for the tile:
-//   M = 128 rank rows (Small^T, MN-major, no swizzle: groups of 8 rank columns;
-//       the TMA view has 16 groups, those past Small's width read as zero),
+//   M = 128 rank rows (Small^T, MN-major, no swizzle: 16 groups of 8 rank columns;
+//       each stage copies the RP / 8 groups of Small's width (those past it read as
+//       zero), the rest of the 16 stay zero from the kernel's start),
 //   N = 256 columns of Big (MN-major, 128-byte swizzle, four 64-column atoms),
 //   K = rows of the chunk, 64 per stage,
 // one TMA copy per operand and stage.  A rank of at most 32 uses a quarter of M,
@@ -73,6 +74,7 @@ struct WgradCfg {
   static constexpr int ATOM = BK * 128;                   // 8 KB: 64 Big columns x BK rows
   static constexpr int B_BYTES = (BN / 64) * ATOM;        // 32 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMALL_COPY = (RP / 8) * SMALL_NG;  // bytes of Small copied per stage
   static constexpr int STAGES = 4;
   static constexpr int ST_LD = BN + 4;                    // fp32 staging row (rank j), padded
   static constexpr int STG_BYTES = RP * ST_LD * 4;
@@ -154,6 +156,11 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
+  // the rank groups past RP of every stage's Small^T tile are zero for the whole launch
+  for (int s = 0; s < C::STAGES; ++s)
+    for (int i = threadIdx.x; i < (C::A_BYTES - C::SMALL_COPY) / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::SMALL_COPY)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -182,9 +189,9 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           const int r0 = ch.row0 + ks * C::BK;
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-          // Small [BK rows][128 rank columns as 16 groups of 8]: groups past its width
-          // read as zero (MN-major, no swizzle: core matrices of 8 rows x 8 columns)
+          mbar_arrive_expect_tx(fb, C::SMALL_COPY + C::B_BYTES);
+          // Small [BK rows][RP / 8 groups of 8 rank columns] (MN-major, no swizzle: core
+          // matrices of 8 rows x 8 columns)
           tma_load_3d(ts, fb, sa, 0, r0, 0);
           if constexpr (C::V) {
             tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
