@@ -327,6 +327,22 @@ __device__ __forceinline__ void bulk_wait() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Every kernel of the library is launched with programmatic stream serialization: it
+// may be scheduled while its predecessor in the stream drains (its prologue - barrier
+// set-up, TMEM allocation, descriptor prefetch - overlaps that tail).  pdl_wait()
+// blocks until the predecessors have completed and their writes are visible; each
+// kernel calls it before its first global-memory access, read or write, and then
+// lets its own dependents be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_begin() {
+  pdl_wait();
+  pdl_launch_dependents();
+}
+
 // ---------------------------------------------------------------- misc
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar(int id, int n) {

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_begin();          // predecessors' outputs visible from here
   const int per_e = p.n_mt * p.n_nt;
   const int total = p.E * per_e;
 

@@ -97,20 +97,9 @@ cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap* maps, c
   const int64_t tiles = (int64_t)g.max_gchunks * p.n_ftiles;
   const int pairs_max = g.num_sms / 2 > 0 ? g.num_sms / 2 : 1;
   const int pairs = (int)(tiles < pairs_max ? (tiles > 0 ? tiles : 1) : pairs_max);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(320, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   ProfScope ps(kind, s);
-  st = cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], p);
+  st = launch_pdl(kern, dim3(2 * pairs), dim3(320), C::SMEM_BYTES, s, 2, maps[0], maps[1], maps[2],
+                  maps[3], p);
   if (st != cudaSuccess) return st;
   return cudaGetLastError();
 }
@@ -194,7 +183,7 @@ static cudaError_t rows_gather_rp(const GemmShape& g, const CUtensorMap* tl, con
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
   ProfScope ps(K_ROWS_GATHER, s);
-  kern<<<g.max_row_tiles, RG_THREADS, C::SMEM_BYTES, s>>>(tl[0], rp_);
+  if (cudaError_t le_ = launch_pdl(kern, dim3(g.max_row_tiles), dim3(RG_THREADS), C::SMEM_BYTES, s, 1, tl[0], rp_); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -209,7 +198,7 @@ static cudaError_t rows_swiglu_rp(const GemmShape& g, const CUtensorMap* tl, con
   int grid = g.num_sms * C::CTAS_PER_SM;
   if (grid > kRowsMaxCtas) grid = kRowsMaxCtas;
   ProfScope ps(MODE == ROWS_SWIGLU ? K_ROWS_SWIGLU : K_ROWS_SWIGLU_BWD, s);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tl[0], tl[1], tl[2], rp_);
+  if (cudaError_t le_ = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, 1, tl[0], tl[1], tl[2], rp_); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -283,7 +272,7 @@ static cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const Wgr
   // at least one CTA per SM: the zero fill of experts without rows runs in every CTA
   const int grid = (int)(units > 0 && units < g.num_sms ? units : g.num_sms);
   ProfScope ps(K_WGRAD, s);
-  kern<<<grid, 192, C::SMEM_BYTES, s>>>(tm[0], tm[1], tm[2], tm[3], wp);
+  if (cudaError_t le_ = launch_pdl(kern, dim3(grid), dim3(192), C::SMEM_BYTES, s, 1, tm[0], tm[1], tm[2], tm[3], wp); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -345,7 +334,7 @@ static cudaError_t expert_dw_launch(int kind, const CUtensorMap* tm, const DwPar
   const int64_t total = (int64_t)p.E * p.n_mt * p.n_nt;
   const int grid = (int)(total < num_sms ? total : num_sms);
   ProfScope ps(kind, s);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(tm[0], tm[1], tm[2], p);
+  if (cudaError_t le_ = launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, s, 1, tm[0], tm[1], tm[2], p); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(320, 1)
   cluster_sync();       // barriers of both CTAs exist before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_begin();          // predecessors' outputs (chunk tables, operands) visible from here
   const int total = (*p.n_chunks) * p.n_ftiles;
 
   if (warp == 0) {

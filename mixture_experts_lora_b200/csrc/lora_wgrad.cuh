@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_begin();          // predecessors' outputs visible from here
   const int nch = *p.n_chunks;
   const int total = nch * (p.pr[0].n_dtiles + (p.n_problems > 1 ? p.pr[1].n_dtiles : 0));
 

@@ -39,6 +39,7 @@ template <int RP, bool L_MN>
 __global__ void __launch_bounds__(RG_THREADS)
     rows_gather_kernel(const __grid_constant__ CUtensorMap tmL, const RowsParams p) {
   using C = RowsGatherCfg<RP>;
+  pdl_begin();          // predecessors' outputs (tile table, rows) visible from here
   const int tile = blockIdx.x;
   if (tile >= *p.n_tiles) return;
   const TileInfo ti = p.tiles[tile];

@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(RowsSwigluCfg<MODE, RP>::THREADS, RowsSwigluCf
     rows_swiglu_kernel(const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmGU,
                        const __grid_constant__ CUtensorMap tmDH, const RowsParams p) {
   using C = RowsSwigluCfg<MODE, RP>;
+  pdl_begin();          // predecessors' outputs (tile table, rows) visible from here
   constexpr int S = C::STAGES;
   const int n_it = (p.n + C::BK - 1) / C::BK;
   const int64_t U = (int64_t)(*p.n_tiles) * n_it;

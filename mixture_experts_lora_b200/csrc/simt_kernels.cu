@@ -53,6 +53,7 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 
 __global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
                                   int32_t* __restrict__ ids, float* __restrict__ wout) {
+  pdl_begin();
   extern __shared__ float s_logits[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
@@ -98,7 +99,7 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
   const int64_t blocks = (T + warps - 1) / warps;
   const size_t smem = (size_t)warps * E * sizeof(float);
   ProfScope ps(K_ROUTE, s);
-  route_topk_kernel<<<(unsigned)blocks, warps * 32, smem, s>>>(logits, T, E, k, ids, w);
+  if (cudaError_t le_ = launch_pdl(route_topk_kernel, dim3((unsigned)blocks), dim3(warps * 32), smem, s, 1, logits, T, E, k, ids, w); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -121,6 +122,7 @@ constexpr int kPermWarps = kPermThreads / 32;
 __global__ void __launch_bounds__(kPermThreads)
     permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
                         int32_t* __restrict__ hist, int* err) {
+  pdl_begin();
   extern __shared__ int s_hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
@@ -138,6 +140,7 @@ __global__ void __launch_bounds__(kPermThreads)
 __global__ void __launch_bounds__(1024)
     permute_scan_kernel(int32_t* __restrict__ hist, int n_chunks, int E, int64_t P,
                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  pdl_begin();
   __shared__ int s_tot[1024];
   __shared__ int s_warp[33];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -178,6 +181,7 @@ __global__ void __launch_bounds__(kPermThreads)
     permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
                            const int32_t* __restrict__ base, int32_t* __restrict__ sorted_pairs,
                            int32_t* __restrict__ pair_pos) {
+  pdl_begin();
   extern __shared__ int s_cnt[];   // [kPermWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_cnt[i] = 0;
@@ -213,13 +217,13 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
   const int n_chunks = (int)((P + kPermuteChunk - 1) / kPermuteChunk);
   if (n_chunks > 0) {
     ProfScope ps(K_PERM_HIST, s);
-    permute_hist_kernel<<<n_chunks, kPermThreads, E * sizeof(int), s>>>(ids, P, E, n_chunks, hist, err);
+    if (cudaError_t le_ = launch_pdl(permute_hist_kernel, dim3(n_chunks), dim3(kPermThreads), E * sizeof(int), s, 1, ids, P, E, n_chunks, hist, err); le_ != cudaSuccess) return le_;
     cudaError_t st = cudaGetLastError();
     if (st != cudaSuccess) return st;
   }
   {
     ProfScope ps(K_PERM_SCAN, s);
-    permute_scan_kernel<<<1, 1024, 0, s>>>(hist, n_chunks, E, P, counts, offsets);
+    if (cudaError_t le_ = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, 1, hist, n_chunks, E, P, counts, offsets); le_ != cudaSuccess) return le_;
   }
   cudaError_t st = cudaGetLastError();
   if (st != cudaSuccess || n_chunks == 0) return st;
@@ -229,8 +233,8 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
     if (st != cudaSuccess) return st;
   }
   ProfScope ps(K_PERM_SCATTER, s);
-  permute_scatter_kernel<<<n_chunks, kPermThreads, smem, s>>>(ids, P, E, n_chunks, hist, sorted_pairs,
-                                                              pair_pos);
+  if (cudaError_t le_ = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads), smem, s, 1, ids, P, E, n_chunks, hist, sorted_pairs,
+                                                              pair_pos); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -245,6 +249,7 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
                                     TileInfo* __restrict__ chunks, int* __restrict__ n_chunks,
                                     int32_t* __restrict__ chunk_start, int* __restrict__ zero,
                                     int n_zero) {
+  pdl_begin();
   for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
   __shared__ int s_warp[33];
   const int e = threadIdx.x;
@@ -296,9 +301,9 @@ cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, Ti
                                 int chunk_rows, TileInfo* chunks, int* n_chunks,
                                 int32_t* chunk_start, int* zero, int n_zero, cudaStream_t s) {
   ProfScope ps(K_TABLES, s);
-  build_tables_kernel<<<1, 1024, 0, s>>>(offsets, E, tile_rows, tiles, n_tiles, gchunk_rows, gchunks,
+  if (cudaError_t le_ = launch_pdl(build_tables_kernel, dim3(1), dim3(1024), 0, s, 1, offsets, E, tile_rows, tiles, n_tiles, gchunk_rows, gchunks,
                                          n_gchunks, chunk_rows, chunks, n_chunks, chunk_start,
-                                         zero, n_zero);
+                                         zero, n_zero); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -325,6 +330,7 @@ static unsigned grid_for(int64_t work, int threads) {
 __global__ void combine_kernel(const uint4* __restrict__ ys, const float* __restrict__ w,
                                const int32_t* __restrict__ pos, int64_t T, int k, int vpr,
                                uint4* __restrict__ y) {
+  pdl_begin();
   const int64_t total = T * vpr;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -356,9 +362,9 @@ cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_
   if (T == 0) return cudaSuccess;
   const int vpr = m / 8;
   ProfScope ps(K_COMBINE, s);
-  combine_kernel<<<grid_for(T * vpr, 256), 256, 0, s>>>(reinterpret_cast<const uint4*>(ysorted), w,
+  if (cudaError_t le_ = launch_pdl(combine_kernel, dim3(grid_for(T * vpr, 256)), dim3(256), 0, s, 1, reinterpret_cast<const uint4*>(ysorted), w,
                                                         pair_pos, T, k, vpr,
-                                                        reinterpret_cast<uint4*>(y));
+                                                        reinterpret_cast<uint4*>(y)); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
@@ -383,6 +389,7 @@ __global__ void __launch_bounds__(256)
                            const int32_t* __restrict__ ids, const float* __restrict__ w,
                            const int32_t* __restrict__ pos, int64_t T, int k, int E, int vpr,
                            float* __restrict__ dlogits) {
+  pdl_begin();
   __shared__ float s_dw[32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tpb = k >= 8 ? 1 : 8 / k;                 // tokens per block
@@ -423,15 +430,16 @@ cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const
   if (T == 0) return cudaSuccess;
   const int tpb = k >= 8 ? 1 : 8 / k;
   ProfScope ps(K_ROUTER_BWD, s);
-  router_backward_kernel<<<(unsigned)((T + tpb - 1) / tpb), 256, 0, s>>>(
+  if (cudaError_t le_ = launch_pdl(router_backward_kernel, dim3((unsigned)((T + tpb - 1) / tpb)), dim3(256), 0, s, 1, 
       reinterpret_cast<const uint4*>(dY), reinterpret_cast<const uint4*>(ys), ids, w, pos, T, k, E,
-      m / 8, dlogits);
+      m / 8, dlogits); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ pad
 __global__ void pad3_kernel(const uint16_t* __restrict__ in, int E, int Ri, int Ci, int Ro, int Co,
                             uint16_t* __restrict__ out) {
+  pdl_begin();
   const int64_t total = (int64_t)E * Ro * Co;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -446,7 +454,7 @@ __global__ void pad3_kernel(const uint16_t* __restrict__ in, int E, int Ri, int 
 cudaError_t launch_pad3(const uint16_t* in, int E, int Ri, int Ci, int Ro, int Co, uint16_t* out,
                         cudaStream_t s) {
   ProfScope ps(K_PAD, s);
-  pad3_kernel<<<grid_for((int64_t)E * Ro * Co, 256), 256, 0, s>>>(in, E, Ri, Ci, Ro, Co, out);
+  if (cudaError_t le_ = launch_pdl(pad3_kernel, dim3(grid_for((int64_t)E * Ro * Co, 256)), dim3(256), 0, s, 1, in, E, Ri, Ci, Ro, Co, out); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
 }
 
