@@ -192,3 +192,33 @@ def test_expert_spanning_several_chunks():
         cpu["logits"][:, 0] += 30.0
     errs, buf = _layer_case(cfg, mutate)
     assert buf.counts.cpu().tolist()[0] == 1500
+
+
+def test_graph_replay_matches_eager_bitwise():
+    # bench.py times CUDA-graph replays of the step (every kernel launched with
+    # programmatic dependent launch): a replay must give the eager results bit for bit
+    cfg = small_config(T=640, m=256, n=128, E=8, k=2, r=16, alpha=16)
+    inp, _ = inputs_on(cfg, seed=11)
+    eager = run_layer(inp, cfg)
+    keys = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU", "save_Xs", "Y_sorted")
+    snap = {k: getattr(eager, k).clone() for k in keys}
+    buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ml.layer_step(inp, cfg.k, cfg.scale, buf)       # warm-up outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            ml.layer_step(inp, cfg.k, cfg.scale, buf)
+        for name in keys:
+            getattr(buf, name).zero_()
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    assert ml.moe_get_device_error() == ml.MOE_OK
+    for k, v in snap.items():
+        a = v.view(torch.int16) if v.dtype == torch.bfloat16 else v
+        b = getattr(buf, k)
+        b = b.view(torch.int16) if b.dtype == torch.bfloat16 else b
+        assert torch.equal(a, b), k
+    del g
