@@ -70,7 +70,8 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than moe_workspace_bytes() */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
   MOE_ERR_DEVICE_INDEX = 5,  /* device-detected: expert id outside [0, E) */
-  MOE_ERR_TIMEOUT = 6        /* device-detected: a bounded wait expired */
+  MOE_ERR_TIMEOUT = 6,       /* device-detected: a bounded wait expired */
+  MOE_ERR_DEVICE_CHECK = 7   /* device-detected: moe_check_permutation() found a broken invariant */
 } moe_status_t;
 
 /* Layer shape.  scale is the LoRA scale c = alpha / r (the caller chooses it). */
@@ -113,6 +114,22 @@ moe_status_t moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k
 moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
                          int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                          int32_t* pair_pos, void* ws, size_t ws_bytes, void* stream);
+
+/* Debug check of a permutation, on the device (the stand-in for a sanitizer run, which
+ * this library's test machines do not offer): every invariant moe_permute() promises.
+ *   offsets[0] = 0, offsets[E] = P, offsets non-decreasing, counts[e] = offsets[e+1] -
+ *   offsets[e]; for every sorted position q: p = sorted_pairs[q] is in [0, P),
+ *   pair_pos[p] = q, q lies in the segment of expert topk_ids[p], and p is larger than
+ *   the pair before it in the same segment (stable order).
+ * Arguments as moe_permute() (all read).  A violation sets MOE_ERR_DEVICE_CHECK in the
+ * device error word (read it with moe_get_device_error()); nothing is written otherwise.
+ * The Python binding runs it after every permutation when the environment variable
+ * MOE_CHECK is set.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+moe_status_t moe_check_permutation(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
+                                   const int32_t* counts, const int32_t* offsets,
+                                   const int32_t* sorted_pairs, const int32_t* pair_pos,
+                                   void* stream);
 
 /* Forward of all experts over their segments (grouped GEMMs, one launch each):
  *   Y_sorted[q] = H[q] W_d[e] + c (H[q] A_d[e]) B_d[e],

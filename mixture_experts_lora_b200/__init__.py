@@ -26,12 +26,14 @@ MOE_ERR_WORKSPACE = 3
 MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_INDEX = 5
 MOE_ERR_TIMEOUT = 6
+MOE_ERR_DEVICE_CHECK = 7
 
 EXPORTED = (
     "moe_workspace_bytes", "moe_route_topk", "moe_permute", "moe_grouped_gemm_lora_fwd",
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
     "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
     "moe_permute_noalloc", "moe_router_backward", "moe_grouped_gemm_full_bwd",
+    "moe_check_permutation",
 )
 
 
@@ -65,6 +67,7 @@ def lib() -> ctypes.CDLL:
         h.moe_route_topk.argtypes = [P, I64, I32, I32, P, P, P]
         h.moe_permute.argtypes = [P, I64, I32, I32, P, P, P, P, P, SZ, P]
         h.moe_permute_noalloc.argtypes = [P, I64, I32, I32, P, P, P, P, P]
+        h.moe_check_permutation.argtypes = [P, I64, I32, I32, P, P, P, P, P]
         h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 16 + [SZ, P]
         h.moe_grouped_gemm_lora_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
         h.moe_grouped_gemm_full_bwd.argtypes = [D] + [P] * 23 + [SZ, P]
@@ -89,9 +92,22 @@ def status_string(status: int) -> str:
     return lib().moe_status_string(int(status)).decode()
 
 
+def debug_checks() -> bool:
+    """True when the environment variable MOE_CHECK is set (and not "0"): every call
+    then synchronises and reads the device error word, and every permutation is
+    checked on the device (moe_check_permutation).  For eager debugging; calls made
+    while a CUDA graph is being captured are not checked."""
+    return os.environ.get("MOE_CHECK", "") not in ("", "0")
+
+
 def _check(fn: str, status: int):
     if status != MOE_OK:
         raise MoEError(fn, status, status_string(status))
+    if debug_checks() and not torch.cuda.is_current_stream_capturing():
+        torch.cuda.synchronize()
+        st = int(lib().moe_get_device_error(_stream()))
+        if st != MOE_OK:
+            raise MoEError(fn, st, status_string(st))
 
 
 def _ptr(t):
@@ -125,6 +141,17 @@ def moe_permute(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, ws, stream
                                             _ptr(offsets), _ptr(sorted_pairs), _ptr(pair_pos),
                                             _ptr(ws), ws.numel() * ws.element_size(),
                                             _stream(stream)))
+    if debug_checks():
+        moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream)
+
+
+def moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream=None):
+    """Device check of every invariant moe_permute promises; a violation sets
+    MOE_ERR_DEVICE_CHECK in the device error word (see moe_get_device_error)."""
+    T, k = topk_ids.shape
+    _check("moe_check_permutation", lib().moe_check_permutation(
+        _ptr(topk_ids), T, k, int(E), _ptr(counts), _ptr(offsets), _ptr(sorted_pairs),
+        _ptr(pair_pos), _stream(stream)))
 
 
 def moe_permute_noalloc(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream=None):
@@ -133,6 +160,8 @@ def moe_permute_noalloc(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, st
     _check("moe_permute_noalloc", lib().moe_permute_noalloc(
         _ptr(topk_ids), T, k, int(E), _ptr(counts), _ptr(offsets), _ptr(sorted_pairs),
         _ptr(pair_pos), _stream(stream)))
+    if debug_checks():
+        moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream)
 
 
 def moe_grouped_gemm_lora_fwd(dims, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,

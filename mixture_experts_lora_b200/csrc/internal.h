@@ -85,6 +85,10 @@ cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, Ti
 cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const int32_t* ids,
                                    const float* w, const int32_t* pos, int64_t T, int k, int E,
                                    int m, float* dlogits, cudaStream_t s);
+// Debug check of moe_permute()'s invariants; sets MOE_ERR_DEVICE_CHECK on a violation.
+cudaError_t launch_check_permutation(const int32_t* ids, int64_t P, int E, const int32_t* counts,
+                                     const int32_t* offsets, const int32_t* sorted_pairs,
+                                     const int32_t* pair_pos, int* err, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_t* pair_pos,
                            int64_t T, int k, int m, uint16_t* y, cudaStream_t s);
 // out [E, Ro, Co] = in [E, Ri, Ci] zero-padded (Ro >= Ri, Co >= Ci)

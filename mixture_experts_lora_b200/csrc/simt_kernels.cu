@@ -324,6 +324,45 @@ static unsigned grid_for(int64_t work, int threads) {
   return (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
 }
 
+// ------------------------------------------------------------------ permutation check
+// Every invariant of the counting sort (debug mode): one thread per sorted position,
+// plus the expert table checked by the first E + 1 threads.
+__global__ void check_permutation_kernel(const int32_t* __restrict__ ids, int64_t P, int E,
+                                         const int32_t* __restrict__ counts,
+                                         const int32_t* __restrict__ offsets,
+                                         const int32_t* __restrict__ sp,
+                                         const int32_t* __restrict__ pos, int* err) {
+  pdl_begin();
+  const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  bool bad = false;
+  if (i0 <= E) {
+    const int e = (int)i0;
+    if (e == 0 && offsets[0] != 0) bad = true;
+    if (e == E && offsets[E] != (int32_t)P) bad = true;
+    if (e < E && (offsets[e + 1] < offsets[e] || counts[e] != offsets[e + 1] - offsets[e])) bad = true;
+  }
+  for (int64_t q = i0; q < P; q += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t p = sp[q];
+    if (p < 0 || p >= P) { bad = true; continue; }
+    if (pos[p] != (int32_t)q) bad = true;
+    const int e = ids[p];
+    if (e < 0 || e >= E || q < offsets[e] || q >= offsets[e + 1]) { bad = true; continue; }
+    if (q > offsets[e] && sp[q - 1] >= p) bad = true;      // stable: ascending pair index
+  }
+  if (bad) report_error(err, MOE_ERR_DEVICE_CHECK);
+}
+
+cudaError_t launch_check_permutation(const int32_t* ids, int64_t P, int E, const int32_t* counts,
+                                     const int32_t* offsets, const int32_t* sorted_pairs,
+                                     const int32_t* pair_pos, int* err, cudaStream_t s) {
+  const int64_t work = P > E + 1 ? P : E + 1;
+  if (cudaError_t le_ = launch_pdl(check_permutation_kernel, dim3(grid_for(work, 256)), dim3(256), 0, s,
+                                   1, ids, P, E, counts, offsets, sorted_pairs, pair_pos, err);
+      le_ != cudaSuccess)
+    return le_;
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ combine
 // y[t, :] = sum_j w[t, j] ysorted[pair_pos[t k + j], :], fp32 over ascending j,
 // one bf16 rounding; w == nullptr means every weight is 1.

@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for s in range(7):
+    for s in range(8):
         assert ml.status_string(s)
     assert ml.status_string(ml.MOE_ERR_WORKSPACE) == "workspace too small"
 
@@ -135,6 +135,24 @@ def test_full_backward_host_validation(L):
     lb = [P(4096)] * 21
     lb[18] = None
     assert L.moe_grouped_gemm_lora_bwd(ctypes.byref(d), *lb, 1 << 30, None) == ml.MOE_ERR_INVALID_ARG
+
+
+def test_check_permutation_host_validation(L):
+    fake = ctypes.c_void_p(256)
+    null = None
+    assert L.moe_check_permutation(fake, 4, 0, 8, fake, fake, fake, fake, null) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_check_permutation(fake, -1, 2, 8, fake, fake, fake, fake, null) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_check_permutation(fake, 4, 2, 8, null, fake, fake, fake, null) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_check_permutation(null, 4, 2, 8, fake, fake, fake, fake, null) == ml.MOE_ERR_INVALID_ARG
+
+
+def test_debug_checks_follow_the_environment(monkeypatch):
+    monkeypatch.delenv("MOE_CHECK", raising=False)
+    assert not ml.debug_checks()
+    monkeypatch.setenv("MOE_CHECK", "0")
+    assert not ml.debug_checks()
+    monkeypatch.setenv("MOE_CHECK", "1")
+    assert ml.debug_checks()
 
 
 def test_router_backward_host_validation(L):

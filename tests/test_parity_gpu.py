@@ -222,3 +222,54 @@ def test_graph_replay_matches_eager_bitwise():
         b = b.view(torch.int16) if b.dtype == torch.bfloat16 else b
         assert torch.equal(a, b), k
     del g
+
+
+def test_check_permutation_accepts_valid_and_flags_broken():
+    T, k, E = 700, 4, 16
+    g = torch.Generator().manual_seed(5)
+    ids, _ = O.route_topk(torch.randn(T, E, generator=g).numpy(), k)
+    d_ids = torch.from_numpy(ids.astype(np.int32)).cuda()
+    P = T * k
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    sp = torch.empty(P, dtype=torch.int32, device="cuda")
+    pos = torch.empty(P, dtype=torch.int32, device="cuda")
+    ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+    ml.moe_permute(d_ids, E, counts, offsets, sp, pos, ws)
+    ml.moe_check_permutation(d_ids, E, counts, offsets, sp, pos)
+    assert ml.moe_get_device_error() == ml.MOE_OK
+
+    def broken(mutate):
+        c, o, s_, p_ = counts.clone(), offsets.clone(), sp.clone(), pos.clone()
+        mutate(c, o, s_, p_)
+        ml.moe_check_permutation(d_ids, E, c, o, s_, p_)
+        return ml.moe_get_device_error()
+
+    off = offsets.cpu().numpy()
+    e = int(np.argmax(np.diff(off)))                       # an expert with at least 2 rows
+    q0 = int(off[e])
+
+    def swap_in_segment(c, o, s_, p_):                     # order inside a segment
+        a, b = s_[q0].item(), s_[q0 + 1].item()
+        s_[q0], s_[q0 + 1] = b, a
+        p_[a], p_[b] = q0 + 1, q0
+
+    def bad_offset(c, o, s_, p_):                          # counts disagree with offsets
+        o[e + 1] += 1
+
+    def bad_inverse(c, o, s_, p_):                         # pair_pos not the inverse
+        p_[0] = (p_[0] + 1) % P
+
+    def out_of_range(c, o, s_, p_):                        # a pair index outside [0, P)
+        s_[5] = P + 3
+
+    for mutate in (swap_in_segment, bad_offset, bad_inverse, out_of_range):
+        assert broken(mutate) == ml.MOE_ERR_DEVICE_CHECK, mutate.__name__
+
+
+def test_layer_with_debug_checks(monkeypatch):
+    monkeypatch.setenv("MOE_CHECK", "1")
+    cfg = CONFIGS["tiny"]
+    inp, cpu = inputs_on(cfg)
+    buf = run_layer(inp, cfg)                              # every call checked on the device
+    check_full_parity(buf, cpu, cfg)
