@@ -240,7 +240,8 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
 
 // ------------------------------------------------------------------ tile tables
 // From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
-// experts (grouped GEMMs), and row chunks of `chunk_rows` rows (adapter
+// experts (row kernels), token chunks of at most `gchunk_rows` rows (grouped
+// GEMMs), and row chunks of `chunk_rows` rows (adapter
 // gradients) with chunk_start[e] = first chunk of expert e.
 __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, int tile_rows,
                                     TileInfo* __restrict__ tiles, int* __restrict__ n_tiles,
@@ -257,13 +258,28 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
   if (e < E) { lo = offsets[e]; hi = offsets[e + 1]; }
   const int cnt = hi - lo;
   int total;
-  // row tiles of exactly tile_rows rows (the last one of an expert may be short)
-  const int nt = (cnt + tile_rows - 1) / tile_rows;
-  const int t0 = block_exclusive_scan_1024(nt, s_warp, &total);
-  for (int i = 0; i < nt; ++i) {
+  // row tiles of tile_rows rows: every expert's full tiles in expert order, then its
+  // short last tile in four size classes from the largest to the smallest (expert
+  // order inside a class).  A launch of one CTA per tile is dispatched in tile
+  // order, breadth-first over the SMs, so the smallest tiles become the CTAs that
+  // share an SM with two others.
+  const int nfull = cnt / tile_rows, rag = cnt - nfull * tile_rows;
+  const int f0 = block_exclusive_scan_1024(nfull, s_warp, &total);
+  for (int i = 0; i < nfull; ++i) {
     TileInfo ti;
-    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = min(hi, lo + (i + 1) * tile_rows); ti.pad = 0;
-    tiles[t0 + i] = ti;
+    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = lo + (i + 1) * tile_rows; ti.pad = 0;
+    tiles[f0 + i] = ti;
+  }
+  for (int cls = 3; cls >= 0; --cls) {
+    const int in = (rag > 0 && (rag * 4) / tile_rows == cls) ? 1 : 0;
+    int ctot;
+    const int r0 = block_exclusive_scan_1024(in, s_warp, &ctot);
+    if (in) {
+      TileInfo ti;
+      ti.e = e; ti.row0 = lo + nfull * tile_rows; ti.row_end = hi; ti.pad = 0;
+      tiles[total + r0] = ti;
+    }
+    total += ctot;
   }
   if (threadIdx.x == 0) *n_tiles = total;
   // token chunks: ceil(cnt / gchunk_rows) chunks of equal size rounded up to 16
