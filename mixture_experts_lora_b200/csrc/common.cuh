@@ -38,6 +38,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// tanh by the hardware approximation (PTX tanh.approx.f32, one special-function
+// op, relative error about 2^-11).  The SwiGLU kernels take the logistic sigmoid
+// through s(x) = (1 + tanh(x / 2)) / 2: one such op per element instead of an
+// exponential and a reciprocal, which bounded their worker warps.  The error stays
+// well below the bf16 rounding of the outputs.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) {
   return __uint_as_float(v << 16);
 }

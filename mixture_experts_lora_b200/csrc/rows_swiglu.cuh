@@ -113,30 +113,37 @@ __global__ void __launch_bounds__(RowsSwigluCfg<MODE, RP>::THREADS, RowsSwigluCf
         uint4* pg = reinterpret_cast<uint4*>(st + off);
         uint4* pu = reinterpret_cast<uint4*>(st + C::TILE_BYTES + off);
         const int q = inf.x + r;
-        const bool valid = q < inf.y && col < p.n;
+        // rows past the tile's end are left as loaded: their rank-r results are never
+        // stored.  Columns past n are computed: with dH (or u) read as zero there they
+        // become the zeros the rank-r product needs against the adapter's next columns.
+        if (q >= inf.y) continue;
+        const bool in_n = col < p.n;
         float g[8], uu[8];
         unpack8(*pg, g);
         unpack8(*pu, uu);
         if constexpr (MODE == ROWS_SWIGLU) {
           float h[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) h[i] = __fdividef(g[i], 1.0f + __expf(-g[i])) * uu[i];
+          for (int i = 0; i < 8; ++i) {
+            const float a = 0.5f * g[i];          // silu(g) = a (1 + tanh(a)), a = g / 2
+            h[i] = fmaf(a, tanh_approx(a), a) * uu[i];
+          }
           const uint4 o = pack8(h);
           *pg = o;
-          if (valid) *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.n + col) = o;
+          if (in_n) *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * p.n + col) = o;
         } else {
           float d[8], dg[8], du[8];
           unpack8(*reinterpret_cast<const uint4*>(st + 2 * C::TILE_BYTES + off), d);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float sg = __fdividef(1.0f, 1.0f + __expf(-g[i]));
+            const float sg = fmaf(0.5f, tanh_approx(0.5f * g[i]), 0.5f);   // sigmoid(g)
             dg[i] = d[i] * uu[i] * sg * (1.0f + g[i] * (1.0f - sg));
             du[i] = d[i] * g[i] * sg;
           }
           const uint4 o0 = pack8(dg), o1 = pack8(du);
           *pg = o0;
           *pu = o1;
-          if (valid) {
+          if (in_n) {
             *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + col) = o0;
             *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * p.n + p.n + col) = o1;
           }
