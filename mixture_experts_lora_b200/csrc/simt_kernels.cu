@@ -8,25 +8,26 @@
 namespace moe {
 
 // ------------------------------------------------------------------ block scan
-// Exclusive scan of one int per thread over a block of up to 1024 threads;
-// *total_out receives the block total.  s_warp holds 33 ints.
-__device__ __forceinline__ int block_exclusive_scan_1024(int v, int* s_warp, int* total_out) {
+// Exclusive scan of one value per thread (int or 64-bit) over a block of up to 1024
+// threads; *total_out receives the block total.  s_warp holds 33 values.
+template <class T>
+__device__ __forceinline__ T block_exclusive_scan_1024(T v, T* s_warp, T* total_out) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
+  T incl = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, off);
+    const T u = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += u;
   }
   __syncthreads();
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
-    int inc2 = w;
+    const T w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : T(0);
+    T inc2 = w;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, inc2, off);
+      const T u = __shfl_up_sync(0xffffffffu, inc2, off);
       if (lane >= off) inc2 += u;
     }
     s_warp[lane] = inc2 - w;
@@ -253,6 +254,7 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
   pdl_begin();
   for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
   __shared__ int s_warp[33];
+  __shared__ unsigned long long s_warp64[33];
   const int e = threadIdx.x;
   int lo = 0, hi = 0;
   if (e < E) { lo = offsets[e]; hi = offsets[e + 1]; }
@@ -270,16 +272,22 @@ __global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, 
     ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = lo + (i + 1) * tile_rows; ti.pad = 0;
     tiles[f0 + i] = ti;
   }
-  for (int cls = 3; cls >= 0; --cls) {
-    const int in = (rag > 0 && (rag * 4) / tile_rows == cls) ? 1 : 0;
-    int ctot;
-    const int r0 = block_exclusive_scan_1024(in, s_warp, &ctot);
-    if (in) {
-      TileInfo ti;
-      ti.e = e; ti.row0 = lo + nfull * tile_rows; ti.row_end = hi; ti.pad = 0;
-      tiles[total + r0] = ti;
+  {
+    // one scan of the four class flags packed 16 bits apart (E <= 1024 per class)
+    const int cls = rag > 0 ? 3 - (rag * 4) / tile_rows : -1;   // 0: largest class
+    unsigned long long ctot;
+    const unsigned long long r = block_exclusive_scan_1024(
+        cls >= 0 ? 1ull << (16 * cls) : 0ull, s_warp64, &ctot);
+    int base = total;
+    for (int c = 0; c < 4; ++c) {
+      if (c == cls) {
+        TileInfo ti;
+        ti.e = e; ti.row0 = lo + nfull * tile_rows; ti.row_end = hi; ti.pad = 0;
+        tiles[base + (int)((r >> (16 * c)) & 0xffffu)] = ti;
+      }
+      base += (int)((ctot >> (16 * c)) & 0xffffu);
     }
-    total += ctot;
+    total = base;
   }
   if (threadIdx.x == 0) *n_tiles = total;
   // token chunks: ceil(cnt / gchunk_rows) chunks of equal size rounded up to 16
