@@ -437,25 +437,43 @@ def run_ours(args, cfg):
         "ms_per_launch": rb_ms, "algorithmic_bytes": rb_bytes,
         "achieved": rb_bytes / (rb_ms / 1e3) / 1e9, "unit": "GB/s"}
 
+    def extra_ms(fn, n):
+        """Mean device time of fn over n runs, L2 flushed before each outside the events:
+        one captured CUDA graph replayed like the timed steps (host launches with
+        --no-graph)."""
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        gph = None
+        if not args.no_graph:
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                fn()
+            gph.replay()
+            torch.cuda.synchronize()
+        xevs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n)]
+        for a, b in xevs:
+            flush.zero_()
+            a.record(stream)
+            if gph is not None:
+                gph.replay()
+            else:
+                fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        del gph
+        return statistics.mean(a.elapsed_time(b) for a, b in xevs)
+
     # the shared expert (dense MLP + LoRA on every token, NEXT-4): the layer with one
     # expert at the same token count and dimensions
     from moe_inputs import LayerConfig
     scfg = LayerConfig("shared_expert", T=cfg.T, m=cfg.m, n=cfg.n, E=1, k=1, r=cfg.r, alpha=cfg.alpha)
     sinp = generate(scfg, seed=7, device=dev)
     sbuf = ml.alloc_buffers(scfg.T, scfg.m, scfg.n, 1, 1, scfg.r, scfg.scale, device=dev)
-    for _ in range(3):
-        ml.shared_expert_step(sinp, scfg.scale, sbuf)
-    se_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(min(args.steps, 50))]
-    for a, b in se_evs:
-        flush.zero_()
-        a.record(stream)
-        ml.shared_expert_step(sinp, scfg.scale, sbuf)
-        b.record(stream)
-    torch.cuda.synchronize()
+    se_ms = extra_ms(lambda: ml.shared_expert_step(sinp, scfg.scale, sbuf), min(args.steps, 50))
     if ml.moe_get_device_error() != ml.MOE_OK:
         raise SystemExit("device error in the shared-expert timing")
-    se_ms = statistics.mean(a.elapsed_time(b) for a, b in se_evs)
     se_flops = acc.flops_step(scfg.T, scfg.m, scfg.n, 1, scfg.r)
     extras["shared_expert"] = {
         "what": f"dense SwiGLU MLP + LoRA on all {scfg.T} tokens, fwd+bwd (NEXT-4 row; not part of the step)",
@@ -477,22 +495,12 @@ def run_ours(args, cfg):
         ad.B_d.copy_(inp["B_d"])
         sp_inp = ad.layer_inputs(inp)
         sp_buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, 2 * cfg.r, cfg.scale, device=dev)
-        for _ in range(3):
-            ml.layer_step(sp_inp, cfg.k, cfg.scale, sp_buf)
-        sp_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(min(args.steps, 50))]
-        for a, b in sp_evs:
-            flush.zero_()
-            a.record(stream)
-            ml.layer_step(sp_inp, cfg.k, cfg.scale, sp_buf)
-            b.record(stream)
-        torch.cuda.synchronize()
+        sp_ms = extra_ms(lambda: ml.layer_step(sp_inp, cfg.k, cfg.scale, sp_buf), min(args.steps, 50))
         if ml.moe_get_device_error() != ml.MOE_OK:
             raise SystemExit("device error in the separate-adapter timing")
-        sp_ms = statistics.mean(a.elapsed_time(b) for a, b in sp_evs)
         extras["separate_gate_up_adapters"] = {
-            "what": f"the step with separate gate and up adapters of rank {cfg.r} (fused rank {2 * cfg.r}, "
-                    "host launches; NEXT-2 row)",
+            "what": f"the step with separate gate and up adapters of rank {cfg.r} (fused rank {2 * cfg.r}; "
+                    "NEXT-2 row)",
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
 
@@ -505,17 +513,7 @@ def run_ours(args, cfg):
         ml.layer_forward(inp, cfg.k, cfg.scale, buf)
         ml.layer_backward_full(inp, inp["dY"], cfg.k, cfg.scale, buf, dWg, dWd, adapters=False)
 
-    for _ in range(3):
-        fft_step()
-    ft_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(min(args.steps, 50))]
-    for a, b in ft_evs:
-        flush.zero_()
-        a.record(stream)
-        fft_step()
-        b.record(stream)
-    torch.cuda.synchronize()
-    ft_ms = statistics.mean(a.elapsed_time(b) for a, b in ft_evs)
+    ft_ms = extra_ms(fft_step, min(args.steps, 50))
     # the two weight-gradient kernels, timed on their own launches in a few more steps
     ml.moe_profile_select(["gemm_dw_gu", "gemm_dw_d"])
     ml.moe_profile_enable(True)
