@@ -95,13 +95,18 @@ __global__ void __launch_bounds__(RG_THREADS)
         if (p.w != nullptr) wrow[j] = p.w[pr];
       }
     }
+    // Rows past the tile's end are not copied: each MMA row depends on its own A row
+    // only, and the rank-r rows of those rows are never stored.  Columns past K of a
+    // real row are zero-filled (the adapter chunk is zero there, and 0 x 0 must not
+    // meet stale non-finite bits).
     auto issue = [&](int it) {
       uint8_t* st = smem + (it % RG_STAGES) * C::TILE_BYTES;
       const int col = it * C::BK + cv * 8;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        if (qrow[j] < 0) continue;
         const int r = rb + 32 * j;
-        const bool v = qrow[j] >= 0 && col < p.K;
+        const bool v = col < p.K;
         // K-major, 128-byte swizzle: 16-byte group cv of row r lands at group cv ^ (r & 7)
         cp_async_16(smem_u32(st + r * 128 + ((cv ^ (r & 7)) << 4)),
                     v ? (const void*)(srow[j] + col) : (const void*)p.src, v ? 16u : 0u);
@@ -128,6 +133,7 @@ __global__ void __launch_bounds__(RG_THREADS)
       const int col = it * C::BK + cv * 8;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        if (qrow[j] < 0) continue;
         const int r = rb + 32 * j;
         uint4* sp = reinterpret_cast<uint4*>(st + r * 128 + ((cv ^ (r & 7)) << 4));
         uint4 v = *sp;
@@ -139,7 +145,7 @@ __global__ void __launch_bounds__(RG_THREADS)
           v = pack8(x);
           *sp = v;
         }
-        if (qrow[j] >= 0 && col < p.K && p.rows_out != nullptr)
+        if (col < p.K && p.rows_out != nullptr)
           *reinterpret_cast<uint4*>(p.rows_out + (size_t)qrow[j] * p.K + col) = v;
       }
       mbar_arrive(smem_u32(&sfull[it % RG_STAGES]));
