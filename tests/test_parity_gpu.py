@@ -142,6 +142,23 @@ def test_hot_expert_and_empty_experts():
     assert counts[3] == 300 and counts[5:].sum() == 0
 
 
+def test_every_tile_size_class():
+    # Expert row counts that give every kind of 128-row tile: exact multiples of 128
+    # (no short tile), a short tile in each of the four size classes the row kernels
+    # order their tiles by (rows >= 96, 64-95, 32-63, < 32), and an empty expert.  n = 96
+    # also leaves the SwiGLU kernels a partial 64-column stage.
+    counts = [128, 256, 100, 70, 40, 10, 0, 230]
+    cfg = small_config(T=sum(counts), m=64, n=96, E=len(counts), k=1, r=16, alpha=16)
+    owner = np.repeat(np.arange(len(counts)), counts)
+    owner = owner[np.random.default_rng(3).permutation(len(owner))]
+
+    def mutate(cpu):
+        cpu["logits"][torch.arange(cfg.T), torch.from_numpy(owner)] += 30.0
+    errs, buf = _layer_case(cfg, mutate)
+    assert buf.counts.cpu().tolist() == counts
+    print(errs)
+
+
 def test_tied_logits_route_to_lowest_indices():
     cfg = small_config(T=64, m=64, n=32, E=6, k=2, r=8, alpha=16)
 
