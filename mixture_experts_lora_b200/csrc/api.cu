@@ -47,9 +47,26 @@ int device_sms() {
 
 inline int rank_padded(int r) { return r <= 16 ? 16 : 32; }
 
-// Row chunk of the adapter-gradient kernel: one chunk covers a whole expert at
-// the shapes served here, so most experts need no second reduction pass.
-inline int64_t chunk_rows_for(int64_t) { return 1024; }
+// Row chunk of the adapter-gradient kernel.  An expert cut into several chunks
+// needs fp32 partials and a last-arriver sum per 256-column unit, and the cut
+// leaves remainder chunks of a few rows whose units are all epilogue; one chunk
+// per expert avoids both.  Start at 1024 rows and double while an expert of 1.5x
+// the average rows would still be cut, as long as the first launch keeps at least
+// kMinWgradUnits units (expert chunks x 256-column tiles of both problems) to
+// spread over the SMs.  At T = 32768, k = 8, E = 256 this gives 2048 rows.
+constexpr int64_t kMinWgradUnits = 296;
+inline int64_t chunk_rows_for(const moe_dims_t& d, int64_t P) {
+  const int64_t avg = d.E > 0 ? (P + d.E - 1) / d.E : 0;
+  const int64_t dtiles = (d.n + 255) / 256 + (d.m + 255) / 256;
+  int64_t chunk = 1024;
+  while (chunk < 8192 && avg + avg / 2 > chunk) {
+    const int64_t nxt = 2 * chunk;
+    const int64_t units = (int64_t)d.E * ((avg + nxt - 1) / nxt) * dtiles;
+    if (units < kMinWgradUnits) break;
+    chunk = nxt;
+  }
+  return chunk;
+}
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -87,7 +104,7 @@ Layout make_layout(const moe_dims_t& d) {
   L.rp = rank_padded(d.r);
   L.max_row_tiles = (int)((L.P + kTileRows - 1) / kTileRows) + d.E;
   L.max_gchunks = (int)((L.P + kGemmChunkRows - 1) / kGemmChunkRows) + d.E;
-  L.chunk_rows = (int)chunk_rows_for(L.P);
+  L.chunk_rows = (int)chunk_rows_for(d, L.P);
   L.max_chunks = (int)((L.P + L.chunk_rows - 1) / L.chunk_rows) + d.E;
   L.perm_chunks = (int)((L.P + kPermuteChunk - 1) / kPermuteChunk);
   const bool pad = d.r != L.rp;
