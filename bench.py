@@ -243,11 +243,23 @@ def oracle_setup(cfg, cpu_inp):
 
 
 def pick_sample_tokens(cfg, cpu_inp, W64, target_s, requested):
+    """Tokens per oracle step for a step time of about target_s.  A step costs a fixed
+    part (every touched expert's fp64 weights are streamed whatever its row count) plus
+    a part per token, so a few tokens cost almost as much as a few hundred: the sample
+    doubles from 64 tokens while a timed step stays under half the budget, instead of
+    extrapolating from a handful of tokens."""
     if requested > 0:
         return requested
-    t = time_oracle_sample(cfg, cpu_inp, W64, 0, 8)
-    per_tok = max(t / 8, 1e-4)
-    return int(max(8, min(cfg.T, target_s / per_tok)))
+    n = min(64, cfg.T)
+    time_oracle_sample(cfg, cpu_inp, W64, 0, n)     # first call: thread pool, page-in
+    spent = 0.0
+    while n < cfg.T and spent < 30.0:
+        ts = [time_oracle_sample(cfg, cpu_inp, W64, 0, n) for _ in range(2)]
+        spent += sum(ts)
+        if min(ts) >= target_s / 2:          # the better of two: host timing is noisy
+            break
+        n = min(cfg.T, 2 * n)
+    return n
 
 
 def cpu_baseline(cfg, cpu_inp, requested, target_s=12.0, cap_s=40.0):
