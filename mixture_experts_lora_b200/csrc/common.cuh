@@ -41,8 +41,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // tanh by the hardware approximation (PTX tanh.approx.f32, one special-function
 // op, relative error about 2^-11).  The SwiGLU kernels take the logistic sigmoid
 // through s(x) = (1 + tanh(x / 2)) / 2: one such op per element instead of an
-// exponential and a reciprocal, which bounded their worker warps.  The error stays
-// well below the bf16 rounding of the outputs.
+// exponential and a reciprocal, whose special-function work was part of what bound
+// their worker warps.  The error stays well below the bf16 rounding of the outputs.
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));

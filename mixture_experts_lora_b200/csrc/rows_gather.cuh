@@ -97,8 +97,8 @@ __global__ void __launch_bounds__(RG_THREADS)
     }
     // Rows past the tile's end are not copied: each MMA row depends on its own A row
     // only, and the rank-r rows of those rows are never stored.  Columns past K of a
-    // real row are zero-filled (the adapter chunk is zero there, and 0 x 0 must not
-    // meet stale non-finite bits).
+    // real row are zero-filled: they meet the adapter chunk's zero rows, and stale
+    // shared-memory bits there could be non-finite (NaN x 0 = NaN).
     auto issue = [&](int it) {
       uint8_t* st = smem + (it % RG_STAGES) * C::TILE_BYTES;
       const int col = it * C::BK + cv * 8;
