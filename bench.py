@@ -491,6 +491,29 @@ def run_ours(args, cfg):
         "what": f"dense SwiGLU MLP + LoRA on all {scfg.T} tokens, fwd+bwd (NEXT-4 row; not part of the step)",
         "ms_per_step": se_ms, "tokens_per_s": scfg.T / (se_ms / 1e3),
         "tflops": se_flops / (se_ms / 1e3) / 1e12}
+
+    # the routed layer and the shared expert together, on two streams of one graph, the
+    # way a model with a shared expert runs them, against the two timed alone
+    side = torch.cuda.Stream(device=dev)
+
+    def routed_and_shared():
+        main = torch.cuda.current_stream(dev)
+        side.wait_stream(main)
+        ml.layer_step(inp, cfg.k, cfg.scale, buf)
+        with torch.cuda.stream(side):
+            ml.shared_expert_step(sinp, scfg.scale, sbuf)
+        main.wait_stream(side)
+
+    routed_ms = extra_ms(lambda: ml.layer_step(inp, cfg.k, cfg.scale, buf), min(args.steps, 50))
+    both_ms = extra_ms(routed_and_shared, min(args.steps, 50))
+    if ml.moe_get_device_error() != ml.MOE_OK:
+        raise SystemExit("device error in the routed + shared timing")
+    extras["routed_plus_shared_expert"] = {
+        "what": "the routed layer and the shared expert concurrently on two streams (one graph), "
+                "fwd+bwd; alone they take routed_ms and shared_ms",
+        "ms_per_step": both_ms, "routed_ms": routed_ms, "shared_ms": se_ms,
+        "tokens_per_s": world * cfg.T / (both_ms / 1e3),
+        "tflops": (acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r) + se_flops) / (both_ms / 1e3) / 1e12}
     del sinp, sbuf
 
     # separate gate/up adapters of rank r (NEXT-2): the same workload run as the fused
