@@ -60,3 +60,39 @@ def test_routed_plus_shared_layer():
     dX = to_np(buf_r.dX) + to_np(buf_s.dX)
     assert rel_err(Y, Yr + Ys) <= TOL
     assert rel_err(dX, gr["dX"] + gs["dX"]) <= TOL
+
+
+def test_routed_and_shared_on_two_streams_match_their_solo_runs():
+    # a model runs the shared expert beside the routed layer: the two share no
+    # library state but the status word, so concurrent calls give the solo bits
+    import torch
+    rcfg = small_config(T=512, m=256, n=128, E=8, k=2, r=16, alpha=16)
+    scfg = small_config(T=512, m=256, n=128, E=1, k=1, r=16, alpha=16)
+    rinp, _ = inputs_on(rcfg, seed=5)
+    sinp, _ = inputs_on(scfg, seed=6)
+    names = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d")
+
+    def solo():
+        rb = ml.alloc_buffers(rcfg.T, rcfg.m, rcfg.n, rcfg.E, rcfg.k, rcfg.r, rcfg.scale)
+        sb = ml.alloc_buffers(scfg.T, scfg.m, scfg.n, 1, 1, scfg.r, scfg.scale)
+        ml.layer_step(rinp, rcfg.k, rcfg.scale, rb)
+        ml.shared_expert_step(sinp, scfg.scale, sb)
+        torch.cuda.synchronize()
+        return rb, sb
+
+    ref_r, ref_s = solo()
+    rb = ml.alloc_buffers(rcfg.T, rcfg.m, rcfg.n, rcfg.E, rcfg.k, rcfg.r, rcfg.scale)
+    sb = ml.alloc_buffers(scfg.T, scfg.m, scfg.n, 1, 1, scfg.r, scfg.scale)
+    side = torch.cuda.Stream()
+    for _ in range(3):
+        main = torch.cuda.current_stream()
+        side.wait_stream(main)
+        ml.layer_step(rinp, rcfg.k, rcfg.scale, rb)
+        with torch.cuda.stream(side):
+            ml.shared_expert_step(sinp, scfg.scale, sb)
+        main.wait_stream(side)
+        torch.cuda.synchronize()
+        assert ml.moe_get_device_error() == ml.MOE_OK
+        for n in names:
+            assert torch.equal(getattr(rb, n), getattr(ref_r, n)), ("routed", n)
+            assert torch.equal(getattr(sb, n), getattr(ref_s, n)), ("shared", n)
