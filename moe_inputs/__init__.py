@@ -61,6 +61,9 @@ CONFIGS = {
     "qwen3_skewed": LayerConfig("qwen3_skewed", T=16384, m=2048, n=768, E=128, k=8, r=16, alpha=16,
                                 zipf_s=1.2, bias_scale=3.0),
     "deepseek_v3": LayerConfig("deepseek_v3", T=32768, m=7168, n=2048, E=256, k=8, r=32, alpha=32),
+    # the DeepSeek-V3 expert geometry (m, n, about 1024 rows per expert) on 16 experts:
+    # a tensor-bound case small enough for a full ncu capture (about 2.5 GB on the device)
+    "deepseek_v3_e16": LayerConfig("deepseek_v3_e16", T=2048, m=7168, n=2048, E=16, k=8, r=32, alpha=32),
 }
 
 DRAW_ORDER = ("logits", "X", "W_gu", "W_d", "A_gu", "B_gu", "A_d", "B_d", "dY")
