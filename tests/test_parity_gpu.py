@@ -191,7 +191,7 @@ def test_empty_input():
 
 
 # ------------------------------------------------------------------ full sizes (sampled)
-@pytest.mark.parametrize("name", ["qwen3_30b_a3b", "gpt_oss_20b", "qwen3_skewed"])
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b", "gpt_oss_20b", "qwen3_skewed", "deepseek_v3_e16"])
 def test_full_size_sampled_parity(name):
     cfg = CONFIGS[name]
     inp, cpu = inputs_on(cfg)
