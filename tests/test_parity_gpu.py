@@ -10,7 +10,7 @@ import torch
 
 import mixture_experts_lora_b200 as ml
 import oracle.moe_lora_oracle as O
-from moe_inputs import CONFIGS, small_config, generate
+from moe_inputs import CONFIGS, LayerConfig, small_config, generate
 
 from gpu_common import (TOL, TOL_W, check_full_parity, check_sampled_parity, ensure_built,
                         inputs_on, rel_err, run_layer, to_np)
@@ -198,6 +198,19 @@ def test_full_size_sampled_parity(name):
     buf = run_layer(inp, cfg)
     errs = check_sampled_parity(buf, cpu, cfg)
     print(name, errs)
+
+
+def test_skewed_experts_across_two_2048_row_chunks():
+    # 1024 rows per expert on average: the adapter-gradient chunk grows to 2048 rows,
+    # and the busiest experts (3200-4100 rows under this skew) take two chunks whose
+    # partials the last arriving unit sums
+    cfg = LayerConfig("skewed_e32", T=4096, m=2048, n=768, E=32, k=8, r=16, alpha=16,
+                      zipf_s=1.0, bias_scale=2.0)
+    inp, cpu = inputs_on(cfg)
+    buf = run_layer(inp, cfg)
+    assert int(buf.counts.max()) > 2048
+    errs = check_sampled_parity(buf, cpu, cfg, n_tokens=16, n_experts=3)
+    print(errs)
 
 
 def test_expert_spanning_several_chunks():
