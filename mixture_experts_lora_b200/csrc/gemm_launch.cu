@@ -99,7 +99,7 @@ cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap* maps, c
   const int pairs = (int)(tiles < pairs_max ? (tiles > 0 ? tiles : 1) : pairs_max);
   ProfScope ps(kind, s);
   st = launch_pdl(kern, dim3(2 * pairs), dim3(320), C::SMEM_BYTES, s, 2, maps[0], maps[1], maps[2],
-                  maps[3], p);
+                  maps[3], maps[4], p);
   if (st != cudaSuccess) return st;
   return cudaGetLastError();
 }
@@ -110,9 +110,16 @@ cudaError_t launch_gemm(int kind, const GemmShape& g, const CUtensorMap* maps, c
 cudaError_t gemm_any(int kind, const GemmShape& g, const uint16_t* W, bool w_fk, int F, int K,
                      const uint16_t* act, const uint16_t* lw, const uint16_t* lrc, uint16_t* out,
                      cudaStream_t s) {
-  CUtensorMap mp[4];
+  CUtensorMap mp[5];
   const uint64_t P = g.P, E = g.E, rp = g.rp;
   using C0 = GemmCfg<true, 16>;
+  {
+    // out [P, F]: 32-token x 32-feature blocks stored from the epilogue's staging
+    const uint64_t dims[2] = {(uint64_t)F, P};
+    const uint64_t str[1] = {(uint64_t)F * 2};
+    const uint32_t box[2] = {32, 32};
+    if (!encode(&mp[4], out, 2, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE)) return cudaErrorInvalidValue;
+  }
   // atom views (one copy per operand and stage) when the K (and MN-major F) extents
   // are whole 64-wide atoms
   const bool v = K % 64 == 0 && (w_fk || F % 64 == 0);

@@ -21,7 +21,8 @@
 // completing on the leader's barriers), warp 1 allocates TMEM and, in the leader
 // CTA, issues tcgen05.mma for the pair; warps 2-9 drain TMEM (two warps per TMEM
 // lane quarter, alternating 32-token chunks), transpose each 32 x 32 block through
-// shared memory and write 16-byte rows of the [tokens, features] output.  The
+// shared memory and write it to the [tokens, features] output with one TMA tensor
+// store (16-byte stores for a chunk's ragged last block).  The
 // accumulator is double buffered (2 x 256 fp32 columns) so the epilogue of one
 // tile overlaps the K-loop of the next.
 //
@@ -101,7 +102,7 @@ template <class C>
 __global__ void __launch_bounds__(320, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmAct,
                     const __grid_constant__ CUtensorMap tmLW, const __grid_constant__ CUtensorMap tmLR,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -354,18 +355,33 @@ __global__ void __launch_bounds__(320, 1)
       for (; c0 < nrows; c0 += 64) {
         const bool more = c0 + 64 < nrows;
         if (more) tmem_ld32(acc + c0 + 64, vn);          // next chunk, in flight meanwhile
+        if (lane == 0) bulk_wait_read<0>();               // the last store from blk has read it
+        __syncwarp();
 #pragma unroll
         for (int i = 0; i < 32; ++i)
           *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
-        __syncwarp();
         const int grow = ch.row0 + c0;
+        if (c0 + 32 <= nrows) {
+          // 32 rows inside the chunk: one TMA tensor store of the block (features past F
+          // are clipped by the tensor map)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, smem_u32(blk), fq, grow);
+            bulk_commit_group();
+          }
+        } else {
+          // the chunk's ragged last block: its rows past the end belong to the next
+          // chunk, so 16-byte stores of the rows inside only
+          __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int rr = rrow + 8 * j;
-          const int f = fq + rpart * 8;
-          if (c0 + rr < nrows && f < p.F) {
-            const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * 64 + rpart * 16);
-            *reinterpret_cast<uint4*>(p.out + (size_t)(grow + rr) * p.F + f) = x;
+          for (int j = 0; j < 4; ++j) {
+            const int rr = rrow + 8 * j;
+            const int f = fq + rpart * 8;
+            if (c0 + rr < nrows && f < p.F) {
+              const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * 64 + rpart * 16);
+              *reinterpret_cast<uint4*>(p.out + (size_t)(grow + rr) * p.F + f) = x;
+            }
           }
         }
         __syncwarp();
@@ -379,6 +395,8 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader + b * 8);
     }
+    if (lane == 0) bulk_wait<0>();                        // every store of this warp complete
+    __syncwarp();
   }
 
   tc_fence_before();
