@@ -217,7 +217,9 @@ moe_status_t moe_grouped_gemm_full_bwd(
  * larger problems return MOE_ERR_WORKSPACE before any launch.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  All calls share the one array: calls that overlap on the
+ * any stream capture.  The address is kept per device and CUDA context, so a call
+ * after a device reset (a new context) looks it up again; the array's contents do
+ * not survive the reset.  All calls share the one array: calls that overlap on the
  * GPU (different streams, no ordering between them) race and must be avoided.
  * Arguments, outputs and errors otherwise as moe_permute(). */
 moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
@@ -252,6 +254,17 @@ moe_status_t moe_router_backward(const moe_bf16_t* dY, const moe_bf16_t* Y_sorte
                                  const int32_t* topk_ids, const float* topk_w,
                                  const int32_t* pair_pos, int64_t T, int32_t k, int32_t E,
                                  int32_t m, float* dlogits, void* stream);
+
+/* Self-test of the failure path (no counterpart on the pages: a check of this
+ * library's own error handling).  Every wait of every kernel here is bounded: it
+ * gives up after a wall-clock limit, sets MOE_ERR_TIMEOUT in the device error word
+ * and lets its kernel return, so a lost arrival cannot hang the GPU.  This call
+ * launches one single-thread kernel that makes that same bounded wait on a barrier
+ * nothing arrives at, with the limit `limit_ns` (1 us to 1 s), and then writes
+ * *done = 1 (device int32) as it returns (2 if the wait had not expired).  After it,
+ * moe_get_device_error() returns MOE_ERR_TIMEOUT and the GPU stays usable.
+ * Errors: INVALID_ARG (limit out of range, done NULL), CUDA. */
+moe_status_t moe_selftest_bounded_wait(uint64_t limit_ns, int32_t* done, void* stream);
 
 /* Synchronises `stream`, returns the device error word of the current device
  * (MOE_OK if no kernel reported a problem) and clears it. */

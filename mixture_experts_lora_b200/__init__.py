@@ -33,7 +33,7 @@ EXPORTED = (
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
     "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
     "moe_permute_noalloc", "moe_router_backward", "moe_grouped_gemm_full_bwd",
-    "moe_check_permutation",
+    "moe_check_permutation", "moe_selftest_bounded_wait",
 )
 
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         h.moe_grouped_gemm_full_bwd.argtypes = [D] + [P] * 23 + [SZ, P]
         h.moe_unpermute_combine.argtypes = [P, P, P, I64, I32, I32, P, P]
         h.moe_router_backward.argtypes = [P, P, P, P, P, I64, I32, I32, I32, P, P]
+        h.moe_selftest_bounded_wait.argtypes = [ctypes.c_uint64, P, P]
         h.moe_get_device_error.argtypes = [P]
         h.moe_status_string.argtypes = [ctypes.c_int]
         h.moe_status_string.restype = ctypes.c_char_p
@@ -211,6 +212,14 @@ def moe_router_backward(dY, Y_sorted, topk_ids, topk_w, pair_pos, E: int, dlogit
     _check("moe_router_backward", lib().moe_router_backward(
         _ptr(dY), _ptr(Y_sorted), _ptr(topk_ids), _ptr(topk_w), _ptr(pair_pos), int(T), int(k),
         int(E), int(m), _ptr(dlogits), _stream(stream)))
+
+
+def moe_selftest_bounded_wait(limit_ns: int, done, stream=None):
+    """Run one bounded wait that nothing ends (see include/moelora.h); afterwards
+    moe_get_device_error() reports MOE_ERR_TIMEOUT and done[0] == 1."""
+    st = lib().moe_selftest_bounded_wait(int(limit_ns), _ptr(done), _stream(stream))
+    if st != MOE_OK:
+        raise MoEError("moe_selftest_bounded_wait", st, status_string(st))
 
 
 def moe_get_device_error(stream=None) -> int:

@@ -3,6 +3,9 @@
 // stream; the library allocates nothing.
 #include <cmath>
 #include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -21,14 +24,21 @@ constexpr int kMaxDevices = 64;
 constexpr int kTileRows = 128;
 constexpr int kGemmChunkRows = 256;
 
+// Device address of g_moe_status in the current context, looked up once per
+// (device, context): a device reset or a new primary context re-resolves it.
 int* status_ptr() {
+  static std::mutex mu;
   static int* ptrs[kMaxDevices] = {nullptr};
+  static void* ctxs[kMaxDevices] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (ptrs[dev] == nullptr) {
+  void* ctx = current_context();
+  std::lock_guard<std::mutex> lk(mu);
+  if (ptrs[dev] == nullptr || ctxs[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_moe_status) != cudaSuccess) return nullptr;
     ptrs[dev] = static_cast<int*>(p);
+    ctxs[dev] = ctx;
   }
   return ptrs[dev];
 }
@@ -297,6 +307,21 @@ moe_status_t backward(
 }
 
 }  // namespace
+
+void* current_context() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
 
 int* moe_status_word() { return status_ptr(); }
 

@@ -81,17 +81,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+// Bounded wait for the phase with the given parity to complete, giving up after
+// limit_ns nanoseconds of %globaltimer (MOE_ERR_TIMEOUT in the status word).
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int* err,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 31u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       report_error(err, MOE_ERR_TIMEOUT);
       return false;
     }
   }
+}
+// The kernels' wait: the same with the library's 1 s limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  return mbar_wait_for(bar, parity, err, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------- fences

@@ -60,6 +60,9 @@ struct ProfScope {
 
 // Device address of the status word of the current device (api.cu), or nullptr.
 int* moe_status_word();
+// The current CUDA context (a CUcontext), or nullptr: caches of device addresses key
+// on it, so that a device reset or a new primary context looks them up again.
+void* current_context();
 
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,

@@ -5,8 +5,11 @@
 // here in a file-scope device array of fixed size, present on every GPU that loads
 // the library until the process exits.  Host code cannot pass the array's name to
 // a kernel (on the host it names a stand-in, not device memory), so the device
-// address is looked up once per device with cudaGetSymbolAddress and cached.
+// address is looked up with cudaGetSymbolAddress, once per device and context, and
+// cached.
 #include <mutex>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -20,17 +23,22 @@ __device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts];
 
 constexpr int kMaxDevices = 64;
 
-// Device address of g_permute_scratch on the current device (nullptr on failure).
+// Device address of g_permute_scratch on the current device (nullptr on failure),
+// looked up with that device current the first time a (device, context) is seen: a
+// device reset or a new primary context gets a fresh lookup, never a stale address.
 int32_t* permute_scratch() {
   static std::mutex mu;
   static int32_t* ptrs[kMaxDevices] = {nullptr};
+  static void* ctxs[kMaxDevices] = {nullptr};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lk(mu);
-  if (ptrs[dev] == nullptr) {
+  if (ptrs[dev] == nullptr || ctxs[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_permute_scratch) != cudaSuccess) return nullptr;
     ptrs[dev] = static_cast<int32_t*>(p);
+    ctxs[dev] = ctx;
   }
   return ptrs[dev];
 }
@@ -44,6 +52,10 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, 
                                             int32_t E, int32_t* counts, int32_t* offsets,
                                             int32_t* sorted_pairs, int32_t* pair_pos,
                                             void* stream) {
+  struct Range {
+    Range() { nvtxRangePushA("moe_permute_noalloc"); }
+    ~Range() { nvtxRangePop(); }
+  } range;
   if (T < 0) return MOE_ERR_INVALID_ARG;
   if (k < 1 || k > 32 || E < k || E > 1024) return MOE_ERR_UNSUPPORTED;
   const int64_t P = T * (int64_t)k;

@@ -177,3 +177,10 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ml, "_lib_handle", None)
     with pytest.raises(RuntimeError):
         ml.lib()
+
+
+def test_selftest_bounded_wait_checks_its_arguments(L):
+    # out-of-range limits and a NULL flag are refused on the host, before any launch
+    assert L.moe_selftest_bounded_wait(999, ctypes.c_void_p(16), None) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(2_000_000_000, ctypes.c_void_p(16), None) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(1_000_000, None, None) == ml.MOE_ERR_INVALID_ARG

@@ -200,6 +200,18 @@ def test_full_size_sampled_parity(name):
     print(name, errs)
 
 
+# Full-size parity in full: every output and saved intermediate of the whole layer,
+# element by element, against the oracle run over the whole workload (the oracle
+# takes seconds to tens of seconds at these sizes on the host's cores).
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b", "qwen3_skewed", "gpt_oss_20b"])
+def test_full_size_full_parity(name):
+    cfg = CONFIGS[name]
+    inp, cpu = inputs_on(cfg)
+    buf = run_layer(inp, cfg)
+    errs = check_full_parity(buf, cpu, cfg)
+    print(name, errs)
+
+
 def test_skewed_experts_across_two_2048_row_chunks():
     # 1024 rows per expert on average: the adapter-gradient chunk grows to 2048 rows,
     # and the busiest experts (3200-4100 rows under this skew) take two chunks whose

@@ -57,3 +57,24 @@ def test_permute_noalloc_rejects_oversized_problem():
     with pytest.raises(ml.MoEError) as e:
         ml.moe_permute_noalloc(ids, E, *outs)
     assert e.value.status == ml.MOE_ERR_WORKSPACE
+
+
+def test_permute_noalloc_at_the_exact_scratch_limit():
+    # ceil(T*k / 512) * E == 2^19 histogram entries: the largest problem the built-in
+    # scratch holds must be accepted and give moe_permute's outputs
+    ensure_built()
+    E, k, T = 1024, 8, 32768
+    assert (T * k + 511) // 512 * E == 1 << 19
+    rng = np.random.default_rng(7)
+    ids = np.argsort(rng.random((T, E), dtype=np.float32), axis=1)[:, :k].astype(np.int32)
+    ids_d = torch.from_numpy(ids).cuda()
+    ws = torch.empty(ml.moe_workspace_bytes(ml.make_dims(T, 64, 64, E, k, 16, 1.0)),
+                     dtype=torch.uint8, device="cuda")
+    ref = _outputs(T, k, E)
+    got = _outputs(T, k, E)
+    ml.moe_permute(ids_d, E, *ref, ws)
+    ml.moe_permute_noalloc(ids_d, E, *got)
+    torch.cuda.synchronize()
+    assert ml.moe_get_device_error() == ml.MOE_OK
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
