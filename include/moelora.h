@@ -45,7 +45,7 @@
  *     (an expert id outside [0, E), a bounded wait that expired) set a device
  *     error word instead of trapping; read it with moe_get_device_error().
  *   - Supported shapes: 1 <= k <= 32, k <= E <= 1024; m and n multiples of 16,
- *     at least 16; r a multiple of 8 with 8 <= r <= 32; P = T*k < 2^31.
+ *     at least 16; r a multiple of 8 with 8 <= r <= 128; P = T*k < 2^31.
  *     T = 0 is valid and produces empty outputs (adapter gradients are zero).
  *     Other shapes return MOE_ERR_UNSUPPORTED.
  *   - Results are deterministic: no floating-point atomics; repeated calls with
@@ -135,25 +135,23 @@ moe_status_t moe_check_permutation(const int32_t* topk_ids, int64_t T, int32_t k
  *   Y_sorted[q] = H[q] W_d[e] + c (H[q] A_d[e]) B_d[e],
  *   H[q]        = silu(GU[q, :n]) * GU[q, n:],
  *   GU[q]       = X[t] W_gu[e] + c (X[t] A_gu[e]) B_gu[e],   t = sorted_pairs[q] / k,
- * for every q in the segment of expert e.
+ * for every q in the segment of expert e.  The rows X[t] are gathered inside the
+ * kernels; no expert-ordered copy of X is written.
  * Inputs (device, read): X bf16 [T, m]; sorted_pairs [P]; offsets [E+1]; the six
  *   weight tensors in the layouts above.
  * Outputs (device, written, bf16, sorted order):
- *   Y_sorted [P, m]; save_Xs [P, m] = X[sorted_pairs / k] (the expert-sorted input
- *   rows, the grouped GEMM's operand, kept for the backward as an autograd
- *   implementation keeps the permuted input); save_GU [P, 2n]; save_H [P, n];
- *   save_XA [P, r] = X A_gu (unscaled); save_HA [P, r] = H A_d (unscaled).  The
- *   save_* tensors are what moe_grouped_gemm_lora_bwd() needs.
- * Accumulation is fp32; every stored value is rounded once to bf16.  The LoRA
- * term multiplies bf16(c * X A) by B.
+ *   Y_sorted [P, m]; save_GU [P, 2n]; save_H [P, n]; save_XA [P, r] = X A_gu
+ *   (unscaled); save_HA [P, r] = H A_d (unscaled).  The save_* tensors are what
+ *   moe_grouped_gemm_lora_bwd() needs besides X.
+ * Accumulation is fp32; every stored value is rounded once to bf16 (H from the
+ * bf16-rounded GU).  The LoRA term multiplies bf16(c * X A) by B.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 moe_status_t moe_grouped_gemm_lora_fwd(
     const moe_dims_t* dims, const moe_bf16_t* X, const int32_t* sorted_pairs,
     const int32_t* offsets, const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
     const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs, moe_bf16_t* save_GU,
-    moe_bf16_t* save_H, moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws,
-    size_t ws_bytes, void* stream);
+    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_GU, moe_bf16_t* save_H,
+    moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws, size_t ws_bytes, void* stream);
 
 /* Backward of all experts (W frozen) for upstream gradient dY:
  *   dy_q     = w[p] dY[t]                          (p = sorted_pairs[q], t = p / k)
@@ -162,21 +160,22 @@ moe_status_t moe_grouped_gemm_lora_fwd(
  *   T2       = dGU B_gu^T, dX_sorted = dGU W_gu^T + c T2 A_gu^T
  *   dA_d[e]  = c H_e^T T1_e,   dB_d[e]  = c HA_e^T dy_e
  *   dA_gu[e] = c X_e^T T2_e,   dB_gu[e] = c XA_e^T dGU_e
- * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; sorted_pairs;
- *   offsets; the six weights; save_Xs, save_GU, save_H, save_XA, save_HA from the
- *   forward.
+ * The rows dY[t] and X[t] are gathered inside the kernels and the routing weight is
+ * applied after the products (by linearity); dH is not written to memory.
+ * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; X bf16 [T, m];
+ *   sorted_pairs; offsets; the six weights; save_GU, save_H, save_XA, save_HA from
+ *   the forward.
  * Outputs (device, written, bf16): dX_sorted [P, m] (sorted order; reduce with
  *   moe_unpermute_combine(topk_w = NULL)); dA_gu [E, m, r]; dB_gu [E, r, 2n];
  *   dA_d [E, n, r]; dB_d [E, r, m].  Experts with no rows get zero gradients.
  * Adapter gradients are reduced over rows in a fixed order (deterministic).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 moe_status_t moe_grouped_gemm_lora_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
     const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
-    const moe_bf16_t* save_XA,
+    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
     const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dA_gu,
     moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream);
@@ -196,12 +195,11 @@ moe_status_t moe_grouped_gemm_lora_bwd(
  * outputs and errors as moe_grouped_gemm_lora_bwd(); each weight-gradient tile
  * sums its rows in one fixed order (deterministic). */
 moe_status_t moe_grouped_gemm_full_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
     const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
-    const moe_bf16_t* save_XA,
+    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
     const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dW_gu,
     moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
     moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream);

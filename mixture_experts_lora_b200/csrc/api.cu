@@ -55,7 +55,7 @@ int device_sms() {
   return sms[dev];
 }
 
-inline int rank_padded(int r) { return r <= 16 ? 16 : 32; }
+inline int rank_padded(int r) { return r <= 16 ? 16 : r <= 32 ? 32 : r <= 64 ? 64 : 128; }
 
 // Row chunk of the adapter-gradient kernel.  An expert cut into several chunks
 // needs fp32 partials and a last-arriver sum per 256-column unit, and the cut
@@ -88,7 +88,7 @@ moe_status_t check_dims(const moe_dims_t* d) {
   if (!std::isfinite(d->scale)) return MOE_ERR_INVALID_ARG;
   if (d->k < 1 || d->k > 32 || d->E < d->k || d->E > 1024) return MOE_ERR_UNSUPPORTED;
   if (d->m < 16 || d->n < 16 || d->m % 16 != 0 || d->n % 16 != 0) return MOE_ERR_UNSUPPORTED;
-  if (d->r < 8 || d->r > 32 || d->r % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (d->r < 8 || d->r > 128 || d->r % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (d->T * (int64_t)d->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
   // largest row index times the widest row must stay within 32-bit tile coordinates
   if ((int64_t)d->m > (1 << 20) || (int64_t)d->n > (1 << 19)) return MOE_ERR_UNSUPPORTED;
@@ -101,10 +101,10 @@ struct Layout {
   int rp;
   int max_row_tiles, max_gchunks, max_chunks, chunk_rows, perm_chunks;
   size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
-  size_t pad_A_gu, pad_B_gu, pad_A_d, pad_B_d;
-  int max_dtiles;             // 128-column tiles of the widest adapter gradient
-  size_t rows, dgu, dh, t1, t2, lrc1, lrc2, partial, partial2, rows_partial;
-  size_t counters;           // [row kernels fwd 2][row kernels bwd 2][gradients 4] sets
+  int max_dtiles;            // 128-column tiles of the widest adapter gradient
+  size_t rows;               // expert-ordered X or w dY (full fine-tuning only)
+  size_t dgu, t1, t2, lrc1, lrc2, wha, partial, partial2;
+  size_t counters;           // arrival counters of the four adapter gradients
   size_t total;
 };
 
@@ -117,7 +117,6 @@ Layout make_layout(const moe_dims_t& d) {
   L.chunk_rows = (int)chunk_rows_for(d, L.P);
   L.max_chunks = (int)((L.P + L.chunk_rows - 1) / L.chunk_rows) + d.E;
   L.perm_chunks = (int)((L.P + kPermuteChunk - 1) / kPermuteChunk);
-  const bool pad = d.r != L.rp;
   const size_t E = d.E, m = d.m, n = d.n, rp = L.rp, P = (size_t)L.P;
   const size_t dmax = m > 2 * n ? m : 2 * n;
   size_t off = 0;
@@ -130,24 +129,17 @@ Layout make_layout(const moe_dims_t& d) {
   L.chunks = take((size_t)L.max_chunks * sizeof(TileInfo));
   L.n_chunks = take(4);
   L.chunk_start = take((E + 1) * 4);
-  L.pad_A_gu = take(pad ? E * m * rp * 2 : 0);
-  L.pad_B_gu = take(pad ? E * rp * 2 * n * 2 : 0);
-  L.pad_A_d = take(pad ? E * n * rp * 2 : 0);
-  L.pad_B_d = take(pad ? E * rp * m * 2 : 0);
   L.rows = take(P * m * 2);
   L.dgu = take(P * 2 * n * 2);
-  L.dh = take(P * n * 2);
   L.t1 = take(P * rp * 2);
   L.t2 = take(P * rp * 2);
   L.lrc1 = take(P * rp * 2);
   L.lrc2 = take(P * rp * 2);
+  L.wha = take(P * rp * 2);
   L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
   L.partial2 = take((size_t)L.max_chunks * dmax * rp * 4);
   L.max_dtiles = (int)((dmax + 127) / 128);
-  L.rows_partial = take((size_t)kRowsMaxCtas * 2 * 128 * rp * 4);
-  // arrival counters: one set of max_row_tiles per row-kernel launch, then one set
-  // of E * max_dtiles per adapter gradient
-  L.counters = take(((size_t)4 * L.max_row_tiles + (size_t)4 * E * L.max_dtiles) * 4);
+  L.counters = take((size_t)4 * E * L.max_dtiles * 4);
   L.total = off;
   return L;
 }
@@ -165,7 +157,8 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
     if (e_ != cudaSuccess) return MOE_ERR_CUDA;        \
   } while (0)
 
-// Common set-up of the grouped GEMMs: tables, padded adapters, operand pointers.
+// Common set-up of the grouped GEMMs: tables and operand pointers.  Adapters are used
+// as given: ranks r .. rp - 1 read as zero through the tensor maps.
 moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32_t* offsets,
                      const uint16_t* W_gu, const uint16_t* W_d, const uint16_t* A_gu,
                      const uint16_t* B_gu, const uint16_t* A_d, const uint16_t* B_d,
@@ -177,25 +170,10 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
                               at<int>(ws, L.n_gchunks), L.chunk_rows,
                               with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
                               at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start),
-                              at<int>(ws, L.counters) + (with_chunks ? 2 * L.max_row_tiles : 0),
-                              with_chunks ? 2 * L.max_row_tiles + 4 * d.E * L.max_dtiles
-                                          : 2 * L.max_row_tiles,
-                              s));
+                              at<int>(ws, L.counters), with_chunks ? 4 * d.E * L.max_dtiles : 0, s));
   w->W_gu = W_gu;
   w->W_d = W_d;
-  if (d.r != L.rp) {
-    uint16_t* pa = at<uint16_t>(ws, L.pad_A_gu);
-    uint16_t* pb = at<uint16_t>(ws, L.pad_B_gu);
-    uint16_t* pc = at<uint16_t>(ws, L.pad_A_d);
-    uint16_t* pd = at<uint16_t>(ws, L.pad_B_d);
-    MOE_TRY(launch_pad3(A_gu, d.E, d.m, d.r, d.m, L.rp, pa, s));
-    MOE_TRY(launch_pad3(B_gu, d.E, d.r, 2 * d.n, L.rp, 2 * d.n, pb, s));
-    MOE_TRY(launch_pad3(A_d, d.E, d.n, d.r, d.n, L.rp, pc, s));
-    MOE_TRY(launch_pad3(B_d, d.E, d.r, d.m, L.rp, d.m, pd, s));
-    w->A_gu = pa; w->B_gu = pb; w->A_d = pc; w->B_d = pd;
-  } else {
-    w->A_gu = A_gu; w->B_gu = B_gu; w->A_d = A_d; w->B_d = B_d;
-  }
+  w->A_gu = A_gu; w->B_gu = B_gu; w->A_d = A_d; w->B_d = B_d;
   g->P = L.P;
   g->m = d.m;
   g->n = d.n;
@@ -215,14 +193,12 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
 }
 
 // The backward pass.  Adapter gradients when dA_gu.. are given (all four or none),
-// expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given; each weight
-// gradient runs while its sorted operands are at hand (dy in the row buffer after
-// the down backward; X sorted saved by the forward).
+// expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given.
 moe_status_t backward(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, moe_bf16_t* dW_gu,
     moe_bf16_t* dW_d, void* ws, size_t ws_bytes, void* stream) {
@@ -248,7 +224,7 @@ moe_status_t backward(
     }
     return MOE_OK;
   }
-  const void* ins[] = {dY, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_Xs, save_GU, save_H, save_XA,
+  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA,
                        save_HA, dX_sorted, ws};
   for (const void* p : ins)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -263,46 +239,53 @@ moe_status_t backward(
   uint16_t* dgu = at<uint16_t>(ws, L.dgu);
   uint16_t* t1 = at<uint16_t>(ws, L.t1);
   uint16_t* t2 = at<uint16_t>(ws, L.t2);
+  uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
+  uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
+  uint16_t* wha = at<uint16_t>(ws, L.wha);
   float* partial = at<float>(ws, L.partial);
+  float* partial2 = at<float>(ws, L.partial2);
   const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
   const int* n_chunks = at<int>(ws, L.n_chunks);
   const int32_t* chunk_start = at<int32_t>(ws, L.chunk_start);
-  uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
-  uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
-  uint16_t* dh = at<uint16_t>(ws, L.dh);
-  float* rpart = at<float>(ws, L.rows_partial);
-  int* rcnt = at<int>(ws, L.counters) + 2 * L.max_row_tiles;   // row-kernel sets 2 and 3
-  // dy = w * dY[t] in expert order, T1 = dy B_d^T (kept for dA_d) and bf16(c T1)
-  MOE_TRY(launch_rows_lowrank(g, 0, d.m, dY, sorted_pairs, topk_w, d.k, nullptr, nullptr, w.B_d,
-                              false, rows, t1, L.rp, L.rp, lrc1, rpart, rcnt, s));
-  // dH = dy W_d^T + (c T1) A_d^T
-  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
-  // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
-  float* partial2 = at<float>(ws, L.partial2);
-  int* counters = at<int>(ws, L.counters) + 4 * L.max_row_tiles;   // gradient sets
+  int* counters = at<int>(ws, L.counters);
   const size_t cstride = (size_t)d.E * L.max_dtiles;
+  const int rp = L.rp;
+  // T1' = dY B_d^T on rows gathered from dY: t1 = bf16(w T1') (the dA_d operand),
+  // lrc1 = bf16(c T1') (the down backward's LoRA operand), wha = bf16(w HA) (dB_d's)
+  MOE_TRY(launch_rank_gathered(K_RANK_T1, g, dY, d.m, sorted_pairs, d.k, topk_w, w.B_d, false, t1,
+                               rp, rp, true, lrc1, save_HA, d.r, wha, s));
+  // dA_d = c H^T (w T1') and dB_d = c (w HA)^T dY (dY rows gathered), one launch
   if (lora) {
     const WgradJob jobs[2] = {
-        {save_H, d.n, t1, L.rp, false, dA_d, partial, counters},
-        {rows, d.m, save_HA, d.r, true, dB_d, partial2, counters + cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+        {save_H, nullptr, d.n, t1, rp, false, dA_d, partial, counters},
+        {nullptr, dY, d.m, wha, rp, true, dB_d, partial2, counters + cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, sorted_pairs,
+                              d.k, s));
   }
-  // dW_d = H^T dy per expert
-  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_D, g, offsets, save_H, d.n, rows, d.m, dW_d, s));
-  // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
-  MOE_TRY(launch_rows_lowrank(g, 2, 2 * d.n, nullptr, nullptr, nullptr, d.k, save_GU, dh, w.B_gu,
-                              false, dgu, t2, L.rp, L.rp, lrc2, rpart, rcnt + L.max_row_tiles, s));
+  // dW_d = H^T (w dY) per expert, on an expert-ordered copy of w dY
+  if (full) {
+    MOE_TRY(launch_gather_rows(dY, sorted_pairs, topk_w, L.P, d.k, d.m, rows, s));
+    MOE_TRY(launch_expert_dw(K_GEMM_DW_D, g, offsets, save_H, d.n, rows, d.m, dW_d, s));
+  }
+  // dGU: the SwiGLU backward of dH = w (dY W_d^T + (c T1') A_d^T), fused
+  MOE_TRY(launch_gemm_down_bwd(g, w, dY, sorted_pairs, d.k, topk_w, save_GU, lrc1, dgu, s));
+  // T2 = dGU B_gu^T (the dA_gu operand) and bf16(c T2)
+  MOE_TRY(launch_rank_sorted(K_RANK_T2, g, dgu, 2 * d.n, w.B_gu, false, t2, rp, rp, lrc2, s));
   // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
-  // dB_gu = c XA^T dGU and dA_gu = c X^T T2 (X in expert order from the forward), one launch
+  // dB_gu = c XA^T dGU and dA_gu = c X^T T2 (X rows gathered), one launch
   if (lora) {
     const WgradJob jobs[2] = {
-        {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
-        {save_Xs, d.m, t2, L.rp, false, dA_gu, partial2, counters + 3 * cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
+        {dgu, nullptr, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
+        {nullptr, X, d.m, t2, rp, false, dA_gu, partial2, counters + 3 * cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, sorted_pairs,
+                              d.k, s));
   }
-  // dW_gu = X^T dGU per expert
-  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, save_Xs, d.m, dgu, 2 * d.n, dW_gu, s));
+  // dW_gu = X^T dGU per expert, on an expert-ordered copy of X
+  if (full) {
+    MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
+    MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, rows, d.m, dgu, 2 * d.n, dW_gu, s));
+  }
   return MOE_OK;
 }
 
@@ -425,8 +408,7 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
                                        const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
                                        const moe_bf16_t* A_gu, const moe_bf16_t* B_gu,
                                        const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs,
-                                       moe_bf16_t* save_GU,
+                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_GU,
                                        moe_bf16_t* save_H, moe_bf16_t* save_XA,
                                        moe_bf16_t* save_HA, void* ws, size_t ws_bytes,
                                        void* stream) {
@@ -435,7 +417,7 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   if (st != MOE_OK) return st;
   const moe_dims_t d = *dims;
   if (d.T == 0) return MOE_OK;
-  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_Xs, save_GU, save_H,
+  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_GU, save_H,
                         save_XA, save_HA, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -447,45 +429,41 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   LayerPtrs w;
   st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, s, &g, &w);
   if (st != MOE_OK) return st;
-  uint16_t* xs = save_Xs;
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
-  float* rpart = at<float>(ws, L.rows_partial);
-  int* rcnt = at<int>(ws, L.counters);           // row-kernel sets 0 and 1 (zeroed above)
-  // X rows in expert order, XA = X A_gu (saved) and bf16(c XA)
-  MOE_TRY(launch_rows_lowrank(g, 0, d.m, X, sorted_pairs, nullptr, d.k, nullptr, nullptr, w.A_gu,
-                              true, xs, save_XA, d.r, d.r, xac, rpart, rcnt, s));
-  // GU = X W_gu + (c XA) B_gu
-  MOE_TRY(launch_gemm_gateup_fwd(g, w, xs, xac, save_GU, s));
-  // H = silu(g) u, HA = H A_d (saved) and bf16(c HA)
-  MOE_TRY(launch_rows_lowrank(g, 1, d.n, nullptr, nullptr, nullptr, d.k, save_GU, nullptr, w.A_d,
-                              true, save_H, save_HA, d.r, d.r, hac, rpart, rcnt + L.max_row_tiles, s));
+  // XA = X A_gu on rows gathered from X (saved) and bf16(c XA)
+  MOE_TRY(launch_rank_gathered(K_RANK_XA, g, X, d.m, sorted_pairs, d.k, nullptr, w.A_gu, true,
+                               save_XA, d.r, d.r, false, xac, nullptr, 0, nullptr, s));
+  // GU = X W_gu + (c XA) B_gu (X rows gathered) and H = silu(g) u, fused
+  MOE_TRY(launch_gemm_gateup_fwd(g, w, X, sorted_pairs, d.k, xac, save_GU, save_H, s));
+  // HA = H A_d (saved) and bf16(c HA)
+  MOE_TRY(launch_rank_sorted(K_RANK_HA, g, save_H, d.n, w.A_d, true, save_HA, d.r, d.r, hac, s));
   // Y = H W_d + (c HA) B_d
   MOE_TRY(launch_gemm_down_fwd(g, w, save_H, hac, Y_sorted, s));
   return MOE_OK;
 }
 
 moe_status_t moe_grouped_gemm_lora_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream) {
   NvtxRange nr("moe_grouped_gemm_lora_bwd");
   if (dA_gu == nullptr || dB_gu == nullptr || dA_d == nullptr || dB_d == nullptr)
     return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
+  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
                   nullptr, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_grouped_gemm_full_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
     const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
     moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
     moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream) {
@@ -493,8 +471,8 @@ moe_status_t moe_grouped_gemm_full_bwd(
   if (dW_gu == nullptr || dW_d == nullptr) return MOE_ERR_INVALID_ARG;
   const int given = (dA_gu != nullptr) + (dB_gu != nullptr) + (dA_d != nullptr) + (dB_d != nullptr);
   if (given != 0 && given != 4) return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
+  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
                   dW_d, ws, ws_bytes, stream);
 }
 

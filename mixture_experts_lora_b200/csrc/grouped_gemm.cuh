@@ -4,65 +4,92 @@
 // Orientation: output features on the MMA's M side, the expert's tokens on the N
 // side.  A pair of CTAs computes 256 features (128 per CTA, each CTA's own TMEM)
 // for a token chunk of at most 256 rows of one expert (granularity 16, each CTA
-// loads half of the token rows, so a token row is read once per pair).  Each
+// holds half of the token rows, so a token row is read once per pair).  Each
 // expert's rows are cut into balanced chunks, so the ragged end of an expert
 // wastes at most 15 columns.  For a tile (token chunk of expert e, feature tile w):
 //
-//   D[f, t] = sum_k Wt[e][f, k] Act[t, k]  +  sum_r Lt[e][f, r] LRc[t, r]
+//   D[f, t] = sum_k Wt[e][f, k] Act[t, k]  +  sum_j Lt[e][f, j] LRc[t, j]
 //
-// where Act is the expert-sorted activation matrix, Wt the weight oriented
-// feature-major and LRc = bf16(c * Act L_A[e]) the rank-r product from the
-// row kernel; the second sum is one extra K-block of the same pipeline.
-// This is Y = XW + (alpha/r)(XA)B of the Split-LoRA reordering ("Accelerating
+// where Act is the activation matrix in expert order, Wt the weight oriented
+// feature-major and LRc = bf16(c * Act L_A[e]) the rank-r product from the rank-r
+// kernel; the second sum is one more K-block of the same accumulation.  This is
+// Y = XW + (alpha/r)(XA)B of the Split-LoRA reordering ("Accelerating
 // Mixture-of-Experts Fine-Tuning", Mathematical Formulation section 2) with no
 // K x N adapter delta.
 //
-// Roles (320 threads per CTA): warp 0 issues TMA loads (each CTA its own half,
-// completing on the leader's barriers), warp 1 allocates TMEM and, in the leader
-// CTA, issues tcgen05.mma for the pair; warps 2-9 drain TMEM (two warps per TMEM
-// lane quarter, alternating 32-token chunks), transpose each 32 x 32 block through
-// shared memory and write it to the [tokens, features] output with one TMA tensor
-// store (16-byte stores for a chunk's ragged last block).  The
-// accumulator is double buffered (2 x 256 fp32 columns) so the epilogue of one
-// tile overlaps the K-loop of the next.
+// Token operand.  Either a sorted [P, K] matrix loaded with TMA, or (GATHER) rows
+// gathered straight from a token matrix [T, K] - row q of the chunk is
+// src[sorted_pairs[q] / k] - by four gather warps with cp.async into the same
+// swizzled layout, so the expert-ordered copy of X or dY is never written to HBM
+// (the "dY gather / scale, not materialised" step of the backward; the routing
+// weight is applied in the epilogue, by linearity).
+//
+// Epilogues (EPI):
+//   EPI_PLAIN    out[q, f] = bf16(D)
+//   EPI_WSCALE   out[q, f] = bf16(w[q] D)                   (w: routing weight of the row)
+//   EPI_SWIGLU   the gate_up projection with the SwiGLU fused (h = silu(g) u, gate = first
+//                n columns; Unsloth docs "What is torch._grouped_mm?", the expert's
+//                gate_up output split in two): each CTA's 128 features are 64 gate
+//                features and the 64 up features of the same indices, so g and u of a
+//                token meet in one CTA; it writes GU (kept for the backward) and H.
+//   EPI_DSWIGLU  the down projection's backward with the SwiGLU backward fused:
+//                dH = w[q] D, then dGU = [dH u s (1 + g (1 - s)), dH g s], s = sigmoid(g),
+//                from the saved GU; only dGU is written.
+//
+// Roles (320 threads per CTA, 448 with GATHER): warp 0 issues TMA loads (each CTA its
+// own half, completing on the leader's barriers), warp 1 allocates TMEM and, in the
+// leader CTA, issues tcgen05.mma for the pair; warps 2-9 drain TMEM (two warps per
+// TMEM lane quarter, alternating 32-token blocks), transpose each 32 x 32 block
+// through shared memory and store it with one TMA tensor store (16-byte stores for a
+// chunk's ragged last block); warps 10-13 (GATHER) gather the token rows.  The
+// accumulator is double buffered (2 x 256 fp32 columns) so the epilogue of one tile
+// overlaps the K-loop of the next.
 //
 // Shared-memory operands (canonical UMMA layouts, per CTA):
-//   A (weights)  forward, W stored [K][F]: MN-major, two 64-feature atoms of 64 K
-//                rows, 128-byte swizzle (one TMA copy through a 4-D view when
-//                F % 64 == 0); backward, W stored [F][K]: K-major,
-//                [128 features][64 K], 128-byte swizzle
+//   A (weights)  forward, W stored [K][F]: MN-major, two 64-feature atoms of 128 K
+//                rows, 128-byte swizzle; backward, W stored [F][K]: K-major,
+//                [128 features][64 K] atoms, 128-byte swizzle
 //   B (tokens)   two K atoms of [128 rows][64 K], K-major, 128-byte swizzle
-// Each stage costs the two issuing threads a fixed number of instructions
-// (waits, TMA copies, MMAs, a commit), so the loaders use as few copies per stage
-// as the layouts allow and the MMA descriptors are advanced by offsets.
-//   LoRA block   A: L_B^T (forward [r][F]: MN-major; backward [F][r]: K-major,
-//                32/64-byte swizzle); B: LRc [N/2 rows][r], K-major, 32/64-byte swizzle
+//   LoRA block   A: L_B^T (forward [r][F]: MN-major; backward [F][r]: K-major), B: LRc
+//                [N/2 rows][r], K-major; 32/64/128-byte swizzle by rank width, two
+//                64-wide K atoms at rank 128.  At rank 16 the block has a double
+//                buffer of its own; wider ranks take one ring stage per tile.
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
+enum GemmEpi : int { EPI_PLAIN = 0, EPI_WSCALE = 1, EPI_SWIGLU = 2, EPI_DSWIGLU = 3 };
+
 struct GemmParams {
   const TileInfo* chunks;  // token chunks {e, row0, row_end}, at most 256 rows each
   const int* n_chunks;
-  int F;                   // output features
-  int n_ftiles;            // feature tiles (256 features per pair) per chunk
-  int nk;                  // K steps of 128 (the LoRA block is step nk)
-  __nv_bfloat16* out;      // [P, F] in sorted token order
+  int F;                   // output features (EPI_SWIGLU: h-features n)
+  int n_ftiles;            // feature tiles per chunk
+  int nk;                  // K steps of 128 (the LoRA block follows them)
+  int K;                   // reduction length
+  // gathered token operand (GATHER): row q = gsrc[sorted_pairs[q] / k]
+  const __nv_bfloat16* gsrc;
+  const int32_t* sorted_pairs;
+  int k;
+  const float* w;          // [P] routing weights in pair order (EPI_WSCALE, EPI_DSWIGLU)
+  const __nv_bfloat16* gu; // [P, 2n] saved GU (EPI_DSWIGLU)
+  int n;                   // expert intermediate size (SwiGLU epilogues)
+  // outputs, for the ragged stores (the full blocks go through the tensor maps)
+  __nv_bfloat16* out;      // PLAIN/WSCALE: [P, F]; SWIGLU: GU [P, 2n]; DSWIGLU: dGU [P, 2n]
+  __nv_bfloat16* out_h;    // SWIGLU: H [P, n]
   int* err;
 };
 
-// A_MN: weights stored [K][F] (MN-major A).  V: operands through atom views, one
-// TMA copy per operand and stage: the weight tile via a 4-D view (64-wide atom,
-// rows, atom index, expert) and the token tile via a 3-D view (64-wide K atom,
-// rows, atom index); needs K % 64 == 0 (and F % 64 == 0 for MN-major weights).
-// Otherwise two copies per operand.
-template <bool A_MN_, int RP_, bool V_ = false>
+// A_MN: weights stored [K][F] (MN-major A).  V: weights through an atom view, one
+// TMA copy per stage (and, for a TMA-loaded token operand, the token tile through
+// one as well); needs whole 64-wide atoms.  Otherwise two copies per operand.
+template <bool A_MN_, int RP_, bool V_, bool GATHER_, int EPI_>
 struct GemmCfg {
   static constexpr int RP = RP_;
-  static constexpr bool A_MN = A_MN_;
-  static constexpr bool V = V_;
+  static constexpr bool A_MN = A_MN_, V = V_, GATHER = GATHER_;
+  static constexpr int EPI = EPI_;
   // BK = 128 per stage as two 64-wide K atoms (one 128-byte swizzle row each): a
   // stage carries 8 MMAs per wait and commit.  BOXR: token rows per LoRA-block copy.
   static constexpr int BM = 128, BK = 128, KA = 64, NMAX = 256, NHALF = NMAX / 2, BOXR = 64;
@@ -73,36 +100,93 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BLK_BYTES = 32 * 32 * 2;        // one 32 x 32 bf16 staging block
   static constexpr int EPI_WARPS = 8;
+  static constexpr int GATHER_WARPS = GATHER ? 4 : 0;
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS + GATHER_WARPS);
   static constexpr int EPI_BYTES = EPI_WARPS * BLK_BYTES;   // one transpose block per warp
   static constexpr int SMEM_LIMIT = 232448;
-  static constexpr int LA_BOX_BYTES = RP * 64 * 2;          // forward: 64 features x RP rows
-  static constexpr int LA_BYTES = A_MN ? 2 * LA_BOX_BYTES : BM * RP * 2;
-  static constexpr int LR_BOX_BYTES = BOXR * RP * 2;        // 64 token rows x RP
-  // LSIDE: the LoRA block's operands (LA: L_B^T, LR: c*LR rows) live in a double
-  // buffer of their own, loaded at the start of a tile, instead of taking a whole
-  // ring stage per tile (fits beside three stages for RP = 16)
+  // LoRA operands.  K-major atoms are LK_W ranks wide.
+  static constexpr int LK_W = RP < 64 ? RP : 64;
+  static constexpr int LK_ATOMS = RP > 64 ? 2 : 1;
+  static constexpr uint32_t LK_SW = LK_W == 16 ? kSw32 : LK_W == 32 ? kSw64 : kSw128;
+  static constexpr uint32_t LK_SBO = 8 * LK_W * 2;
+  static constexpr int LA_ATOM = BM * LK_W * 2;             // K-major A atom (128 features)
+  static constexpr int LR_ATOM = NHALF * LK_W * 2;          // K-major B atom (128 token rows)
+  static constexpr int LA_BOX_BYTES = RP * 64 * 2;          // forward: RP rows x 64 features
+  static constexpr int LA_BYTES = A_MN ? 2 * LA_BOX_BYTES : LK_ATOMS * LA_ATOM;
+  static constexpr int LR_BOX_BYTES = BOXR * LK_W * 2;      // 64 token rows x LK_W ranks
+  // LSIDE: at rank 16 the LoRA block's operands live in a double buffer of their own,
+  // loaded at the start of a tile, instead of taking a whole ring stage per tile
   static constexpr bool LSIDE = RP == 16;
-  static constexpr int LS_BYTES = LA_BYTES + NHALF * RP * 2;
+  static constexpr int LS_BYTES = LA_BYTES + LK_ATOMS * LR_ATOM;
   static constexpr int LS_TOTAL = LSIDE ? 2 * LS_BYTES : 0;
   static constexpr int STAGES_FIT = (SMEM_LIMIT - EPI_BYTES - LS_TOTAL - 2048) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LS_TOTAL + EPI_BYTES + 2048;
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t LR_SWZ = RP == 16 ? kSw32 : kSw64;
-  static constexpr uint32_t LR_SBO = RP == 16 ? 256 : 512;
-  static_assert(RP == 16 || RP == 32, "RP");
+  static_assert(RP == 16 || RP == 32 || RP == 64 || RP == 128, "RP");
+  static_assert(LA_BYTES <= A_BYTES && LK_ATOMS * LR_ATOM <= B_BYTES, "LoRA block fits a stage");
   static_assert(STAGES >= 3, "pipeline depth");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory");
+  static_assert(!(EPI == EPI_SWIGLU) || A_MN, "SwiGLU epilogue is the gate_up forward");
 };
 
-// First feature of this CTA's 64-feature A box i for feature tile w (pair rank r).
-__device__ __forceinline__ int feat_box(int w, int r, int i) { return w * 256 + r * 128 + i * 64; }
+// Descriptor offset (in 16-byte units) of 16-wide K step kk inside K-major LoRA
+// operand atoms of `atom_bytes` bytes, LK_W ranks wide.
+template <class C>
+__device__ __forceinline__ uint32_t lk_step(int kk, int atom_bytes) {
+  const int k0 = kk * 16;
+  return (uint32_t)((k0 / C::LK_W) * atom_bytes + (k0 % C::LK_W) * 2) >> 4;
+}
+
+// Stores one 32-token x 32-feature staging block (token-major rows of 64 bytes) at
+// (column fcol of the tensor map, row grow).  A block with all 32 rows inside the
+// chunk goes out as one TMA tensor store (columns past the map's width and rows past
+// P clipped); the chunk's ragged last block, whose rows past the end belong to the
+// next chunk, as 16-byte stores of its rows_left rows and columns below fmax, at
+// base + row * ld + fcol.
+__device__ __forceinline__ void epi_store_block(const CUtensorMap* tm, uint8_t* blk, int fcol,
+                                                int grow, int rows_left, __nv_bfloat16* base,
+                                                size_t ld, int fmax) {
+  const int lane = lane_id();
+  if (rows_left >= 32) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm, smem_u32(blk), fcol, grow);
+      bulk_commit_group();
+    }
+  } else {
+    __syncwarp();
+    const int rrow = lane >> 2, rpart = lane & 3;   // 8 rows x 4 parts per pass
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int rr = rrow + 8 * j;
+      const int f = fcol + rpart * 8;
+      if (rr < rows_left && f < fmax) {
+        const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * 64 + rpart * 16);
+        *reinterpret_cast<uint4*>(base + (size_t)(grow + rr) * ld + f) = x;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// First feature (global column of W) of this CTA's 64-feature A box i for feature
+// tile w (pair rank r): plain tiles cover 256 output features per pair; SwiGLU tiles
+// cover 128 h-features per pair, each CTA 64 gate columns (box 0) and the 64 up
+// columns n later (box 1).
+template <class C>
+__device__ __forceinline__ int feat_box(int w, int r, int i, int n) {
+  if constexpr (C::EPI == EPI_SWIGLU) return w * 128 + r * 64 + i * n;
+  else return w * 256 + r * 128 + i * 64;
+}
 
 template <class C>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(C::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmAct,
                     const __grid_constant__ CUtensorMap tmLW, const __grid_constant__ CUtensorMap tmLR,
-                    const __grid_constant__ CUtensorMap tmOut, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmOut2,
+                    const __grid_constant__ CUtensorMap tmOut3, const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -123,10 +207,12 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  constexpr int NST = C::LSIDE ? 0 : 1;        // ring stages of the LoRA block per tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      // the producer's expect_tx arrival, plus one per gather warp of both CTAs
+      mbar_init(smem_u32(&full[s]), 1 + 2 * C::GATHER_WARPS);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -141,7 +227,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmW);
-    tma_prefetch_desc(&tmAct);
+    if constexpr (!C::GATHER) tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmLW);
     tma_prefetch_desc(&tmLR);
   }
@@ -157,6 +243,23 @@ __global__ void __launch_bounds__(320, 1)
   pdl_begin();          // predecessors' outputs (chunk tables, operands) visible from here
   const int total = (*p.n_chunks) * p.n_ftiles;
 
+  // Issue the LoRA block's copies (L_B^T rows of this CTA's features and its half of
+  // the LRc rows) into the A and B areas at la / lr, completing on the leader's bar.
+  auto load_lora = [&](uint32_t bar, uint32_t la, uint32_t lr, int w, int e, int r0, int nbh) {
+    if constexpr (C::A_MN) {
+      tma_load_3d_pair(&tmLW, bar, la, feat_box<C>(w, rank, 0, p.n), 0, e);
+      tma_load_3d_pair(&tmLW, bar, la + C::LA_BOX_BYTES, feat_box<C>(w, rank, 1, p.n), 0, e);
+    } else {
+#pragma unroll
+      for (int a = 0; a < C::LK_ATOMS; ++a)
+        tma_load_3d_pair(&tmLW, bar, la + a * C::LA_ATOM, a * 64, feat_box<C>(w, rank, 0, p.n), e);
+    }
+#pragma unroll
+    for (int a = 0; a < C::LK_ATOMS; ++a)
+      for (int j = 0; j < nbh; ++j)
+        tma_load_2d_pair(&tmLR, bar, lr + a * C::LR_ATOM + j * C::LR_BOX_BYTES, a * 64, r0 + j * C::BOXR);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     // The whole warp waits (converged), lane 0 issues the copies.
@@ -171,6 +274,7 @@ __global__ void __launch_bounds__(320, 1)
       const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
       const int nbh = (half + C::BOXR - 1) / C::BOXR;
       const int r0 = ch.row0 + (int)rank * half;
+      const uint32_t lbytes = C::LA_BYTES + C::LK_ATOMS * nbh * C::LR_BOX_BYTES;
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       if constexpr (C::LSIDE) {
         // LoRA operands of this tile into side buffer it & 1
@@ -178,22 +282,13 @@ __global__ void __launch_bounds__(320, 1)
         const bool lok = mbar_wait(smem_u32(&lempty[lb]), ((it >> 1) & 1) ^ 1, p.err);
         if (!__all_sync(0xffffffffu, lok)) { ok = false; break; }
         if (lane == 0) {
-          const uint32_t lfb = mapa_smem(smem_u32(&lfull[lb]), 0);
           const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
-          const uint32_t lr = la + C::LA_BYTES;
-          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&lfull[lb]), 2 * (C::LA_BYTES + nbh * C::LR_BOX_BYTES));
-          if constexpr (C::A_MN) {
-            tma_load_3d_pair(&tmLW, lfb, la, feat_box(w, rank, 0), 0, ch.e);
-            tma_load_3d_pair(&tmLW, lfb, la + C::LA_BOX_BYTES, feat_box(w, rank, 1), 0, ch.e);
-          } else {
-            tma_load_3d_pair(&tmLW, lfb, la, 0, feat_box(w, rank, 0), ch.e);
-          }
-          for (int j = 0; j < nbh; ++j)
-            tma_load_2d_pair(&tmLR, lfb, lr + j * C::LR_BOX_BYTES, 0, r0 + j * C::BOXR);
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&lfull[lb]), 2 * lbytes);
+          load_lora(mapa_smem(smem_u32(&lfull[lb]), 0), la, la + C::LA_BYTES, w, ch.e, r0, nbh);
         }
         __syncwarp();
       }
-      for (int ks = 0; ks < p.nk + (C::LSIDE ? 0 : 1); ++ks) {
+      for (int ks = 0; ks < p.nk + NST; ++ks) {
         const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
         if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
         if (lane == 0) {
@@ -204,35 +299,32 @@ __global__ void __launch_bounds__(320, 1)
             // every copy is full-size (rows past the chunk are loaded and ignored,
             // rows past P and K past the end read as zero)
             const int k0 = ks * C::BK;
-            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + C::B_BYTES));
+            if (rank == 0)
+              mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + (C::GATHER ? 0 : C::B_BYTES)));
             if constexpr (C::V) {
-              if constexpr (C::A_MN)
-                tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box(w, rank, 0) / 64, ch.e);
+              if constexpr (C::EPI == EPI_SWIGLU)
+                tma_load_5d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, 0, ch.e);
+              else if constexpr (C::A_MN)
+                tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, ch.e);
               else
-                tma_load_4d_pair(&tmW, fb, sa, 0, feat_box(w, rank, 0), k0 / C::KA, ch.e);
-              tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
+                tma_load_4d_pair(&tmW, fb, sa, 0, feat_box<C>(w, rank, 0, p.n), k0 / C::KA, ch.e);
+              if constexpr (!C::GATHER) tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
             } else {
               if constexpr (C::A_MN) {
-                tma_load_3d_pair(&tmW, fb, sa, feat_box(w, rank, 0), k0, ch.e);
-                tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box(w, rank, 1), k0, ch.e);
+                tma_load_3d_pair(&tmW, fb, sa, feat_box<C>(w, rank, 0, p.n), k0, ch.e);
+                tma_load_3d_pair(&tmW, fb, sa + C::A_BYTES / 2, feat_box<C>(w, rank, 1, p.n), k0, ch.e);
               } else {
-                tma_load_3d_pair(&tmW, fb, sa, k0, feat_box(w, rank, 0), ch.e);
-                tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box(w, rank, 0), ch.e);
+                tma_load_3d_pair(&tmW, fb, sa, k0, feat_box<C>(w, rank, 0, p.n), ch.e);
+                tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box<C>(w, rank, 0, p.n), ch.e);
               }
-              tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
-              tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
+              if constexpr (!C::GATHER) {
+                tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
+                tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
+              }
             }
           } else {
-            const uint32_t bytes = C::LA_BYTES + nbh * C::LR_BOX_BYTES;
-            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * bytes);
-            if constexpr (C::A_MN) {
-              tma_load_3d_pair(&tmLW, fb, sa, feat_box(w, rank, 0), 0, ch.e);
-              tma_load_3d_pair(&tmLW, fb, sa + C::LA_BOX_BYTES, feat_box(w, rank, 1), 0, ch.e);
-            } else {
-              tma_load_3d_pair(&tmLW, fb, sa, 0, feat_box(w, rank, 0), ch.e);
-            }
-            for (int j = 0; j < nbh; ++j)
-              tma_load_2d_pair(&tmLR, fb, sb + j * C::LR_BOX_BYTES, 0, r0 + j * C::BOXR);
+            if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * lbytes);
+            load_lora(fb, sa, sb, w, ch.e, r0, nbh);
           }
         }
         __syncwarp();
@@ -251,13 +343,22 @@ __global__ void __launch_bounds__(320, 1)
                                        : smem_desc(s_base, 16, 1024, kSw128);
       const uint64_t b_desc0 = smem_desc(s_base + C::A_BYTES, 16, 1024, kSw128);
       const uint64_t la_desc0 = C::A_MN ? smem_desc(s_base, C::LA_BOX_BYTES, 1024, kSw128)
-                                        : smem_desc(s_base, 16, C::LR_SBO, C::LR_SWZ);
-      const uint64_t lr_desc0 = smem_desc(s_base + C::A_BYTES, 16, C::LR_SBO, C::LR_SWZ);
+                                        : smem_desc(s_base, 16, C::LK_SBO, C::LK_SW);
+      const uint64_t lr_desc0 = smem_desc(s_base + C::A_BYTES, 16, C::LK_SBO, C::LK_SW);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       bool issued_any = false;
+      // the LoRA block's K steps at LoRA operands la (A) / lr (B) + offsets
+      auto lora_mmas = [&](uint32_t d, uint64_t la0, uint64_t lr0, uint32_t idesc, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < C::RP / 16; ++kk) {
+          const uint32_t ao = C::A_MN ? (uint32_t)(kk * 2048) >> 4 : lk_step<C>(kk, C::LA_ATOM);
+          umma_bf16_pair(d, la0 + ao, lr0 + lk_step<C>(kk, C::LR_ATOM), idesc,
+                         (first && kk == 0) ? 0u : 1u);
+        }
+      };
       for (int t = pair; t < total && ok; t += npairs, ++it) {
         const int c = t / p.n_ftiles;
         const TileInfo ch = p.chunks[c];
@@ -277,20 +378,17 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
           if (lane == 0) {
             const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
-            const uint32_t lr = la + C::LA_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < C::RP / 16; ++kk) {
-              const uint64_t ad = C::A_MN ? smem_desc(la + kk * 2048, C::LA_BOX_BYTES, 1024, kSw128)
-                                          : smem_desc(la + kk * 32, 16, C::LR_SBO, C::LR_SWZ);
-              umma_bf16_pair(d, ad, smem_desc(lr + kk * 32, 16, C::LR_SBO, C::LR_SWZ), idesc,
-                             kk ? 1u : 0u);
-            }
+            const uint64_t la0 = C::A_MN ? smem_desc(la, C::LA_BOX_BYTES, 1024, kSw128)
+                                         : smem_desc(la, 16, C::LK_SBO, C::LK_SW);
+            lora_mmas(d, la0, smem_desc(la + C::LA_BYTES, 16, C::LK_SBO, C::LK_SW), idesc, true);
             umma_commit_pair(smem_u32(&lempty[lb]), 0x3);
           }
           __syncwarp();
         }
-        for (int ks = 0; ks < p.nk + (C::LSIDE ? 0 : 1); ++ks) {
-          const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
+        for (int ks = 0; ks < p.nk + NST; ++ks) {
+          bool fok;
+          if constexpr (C::GATHER) fok = mbar_wait_cluster(smem_u32(&full[stage]), phase, p.err);
+          else fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
           if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
           tc_fence_after();
           if (lane == 0) {
@@ -307,10 +405,7 @@ __global__ void __launch_bounds__(320, 1)
                                idesc, (C::LSIDE || (ks | kk)) ? 1u : 0u);
               }
             } else {
-#pragma unroll
-              for (int kk = 0; kk < C::RP / 16; ++kk)
-                umma_bf16_pair(d, la_desc0 + so + kk * (C::A_MN ? 2048 / 16 : 32 / 16),
-                               lr_desc0 + so + kk * (32 / 16), idesc, 1u);
+              lora_mmas(d, la_desc0 + so, lr_desc0 + so, idesc, false);
             }
             umma_commit_pair(smem_u32(&empty[stage]), 0x3);
           }
@@ -330,73 +425,194 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 2 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue (warps 2..9, both CTAs)
     const int q = warp & 3;                         // TMEM lane quarter of this warp
-    const int hsel = (warp - 2) >> 2;               // which alternate 32-token chunks
+    const int hsel = (warp - 2) >> 2;               // which alternate 32-token blocks
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const uint32_t acc_empty_leader = mapa_smem(smem_u32(acc_empty), 0);
     uint8_t* blk = epi + (warp - 2) * C::BLK_BYTES; // 32 tokens x 32 features bf16, 64-byte rows
-    const int rrow = lane >> 2, rpart = lane & 3;   // transposed read: 8 rows x 4 parts per pass
+    // SwiGLU: lane quarters 0-1 hold gate features, 2-3 the up features of the same
+    // indices; each gate warp pairs with the up warp two below it (same token blocks).
+    const bool gate_w = q < 2;
+    uint8_t* blk_up = epi + (warp - 4) * C::BLK_BYTES;              // gate warps only
+    const int pbar = 2 + 2 * ((q & 1) + 2 * hsel);                  // 2,4,6,8 and +1
+    if constexpr (C::EPI == EPI_SWIGLU) {
+      if (gate_w) named_bar_arrive(pbar + 1, 64);   // the up warp may stage its first block
+    }
+    const size_t ldo = C::EPI == EPI_PLAIN || C::EPI == EPI_WSCALE ? (size_t)p.F : (size_t)2 * p.n;
     int it = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const int c = t / p.n_ftiles, w = t % p.n_ftiles;
       const TileInfo ch = p.chunks[c];
       const int nrows = ch.row_end - ch.row0;
       const int b = it & 1;
-      const int fq = w * 256 + (int)rank * 128 + q * 32;   // first feature of this warp
+      // first feature of this warp: SwiGLU h-feature index, else the output column
+      const int fq = C::EPI == EPI_SWIGLU ? w * 128 + (int)rank * 64 + (q & 1) * 32
+                                          : w * 256 + (int)rank * 128 + q * 32;
       const bool ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
       if (named_bar_or(1, 32 * C::EPI_WARPS, !ok || *abort_flag != 0)) { *abort_flag = 1; break; }
       tc_fence_after();
       const uint32_t acc = tmem + lane_base + b * C::NMAX;
-      uint32_t v[32], vn[32];
-      int c0 = hsel * 32;
-      if (c0 < nrows) { tmem_ld32(acc + c0, v); tmem_wait_ld(); }
-      for (; c0 < nrows; c0 += 64) {
-        const bool more = c0 + 64 < nrows;
-        if (more) tmem_ld32(acc + c0 + 64, vn);          // next chunk, in flight meanwhile
-        if (lane == 0) bulk_wait_read<0>();               // the last store from blk has read it
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
+      uint32_t v[32];
+      for (int c0 = hsel * 32; c0 < nrows; c0 += 64) {
+        tmem_ld32(acc + c0, v);
+        tmem_wait_ld();
         const int grow = ch.row0 + c0;
-        if (c0 + 32 <= nrows) {
-          // 32 rows inside the chunk: one TMA tensor store of the block (features past F
-          // are clipped by the tensor map)
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmOut, smem_u32(blk), fq, grow);
-            bulk_commit_group();
+        const int rows_left = nrows - c0;
+        if constexpr (C::EPI == EPI_WSCALE || C::EPI == EPI_DSWIGLU) {
+          // the routing weight of each token of the block (lane i holds token i's)
+          const float wl = lane < rows_left ? p.w[p.sorted_pairs[grow + lane]] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            v[i] = __float_as_uint(__uint_as_float(v[i]) * __shfl_sync(0xffffffffu, wl, i));
+        }
+        if (lane == 0) bulk_wait_read<0>();         // the last store from blk has read it
+        __syncwarp();
+        if constexpr (C::EPI == EPI_PLAIN || C::EPI == EPI_WSCALE) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
+          epi_store_block(&tmOut, blk, fq, grow, rows_left, p.out, ldo, p.F);
+        } else if constexpr (C::EPI == EPI_SWIGLU) {
+          if (!gate_w) {
+            // u: stage it once the gate warp has read the previous block, store it
+            // (GU columns n + f), then hand the staging block to the gate warp
+            named_bar(pbar + 1, 64);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
+            epi_store_block(&tmOut2, blk, fq, grow, rows_left, p.out + p.n, ldo, p.n);
+            named_bar_arrive(pbar, 64);
+          } else {
+            // g: store it (GU columns f), then h = silu(g) u from the bf16-rounded g and
+            // the up warp's staged u, stored to H
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat16 gb = __float2bfloat16_rn(__uint_as_float(v[i]));
+              *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = gb;
+              v[i] = __float_as_uint(__bfloat162float(gb));
+            }
+            epi_store_block(&tmOut, blk, fq, grow, rows_left, p.out, ldo, p.n);
+            named_bar(pbar, 64);                     // u staged
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float u = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(blk_up + i * 64 + lane * 2));
+              const float a = 0.5f * __uint_as_float(v[i]);   // silu(g) = a (1 + tanh(a)), a = g / 2
+              v[i] = __float_as_uint(fmaf(a, tanh_approx(a), a) * u);
+            }
+            named_bar_arrive(pbar + 1, 64);          // done with the up block
+            if (lane == 0) bulk_wait_read<0>();      // the g store has read blk
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
+            epi_store_block(&tmOut3, blk, fq, grow, rows_left, p.out_h, (size_t)p.n, p.n);
           }
         } else {
-          // the chunk's ragged last block: its rows past the end belong to the next
-          // chunk, so 16-byte stores of the rows inside only
+          // EPI_DSWIGLU: v = dH of feature fq + lane for the block's tokens
+          const int f = fq + lane;
+          uint32_t gu2[32];                          // (u << 16) | g, bf16 bits
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            uint32_t g16 = 0, u16 = 0;
+            if (i < rows_left && f < p.n) {
+              const unsigned short* row = reinterpret_cast<const unsigned short*>(p.gu + (size_t)(grow + i) * ldo);
+              g16 = __ldg(row + f);
+              u16 = __ldg(row + p.n + f);
+            }
+            gu2[i] = g16 | (u16 << 16);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = bf16_lo(gu2[i]), u = bf16_hi(gu2[i]);
+            const float dh = __uint_as_float(v[i]);
+            const float s = fmaf(0.5f, tanh_approx(0.5f * g), 0.5f);          // sigmoid(g)
+            const float dg = dh * u * s * (1.0f + g * (1.0f - s));
+            const float du = dh * g * s;
+            *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(dg);
+            v[i] = __float_as_uint(du);
+          }
+          epi_store_block(&tmOut, blk, fq, grow, rows_left, p.out, ldo, p.n);
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int rr = rrow + 8 * j;
-            const int f = fq + rpart * 8;
-            if (c0 + rr < nrows && f < p.F) {
-              const uint4 x = *reinterpret_cast<const uint4*>(blk + rr * 64 + rpart * 16);
-              *reinterpret_cast<uint4*>(p.out + (size_t)(grow + rr) * p.F + f) = x;
-            }
-          }
-        }
-        __syncwarp();
-        if (more) {
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = vn[i];
+          for (int i = 0; i < 32; ++i)
+            *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
+          epi_store_block(&tmOut2, blk, fq, grow, rows_left, p.out + p.n, ldo, p.n);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_leader + b * 8);
     }
+    if constexpr (C::EPI == EPI_SWIGLU) {
+      if (!gate_w) named_bar(pbar + 1, 64);   // the gate warp's last hand-back
+    }
     if (lane == 0) bulk_wait<0>();                        // every store of this warp complete
     __syncwarp();
+  } else {
+    // ------------------------------------------------------------ gather warps (GATHER, both CTAs)
+    // Rows of this CTA's half of the chunk, 16-byte pieces into the two K atoms of the
+    // stage's B area; each warp arrives on the leader's full barrier once its lanes'
+    // pieces of the stage have landed (one stage in flight behind the one issued).
+    if constexpr (C::GATHER) {
+      const int gt = (warp - 2 - C::EPI_WARPS) * 32 + lane;   // 0..127
+      const int cv = gt & 7, rb = gt >> 3;                     // rows rb + 16 j
+      const uint32_t full_leader = mapa_smem(smem_u32(full), 0);
+      int stage = 0, pend = -1;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const int c = t / p.n_ftiles;
+        const TileInfo ch = p.chunks[c];
+        const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
+        const int r0 = ch.row0 + (int)rank * half;
+        int nv = ch.row_end - r0;                  // rows of this half inside the chunk
+        nv = nv < 0 ? 0 : (nv > half ? half : nv);
+        const __nv_bfloat16* rp[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = rb + 16 * j;
+          rp[j] = r < nv ? p.gsrc + (size_t)(p.sorted_pairs[r0 + r] / p.k) * p.K : nullptr;
+        }
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+        for (int ks = 0; ks < p.nk + NST; ++ks) {
+          const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
+          if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
+          if (ks < p.nk) {
+            const uint32_t sb = s_base + stage * C::STAGE_BYTES + C::A_BYTES;
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              const int col = ks * C::BK + a * C::KA + cv * 8;
+              const bool v = col < p.K;            // columns past K are zero
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (rp[j] == nullptr) continue;    // rows past the chunk: never stored
+                const int r = rb + 16 * j;
+                cp_async_16(sb + a * C::ATOM_B + r * 128 + ((cv ^ (r & 7)) << 4),
+                            v ? (const void*)(rp[j] + col) : (const void*)p.gsrc, v ? 16u : 0u);
+              }
+            }
+          }
+          cp_async_commit();
+          if (pend >= 0) {
+            cp_async_wait<1>();                    // the previous stage's pieces landed
+            fence_proxy_async_smem();              // generic-proxy writes -> tcgen05 reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(full_leader + pend * 8);
+          }
+          pend = stage;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (pend >= 0 && lane == 0) mbar_arrive_cluster(full_leader + pend * 8);
+      if (!ok && lane == 0) *abort_flag = 1;
+      __syncwarp();
+    }
   }
 
   tc_fence_before();

@@ -17,7 +17,10 @@
 //       zero), the rest of the 16 stay zero from the kernel's start),
 //   N = 256 columns of Big (MN-major, 128-byte swizzle, four 64-column atoms),
 //   K = rows of the chunk, 64 per stage,
-// one TMA copy per operand and stage.  A rank of at most 32 uses a quarter of M,
+// one TMA copy per operand and stage (a Big gathered from a token matrix - X for
+// dA_gu, dY for dB_d - comes instead from four gather warps with cp.async into the
+// same layout, so no expert-ordered copy of X or dY exists).  A rank of 16 uses an
+// eighth of M,
 // but each MMA then moves 256 columns of Big: a thin N = r MMA costs the tensor
 // pipe about as long as a full one and would bound the kernel instead of HBM.
 // Every copy is full-size from the chunk's first row, so the stage that crosses the
@@ -25,9 +28,9 @@
 // 16-row K steps that reach into the chunk and zeroes Small's rows past its end in
 // the last of them.
 // The accumulator (128 lanes x 256 fp32 columns) is double buffered in TMEM.  The
-// warp that owns TMEM lanes 0-31 (the rank rows) copies them to shared memory; all
-// four epilogue warps then write the gradient with 16-byte stores in its output
-// orientation.  A unit of an expert whose rows fit in one chunk writes the final
+// warps that own the TMEM lanes of the rank rows copy them to shared memory (in two
+// column halves at ranks above 32); all four epilogue warps then write the gradient
+// with 16-byte stores in its output orientation.  A unit of an expert whose rows fit in one chunk writes the final
 // bf16 gradient (scaled).  Otherwise each unit writes an fp32 partial and counts
 // itself in a per-(expert, column tile) arrival counter; the unit that arrives
 // last sums the expert's partials in chunk order (deterministic, whatever the
@@ -40,6 +43,9 @@
 namespace moe {
 
 struct WgradProblem {
+  // Big gathered from a token matrix when gsrc is set (row q = gsrc[sorted_pairs[q] / k],
+  // D columns), else loaded with TMA from the sorted [P, D] matrix of the tensor map
+  const __nv_bfloat16* gsrc;
   const __nv_bfloat16* small;  // [P, ld_small]
   int ld_small;
   int r_small;                 // columns of `small` to read (rest zero)
@@ -60,12 +66,17 @@ struct WgradParams {
   int E;
   int r;                       // output rank
   float scale;
+  const int32_t* sorted_pairs; // gathered Big rows
+  int k;
   int* err;
 };
 
-template <int RP, bool V_ = true>
+template <int RP, bool V_ = true, bool G_ = false>
 struct WgradCfg {
   static constexpr bool V = V_;             // Big through the atom view (D % 64 == 0)
+  static constexpr bool G = G_;             // gather warps for a gathered Big
+  static constexpr int GATHER_WARPS = G ? 4 : 0;
+  static constexpr int THREADS = 192 + 32 * GATHER_WARPS;
   static constexpr int BM = 128;            // rank rows on M (RP of them are used)
   static constexpr int BN = 256;            // Big columns per unit
   static constexpr int BK = 64;             // rows per stage
@@ -75,8 +86,11 @@ struct WgradCfg {
   static constexpr int B_BYTES = (BN / 64) * ATOM;        // 32 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SMALL_COPY = (RP / 8) * SMALL_NG;  // bytes of Small copied per stage
-  static constexpr int STAGES = 4;
-  static constexpr int ST_LD = BN + 4;                    // fp32 staging row (rank j), padded
+  static constexpr int STAGES = RP > 64 ? 3 : 4;
+  // fp32 staging of the accumulator's rank rows, in column halves of SC columns when
+  // the rank is wide (the staging of all 256 columns would not fit beside the ring)
+  static constexpr int SC = RP > 32 ? BN / 2 : BN;
+  static constexpr int ST_LD = SC + 4;                    // fp32 staging row (rank j), padded
   static constexpr int STG_BYTES = RP * ST_LD * 4;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_BYTES + 512 + 1024;
   static constexpr int TMEM_COLS = 2 * BN;
@@ -109,13 +123,14 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, float s, const 
   *reinterpret_cast<uint4*>(dst) = o;
 }
 
-template <int RP, bool V>
-__global__ void __launch_bounds__(192, 1)
+template <int RP, bool V, bool G>
+__global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
     lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig0,
                       const __grid_constant__ CUtensorMap tmBig1,
                       const __grid_constant__ CUtensorMap tmSmall0,
                       const __grid_constant__ CUtensorMap tmSmall1, const WgradParams p) {
-  using C = WgradCfg<RP, V>;
+  using C = WgradCfg<RP, V, G>;
+  constexpr int OWNERS = RP <= 32 ? 1 : RP / 32;   // epilogue warps holding rank rows
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -134,21 +149,21 @@ __global__ void __launch_bounds__(192, 1)
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&full[s]), 1 + C::GATHER_WARPS);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), OWNERS);
     }
     mbar_init(smem_u32(drain), 1);
     *abort_flag = 0;
     *last_flag = 0;
     mbar_fence_init();
-    tma_prefetch_desc(&tmBig0);
+    if (p.pr[0].gsrc == nullptr) tma_prefetch_desc(&tmBig0);
     tma_prefetch_desc(&tmSmall0);
     if (p.n_problems > 1) {
-      tma_prefetch_desc(&tmBig1);
+      if (p.pr[1].gsrc == nullptr) tma_prefetch_desc(&tmBig1);
       tma_prefetch_desc(&tmSmall1);
     }
   }
@@ -178,6 +193,7 @@ __global__ void __launch_bounds__(192, 1)
       const WgradUnit u = wgrad_unit(p, nch, t);
       const CUtensorMap* tb = u.prob == 0 ? &tmBig0 : &tmBig1;
       const CUtensorMap* ts = u.prob == 0 ? &tmSmall0 : &tmSmall1;
+      const bool gathered = p.pr[u.prob].gsrc != nullptr;
       const TileInfo ch = p.chunks[u.c];
       const int d0 = u.dt * C::BN;
       const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
@@ -190,15 +206,17 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           const int r0 = ch.row0 + ks * C::BK;
-          mbar_arrive_expect_tx(fb, C::SMALL_COPY + C::B_BYTES);
+          mbar_arrive_expect_tx(fb, C::SMALL_COPY + (gathered ? 0 : C::B_BYTES));
           // Small [BK rows][RP / 8 groups of 8 rank columns] (MN-major, no swizzle: core
           // matrices of 8 rows x 8 columns)
           tma_load_3d(ts, fb, sa, 0, r0, 0);
-          if constexpr (C::V) {
-            tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
-          } else {
+          if (!gathered) {
+            if constexpr (C::V) {
+              tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
+            } else {
 #pragma unroll
-            for (int a = 0; a < C::BN / 64; ++a) tma_load_2d(tb, fb, sb + a * C::ATOM, d0 + a * 64, r0);
+              for (int a = 0; a < C::BN / 64; ++a) tma_load_2d(tb, fb, sb + a * C::ATOM, d0 + a * 64, r0);
+            }
           }
         }
         __syncwarp();
@@ -267,80 +285,90 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(smem_u32(drain), 0, p.err);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ---------------------------------------------------------- epilogue (warps 2..5)
     const int et = (warp - 2) * 32 + lane;         // 0..127
-    const bool owner = (warp & 3) == 0;            // the warp of TMEM lanes 0-31 (rank rows)
+    const int q4 = warp & 3;                       // TMEM lane quarter: rank rows 32 q4 ..
+    const bool owner = q4 < OWNERS;
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const WgradUnit u = wgrad_unit(p, nch, t);
       const WgradProblem& q = p.pr[u.prob];
       const TileInfo ch = p.chunks[u.c];
       const int b = it & 1;
+      const int d0 = u.dt * C::BN;
+      const int c0 = p.chunk_start[ch.e], c1 = p.chunk_start[ch.e + 1];
       bool ok = true;
       if (owner) {
         ok = mbar_wait(smem_u32(&acc_full[b]), (it >> 1) & 1, p.err);
-        if (ok) {
-          // rank row `lane` of the accumulator -> staging row lane (fp32)
-          tc_fence_after();
-          const uint32_t acc = tmem + b * C::BN;
+        tc_fence_after();
+      }
+      if (named_bar_or(1, C::EPI_THREADS, !ok || *abort_flag != 0)) { *abort_flag = 1; break; }
 #pragma unroll 1
-          for (int c0 = 0; c0 < C::BN; c0 += 32) {
+      for (int hf = 0; hf < C::BN / C::SC; ++hf) {
+        const int cb = d0 + hf * C::SC;            // first Big column of this half
+        if (owner) {
+          // rank row 32 q4 + lane of the accumulator -> staging row (fp32)
+          const uint32_t acc = tmem + ((uint32_t)(q4 * 32) << 16) + b * C::BN + hf * C::SC;
+          const int j = q4 * 32 + lane;
+#pragma unroll 1
+          for (int cc = 0; cc < C::SC; cc += 32) {
             uint32_t v[32];
-            tmem_ld32(acc + c0, v);
+            tmem_ld32(acc + cc, v);
             tmem_wait_ld();
-            if (lane < RP) {
-              float4* dst = reinterpret_cast<float4*>(stg + lane * C::ST_LD + c0);
+            if (j < RP) {
+              float4* dst = reinterpret_cast<float4*>(stg + j * C::ST_LD + cc);
 #pragma unroll
               for (int i = 0; i < 8; ++i)
                 dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
                                      __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
             }
           }
-          tc_fence_before();
+          if (hf == C::BN / C::SC - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
-      }
-      // every epilogue warp takes the same branch (named barriers follow)
-      if (named_bar_or(1, C::EPI_THREADS, !ok || *abort_flag != 0)) { *abort_flag = 1; break; }
-      const int d0 = u.dt * C::BN;
-      const int c0 = p.chunk_start[ch.e], c1 = p.chunk_start[ch.e + 1];
-      if (c1 - c0 == 1) {
-        if (q.transpose) {
-          // out [E][r][D]: row j, 8 consecutive columns per store
-          for (int i = et; i < p.r * (C::BN / 8); i += C::EPI_THREADS) {
-            const int j = i / (C::BN / 8), cc = (i - j * (C::BN / 8)) * 8;
-            if (d0 + cc >= q.D) continue;
-            float v[8];
+        named_bar(1, C::EPI_THREADS);              // staging of this half complete
+        if (c1 - c0 == 1) {
+          if (q.transpose) {
+            // out [E][r][D]: row j, 8 consecutive columns per store
+            for (int i = et; i < p.r * (C::SC / 8); i += C::EPI_THREADS) {
+              const int j = i / (C::SC / 8), cc = (i - j * (C::SC / 8)) * 8;
+              if (cb + cc >= q.D) continue;
+              float v[8];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v[x] = stg[j * C::ST_LD + cc + x];
-            store_bf16x8(q.out + ((size_t)ch.e * p.r + j) * q.D + d0 + cc, p.scale, v);
+              for (int x = 0; x < 8; ++x) v[x] = stg[j * C::ST_LD + cc + x];
+              store_bf16x8(q.out + ((size_t)ch.e * p.r + j) * q.D + cb + cc, p.scale, v);
+            }
+          } else {
+            // out [E][D][r]: column d, 8 consecutive rank entries per store
+            for (int i = et; i < C::SC * (p.r / 8); i += C::EPI_THREADS) {
+              const int dd = i / (p.r / 8), g = i - dd * (p.r / 8);
+              if (cb + dd >= q.D) continue;
+              float v[8];
+#pragma unroll
+              for (int x = 0; x < 8; ++x) v[x] = stg[(g * 8 + x) * C::ST_LD + dd];
+              store_bf16x8(q.out + ((size_t)ch.e * q.D + cb + dd) * p.r + g * 8, p.scale, v);
+            }
           }
         } else {
-          // out [E][D][r]: column d, 8 consecutive rank entries per store
-          for (int i = et; i < C::BN * (p.r / 8); i += C::EPI_THREADS) {
-            const int dd = i / (p.r / 8), g = i - dd * (p.r / 8);
-            if (d0 + dd >= q.D) continue;
-            float v[8];
+          // several chunks: fp32 partial [chunk][d][RP] of this half
+          for (int dd = et; dd < C::SC; dd += C::EPI_THREADS) {
+            if (cb + dd >= q.D) continue;
+            float4* dst = reinterpret_cast<float4*>(q.partial + ((size_t)u.c * q.D + cb + dd) * RP);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v[x] = stg[(g * 8 + x) * C::ST_LD + dd];
-            store_bf16x8(q.out + ((size_t)ch.e * q.D + d0 + dd) * p.r + g * 8, p.scale, v);
+            for (int i = 0; i < RP / 4; ++i)
+              dst[i] = make_float4(stg[(4 * i) * C::ST_LD + dd], stg[(4 * i + 1) * C::ST_LD + dd],
+                                   stg[(4 * i + 2) * C::ST_LD + dd], stg[(4 * i + 3) * C::ST_LD + dd]);
           }
         }
-        named_bar(1, C::EPI_THREADS);             // staging is rewritten by the next unit
-        continue;
+        named_bar(1, C::EPI_THREADS);              // staging is rewritten by the next half
       }
-      // several chunks: fp32 partial [chunk][d][RP], then the last arriving unit sums
-      // the expert's partials in chunk order and writes the gradient
-      for (int dd = et; dd < C::BN; dd += C::EPI_THREADS) {
-        if (d0 + dd >= q.D) continue;
-        float4* dst = reinterpret_cast<float4*>(q.partial + ((size_t)u.c * q.D + d0 + dd) * RP);
-#pragma unroll
-        for (int i = 0; i < RP / 4; ++i)
-          dst[i] = make_float4(stg[(4 * i) * C::ST_LD + dd], stg[(4 * i + 1) * C::ST_LD + dd],
-                               stg[(4 * i + 2) * C::ST_LD + dd], stg[(4 * i + 3) * C::ST_LD + dd]);
-      }
+      if (c1 - c0 == 1) continue;
+      // the last arriving unit of the expert's chunks sums their partials in chunk order
+      // and writes the gradient
       __threadfence();
       named_bar(1, C::EPI_THREADS);
       if (et == 0) {
@@ -354,40 +382,29 @@ __global__ void __launch_bounds__(192, 1)
       }
       named_bar(1, C::EPI_THREADS);
       if (*last_flag) {
-        for (int dd = et; dd < C::BN; dd += C::EPI_THREADS) {
+        for (int i = et; i < C::BN * (RP / 8); i += C::EPI_THREADS) {
+          const int dd = i / (RP / 8), g = i - dd * (RP / 8);
           const int dg = d0 + dd;
-          if (dg >= q.D) continue;
-          float acc[RP];
+          if (dg >= q.D || g * 8 >= p.r) continue;
+          float acc[8];
 #pragma unroll
-          for (int i = 0; i < RP; ++i) acc[i] = 0.f;
+          for (int x = 0; x < 8; ++x) acc[x] = 0.f;
           for (int cc = c0; cc < c1; ++cc) {
-            const float4* src = reinterpret_cast<const float4*>(q.partial + ((size_t)cc * q.D + dg) * RP);
-#pragma unroll
-            for (int i = 0; i < RP / 4; ++i) {
-              const float4 x = __ldcg(src + i);
-              acc[4 * i] += x.x;
-              acc[4 * i + 1] += x.y;
-              acc[4 * i + 2] += x.z;
-              acc[4 * i + 3] += x.w;
-            }
+            const float4* src = reinterpret_cast<const float4*>(q.partial + ((size_t)cc * q.D + dg) * RP + g * 8);
+            const float4 x0 = __ldcg(src), x1 = __ldcg(src + 1);
+            acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+            acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
           }
           if (q.transpose) {
 #pragma unroll
-            for (int i = 0; i < RP; ++i)
-              if (i < p.r) q.out[((size_t)ch.e * p.r + i) * q.D + dg] = __float2bfloat16_rn(p.scale * acc[i]);
+            for (int x = 0; x < 8; ++x)
+              q.out[((size_t)ch.e * p.r + g * 8 + x) * q.D + dg] = __float2bfloat16_rn(p.scale * acc[x]);
           } else {
-#pragma unroll
-            for (int g = 0; g < RP / 8; ++g)
-              if (g * 8 < p.r) {
-                float v[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) v[x] = acc[8 * g + x];
-                store_bf16x8(q.out + ((size_t)ch.e * q.D + dg) * p.r + 8 * g, p.scale, v);
-              }
+            store_bf16x8(q.out + ((size_t)ch.e * q.D + dg) * p.r + 8 * g, p.scale, acc);
           }
         }
       }
-      named_bar(1, C::EPI_THREADS);                 // the flag and staging are rewritten next
+      named_bar(1, C::EPI_THREADS);                 // the flag is rewritten next
     }
     // gradients of experts without rows are zero (D * r contiguous values in either
     // orientation): after the units, so the scan never holds up the accumulators;
@@ -401,6 +418,64 @@ __global__ void __launch_bounds__(192, 1)
         for (int64_t i = et; i < n8; i += C::EPI_THREADS)
           store_bf16x8(q.out + (size_t)e * q.D * p.r + i * 8, 0.f, z);
       }
+    }
+  } else {
+    // ---------------------------------------------------------- gather warps (G)
+    // For units whose Big is gathered: the stage's 64 rows x 256 columns, 16-byte
+    // pieces into the four 64-column atoms (rows past the chunk and columns past D
+    // zero: they meet zero rows of Small, and stale bits could be NaN).  Every stage
+    // of every unit gets one arrival per warp, data or not, once the lanes' pieces of
+    // the stage have landed (one stage in flight behind the one issued).
+    if constexpr (C::G) {
+      const int gt = (warp - 6) * 32 + lane;       // 0..127
+      const int cv = gt & 7, rb = gt >> 3;         // rows rb + 16 j
+      int stage = 0, pend = -1;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const WgradUnit u = wgrad_unit(p, nch, t);
+        const WgradProblem& q = p.pr[u.prob];
+        const TileInfo ch = p.chunks[u.c];
+        const int d0 = u.dt * C::BN;
+        const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+        for (int ks = 0; ks < nk; ++ks) {
+          const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
+          if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
+          if (q.gsrc != nullptr) {
+            const uint32_t sb = s_base + stage * C::STAGE_BYTES + C::A_BYTES;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int r = rb + 16 * j;
+              const int row = ch.row0 + ks * C::BK + r;
+              const __nv_bfloat16* src = row < ch.row_end
+                  ? q.gsrc + (size_t)(p.sorted_pairs[row] / p.k) * q.D : nullptr;
+#pragma unroll
+              for (int a = 0; a < 4; ++a) {
+                const int col = d0 + a * 64 + cv * 8;
+                const bool v = src != nullptr && col < q.D;
+                cp_async_16(sb + a * C::ATOM + r * 128 + ((cv ^ (r & 7)) << 4),
+                            v ? (const void*)(src + col) : (const void*)q.gsrc, v ? 16u : 0u);
+              }
+            }
+          }
+          cp_async_commit();
+          if (pend >= 0) {
+            cp_async_wait<1>();                    // the previous stage's pieces landed
+            fence_proxy_async_smem();              // generic-proxy writes -> tcgen05 reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&full[pend]));
+          }
+          pend = stage;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (pend >= 0 && lane == 0) mbar_arrive(smem_u32(&full[pend]));
+      if (!ok && lane == 0) *abort_flag = 1;
+      __syncwarp();
     }
   }
 

@@ -1,5 +1,6 @@
 // SIMT kernels of the layer: top-k routing, the stable counting-sort permute,
-// tile tables, row gather, weighted un-permute combine and LoRA padding.
+// tile tables, weighted un-permute combine, router backward and the gathered-row
+// copies of full fine-tuning.
 // All are HBM- or latency-bound; they use coalesced 16-byte accesses and warp
 // primitives, no floating-point atomics.
 #include "common.cuh"
@@ -499,25 +500,42 @@ cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ pad
-__global__ void pad3_kernel(const uint16_t* __restrict__ in, int E, int Ri, int Ci, int Ro, int Co,
-                            uint16_t* __restrict__ out) {
+// ------------------------------------------------------------------ gathered rows
+// The expert-ordered copy of X (or of w dY) for the expert-weight gradients of full
+// fine-tuning: out[q] = (w ? w[p] : 1) src[p / k], p = sorted_pairs[q], 16-byte pieces.
+__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ sp,
+                                   const float* __restrict__ w, int64_t P, int k, int vpr,
+                                   uint4* __restrict__ out) {
   pdl_begin();
-  const int64_t total = (int64_t)E * Ro * Co;
+  const int64_t total = P * vpr;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const int c = (int)(i % Co);
-    const int64_t rr = i / Co;
-    const int r = (int)(rr % Ro);
-    const int64_t e = rr / Ro;
-    out[i] = (r < Ri && c < Ci) ? in[(e * Ri + r) * Ci + c] : (uint16_t)0;
+    const int64_t q = i / vpr;
+    const int v = (int)(i - q * vpr);
+    const int32_t p = sp[q];
+    uint4 x = src[(int64_t)(p / k) * vpr + v];
+    if (w != nullptr) {
+      float f[8];
+      unpack8(x, f);
+      const float s = w[p];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) f[c] *= s;
+      x = pack8(f);
+    }
+    out[i] = x;
   }
 }
 
-cudaError_t launch_pad3(const uint16_t* in, int E, int Ri, int Ci, int Ro, int Co, uint16_t* out,
-                        cudaStream_t s) {
-  ProfScope ps(K_PAD, s);
-  if (cudaError_t le_ = launch_pdl(pad3_kernel, dim3(grid_for((int64_t)E * Ro * Co, 256)), dim3(256), 0, s, 1, in, E, Ri, Ci, Ro, Co, out); le_ != cudaSuccess) return le_;
+cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
+                               int64_t P, int k, int K, uint16_t* out, cudaStream_t s) {
+  if (P == 0) return cudaSuccess;
+  const int vpr = K / 8;
+  ProfScope ps(K_GATHER_ROWS, s);
+  if (cudaError_t le_ = launch_pdl(gather_rows_kernel, dim3(grid_for(P * vpr, 256)), dim3(256), 0, s, 1,
+                                   reinterpret_cast<const uint4*>(src), sorted_pairs, w, P, k, vpr,
+                                   reinterpret_cast<uint4*>(out));
+      le_ != cudaSuccess)
+    return le_;
   return cudaGetLastError();
 }
 

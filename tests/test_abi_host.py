@@ -57,7 +57,7 @@ def dims(**kw):
 def test_workspace_bytes_supported_and_not(L):
     assert ml.moe_workspace_bytes(dims()) > 0
     for bad in (dict(k=0), dict(k=33, E=64), dict(E=1025), dict(m=120), dict(n=8), dict(r=12),
-                dict(r=40), dict(E=1, k=2), dict(T=-1)):
+                dict(r=136), dict(r=44), dict(E=1, k=2), dict(T=-1)):
         assert ml.moe_workspace_bytes(dims(**bad)) == 0, bad
 
 
@@ -85,7 +85,7 @@ def test_host_validation_returns_before_launch(L):
     assert L.moe_permute(fake, 4, 2, 8, fake, fake, fake, fake, fake, 8, null) == ml.MOE_ERR_WORKSPACE
     # forward: bad dims, NULL / misaligned pointers, small workspace
     d = dims()
-    ptrs = [P(4096)] * 16
+    ptrs = [P(4096)] * 15
     assert L.moe_grouped_gemm_lora_fwd(ctypes.byref(dims(m=100)), *ptrs, 1 << 30, null) == ml.MOE_ERR_UNSUPPORTED
     assert L.moe_grouped_gemm_lora_fwd(None, *ptrs, 1 << 30, null) == ml.MOE_ERR_INVALID_ARG
     bad = list(ptrs)

@@ -122,6 +122,12 @@ EDGE = {
     "rank24_padded": small_config(T=90, m=96, n=48, E=5, k=3, r=24, alpha=48),
     "k_equals_E": small_config(T=70, m=64, n=32, E=8, k=8, r=8, alpha=8),
     "long_K": small_config(T=130, m=1024, n=320, E=4, k=2, r=16, alpha=16),
+    # wide ranks: the rank the pages benchmark at (64), the widest supported (128),
+    # and ranks padded up to them (48 -> 64, 96 -> 128)
+    "rank64": small_config(T=200, m=128, n=96, E=8, k=2, r=64, alpha=64),
+    "rank48_padded": small_config(T=90, m=192, n=64, E=5, k=3, r=48, alpha=48),
+    "rank128": small_config(T=150, m=256, n=128, E=4, k=2, r=128, alpha=128),
+    "rank96_padded_odd_dims": small_config(T=110, m=144, n=80, E=6, k=2, r=96, alpha=96),
 }
 
 
@@ -242,7 +248,7 @@ def test_graph_replay_matches_eager_bitwise():
     cfg = small_config(T=640, m=256, n=128, E=8, k=2, r=16, alpha=16)
     inp, _ = inputs_on(cfg, seed=11)
     eager = run_layer(inp, cfg)
-    keys = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU", "save_Xs", "Y_sorted")
+    keys = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU", "save_H", "Y_sorted")
     snap = {k: getattr(eager, k).clone() for k in keys}
     buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale)
     s = torch.cuda.Stream()
