@@ -139,31 +139,32 @@ def kernel_work(cfg, active_experts=None):
     P = T * k
     rp = 16 if r <= 16 else 32 if r <= 32 else 64 if r <= 64 else 128
     tok = T * m * 2                                       # X or dY, read once
+    rows = P * m * 2                                      # expert-ordered X or w dY
     lrc = P * rp * 2                                      # one [P, rp] rank-r operand
     return {
         "gemm_gateup_fwd": {"flop": acc.flops_gemm_gate_up_fwd(T, m, n, k, r),
-                            "byte": Ea * m * 2 * n * 2 + tok + lrc + Ea * r * 2 * n * 2
+                            "byte": Ea * m * 2 * n * 2 + rows + lrc + Ea * r * 2 * n * 2
                                     + P * 2 * n * 2 + P * n * 2},            # GU and H written
         "gemm_down_fwd": {"flop": acc.flops_gemm_down_fwd(T, m, n, k, r),
                           "byte": Ea * n * m * 2 + P * n * 2 + lrc + Ea * r * m * 2 + P * m * 2},
         "gemm_down_bwd": {"flop": acc.flops_gemm_down_bwd(T, m, n, k, r),
-                          "byte": Ea * n * m * 2 + tok + lrc + Ea * n * r * 2 + P * 4
-                                  + P * 2 * n * 2 + P * 2 * n * 2},          # GU read, dGU written
+                          "byte": Ea * n * m * 2 + rows + lrc + Ea * n * r * 2 + P * n * 2},
         "gemm_gateup_bwd": {"flop": acc.flops_gemm_gate_up_bwd(T, m, n, k, r),
                             "byte": Ea * m * 2 * n * 2 + P * 2 * n * 2 + lrc + Ea * m * r * 2 + P * m * 2},
-        "rank_xa": {"byte": tok + E * m * r * 2 + P * r * 2 + lrc},
+        # gathered X rows written in expert order, XA (saved) and bf16(c XA)
+        "rank_xa": {"byte": tok + P * 4 + rows + E * m * r * 2 + P * r * 2 + lrc},
         "rank_ha": {"byte": P * n * 2 + E * n * r * 2 + P * r * 2 + lrc},
-        "rank_t1": {"byte": tok + E * r * m * 2 + P * r * 2 + P * 4 + 3 * lrc},
-        "rank_t2": {"byte": P * 2 * n * 2 + E * r * 2 * n * 2 + 2 * lrc},
-        # two launches: (H, dY gathered) -> dA_d, dB_d; (dGU, X gathered) -> dB_gu, dA_gu
-        "lora_wgrad": {"byte": P * n * 2 + tok + 2 * lrc + E * r * (n + m) * 2
-                               + P * 2 * n * 2 + tok + P * r * 2 + lrc + E * r * (m + 2 * n) * 2},
+        # gathered w dY rows written in expert order, T1 and bf16(c T1)
+        "rank_t1": {"byte": tok + P * 8 + rows + E * r * m * 2 + 2 * lrc},
+        # the SwiGLU backward (dH and GU read, dGU written) with T2 and bf16(c T2)
+        "rank_t2": {"byte": P * n * 2 + P * 2 * n * 2 + P * 2 * n * 2 + E * r * 2 * n * 2 + 2 * lrc},
+        # two launches: (H, w dY) -> dA_d, dB_d; (dGU, X) -> dB_gu, dA_gu
+        "lora_wgrad": {"byte": P * n * 2 + rows + lrc + P * r * 2 + E * r * (n + m) * 2
+                               + P * 2 * n * 2 + rows + P * r * 2 + lrc + E * r * (m + 2 * n) * 2},
         "route_topk": {"byte": acc.bytes_route(T, E, k)},
         "unpermute_combine": {"byte": 2 * acc.bytes_combine(T, m, k)},  # Y and dX
-        # full fine-tuning only: expert-ordered copies of w dY and X, then the
-        # expert-weight gradients (sorted operands read once, every expert's gradient
-        # written once)
-        "gather_rows": {"byte": 2 * (tok + P * m * 2)},
+        # full fine-tuning only: the expert-weight gradients (sorted operands read once,
+        # every expert's gradient written once)
         "gemm_dw_gu": {"flop": 4 * P * m * n, "byte": P * m * 2 + P * 2 * n * 2 + E * m * 2 * n * 2},
         "gemm_dw_d": {"flop": 2 * P * n * m, "byte": P * n * 2 + P * m * 2 + E * n * m * 2},
     }

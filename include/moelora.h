@@ -115,6 +115,19 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
                          int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                          int32_t* pair_pos, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_route_topk() and moe_permute() in one call, for the common case where the
+ * permutation follows the routing directly: the routing kernel also counts each
+ * block's pairs per expert, so routing and the counting sort take two launches
+ * instead of three.  Same definitions and outputs as the two calls (stable order,
+ * ties to the lower expert index).
+ * ws, ws_bytes: scratch of at least moe_workspace_bytes() for any dims with this T,
+ * E, k (per-chunk histograms of ceil(T / floor(512 / k)) chunks).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+moe_status_t moe_route_permute(const float* logits, int64_t T, int32_t E, int32_t k,
+                               int32_t* topk_ids, float* topk_w, int32_t* counts,
+                               int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
+                               void* ws, size_t ws_bytes, void* stream);
+
 /* Debug check of a permutation, on the device (the stand-in for a sanitizer run, which
  * this library's test machines do not offer): every invariant moe_permute() promises.
  *   offsets[0] = 0, offsets[E] = P, offsets non-decreasing, counts[e] = offsets[e+1] -
@@ -135,14 +148,15 @@ moe_status_t moe_check_permutation(const int32_t* topk_ids, int64_t T, int32_t k
  *   Y_sorted[q] = H[q] W_d[e] + c (H[q] A_d[e]) B_d[e],
  *   H[q]        = silu(GU[q, :n]) * GU[q, n:],
  *   GU[q]       = X[t] W_gu[e] + c (X[t] A_gu[e]) B_gu[e],   t = sorted_pairs[q] / k,
- * for every q in the segment of expert e.  The rows X[t] are gathered inside the
- * kernels; no expert-ordered copy of X is written.
+ * for every q in the segment of expert e.
  * Inputs (device, read): X bf16 [T, m]; sorted_pairs [P]; offsets [E+1]; the six
  *   weight tensors in the layouts above.
  * Outputs (device, written, bf16, sorted order):
- *   Y_sorted [P, m]; save_GU [P, 2n]; save_H [P, n]; save_XA [P, r] = X A_gu
- *   (unscaled); save_HA [P, r] = H A_d (unscaled).  The save_* tensors are what
- *   moe_grouped_gemm_lora_bwd() needs besides X.
+ *   Y_sorted [P, m]; save_Xs [P, m] = X[sorted_pairs / k] (the expert-sorted input
+ *   rows, the grouped GEMM's operand, kept for the backward as an autograd
+ *   implementation keeps the permuted input); save_GU [P, 2n]; save_H [P, n];
+ *   save_XA [P, r] = X A_gu (unscaled); save_HA [P, r] = H A_d (unscaled).  The
+ *   save_* tensors are what moe_grouped_gemm_lora_bwd() needs.
  * Accumulation is fp32; every stored value is rounded once to bf16 (H from the
  * bf16-rounded GU).  The LoRA term multiplies bf16(c * X A) by B.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
@@ -150,8 +164,9 @@ moe_status_t moe_grouped_gemm_lora_fwd(
     const moe_dims_t* dims, const moe_bf16_t* X, const int32_t* sorted_pairs,
     const int32_t* offsets, const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
     const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_GU, moe_bf16_t* save_H,
-    moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws, size_t ws_bytes, void* stream);
+    const moe_bf16_t* B_d, moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs, moe_bf16_t* save_GU,
+    moe_bf16_t* save_H, moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws,
+    size_t ws_bytes, void* stream);
 
 /* Backward of all experts (W frozen) for upstream gradient dY:
  *   dy_q     = w[p] dY[t]                          (p = sorted_pairs[q], t = p / k)
@@ -160,24 +175,22 @@ moe_status_t moe_grouped_gemm_lora_fwd(
  *   T2       = dGU B_gu^T, dX_sorted = dGU W_gu^T + c T2 A_gu^T
  *   dA_d[e]  = c H_e^T T1_e,   dB_d[e]  = c HA_e^T dy_e
  *   dA_gu[e] = c X_e^T T2_e,   dB_gu[e] = c XA_e^T dGU_e
- * The rows dY[t] and X[t] are gathered inside the kernels and the routing weight is
- * applied after the products (by linearity); dH is not written to memory.
- * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; X bf16 [T, m];
- *   sorted_pairs; offsets; the six weights; save_GU, save_H, save_XA, save_HA from
- *   the forward.
+ * Inputs (device, read): dY bf16 [T, m]; topk_w fp32 [T, k]; sorted_pairs;
+ *   offsets; the six weights; save_Xs, save_GU, save_H, save_XA, save_HA from the
+ *   forward.
  * Outputs (device, written, bf16): dX_sorted [P, m] (sorted order; reduce with
  *   moe_unpermute_combine(topk_w = NULL)); dA_gu [E, m, r]; dB_gu [E, r, 2n];
  *   dA_d [E, n, r]; dB_d [E, r, m].  Experts with no rows get zero gradients.
  * Adapter gradients are reduced over rows in a fixed order (deterministic).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
 moe_status_t moe_grouped_gemm_lora_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
-    const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dA_gu,
-    moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
+    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
+    moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
     size_t ws_bytes, void* stream);
 
 /* Backward for full fine-tuning: everything moe_grouped_gemm_lora_bwd() computes,
@@ -195,21 +208,21 @@ moe_status_t moe_grouped_gemm_lora_bwd(
  * outputs and errors as moe_grouped_gemm_lora_bwd(); each weight-gradient tile
  * sums its rows in one fixed order (deterministic). */
 moe_status_t moe_grouped_gemm_full_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets,
     const moe_bf16_t* W_gu, const moe_bf16_t* W_d, const moe_bf16_t* A_gu,
     const moe_bf16_t* B_gu, const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-    const moe_bf16_t* save_GU, const moe_bf16_t* save_H, const moe_bf16_t* save_XA,
-    const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted, moe_bf16_t* dW_gu,
-    moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
-    moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream);
+    const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
+    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
+    moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu,
+    moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream);
 
 /* The same permutation as moe_permute(), for callers that cannot allocate device
  * memory: plug-ins hosted inside another framework that owns all device memory
  * and hands them no allocator, or code that must run with a fixed device-memory
  * footprint decided before it starts.  It takes no workspace; its scratch (the
- * per-chunk histograms) is a 2 MiB array built into the library, which every GPU
- * that loads the library holds until the process exits.  There is no
+ * per-chunk histograms) is a 2 MiB array built into the library (with one counter
+ * after it), which every GPU that loads the library holds until the process exits.  There is no
  * counterpart on the pages: this is an interface convenience.
  * Limit: ceil(T*k / 512) * E <= 524288 (e.g. T*k <= 2^21 pairs at E = 128);
  * larger problems return MOE_ERR_WORKSPACE before any launch.

@@ -33,7 +33,7 @@ EXPORTED = (
     "moe_grouped_gemm_lora_bwd", "moe_unpermute_combine", "moe_get_device_error",
     "moe_status_string", "moe_profile_enable", "moe_profile_select", "moe_profile_read",
     "moe_permute_noalloc", "moe_router_backward", "moe_grouped_gemm_full_bwd",
-    "moe_check_permutation", "moe_selftest_bounded_wait",
+    "moe_check_permutation", "moe_selftest_bounded_wait", "moe_route_permute",
 )
 
 
@@ -67,8 +67,9 @@ def lib() -> ctypes.CDLL:
         h.moe_route_topk.argtypes = [P, I64, I32, I32, P, P, P]
         h.moe_permute.argtypes = [P, I64, I32, I32, P, P, P, P, P, SZ, P]
         h.moe_permute_noalloc.argtypes = [P, I64, I32, I32, P, P, P, P, P]
+        h.moe_route_permute.argtypes = [P, I64, I32, I32, P, P, P, P, P, P, P, SZ, P]
         h.moe_check_permutation.argtypes = [P, I64, I32, I32, P, P, P, P, P]
-        h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 15 + [SZ, P]
+        h.moe_grouped_gemm_lora_fwd.argtypes = [D] + [P] * 16 + [SZ, P]
         h.moe_grouped_gemm_lora_bwd.argtypes = [D] + [P] * 21 + [SZ, P]
         h.moe_grouped_gemm_full_bwd.argtypes = [D] + [P] * 23 + [SZ, P]
         h.moe_unpermute_combine.argtypes = [P, P, P, I64, I32, I32, P, P]
@@ -146,6 +147,18 @@ def moe_permute(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, ws, stream
         moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream)
 
 
+def moe_route_permute(logits, k, topk_ids, topk_w, counts, offsets, sorted_pairs, pair_pos, ws,
+                      stream=None):
+    """moe_route_topk and moe_permute in one call (two launches)."""
+    T, E = logits.shape
+    _check("moe_route_permute", lib().moe_route_permute(
+        _ptr(logits), T, E, int(k), _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(offsets),
+        _ptr(sorted_pairs), _ptr(pair_pos), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    if debug_checks():
+        moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream)
+
+
 def moe_check_permutation(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, stream=None):
     """Device check of every invariant moe_permute promises; a violation sets
     MOE_ERR_DEVICE_CHECK in the device error word (see moe_get_device_error)."""
@@ -166,33 +179,33 @@ def moe_permute_noalloc(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, st
 
 
 def moe_grouped_gemm_lora_fwd(dims, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                              Y_sorted, save_GU, save_H, save_XA, save_HA, ws, stream=None):
-    args = [X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_GU,
+                              Y_sorted, save_Xs, save_GU, save_H, save_XA, save_HA, ws, stream=None):
+    args = [X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_Xs, save_GU,
             save_H, save_XA, save_HA, ws]
     _check("moe_grouped_gemm_lora_fwd", lib().moe_grouped_gemm_lora_fwd(
         ctypes.byref(dims), *[_ptr(a) for a in args], ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
-def moe_grouped_gemm_lora_bwd(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu,
-                              A_d, B_d, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu,
+def moe_grouped_gemm_lora_bwd(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu,
+                              A_d, B_d, save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu,
                               dB_gu, dA_d, dB_d, ws, stream=None):
-    args = [dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU,
+    args = [dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_Xs, save_GU,
             save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, ws]
     _check("moe_grouped_gemm_lora_bwd", lib().moe_grouped_gemm_lora_bwd(
         ctypes.byref(dims), *[_ptr(a) for a in args], ws.numel() * ws.element_size(),
         _stream(stream)))
 
 
-def moe_grouped_gemm_full_bwd(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu,
-                              A_d, B_d, save_GU, save_H, save_XA, save_HA, dX_sorted, dW_gu,
+def moe_grouped_gemm_full_bwd(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu,
+                              A_d, B_d, save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dW_gu,
                               dW_d, dA_gu=None, dB_gu=None, dA_d=None, dB_d=None, ws=None,
                               stream=None):
     """Backward with the expert-weight gradients dW_gu [E, m, 2n] and dW_d [E, n, m]
     (full fine-tuning); the adapter gradients are computed when all four are given."""
     if ws is None:
         raise ValueError("moe_grouped_gemm_full_bwd needs the workspace")
-    args = [dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU,
+    args = [dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_Xs, save_GU,
             save_H, save_XA, save_HA, dX_sorted, dW_gu, dW_d, dA_gu, dB_gu, dA_d, dB_d, ws]
     _check("moe_grouped_gemm_full_bwd", lib().moe_grouped_gemm_full_bwd(
         ctypes.byref(dims), *[_ptr(a) for a in args], ws.numel() * ws.element_size(),
@@ -262,6 +275,7 @@ class LayerBuffers:
     sorted_pairs: torch.Tensor
     pair_pos: torch.Tensor
     Y_sorted: torch.Tensor
+    save_Xs: torch.Tensor
     save_GU: torch.Tensor
     save_H: torch.Tensor
     save_XA: torch.Tensor
@@ -287,7 +301,8 @@ def alloc_buffers(T, m, n, E, k, r, scale, device="cuda") -> LayerBuffers:
         ids=torch.empty(T, k, **i32), w=torch.empty(T, k, dtype=torch.float32, device=device),
         counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
         sorted_pairs=torch.empty(P, **i32), pair_pos=torch.empty(P, **i32),
-        Y_sorted=torch.empty(P, m, **bf), save_GU=torch.empty(P, 2 * n, **bf),
+        Y_sorted=torch.empty(P, m, **bf), save_Xs=torch.empty(P, m, **bf),
+        save_GU=torch.empty(P, 2 * n, **bf),
         save_H=torch.empty(P, n, **bf), save_XA=torch.empty(P, r, **bf),
         save_HA=torch.empty(P, r, **bf), Y=torch.empty(T, m, **bf),
         dX_sorted=torch.empty(P, m, **bf), dX=torch.empty(T, m, **bf),
@@ -302,11 +317,11 @@ def layer_forward(inp: dict, k: int, scale: float, buf: LayerBuffers, stream=Non
     E, _, n2 = inp["W_gu"].shape
     r = inp["A_gu"].shape[2]
     dims = make_dims(T, m, n2 // 2, E, k, r, scale)
-    moe_route_topk(inp["logits"], k, buf.ids, buf.w, stream)
-    moe_permute(buf.ids, E, buf.counts, buf.offsets, buf.sorted_pairs, buf.pair_pos, buf.ws, stream)
+    moe_route_permute(inp["logits"], k, buf.ids, buf.w, buf.counts, buf.offsets, buf.sorted_pairs,
+                      buf.pair_pos, buf.ws, stream)
     moe_grouped_gemm_lora_fwd(dims, inp["X"], buf.sorted_pairs, buf.offsets, inp["W_gu"],
                               inp["W_d"], inp["A_gu"], inp["B_gu"], inp["A_d"], inp["B_d"],
-                              buf.Y_sorted, buf.save_GU, buf.save_H, buf.save_XA,
+                              buf.Y_sorted, buf.save_Xs, buf.save_GU, buf.save_H, buf.save_XA,
                               buf.save_HA, buf.ws, stream)
     moe_unpermute_combine(buf.Y_sorted, buf.w, buf.pair_pos, T, k, m, buf.Y, stream)
     return buf.Y
@@ -318,9 +333,9 @@ def layer_backward(inp: dict, dY, k: int, scale: float, buf: LayerBuffers, strea
     E, _, n2 = inp["W_gu"].shape
     r = inp["A_gu"].shape[2]
     dims = make_dims(T, m, n2 // 2, E, k, r, scale)
-    moe_grouped_gemm_lora_bwd(dims, dY, buf.w, inp["X"], buf.sorted_pairs, buf.offsets,
+    moe_grouped_gemm_lora_bwd(dims, dY, buf.w, buf.sorted_pairs, buf.offsets,
                               inp["W_gu"], inp["W_d"], inp["A_gu"], inp["B_gu"], inp["A_d"],
-                              inp["B_d"], buf.save_GU, buf.save_H, buf.save_XA,
+                              inp["B_d"], buf.save_Xs, buf.save_GU, buf.save_H, buf.save_XA,
                               buf.save_HA,
                               buf.dX_sorted, buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d, buf.ws,
                               stream)
@@ -337,9 +352,9 @@ def layer_backward_full(inp: dict, dY, k: int, scale: float, buf: LayerBuffers, 
     r = inp["A_gu"].shape[2]
     dims = make_dims(T, m, n2 // 2, E, k, r, scale)
     lora = (buf.dA_gu, buf.dB_gu, buf.dA_d, buf.dB_d) if adapters else (None,) * 4
-    moe_grouped_gemm_full_bwd(dims, dY, buf.w, inp["X"], buf.sorted_pairs, buf.offsets,
+    moe_grouped_gemm_full_bwd(dims, dY, buf.w, buf.sorted_pairs, buf.offsets,
                               inp["W_gu"], inp["W_d"], inp["A_gu"], inp["B_gu"], inp["A_d"],
-                              inp["B_d"], buf.save_GU, buf.save_H, buf.save_XA,
+                              inp["B_d"], buf.save_Xs, buf.save_GU, buf.save_H, buf.save_XA,
                               buf.save_HA,
                               buf.dX_sorted, dW_gu, dW_d, *lora, ws=buf.ws, stream=stream)
     moe_unpermute_combine(buf.dX_sorted, None, buf.pair_pos, T, k, m, buf.dX, stream)

@@ -102,8 +102,8 @@ struct Layout {
   int max_row_tiles, max_gchunks, max_chunks, chunk_rows, perm_chunks;
   size_t hist, tiles, n_tiles, gchunks, n_gchunks, chunks, n_chunks, chunk_start;
   int max_dtiles;            // 128-column tiles of the widest adapter gradient
-  size_t rows;               // expert-ordered X or w dY (full fine-tuning only)
-  size_t dgu, t1, t2, lrc1, lrc2, wha, partial, partial2;
+  size_t rows;               // expert-ordered w dY (the backward's token operand)
+  size_t dh, dgu, t1, t2, lrc1, lrc2, partial, partial2;
   size_t counters;           // arrival counters of the four adapter gradients
   size_t total;
 };
@@ -116,7 +116,12 @@ Layout make_layout(const moe_dims_t& d) {
   L.max_gchunks = (int)((L.P + kGemmChunkRows - 1) / kGemmChunkRows) + d.E;
   L.chunk_rows = (int)chunk_rows_for(d, L.P);
   L.max_chunks = (int)((L.P + L.chunk_rows - 1) / L.chunk_rows) + d.E;
-  L.perm_chunks = (int)((L.P + kPermuteChunk - 1) / kPermuteChunk);
+  {
+    // chunks of moe_permute (kPermuteChunk pairs) or of moe_route_permute (whole tokens)
+    const int64_t tpb = route_tokens_per_chunk(d.k);
+    const int64_t a = (L.P + kPermuteChunk - 1) / kPermuteChunk, b = (d.T + tpb - 1) / tpb;
+    L.perm_chunks = (int)(a > b ? a : b);
+  }
   const size_t E = d.E, m = d.m, n = d.n, rp = L.rp, P = (size_t)L.P;
   const size_t dmax = m > 2 * n ? m : 2 * n;
   size_t off = 0;
@@ -130,12 +135,12 @@ Layout make_layout(const moe_dims_t& d) {
   L.n_chunks = take(4);
   L.chunk_start = take((E + 1) * 4);
   L.rows = take(P * m * 2);
+  L.dh = take(P * n * 2);
   L.dgu = take(P * 2 * n * 2);
   L.t1 = take(P * rp * 2);
   L.t2 = take(P * rp * 2);
   L.lrc1 = take(P * rp * 2);
   L.lrc2 = take(P * rp * 2);
-  L.wha = take(P * rp * 2);
   L.partial = take((size_t)L.max_chunks * dmax * rp * 4);
   L.partial2 = take((size_t)L.max_chunks * dmax * rp * 4);
   L.max_dtiles = (int)((dmax + 127) / 128);
@@ -193,15 +198,18 @@ moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32
 }
 
 // The backward pass.  Adapter gradients when dA_gu.. are given (all four or none),
-// expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given.
+// expert-weight gradients (full fine-tuning) when dW_gu, dW_d are given; each weight
+// gradient runs while its sorted operands are at hand (w dY in the row buffer after
+// the rank-r kernel; X sorted saved by the forward).
 moe_status_t backward(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
-    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
-    moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, moe_bf16_t* dW_gu,
-    moe_bf16_t* dW_d, void* ws, size_t ws_bytes, void* stream) {
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU,
+    const moe_bf16_t* save_H, const moe_bf16_t* save_XA, const moe_bf16_t* save_HA,
+    moe_bf16_t* dX_sorted, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
+    moe_bf16_t* dB_d, moe_bf16_t* dW_gu, moe_bf16_t* dW_d, void* ws, size_t ws_bytes,
+    void* stream) {
   moe_status_t st = check_dims(dims);
   if (st != MOE_OK) return st;
   const moe_dims_t d = *dims;
@@ -224,7 +232,7 @@ moe_status_t backward(
     }
     return MOE_OK;
   }
-  const void* ins[] = {dY, X, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_GU, save_H, save_XA,
+  const void* ins[] = {dY, W_gu, W_d, A_gu, B_gu, A_d, B_d, save_Xs, save_GU, save_H, save_XA,
                        save_HA, dX_sorted, ws};
   for (const void* p : ins)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -236,12 +244,12 @@ moe_status_t backward(
   st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, s, &g, &w);
   if (st != MOE_OK) return st;
   uint16_t* rows = at<uint16_t>(ws, L.rows);
+  uint16_t* dh = at<uint16_t>(ws, L.dh);
   uint16_t* dgu = at<uint16_t>(ws, L.dgu);
   uint16_t* t1 = at<uint16_t>(ws, L.t1);
   uint16_t* t2 = at<uint16_t>(ws, L.t2);
   uint16_t* lrc1 = at<uint16_t>(ws, L.lrc1);
   uint16_t* lrc2 = at<uint16_t>(ws, L.lrc2);
-  uint16_t* wha = at<uint16_t>(ws, L.wha);
   float* partial = at<float>(ws, L.partial);
   float* partial2 = at<float>(ws, L.partial2);
   const TileInfo* chunks = at<TileInfo>(ws, L.chunks);
@@ -250,42 +258,33 @@ moe_status_t backward(
   int* counters = at<int>(ws, L.counters);
   const size_t cstride = (size_t)d.E * L.max_dtiles;
   const int rp = L.rp;
-  // T1' = dY B_d^T on rows gathered from dY: t1 = bf16(w T1') (the dA_d operand),
-  // lrc1 = bf16(c T1') (the down backward's LoRA operand), wha = bf16(w HA) (dB_d's)
-  MOE_TRY(launch_rank_gathered(K_RANK_T1, g, dY, d.m, sorted_pairs, d.k, topk_w, w.B_d, false, t1,
-                               rp, rp, true, lrc1, save_HA, d.r, wha, s));
-  // dA_d = c H^T (w T1') and dB_d = c (w HA)^T dY (dY rows gathered), one launch
+  // dy = w dY[t] in expert order (the row buffer), T1 = dy B_d^T (kept for dA_d) and
+  // bf16(c T1)
+  MOE_TRY(launch_rank_gathered(K_RANK_T1, g, dY, d.m, sorted_pairs, d.k, topk_w, rows, w.B_d,
+                               false, t1, rp, rp, lrc1, s));
+  // dH = dy W_d^T + (c T1) A_d^T
+  MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
+  // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
   if (lora) {
-    const WgradJob jobs[2] = {
-        {save_H, nullptr, d.n, t1, rp, false, dA_d, partial, counters},
-        {nullptr, dY, d.m, wha, rp, true, dB_d, partial2, counters + cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, sorted_pairs,
-                              d.k, s));
+    const WgradJob jobs[2] = {{save_H, d.n, t1, rp, false, dA_d, partial, counters},
+                              {rows, d.m, save_HA, d.r, true, dB_d, partial2, counters + cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
   }
-  // dW_d = H^T (w dY) per expert, on an expert-ordered copy of w dY
-  if (full) {
-    MOE_TRY(launch_gather_rows(dY, sorted_pairs, topk_w, L.P, d.k, d.m, rows, s));
-    MOE_TRY(launch_expert_dw(K_GEMM_DW_D, g, offsets, save_H, d.n, rows, d.m, dW_d, s));
-  }
-  // dGU: the SwiGLU backward of dH = w (dY W_d^T + (c T1') A_d^T), fused
-  MOE_TRY(launch_gemm_down_bwd(g, w, dY, sorted_pairs, d.k, topk_w, save_GU, lrc1, dgu, s));
-  // T2 = dGU B_gu^T (the dA_gu operand) and bf16(c T2)
-  MOE_TRY(launch_rank_sorted(K_RANK_T2, g, dgu, 2 * d.n, w.B_gu, false, t2, rp, rp, lrc2, s));
+  // dW_d = H^T dy per expert
+  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_D, g, offsets, save_H, d.n, rows, d.m, dW_d, s));
+  // dGU = SwiGLU backward of dH, T2 = dGU B_gu^T and bf16(c T2)
+  MOE_TRY(launch_rank_dswiglu(g, dh, save_GU, w.B_gu, dgu, t2, rp, rp, lrc2, s));
   // dX_sorted = dGU W_gu^T + (c T2) A_gu^T
   MOE_TRY(launch_gemm_gateup_bwd(g, w, dgu, lrc2, dX_sorted, s));
-  // dB_gu = c XA^T dGU and dA_gu = c X^T T2 (X rows gathered), one launch
+  // dB_gu = c XA^T dGU and dA_gu = c X^T T2 (X in expert order from the forward), one launch
   if (lora) {
     const WgradJob jobs[2] = {
-        {dgu, nullptr, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
-        {nullptr, X, d.m, t2, rp, false, dA_gu, partial2, counters + 3 * cstride}};
-    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, sorted_pairs,
-                              d.k, s));
+        {dgu, 2 * d.n, save_XA, d.r, true, dB_gu, partial, counters + 2 * cstride},
+        {save_Xs, d.m, t2, rp, false, dA_gu, partial2, counters + 3 * cstride}};
+    MOE_TRY(launch_lora_wgrad(g, jobs, 2, chunks, n_chunks, L.max_chunks, chunk_start, s));
   }
-  // dW_gu = X^T dGU per expert, on an expert-ordered copy of X
-  if (full) {
-    MOE_TRY(launch_gather_rows(X, sorted_pairs, nullptr, L.P, d.k, d.m, rows, s));
-    MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, rows, d.m, dgu, 2 * d.n, dW_gu, s));
-  }
+  // dW_gu = X^T dGU per expert
+  if (full) MOE_TRY(launch_expert_dw(K_GEMM_DW_GU, g, offsets, save_Xs, d.m, dgu, 2 * d.n, dW_gu, s));
   return MOE_OK;
 }
 
@@ -376,13 +375,35 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
   if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
   if (P > 0 && (topk_ids == nullptr || sorted_pairs == nullptr || pair_pos == nullptr))
     return MOE_ERR_INVALID_ARG;
-  const size_t need = align256((size_t)((P + kPermuteChunk - 1) / kPermuteChunk) * E * 4 + 4);
-  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
+  const size_t n_hist = (size_t)((P + kPermuteChunk - 1) / kPermuteChunk) * E;
+  if (ws_bytes < align256(n_hist * 4 + 4)) return MOE_ERR_WORKSPACE;
   int* err = status_ptr();
   if (err == nullptr) return MOE_ERR_CUDA;
-  return cuda_status(launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos,
-                                    static_cast<int32_t*>(ws), err,
-                                    static_cast<cudaStream_t>(stream)));
+  int32_t* hist = static_cast<int32_t*>(ws);
+  return cuda_status(launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos, hist,
+                                    hist + n_hist, err, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_route_permute(const float* logits, int64_t T, int32_t E, int32_t k,
+                               int32_t* topk_ids, float* topk_w, int32_t* counts, int32_t* offsets,
+                               int32_t* sorted_pairs, int32_t* pair_pos, void* ws, size_t ws_bytes,
+                               void* stream) {
+  NvtxRange nr("moe_route_permute");
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if (k < 1 || k > 32 || E < k || E > 1024) return MOE_ERR_UNSUPPORTED;
+  if (T * (int64_t)k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (logits == nullptr || topk_ids == nullptr || topk_w == nullptr ||
+                sorted_pairs == nullptr || pair_pos == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t tpb = route_tokens_per_chunk(k);
+  const size_t n_hist = (size_t)((T + tpb - 1) / tpb) * E;
+  if (ws_bytes < align256(n_hist * 4 + 4)) return MOE_ERR_WORKSPACE;
+  if (status_ptr() == nullptr) return MOE_ERR_CUDA;
+  int32_t* hist = static_cast<int32_t*>(ws);
+  return cuda_status(launch_route_permute(logits, T, E, k, topk_ids, topk_w, counts, offsets,
+                                          sorted_pairs, pair_pos, hist, hist + n_hist,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_check_permutation(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E,
@@ -408,16 +429,16 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
                                        const moe_bf16_t* W_gu, const moe_bf16_t* W_d,
                                        const moe_bf16_t* A_gu, const moe_bf16_t* B_gu,
                                        const moe_bf16_t* A_d, const moe_bf16_t* B_d,
-                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_GU,
-                                       moe_bf16_t* save_H, moe_bf16_t* save_XA,
-                                       moe_bf16_t* save_HA, void* ws, size_t ws_bytes,
-                                       void* stream) {
+                                       moe_bf16_t* Y_sorted, moe_bf16_t* save_Xs,
+                                       moe_bf16_t* save_GU, moe_bf16_t* save_H,
+                                       moe_bf16_t* save_XA, moe_bf16_t* save_HA, void* ws,
+                                       size_t ws_bytes, void* stream) {
   NvtxRange nr("moe_grouped_gemm_lora_fwd");
   moe_status_t st = check_dims(dims);
   if (st != MOE_OK) return st;
   const moe_dims_t d = *dims;
   if (d.T == 0) return MOE_OK;
-  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_GU, save_H,
+  const void* ptrs[] = {X, W_gu, W_d, A_gu, B_gu, A_d, B_d, Y_sorted, save_Xs, save_GU, save_H,
                         save_XA, save_HA, ws};
   for (const void* p : ptrs)
     if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
@@ -431,11 +452,11 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   if (st != MOE_OK) return st;
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
-  // XA = X A_gu on rows gathered from X (saved) and bf16(c XA)
-  MOE_TRY(launch_rank_gathered(K_RANK_XA, g, X, d.m, sorted_pairs, d.k, nullptr, w.A_gu, true,
-                               save_XA, d.r, d.r, false, xac, nullptr, 0, nullptr, s));
-  // GU = X W_gu + (c XA) B_gu (X rows gathered) and H = silu(g) u, fused
-  MOE_TRY(launch_gemm_gateup_fwd(g, w, X, sorted_pairs, d.k, xac, save_GU, save_H, s));
+  // X rows in expert order (saved), XA = X A_gu (saved) and bf16(c XA)
+  MOE_TRY(launch_rank_gathered(K_RANK_XA, g, X, d.m, sorted_pairs, d.k, nullptr, save_Xs, w.A_gu,
+                               true, save_XA, d.r, d.r, xac, s));
+  // GU = X W_gu + (c XA) B_gu and H = silu(g) u, fused
+  MOE_TRY(launch_gemm_gateup_fwd(g, w, save_Xs, xac, save_GU, save_H, s));
   // HA = H A_d (saved) and bf16(c HA)
   MOE_TRY(launch_rank_sorted(K_RANK_HA, g, save_H, d.n, w.A_d, true, save_HA, d.r, d.r, hac, s));
   // Y = H W_d + (c HA) B_d
@@ -444,36 +465,37 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
 }
 
 moe_status_t moe_grouped_gemm_lora_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
-    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
-    moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws,
-    size_t ws_bytes, void* stream) {
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU,
+    const moe_bf16_t* save_H, const moe_bf16_t* save_XA, const moe_bf16_t* save_HA,
+    moe_bf16_t* dX_sorted, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
+    moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream) {
   NvtxRange nr("moe_grouped_gemm_lora_bwd");
   if (dA_gu == nullptr || dB_gu == nullptr || dA_d == nullptr || dB_d == nullptr)
     return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, nullptr,
-                  nullptr, ws, ws_bytes, stream);
+  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d,
+                  nullptr, nullptr, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_grouped_gemm_full_bwd(
-    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w, const moe_bf16_t* X,
+    const moe_dims_t* dims, const moe_bf16_t* dY, const float* topk_w,
     const int32_t* sorted_pairs, const int32_t* offsets, const moe_bf16_t* W_gu,
     const moe_bf16_t* W_d, const moe_bf16_t* A_gu, const moe_bf16_t* B_gu, const moe_bf16_t* A_d,
-    const moe_bf16_t* B_d, const moe_bf16_t* save_GU, const moe_bf16_t* save_H,
-    const moe_bf16_t* save_XA, const moe_bf16_t* save_HA, moe_bf16_t* dX_sorted,
-    moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu, moe_bf16_t* dB_gu, moe_bf16_t* dA_d,
-    moe_bf16_t* dB_d, void* ws, size_t ws_bytes, void* stream) {
+    const moe_bf16_t* B_d, const moe_bf16_t* save_Xs, const moe_bf16_t* save_GU,
+    const moe_bf16_t* save_H, const moe_bf16_t* save_XA, const moe_bf16_t* save_HA,
+    moe_bf16_t* dX_sorted, moe_bf16_t* dW_gu, moe_bf16_t* dW_d, moe_bf16_t* dA_gu,
+    moe_bf16_t* dB_gu, moe_bf16_t* dA_d, moe_bf16_t* dB_d, void* ws, size_t ws_bytes,
+    void* stream) {
   NvtxRange nr("moe_grouped_gemm_full_bwd");
   if (dW_gu == nullptr || dW_d == nullptr) return MOE_ERR_INVALID_ARG;
   const int given = (dA_gu != nullptr) + (dB_gu != nullptr) + (dA_d != nullptr) + (dB_d != nullptr);
   if (given != 0 && given != 4) return MOE_ERR_INVALID_ARG;
-  return backward(dims, dY, topk_w, X, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
-                  save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d, dW_gu,
-                  dW_d, ws, ws_bytes, stream);
+  return backward(dims, dY, topk_w, sorted_pairs, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d,
+                  save_Xs, save_GU, save_H, save_XA, save_HA, dX_sorted, dA_gu, dB_gu, dA_d, dB_d,
+                  dW_gu, dW_d, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_router_backward(const moe_bf16_t* dY, const moe_bf16_t* Y_sorted,

@@ -22,11 +22,10 @@ cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const u
   p.F = g.m;
   p.n_ftiles = (g.m + 255) / 256;
   p.nk = (g.n + 127) / 128;
-  p.K = g.n;
   p.n = g.n;
   p.out = reinterpret_cast<__nv_bfloat16*>(Yp);
   p.err = g.err;
-  return dispatch_gemm<true, false, EPI_PLAIN>(K_GEMM_DOWN_FWD, g, v, mp, p, s);
+  return dispatch_gemm<true, EPI_PLAIN>(K_GEMM_DOWN_FWD, g, v, mp, p, s);
 }
 
 }  // namespace moe

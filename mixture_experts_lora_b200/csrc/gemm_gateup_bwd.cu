@@ -23,11 +23,10 @@ cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const
   p.F = g.m;
   p.n_ftiles = (g.m + 255) / 256;
   p.nk = (2 * g.n + 127) / 128;
-  p.K = 2 * g.n;
   p.n = g.n;
   p.out = reinterpret_cast<__nv_bfloat16*>(dXp);
   p.err = g.err;
-  return dispatch_gemm<false, false, EPI_PLAIN>(K_GEMM_GATEUP_BWD, g, v, mp, p, s);
+  return dispatch_gemm<false, EPI_PLAIN>(K_GEMM_GATEUP_BWD, g, v, mp, p, s);
 }
 
 }  // namespace moe

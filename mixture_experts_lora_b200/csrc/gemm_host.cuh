@@ -30,13 +30,13 @@ cudaError_t launch_gemm_cfg(int kind, const GemmShape& g, const GemmMaps& mp, co
   return cudaGetLastError();
 }
 
-template <bool A_MN, bool GATHER, int EPI>
+template <bool A_MN, int EPI>
 cudaError_t dispatch_gemm(int kind, const GemmShape& g, bool v, const GemmMaps& mp,
                           const GemmParams& p, cudaStream_t s) {
-#define MOE_GEMM_RP(RPV)                                                                      \
-  case RPV:                                                                                   \
-    return v ? launch_gemm_cfg<GemmCfg<A_MN, RPV, true, GATHER, EPI>>(kind, g, mp, p, s)      \
-             : launch_gemm_cfg<GemmCfg<A_MN, RPV, false, GATHER, EPI>>(kind, g, mp, p, s);
+#define MOE_GEMM_RP(RPV)                                                                 \
+  case RPV:                                                                              \
+    return v ? launch_gemm_cfg<GemmCfg<A_MN, RPV, true, EPI>>(kind, g, mp, p, s)         \
+             : launch_gemm_cfg<GemmCfg<A_MN, RPV, false, EPI>>(kind, g, mp, p, s);
   switch (g.rp) {
     MOE_GEMM_RP(16)
     MOE_GEMM_RP(32)

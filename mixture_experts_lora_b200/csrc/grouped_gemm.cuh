@@ -17,33 +17,24 @@
 // Mixture-of-Experts Fine-Tuning", Mathematical Formulation section 2) with no
 // K x N adapter delta.
 //
-// Token operand.  Either a sorted [P, K] matrix loaded with TMA, or (GATHER) rows
-// gathered straight from a token matrix [T, K] - row q of the chunk is
-// src[sorted_pairs[q] / k] - by four gather warps with cp.async into the same
-// swizzled layout, so the expert-ordered copy of X or dY is never written to HBM
-// (the "dY gather / scale, not materialised" step of the backward; the routing
-// weight is applied in the epilogue, by linearity).
+// The token operand is the expert-ordered [P, K] matrix (sorted X, H, w dY or dGU)
+// loaded with TMA.
 //
 // Epilogues (EPI):
 //   EPI_PLAIN    out[q, f] = bf16(D)
-//   EPI_WSCALE   out[q, f] = bf16(w[q] D)                   (w: routing weight of the row)
 //   EPI_SWIGLU   the gate_up projection with the SwiGLU fused (h = silu(g) u, gate = first
 //                n columns; Unsloth docs "What is torch._grouped_mm?", the expert's
 //                gate_up output split in two): each CTA's 128 features are 64 gate
 //                features and the 64 up features of the same indices, so g and u of a
 //                token meet in one CTA; it writes GU (kept for the backward) and H.
-//   EPI_DSWIGLU  the down projection's backward with the SwiGLU backward fused:
-//                dH = w[q] D, then dGU = [dH u s (1 + g (1 - s)), dH g s], s = sigmoid(g),
-//                from the saved GU; only dGU is written.
 //
-// Roles (320 threads per CTA, 448 with GATHER): warp 0 issues TMA loads (each CTA its
-// own half, completing on the leader's barriers), warp 1 allocates TMEM and, in the
-// leader CTA, issues tcgen05.mma for the pair; warps 2-9 drain TMEM (two warps per
-// TMEM lane quarter, alternating 32-token blocks), transpose each 32 x 32 block
-// through shared memory and store it with one TMA tensor store (16-byte stores for a
-// chunk's ragged last block); warps 10-13 (GATHER) gather the token rows.  The
-// accumulator is double buffered (2 x 256 fp32 columns) so the epilogue of one tile
-// overlaps the K-loop of the next.
+// Roles (320 threads per CTA): warp 0 issues TMA loads (each CTA its own half,
+// completing on the leader's barriers), warp 1 allocates TMEM and, in the leader CTA,
+// issues tcgen05.mma for the pair; warps 2-9 drain TMEM (two warps per TMEM lane
+// quarter, alternating 32-token blocks), transpose each 32 x 32 block through shared
+// memory and store it with one TMA tensor store (16-byte stores for a chunk's ragged
+// last block).  The accumulator is double buffered (2 x 256 fp32 columns) so the
+// epilogue of one tile overlaps the K-loop of the next.
 //
 // Shared-memory operands (canonical UMMA layouts, per CTA):
 //   A (weights)  forward, W stored [K][F]: MN-major, two 64-feature atoms of 128 K
@@ -60,7 +51,7 @@
 
 namespace moe {
 
-enum GemmEpi : int { EPI_PLAIN = 0, EPI_WSCALE = 1, EPI_SWIGLU = 2, EPI_DSWIGLU = 3 };
+enum GemmEpi : int { EPI_PLAIN = 0, EPI_SWIGLU = 1 };
 
 struct GemmParams {
   const TileInfo* chunks;  // token chunks {e, row0, row_end}, at most 256 rows each
@@ -68,27 +59,20 @@ struct GemmParams {
   int F;                   // output features (EPI_SWIGLU: h-features n)
   int n_ftiles;            // feature tiles per chunk
   int nk;                  // K steps of 128 (the LoRA block follows them)
-  int K;                   // reduction length
-  // gathered token operand (GATHER): row q = gsrc[sorted_pairs[q] / k]
-  const __nv_bfloat16* gsrc;
-  const int32_t* sorted_pairs;
-  int k;
-  const float* w;          // [P] routing weights in pair order (EPI_WSCALE, EPI_DSWIGLU)
-  const __nv_bfloat16* gu; // [P, 2n] saved GU (EPI_DSWIGLU)
-  int n;                   // expert intermediate size (SwiGLU epilogues)
+  int n;                   // expert intermediate size (SwiGLU epilogue)
   // outputs, for the ragged stores (the full blocks go through the tensor maps)
-  __nv_bfloat16* out;      // PLAIN/WSCALE: [P, F]; SWIGLU: GU [P, 2n]; DSWIGLU: dGU [P, 2n]
+  __nv_bfloat16* out;      // PLAIN: [P, F]; SWIGLU: GU [P, 2n]
   __nv_bfloat16* out_h;    // SWIGLU: H [P, n]
   int* err;
 };
 
-// A_MN: weights stored [K][F] (MN-major A).  V: weights through an atom view, one
-// TMA copy per stage (and, for a TMA-loaded token operand, the token tile through
-// one as well); needs whole 64-wide atoms.  Otherwise two copies per operand.
-template <bool A_MN_, int RP_, bool V_, bool GATHER_, int EPI_>
+// A_MN: weights stored [K][F] (MN-major A).  V: operands through atom views, one TMA
+// copy per operand and stage; needs whole 64-wide atoms.  Otherwise two copies per
+// operand.
+template <bool A_MN_, int RP_, bool V_, int EPI_>
 struct GemmCfg {
   static constexpr int RP = RP_;
-  static constexpr bool A_MN = A_MN_, V = V_, GATHER = GATHER_;
+  static constexpr bool A_MN = A_MN_, V = V_;
   static constexpr int EPI = EPI_;
   // BK = 128 per stage as two 64-wide K atoms (one 128-byte swizzle row each): a
   // stage carries 8 MMAs per wait and commit.  BOXR: token rows per LoRA-block copy.
@@ -100,8 +84,7 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BLK_BYTES = 32 * 32 * 2;        // one 32 x 32 bf16 staging block
   static constexpr int EPI_WARPS = 8;
-  static constexpr int GATHER_WARPS = GATHER ? 4 : 0;
-  static constexpr int THREADS = 32 * (2 + EPI_WARPS + GATHER_WARPS);
+  static constexpr int THREADS = 32 * (2 + EPI_WARPS);
   static constexpr int EPI_BYTES = EPI_WARPS * BLK_BYTES;   // one transpose block per warp
   static constexpr int SMEM_LIMIT = 232448;
   // LoRA operands.  K-major atoms are LK_W ranks wide.
@@ -211,8 +194,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      // the producer's expect_tx arrival, plus one per gather warp of both CTAs
-      mbar_init(smem_u32(&full[s]), 1 + 2 * C::GATHER_WARPS);
+      mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -227,7 +209,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     *abort_flag = 0;
     mbar_fence_init();
     tma_prefetch_desc(&tmW);
-    if constexpr (!C::GATHER) tma_prefetch_desc(&tmAct);
+    tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmLW);
     tma_prefetch_desc(&tmLR);
   }
@@ -300,7 +282,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             // rows past P and K past the end read as zero)
             const int k0 = ks * C::BK;
             if (rank == 0)
-              mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + (C::GATHER ? 0 : C::B_BYTES)));
+              mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + C::B_BYTES));
             if constexpr (C::V) {
               if constexpr (C::EPI == EPI_SWIGLU)
                 tma_load_5d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, 0, ch.e);
@@ -308,7 +290,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, ch.e);
               else
                 tma_load_4d_pair(&tmW, fb, sa, 0, feat_box<C>(w, rank, 0, p.n), k0 / C::KA, ch.e);
-              if constexpr (!C::GATHER) tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
+              tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
             } else {
               if constexpr (C::A_MN) {
                 tma_load_3d_pair(&tmW, fb, sa, feat_box<C>(w, rank, 0, p.n), k0, ch.e);
@@ -317,10 +299,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tma_load_3d_pair(&tmW, fb, sa, k0, feat_box<C>(w, rank, 0, p.n), ch.e);
                 tma_load_3d_pair(&tmW, fb, sa + C::ATOM_A, k0 + C::KA, feat_box<C>(w, rank, 0, p.n), ch.e);
               }
-              if constexpr (!C::GATHER) {
-                tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
-                tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
-              }
+              tma_load_2d_pair(&tmAct, fb, sb, k0, r0);
+              tma_load_2d_pair(&tmAct, fb, sb + C::ATOM_B, k0 + C::KA, r0);
             }
           } else {
             if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * lbytes);
@@ -386,9 +366,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           __syncwarp();
         }
         for (int ks = 0; ks < p.nk + NST; ++ks) {
-          bool fok;
-          if constexpr (C::GATHER) fok = mbar_wait_cluster(smem_u32(&full[stage]), phase, p.err);
-          else fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
+          const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
           if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
           tc_fence_after();
           if (lane == 0) {
@@ -440,7 +418,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if constexpr (C::EPI == EPI_SWIGLU) {
       if (gate_w) named_bar_arrive(pbar + 1, 64);   // the up warp may stage its first block
     }
-    const size_t ldo = C::EPI == EPI_PLAIN || C::EPI == EPI_WSCALE ? (size_t)p.F : (size_t)2 * p.n;
+    const size_t ldo = C::EPI == EPI_PLAIN ? (size_t)p.F : (size_t)2 * p.n;
     int it = 0;
     for (int t = pair; t < total; t += npairs, ++it) {
       const int c = t / p.n_ftiles, w = t % p.n_ftiles;
@@ -460,21 +438,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tmem_wait_ld();
         const int grow = ch.row0 + c0;
         const int rows_left = nrows - c0;
-        if constexpr (C::EPI == EPI_WSCALE || C::EPI == EPI_DSWIGLU) {
-          // the routing weight of each token of the block (lane i holds token i's)
-          const float wl = lane < rows_left ? p.w[p.sorted_pairs[grow + lane]] : 0.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            v[i] = __float_as_uint(__uint_as_float(v[i]) * __shfl_sync(0xffffffffu, wl, i));
-        }
         if (lane == 0) bulk_wait_read<0>();         // the last store from blk has read it
         __syncwarp();
-        if constexpr (C::EPI == EPI_PLAIN || C::EPI == EPI_WSCALE) {
+        if constexpr (C::EPI == EPI_PLAIN) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
           epi_store_block(&tmOut, blk, fq, grow, rows_left, p.out, ldo, p.F);
-        } else if constexpr (C::EPI == EPI_SWIGLU) {
+        } else {
           if (!gate_w) {
             // u: stage it once the gate warp has read the previous block, store it
             // (GU columns n + f), then hand the staging block to the gate warp
@@ -509,37 +480,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
             epi_store_block(&tmOut3, blk, fq, grow, rows_left, p.out_h, (size_t)p.n, p.n);
           }
-        } else {
-          // EPI_DSWIGLU: v = dH of feature fq + lane for the block's tokens
-          const int f = fq + lane;
-          uint32_t gu2[32];                          // (u << 16) | g, bf16 bits
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            uint32_t g16 = 0, u16 = 0;
-            if (i < rows_left && f < p.n) {
-              const unsigned short* row = reinterpret_cast<const unsigned short*>(p.gu + (size_t)(grow + i) * ldo);
-              g16 = __ldg(row + f);
-              u16 = __ldg(row + p.n + f);
-            }
-            gu2[i] = g16 | (u16 << 16);
-          }
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float g = bf16_lo(gu2[i]), u = bf16_hi(gu2[i]);
-            const float dh = __uint_as_float(v[i]);
-            const float s = fmaf(0.5f, tanh_approx(0.5f * g), 0.5f);          // sigmoid(g)
-            const float dg = dh * u * s * (1.0f + g * (1.0f - s));
-            const float du = dh * g * s;
-            *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(dg);
-            v[i] = __float_as_uint(du);
-          }
-          epi_store_block(&tmOut, blk, fq, grow, rows_left, p.out, ldo, p.n);
-          if (lane == 0) bulk_wait_read<0>();
-          __syncwarp();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            *reinterpret_cast<__nv_bfloat16*>(blk + i * 64 + lane * 2) = __float2bfloat16_rn(__uint_as_float(v[i]));
-          epi_store_block(&tmOut2, blk, fq, grow, rows_left, p.out + p.n, ldo, p.n);
         }
       }
       tc_fence_before();
@@ -551,68 +491,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     if (lane == 0) bulk_wait<0>();                        // every store of this warp complete
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ gather warps (GATHER, both CTAs)
-    // Rows of this CTA's half of the chunk, 16-byte pieces into the two K atoms of the
-    // stage's B area; each warp arrives on the leader's full barrier once its lanes'
-    // pieces of the stage have landed (one stage in flight behind the one issued).
-    if constexpr (C::GATHER) {
-      const int gt = (warp - 2 - C::EPI_WARPS) * 32 + lane;   // 0..127
-      const int cv = gt & 7, rb = gt >> 3;                     // rows rb + 16 j
-      const uint32_t full_leader = mapa_smem(smem_u32(full), 0);
-      int stage = 0, pend = -1;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = pair; t < total && ok; t += npairs) {
-        const int c = t / p.n_ftiles;
-        const TileInfo ch = p.chunks[c];
-        const int half = ((((ch.row_end - ch.row0) + 15) & ~15) >> 1);
-        const int r0 = ch.row0 + (int)rank * half;
-        int nv = ch.row_end - r0;                  // rows of this half inside the chunk
-        nv = nv < 0 ? 0 : (nv > half ? half : nv);
-        const __nv_bfloat16* rp[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int r = rb + 16 * j;
-          rp[j] = r < nv ? p.gsrc + (size_t)(p.sorted_pairs[r0 + r] / p.k) * p.K : nullptr;
-        }
-        if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-        for (int ks = 0; ks < p.nk + NST; ++ks) {
-          const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
-          if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
-          if (ks < p.nk) {
-            const uint32_t sb = s_base + stage * C::STAGE_BYTES + C::A_BYTES;
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-              const int col = ks * C::BK + a * C::KA + cv * 8;
-              const bool v = col < p.K;            // columns past K are zero
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if (rp[j] == nullptr) continue;    // rows past the chunk: never stored
-                const int r = rb + 16 * j;
-                cp_async_16(sb + a * C::ATOM_B + r * 128 + ((cv ^ (r & 7)) << 4),
-                            v ? (const void*)(rp[j] + col) : (const void*)p.gsrc, v ? 16u : 0u);
-              }
-            }
-          }
-          cp_async_commit();
-          if (pend >= 0) {
-            cp_async_wait<1>();                    // the previous stage's pieces landed
-            fence_proxy_async_smem();              // generic-proxy writes -> tcgen05 reads
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(full_leader + pend * 8);
-          }
-          pend = stage;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-        }
-      }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (pend >= 0 && lane == 0) mbar_arrive_cluster(full_leader + pend * 8);
-      if (!ok && lane == 0) *abort_flag = 1;
-      __syncwarp();
-    }
   }
 
   tc_fence_before();

@@ -40,10 +40,10 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // ---- kernel timing (profile.cu): while enabled, each launch is bracketed by
 // CUDA events on its stream and attributed to one of these kinds.
 enum KernelKind : int {
-  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_TABLES,
+  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCATTER, K_TABLES,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
   K_COMBINE, K_MEMSET, K_RANK_XA, K_RANK_HA, K_RANK_T1, K_RANK_T2,
-  K_ROUTER_BWD, K_GEMM_DW_GU, K_GEMM_DW_D, K_GATHER_ROWS, K_NUM_KINDS
+  K_ROUTER_BWD, K_GEMM_DW_GU, K_GEMM_DW_D, K_NUM_KINDS
 };
 extern const char* const kKernelNames[K_NUM_KINDS];
 bool prof_enabled();
@@ -67,11 +67,18 @@ void* current_context();
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
-// one block per chunk of kPermuteChunk pairs; hist holds n_chunks * E ints
+// one block per chunk of kPermuteChunk pairs; hist holds n_chunks * E ints; arrive is
+// an int the call zeroes (the last block of the histogram launch is the one that scans)
 constexpr int kPermuteChunk = 512;
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
-                           int32_t* hist, int* err, cudaStream_t s);
+                           int32_t* hist, int* arrive, int* err, cudaStream_t s);
+// Routing fused with the permutation's histogram: chunks of route_tokens_per_chunk(k)
+// tokens (their k pairs each), hist holds ceil(T / that) * E ints.
+int route_tokens_per_chunk(int k);
+cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
+                                 float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
+                                 int32_t* pair_pos, int32_t* hist, int* arrive, cudaStream_t s);
 // From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
 // experts (row kernels), token chunks of at most `gchunk_rows` rows split
 // evenly inside each expert (grouped GEMMs; all but the last chunk of an expert
@@ -92,11 +99,6 @@ cudaError_t launch_check_permutation(const int32_t* ids, int64_t P, int E, const
                                      const int32_t* pair_pos, int* err, cudaStream_t s);
 cudaError_t launch_combine(const uint16_t* ysorted, const float* w, const int32_t* pair_pos,
                            int64_t T, int k, int m, uint16_t* y, cudaStream_t s);
-// out[q] = (w ? w[sorted_pairs[q]] : 1) * src[sorted_pairs[q] / k] for q < P, rows of
-// K bf16 (K % 8 == 0): the expert-ordered copy of X or w dY that only the weight
-// gradients of full fine-tuning read.
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
-                               int64_t P, int k, int K, uint16_t* out, cudaStream_t s);
 cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t s);
 
 // ---- tcgen05 GEMMs (gemm_*.cu), rank-r products (rank_launch.cu), adapter and
@@ -125,41 +127,42 @@ struct GemmShape {
 };
 
 // Grouped GEMMs (features on M, expert tokens on N, CTA pairs), sorted token order.
-// GU, H = SwiGLU(X W_gu + XAc B_gu), X rows gathered (XAc = bf16(c X A_gu))
-cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* X,
-                                   const int32_t* sorted_pairs, int k, const uint16_t* XAc,
-                                   uint16_t* GU, uint16_t* H, cudaStream_t s);
+// GU, H = SwiGLU(Xs W_gu + XAc B_gu)   (XAc = bf16(c Xs A_gu))
+cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* Xs,
+                                   const uint16_t* XAc, uint16_t* GU, uint16_t* H, cudaStream_t s);
 // Yp = H W_d + HAc B_d
 cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* H,
                                  const uint16_t* HAc, uint16_t* Yp, cudaStream_t s);
-// dGU = SwiGLU'(GU) of dH = w (dY W_d^T + T1c A_d^T), dY rows gathered
-cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dY,
-                                 const int32_t* sorted_pairs, int k, const float* topk_w,
-                                 const uint16_t* GU, const uint16_t* T1c, uint16_t* dGU,
-                                 cudaStream_t s);
+// dH = dy W_d^T + T1c A_d^T
+cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dys,
+                                 const uint16_t* T1c, uint16_t* dH, cudaStream_t s);
 // dXp = dGU W_gu^T + T2c A_gu^T
 cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const uint16_t* dGU,
                                    const uint16_t* T2c, uint16_t* dXp, cudaStream_t s);
 
-// Rank-r products LR = Rows L[e] (rank_r.cuh).  Gathered rows src[sorted_pairs[q] / k]
-// of K columns; L [E, K, r] (l_mn) or [E, r, K].  Writes out_save [P, ld_save] (first
-// r_save columns; times w[pair] with save_w), out_c = bf16(scale LR) [P, rp] and, if
-// out_w is given, out_w = bf16(w wsrc) [P, rp] from wsrc [P, r_wsrc].
+// Rank-r products LR = Rows L[e] (rank_r.cuh); every variant writes out_save [P, ld_save]
+// (first r_save columns, unscaled) and out_c = bf16(scale LR) [P, rp].
+// Gathered rows s_q src[sorted_pairs[q] / k] of K columns (s_q = w[pair] if w is
+// given), written to rows_out [P, K]; L [E, K, r] (l_mn) or [E, r, K].
 cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* src, int K,
                                  const int32_t* sorted_pairs, int k, const float* w,
-                                 const uint16_t* L, bool l_mn, uint16_t* out_save, int ld_save,
-                                 int r_save, bool save_w, uint16_t* out_c, const uint16_t* wsrc,
-                                 int r_wsrc, uint16_t* out_w, cudaStream_t s);
+                                 uint16_t* rows_out, const uint16_t* L, bool l_mn,
+                                 uint16_t* out_save, int ld_save, int r_save, uint16_t* out_c,
+                                 cudaStream_t s);
 // Sorted rows [P, K].
 cudaError_t launch_rank_sorted(int kind, const GemmShape& g, const uint16_t* rows, int K,
                                const uint16_t* L, bool l_mn, uint16_t* out_save, int ld_save,
                                int r_save, uint16_t* out_c, cudaStream_t s);
+// The SwiGLU backward dGU [P, 2n] of dH [P, n] and GU [P, 2n], written out, with
+// T2 = dGU B_gu^T.
+cudaError_t launch_rank_dswiglu(const GemmShape& g, const uint16_t* dH, const uint16_t* GU,
+                                const uint16_t* B_gu, uint16_t* dGU, uint16_t* out_save,
+                                int ld_save, int r_save, uint16_t* out_c, cudaStream_t s);
 
 // One adapter-gradient problem G_e = Big_e^T Small_e (see lora_wgrad.cuh):
 // out = scale * G per expert, out [E, D, r] or (transpose) [E, r, D].
 struct WgradJob {
-  const uint16_t* big;   // [P, D] sorted rows (when gsrc is null)
-  const uint16_t* gsrc;  // [T, D] token matrix whose rows are gathered, or null
+  const uint16_t* big;   // [P, D] sorted rows
   int D;
   const uint16_t* small; // [P, ld_small]
   int ld_small;
@@ -171,8 +174,7 @@ struct WgradJob {
 // One launch for one or two problems.
 cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jobs,
                               const TileInfo* chunks, const int* n_chunks, int max_chunks,
-                              const int32_t* chunk_start, const int32_t* sorted_pairs, int k,
-                              cudaStream_t s);
+                              const int32_t* chunk_start, cudaStream_t s);
 
 // Expert-weight gradients (expert_dw.cuh): out[e] = Lm_e^T Rm_e over the rows of expert
 // e (offsets), Lm [P, Mdim], Rm [P, Ndim] sorted rows, out [E, Mdim, Ndim] bf16.

@@ -17,10 +17,7 @@
 //       zero), the rest of the 16 stay zero from the kernel's start),
 //   N = 256 columns of Big (MN-major, 128-byte swizzle, four 64-column atoms),
 //   K = rows of the chunk, 64 per stage,
-// one TMA copy per operand and stage (a Big gathered from a token matrix - X for
-// dA_gu, dY for dB_d - comes instead from four gather warps with cp.async into the
-// same layout, so no expert-ordered copy of X or dY exists).  A rank of 16 uses an
-// eighth of M,
+// one TMA copy per operand and stage.  A rank of 16 uses an eighth of M,
 // but each MMA then moves 256 columns of Big: a thin N = r MMA costs the tensor
 // pipe about as long as a full one and would bound the kernel instead of HBM.
 // Every copy is full-size from the chunk's first row, so the stage that crosses the
@@ -43,9 +40,6 @@
 namespace moe {
 
 struct WgradProblem {
-  // Big gathered from a token matrix when gsrc is set (row q = gsrc[sorted_pairs[q] / k],
-  // D columns), else loaded with TMA from the sorted [P, D] matrix of the tensor map
-  const __nv_bfloat16* gsrc;
   const __nv_bfloat16* small;  // [P, ld_small]
   int ld_small;
   int r_small;                 // columns of `small` to read (rest zero)
@@ -66,17 +60,13 @@ struct WgradParams {
   int E;
   int r;                       // output rank
   float scale;
-  const int32_t* sorted_pairs; // gathered Big rows
-  int k;
   int* err;
 };
 
-template <int RP, bool V_ = true, bool G_ = false>
+template <int RP, bool V_ = true>
 struct WgradCfg {
   static constexpr bool V = V_;             // Big through the atom view (D % 64 == 0)
-  static constexpr bool G = G_;             // gather warps for a gathered Big
-  static constexpr int GATHER_WARPS = G ? 4 : 0;
-  static constexpr int THREADS = 192 + 32 * GATHER_WARPS;
+  static constexpr int THREADS = 192;
   static constexpr int BM = 128;            // rank rows on M (RP of them are used)
   static constexpr int BN = 256;            // Big columns per unit
   static constexpr int BK = 64;             // rows per stage
@@ -123,13 +113,13 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, float s, const 
   *reinterpret_cast<uint4*>(dst) = o;
 }
 
-template <int RP, bool V, bool G>
-__global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
+template <int RP, bool V>
+__global__ void __launch_bounds__(WgradCfg<RP, V>::THREADS, 1)
     lora_wgrad_kernel(const __grid_constant__ CUtensorMap tmBig0,
                       const __grid_constant__ CUtensorMap tmBig1,
                       const __grid_constant__ CUtensorMap tmSmall0,
                       const __grid_constant__ CUtensorMap tmSmall1, const WgradParams p) {
-  using C = WgradCfg<RP, V, G>;
+  using C = WgradCfg<RP, V>;
   constexpr int OWNERS = RP <= 32 ? 1 : RP / 32;   // epilogue warps holding rank rows
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -149,7 +139,7 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&full[s]), 1 + C::GATHER_WARPS);
+      mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -160,10 +150,10 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
     *abort_flag = 0;
     *last_flag = 0;
     mbar_fence_init();
-    if (p.pr[0].gsrc == nullptr) tma_prefetch_desc(&tmBig0);
+    tma_prefetch_desc(&tmBig0);
     tma_prefetch_desc(&tmSmall0);
     if (p.n_problems > 1) {
-      if (p.pr[1].gsrc == nullptr) tma_prefetch_desc(&tmBig1);
+      tma_prefetch_desc(&tmBig1);
       tma_prefetch_desc(&tmSmall1);
     }
   }
@@ -193,7 +183,6 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
       const WgradUnit u = wgrad_unit(p, nch, t);
       const CUtensorMap* tb = u.prob == 0 ? &tmBig0 : &tmBig1;
       const CUtensorMap* ts = u.prob == 0 ? &tmSmall0 : &tmSmall1;
-      const bool gathered = p.pr[u.prob].gsrc != nullptr;
       const TileInfo ch = p.chunks[u.c];
       const int d0 = u.dt * C::BN;
       const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
@@ -206,17 +195,15 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           const int r0 = ch.row0 + ks * C::BK;
-          mbar_arrive_expect_tx(fb, C::SMALL_COPY + (gathered ? 0 : C::B_BYTES));
+          mbar_arrive_expect_tx(fb, C::SMALL_COPY + C::B_BYTES);
           // Small [BK rows][RP / 8 groups of 8 rank columns] (MN-major, no swizzle: core
           // matrices of 8 rows x 8 columns)
           tma_load_3d(ts, fb, sa, 0, r0, 0);
-          if (!gathered) {
-            if constexpr (C::V) {
-              tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
-            } else {
+          if constexpr (C::V) {
+            tma_load_3d(tb, fb, sb, 0, r0, d0 / 64);
+          } else {
 #pragma unroll
-              for (int a = 0; a < C::BN / 64; ++a) tma_load_2d(tb, fb, sb + a * C::ATOM, d0 + a * 64, r0);
-            }
+            for (int a = 0; a < C::BN / 64; ++a) tma_load_2d(tb, fb, sb + a * C::ATOM, d0 + a * 64, r0);
           }
         }
         __syncwarp();
@@ -285,7 +272,7 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
       mbar_wait(smem_u32(drain), 0, p.err);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else {
     // ---------------------------------------------------------- epilogue (warps 2..5)
     const int et = (warp - 2) * 32 + lane;         // 0..127
     const int q4 = warp & 3;                       // TMEM lane quarter: rank rows 32 q4 ..
@@ -418,64 +405,6 @@ __global__ void __launch_bounds__(WgradCfg<RP, V, G>::THREADS, 1)
         for (int64_t i = et; i < n8; i += C::EPI_THREADS)
           store_bf16x8(q.out + (size_t)e * q.D * p.r + i * 8, 0.f, z);
       }
-    }
-  } else {
-    // ---------------------------------------------------------- gather warps (G)
-    // For units whose Big is gathered: the stage's 64 rows x 256 columns, 16-byte
-    // pieces into the four 64-column atoms (rows past the chunk and columns past D
-    // zero: they meet zero rows of Small, and stale bits could be NaN).  Every stage
-    // of every unit gets one arrival per warp, data or not, once the lanes' pieces of
-    // the stage have landed (one stage in flight behind the one issued).
-    if constexpr (C::G) {
-      const int gt = (warp - 6) * 32 + lane;       // 0..127
-      const int cv = gt & 7, rb = gt >> 3;         // rows rb + 16 j
-      int stage = 0, pend = -1;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const WgradUnit u = wgrad_unit(p, nch, t);
-        const WgradProblem& q = p.pr[u.prob];
-        const TileInfo ch = p.chunks[u.c];
-        const int d0 = u.dt * C::BN;
-        const int nk = (ch.row_end - ch.row0 + C::BK - 1) / C::BK;
-        if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-        for (int ks = 0; ks < nk; ++ks) {
-          const bool wok = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err);
-          if (!__all_sync(0xffffffffu, wok)) { ok = false; break; }
-          if (q.gsrc != nullptr) {
-            const uint32_t sb = s_base + stage * C::STAGE_BYTES + C::A_BYTES;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int r = rb + 16 * j;
-              const int row = ch.row0 + ks * C::BK + r;
-              const __nv_bfloat16* src = row < ch.row_end
-                  ? q.gsrc + (size_t)(p.sorted_pairs[row] / p.k) * q.D : nullptr;
-#pragma unroll
-              for (int a = 0; a < 4; ++a) {
-                const int col = d0 + a * 64 + cv * 8;
-                const bool v = src != nullptr && col < q.D;
-                cp_async_16(sb + a * C::ATOM + r * 128 + ((cv ^ (r & 7)) << 4),
-                            v ? (const void*)(src + col) : (const void*)q.gsrc, v ? 16u : 0u);
-              }
-            }
-          }
-          cp_async_commit();
-          if (pend >= 0) {
-            cp_async_wait<1>();                    // the previous stage's pieces landed
-            fence_proxy_async_smem();              // generic-proxy writes -> tcgen05 reads
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&full[pend]));
-          }
-          pend = stage;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
-        }
-      }
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (pend >= 0 && lane == 0) mbar_arrive(smem_u32(&full[pend]));
-      if (!ok && lane == 0) *abort_flag = 1;
-      __syncwarp();
     }
   }
 

@@ -17,9 +17,10 @@
 namespace moe {
 namespace {
 
-// 2^19 int32 = 2 MiB: room for ceil(T*k / kPermuteChunk) * E histogram entries.
+// 2^19 int32 = 2 MiB: room for ceil(T*k / kPermuteChunk) * E histogram entries, then
+// the arrival counter of the histogram launch.
 constexpr size_t kPermuteScratchInts = size_t(1) << 19;
-__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts];
+__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts + 64];
 
 constexpr int kMaxDevices = 64;
 
@@ -63,13 +64,15 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, 
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
   if (P > 0 && (topk_ids == nullptr || sorted_pairs == nullptr || pair_pos == nullptr))
     return MOE_ERR_INVALID_ARG;
-  // every histogram entry is written before it is read, so the scratch needs no clearing
+  // every histogram entry is written before it is read; the arrival counter after them
+  // is zeroed by the call itself
   const int64_t need = ((P + kPermuteChunk - 1) / kPermuteChunk) * (int64_t)E;
   if (need > (int64_t)kPermuteScratchInts) return MOE_ERR_WORKSPACE;
   int32_t* scratch = permute_scratch();
   int* err = moe_status_word();
   if (scratch == nullptr || err == nullptr) return MOE_ERR_CUDA;
   const cudaError_t st = launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos,
-                                        scratch, err, static_cast<cudaStream_t>(stream));
+                                        scratch, scratch + kPermuteScratchInts, err,
+                                        static_cast<cudaStream_t>(stream));
   return st == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

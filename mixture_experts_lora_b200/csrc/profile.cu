@@ -15,11 +15,11 @@
 namespace moe {
 
 const char* const kKernelNames[K_NUM_KINDS] = {
-    "route_topk",        "permute_hist",      "permute_scan",     "permute_scatter",
-    "build_tables",      "gemm_gateup_fwd",   "gemm_down_fwd",    "gemm_down_bwd",
+    "route_topk",        "permute_hist",      "permute_scatter",  "build_tables",
+    "gemm_gateup_fwd",   "gemm_down_fwd",     "gemm_down_bwd",
     "gemm_gateup_bwd",   "lora_wgrad",        "unpermute_combine", "memset",
     "rank_xa",           "rank_ha",           "rank_t1",          "rank_t2",
-    "router_backward",   "gemm_dw_gu",        "gemm_dw_d",        "gather_rows"};
+    "router_backward",   "gemm_dw_gu",        "gemm_dw_d"};
 
 namespace {
 struct Rec {

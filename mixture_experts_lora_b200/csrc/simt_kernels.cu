@@ -1,6 +1,5 @@
 // SIMT kernels of the layer: top-k routing, the stable counting-sort permute,
-// tile tables, weighted un-permute combine, router backward and the gathered-row
-// copies of full fine-tuning.
+// tile tables, weighted un-permute combine and router backward.
 // All are HBM- or latency-bound; they use coalesced 16-byte accesses and warp
 // primitives, no floating-point atomics.
 #include "common.cuh"
@@ -106,26 +105,89 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 }
 
 // ------------------------------------------------------------------ permute
-// Counting sort in three launches.  Pairs are cut into chunks of kPermuteChunk
-// consecutive pair indices, one 512-thread block per chunk, one pair per thread:
-//   1. histogram of each chunk (shared-memory atomics)     -> hist[e][c]
-//   2. one block: per expert, an exclusive scan over the chunks (a warp per
-//      expert column), counts and offsets from a block scan over the experts,
-//      then hist[e][c] = offsets[e] + pairs of expert e in chunks before c
-//   3. each block ranks its pairs: __match_any_sync groups the lanes of a warp by
+// Counting sort in two launches.  Pairs are cut into chunks of consecutive pair
+// indices, one block per chunk:
+//   1. each block counts its chunk's pairs per expert (shared-memory atomics) into
+//      hist[c][e]; the block that finishes last (an arrival counter decides which,
+//      never the order of any sum) scans every expert's counts over the chunks,
+//      forms counts and offsets with a block scan over the experts, and turns
+//      hist[c][e] into the sorted position of the first pair of e in chunk c;
+//   2. each block ranks its pairs: __match_any_sync groups the lanes of a warp by
 //      expert (rank = earlier lanes of the group), a shared [warp][expert] table
 //      prefix-summed over the warps orders the warps, hist gives the chunk base;
 //      positions are therefore stable (ascending pair index inside every segment).
+// Routing can fill launch 1 as well: in moe_route_permute each routing warp counts
+// its token's pairs.
 // Replaces the per-expert mask lookup of the loop form ("What is
 // torch._grouped_mm?", Unsloth faster-moe docs).
 constexpr int kPermThreads = kPermuteChunk;
 constexpr int kPermWarps = kPermThreads / 32;
 
+// Run by every thread of the last block of a histogram launch (any block size that is
+// a multiple of 32, at most 1024): see step 1 above.  hist is [n_chunks][E]; s_tot
+// holds E ints.  A thread per expert walks the chunks in batches of independent loads.
+__device__ void scan_histograms(int32_t* __restrict__ hist, int n_chunks, int E, int64_t P,
+                                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                int* s_tot, int* s_warp) {
+  constexpr int B = 16;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c0 = 0; c0 < n_chunks; c0 += B) {
+      int v[B];
+#pragma unroll
+      for (int j = 0; j < B; ++j) v[j] = c0 + j < n_chunks ? __ldcg(hist + (int64_t)(c0 + j) * E + e) : 0;
+#pragma unroll
+      for (int j = 0; j < B; ++j) {
+        if (c0 + j < n_chunks) hist[(int64_t)(c0 + j) * E + e] = run;
+        run += v[j];
+      }
+    }
+    s_tot[e] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the expert totals: each thread owns a run of `per` experts
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int mine = 0;
+  for (int e = e0; e < e0 + per && e < E; ++e) mine += s_tot[e];
+  int all;
+  int run = block_exclusive_scan_1024(mine, s_warp, &all);
+  for (int e = e0; e < e0 + per && e < E; ++e) {
+    const int t = s_tot[e];
+    counts[e] = t;
+    offsets[e] = run;
+    s_tot[e] = run;
+    run += t;
+  }
+  if (threadIdx.x == 0) offsets[E] = (int32_t)P;
+  __syncthreads();
+  const int64_t total = (int64_t)n_chunks * E;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) hist[i] += s_tot[i % E];
+}
+
+// The block's histogram is in s_hist: publish it, and let the last block scan.
+__device__ __forceinline__ void publish_histogram(const int* s_hist, int32_t* __restrict__ hist,
+                                                  int n_chunks, int E, int64_t P,
+                                                  int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ offsets, int* arrive,
+                                                  int* s_tot, int* s_warp, int* s_last) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *s_last = atomicAdd(arrive, 1) == n_chunks - 1;
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  scan_histograms(hist, n_chunks, E, P, counts, offsets, s_tot, s_warp);
+  if (threadIdx.x == 0) *arrive = 0;                 // ready for the next call
+}
+
 __global__ void __launch_bounds__(kPermThreads)
     permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
-                        int32_t* __restrict__ hist, int* err) {
+                        int32_t* __restrict__ hist, int32_t* __restrict__ counts,
+                        int32_t* __restrict__ offsets, int* arrive, int* err) {
   pdl_begin();
-  extern __shared__ int s_hist[];
+  __shared__ int s_hist[1024], s_tot[1024], s_warp[33], s_last;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
   const int64_t p = (int64_t)blockIdx.x * kPermuteChunk + threadIdx.x;
@@ -135,70 +197,88 @@ __global__ void __launch_bounds__(kPermThreads)
     else report_error(err, MOE_ERR_DEVICE_INDEX);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    hist[(int64_t)e * n_chunks + blockIdx.x] = s_hist[e];
+  publish_histogram(s_hist, hist, n_chunks, E, P, counts, offsets, arrive, s_tot, s_warp, &s_last);
 }
 
-__global__ void __launch_bounds__(1024)
-    permute_scan_kernel(int32_t* __restrict__ hist, int n_chunks, int E, int64_t P,
-                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+// Routing (a warp per token, as route_topk_kernel, 8 tokens per block) fused with the
+// permutation's histogram: chunk c holds the pairs of tokens [c tpc, (c + 1) tpc), and
+// each warp adds its token's k pairs to hist[c][e] with integer atomics (the counts
+// do not depend on their order); the last block to finish scans.  hist and the
+// arrival counter after it are zero on entry.
+__global__ void __launch_bounds__(256)
+    route_hist_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int tpc,
+                      int32_t* __restrict__ ids, float* __restrict__ wout, int n_chunks,
+                      int32_t* __restrict__ hist, int32_t* __restrict__ counts,
+                      int32_t* __restrict__ offsets, int* arrive) {
   pdl_begin();
-  __shared__ int s_tot[1024];
-  __shared__ int s_warp[33];
+  extern __shared__ float s_logits[];               // [8 warps][E]
+  __shared__ int s_tot[1024], s_warp[33], s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = warp; e < E; e += 32) {
-    int32_t* col = hist + (int64_t)e * n_chunks;
-    int run = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int v = c < n_chunks ? col[c] : 0;
-      int incl = v;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += u;
+  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
+  if (t < T) {
+    float* row = s_logits + warp * E;
+    const float* src = logits + t * E;
+    for (int e = lane; e < E; e += 32) row[e] = src[e];
+    __syncwarp();
+    const int per_lane = (E + 31) >> 5;
+    uint32_t taken = 0;
+    float my_val = 0.f;
+    int my_id = 0;
+    for (int j = 0; j < k; ++j) {
+      uint32_t bkey = 0, blo = 0;
+      for (int q = 0; q < per_lane; ++q) {
+        const int e = lane + 32 * q;
+        if (e >= E || ((taken >> q) & 1u)) continue;
+        const uint32_t key = order_key(row[e]);
+        if (blo == 0 || key > bkey) { bkey = key; blo = ~(uint32_t)e; }
       }
-      if (c < n_chunks) col[c] = run + incl - v;
-      run += __shfl_sync(0xffffffffu, incl, 31);
+      const uint32_t wkey = __reduce_max_sync(0xffffffffu, blo != 0 ? bkey : 0u);
+      const uint32_t wlo = __reduce_max_sync(0xffffffffu, (blo != 0 && bkey == wkey) ? blo : 0u);
+      const int bi = (int)(~wlo);
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (lane == j) { my_val = row[bi]; my_id = bi; }
     }
-    if (lane == 0) s_tot[e] = run;
+    const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
+    const float z = lane < k ? expf(my_val - vmax) : 0.f;
+    float sum = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+      ids[t * k + lane] = my_id;
+      wout[t * k + lane] = z / sum;
+      atomicAdd(&hist[(t / tpc) * E + my_id], 1);
+    }
   }
+  __threadfence();
   __syncthreads();
-  const int e = threadIdx.x;
-  const int tot = e < E ? s_tot[e] : 0;
-  int all;
-  const int excl = block_exclusive_scan_1024(tot, s_warp, &all);
-  if (e < E) {
-    counts[e] = tot;
-    offsets[e] = excl;
-    s_tot[e] = excl;
-  }
-  if (e == 0) offsets[E] = (int32_t)P;
+  if (threadIdx.x == 0) s_last = atomicAdd(arrive, 1) == (int)gridDim.x - 1;
   __syncthreads();
-  const int64_t total = (int64_t)n_chunks * E;
-  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) hist[i] += s_tot[i / n_chunks];
+  if (!s_last) return;
+  __threadfence();
+  scan_histograms(hist, n_chunks, E, T * k, counts, offsets, s_tot, s_warp);
 }
 
 __global__ void __launch_bounds__(kPermThreads)
     permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
-                           const int32_t* __restrict__ base, int32_t* __restrict__ sorted_pairs,
-                           int32_t* __restrict__ pair_pos) {
+                           int chunk_pairs, const int32_t* __restrict__ base,
+                           int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos) {
   pdl_begin();
   extern __shared__ int s_cnt[];   // [kPermWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_cnt[i] = 0;
   __syncthreads();
-  const int64_t p = (int64_t)blockIdx.x * kPermuteChunk + threadIdx.x;
+  const int64_t p = (int64_t)blockIdx.x * chunk_pairs + threadIdx.x;
+  const bool in = (int)threadIdx.x < chunk_pairs && p < P;
   int e = -1;
-  if (p < P) e = ids[p];
-  const bool ok = p < P && e >= 0 && e < E;
+  if (in) e = ids[p];
+  const bool ok = in && e >= 0 && e < E;
   const int key = ok ? e : -1 - lane;  // invalid lanes never group
   const unsigned grp = __match_any_sync(0xffffffffu, key);
   const int rank = __popc(grp & ((1u << lane) - 1u));
   if (ok && (31 - __clz(grp)) == lane) s_cnt[warp * E + e] = __popc(grp);
   __syncthreads();
   for (int ee = threadIdx.x; ee < E; ee += blockDim.x) {
-    int run = base[(int64_t)ee * n_chunks + blockIdx.x];
+    int run = base[(int64_t)blockIdx.x * E + ee];
     for (int w = 0; w < kPermWarps; ++w) {
       const int t = s_cnt[w * E + ee];
       s_cnt[w * E + ee] = run;
@@ -213,31 +293,76 @@ __global__ void __launch_bounds__(kPermThreads)
   }
 }
 
-cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* sorted_pairs, int32_t* pair_pos, int32_t* hist, int* err,
-                           cudaStream_t s) {
-  const int n_chunks = (int)((P + kPermuteChunk - 1) / kPermuteChunk);
-  if (n_chunks > 0) {
-    ProfScope ps(K_PERM_HIST, s);
-    if (cudaError_t le_ = launch_pdl(permute_hist_kernel, dim3(n_chunks), dim3(kPermThreads), E * sizeof(int), s, 1, ids, P, E, n_chunks, hist, err); le_ != cudaSuccess) return le_;
-    cudaError_t st = cudaGetLastError();
-    if (st != cudaSuccess) return st;
-  }
-  {
-    ProfScope ps(K_PERM_SCAN, s);
-    if (cudaError_t le_ = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, s, 1, hist, n_chunks, E, P, counts, offsets); le_ != cudaSuccess) return le_;
-  }
-  cudaError_t st = cudaGetLastError();
-  if (st != cudaSuccess || n_chunks == 0) return st;
+static cudaError_t launch_scatter(const int32_t* ids, int64_t P, int E, int n_chunks, int chunk_pairs,
+                                  const int32_t* hist, int32_t* sorted_pairs, int32_t* pair_pos,
+                                  cudaStream_t s) {
   const int smem = kPermWarps * E * (int)sizeof(int);
   if (smem > 48 * 1024) {
-    st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (st != cudaSuccess) return st;
   }
   ProfScope ps(K_PERM_SCATTER, s);
-  if (cudaError_t le_ = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads), smem, s, 1, ids, P, E, n_chunks, hist, sorted_pairs,
-                                                              pair_pos); le_ != cudaSuccess) return le_;
+  if (cudaError_t le_ = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads), smem, s, 1, ids,
+                                   P, E, n_chunks, chunk_pairs, hist, sorted_pairs, pair_pos);
+      le_ != cudaSuccess)
+    return le_;
   return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts, int32_t* offsets,
+                           int32_t* sorted_pairs, int32_t* pair_pos, int32_t* hist, int* arrive,
+                           int* err, cudaStream_t s) {
+  const int n_chunks = (int)((P + kPermuteChunk - 1) / kPermuteChunk);
+  if (n_chunks == 0) {
+    // no pairs: zero counts, offsets all zero
+    cudaError_t st = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s);
+    if (st != cudaSuccess) return st;
+    return cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
+  }
+  cudaError_t st = cudaMemsetAsync(arrive, 0, sizeof(int), s);
+  if (st != cudaSuccess) return st;
+  {
+    ProfScope ps(K_PERM_HIST, s);
+    if (cudaError_t le_ = launch_pdl(permute_hist_kernel, dim3(n_chunks), dim3(kPermThreads), 0, s, 1,
+                                     ids, P, E, n_chunks, hist, counts, offsets, arrive, err);
+        le_ != cudaSuccess)
+      return le_;
+    st = cudaGetLastError();
+    if (st != cudaSuccess) return st;
+  }
+  return launch_scatter(ids, P, E, n_chunks, kPermuteChunk, hist, sorted_pairs, pair_pos, s);
+}
+
+int route_tokens_per_chunk(int k) { return kPermuteChunk / k; }
+
+cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
+                                 float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
+                                 int32_t* pair_pos, int32_t* hist, int* arrive, cudaStream_t s) {
+  const int tpc = route_tokens_per_chunk(k);
+  const int n_chunks = (int)((T + tpc - 1) / tpc);
+  const int64_t P = T * (int64_t)k;
+  if (n_chunks == 0) {
+    cudaError_t st = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s);
+    if (st != cudaSuccess) return st;
+    return cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
+  }
+  // the histogram and, right after it, the arrival counter start at zero
+  const size_t n_hist = (size_t)n_chunks * E;
+  if (arrive != hist + n_hist) return cudaErrorInvalidValue;
+  cudaError_t st = cudaMemsetAsync(hist, 0, (n_hist + 1) * sizeof(int32_t), s);
+  if (st != cudaSuccess) return st;
+  {
+    const size_t smem = (size_t)8 * E * sizeof(float);
+    ProfScope ps(K_ROUTE, s);
+    if (cudaError_t le_ = launch_pdl(route_hist_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), smem, s,
+                                     1, logits, T, E, k, tpc, ids, w, n_chunks, hist, counts, offsets,
+                                     arrive);
+        le_ != cudaSuccess)
+      return le_;
+    st = cudaGetLastError();
+    if (st != cudaSuccess) return st;
+  }
+  return launch_scatter(ids, P, E, n_chunks, tpc * k, hist, sorted_pairs, pair_pos, s);
 }
 
 // ------------------------------------------------------------------ tile tables
@@ -497,45 +622,6 @@ cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const
   if (cudaError_t le_ = launch_pdl(router_backward_kernel, dim3((unsigned)((T + tpb - 1) / tpb)), dim3(256), 0, s, 1, 
       reinterpret_cast<const uint4*>(dY), reinterpret_cast<const uint4*>(ys), ids, w, pos, T, k, E,
       m / 8, dlogits); le_ != cudaSuccess) return le_;
-  return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------ gathered rows
-// The expert-ordered copy of X (or of w dY) for the expert-weight gradients of full
-// fine-tuning: out[q] = (w ? w[p] : 1) src[p / k], p = sorted_pairs[q], 16-byte pieces.
-__global__ void gather_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ sp,
-                                   const float* __restrict__ w, int64_t P, int k, int vpr,
-                                   uint4* __restrict__ out) {
-  pdl_begin();
-  const int64_t total = P * vpr;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t q = i / vpr;
-    const int v = (int)(i - q * vpr);
-    const int32_t p = sp[q];
-    uint4 x = src[(int64_t)(p / k) * vpr + v];
-    if (w != nullptr) {
-      float f[8];
-      unpack8(x, f);
-      const float s = w[p];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) f[c] *= s;
-      x = pack8(f);
-    }
-    out[i] = x;
-  }
-}
-
-cudaError_t launch_gather_rows(const uint16_t* src, const int32_t* sorted_pairs, const float* w,
-                               int64_t P, int k, int K, uint16_t* out, cudaStream_t s) {
-  if (P == 0) return cudaSuccess;
-  const int vpr = K / 8;
-  ProfScope ps(K_GATHER_ROWS, s);
-  if (cudaError_t le_ = launch_pdl(gather_rows_kernel, dim3(grid_for(P * vpr, 256)), dim3(256), 0, s, 1,
-                                   reinterpret_cast<const uint4*>(src), sorted_pairs, w, P, k, vpr,
-                                   reinterpret_cast<uint4*>(out));
-      le_ != cudaSuccess)
-    return le_;
   return cudaGetLastError();
 }
 

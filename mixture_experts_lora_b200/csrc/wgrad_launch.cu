@@ -11,8 +11,8 @@ namespace {
 template <int RP, bool V>
 cudaError_t wgrad_rp(const GemmShape& g, const CUtensorMap* tm, const WgradParams& wp,
                      int max_chunks, cudaStream_t s) {
-  using C = WgradCfg<RP, V, true>;
-  auto kern = lora_wgrad_kernel<RP, V, true>;
+  using C = WgradCfg<RP, V>;
+  auto kern = lora_wgrad_kernel<RP, V>;
   cudaError_t st = ensure_smem(kern, C::SMEM_BYTES);
   if (st != cudaSuccess) return st;
   int dtiles = wp.pr[0].n_dtiles + (wp.n_problems > 1 ? wp.pr[1].n_dtiles : 0);
@@ -55,15 +55,14 @@ cudaError_t expert_dw_launch(int kind, const CUtensorMap* tm, const DwParams& p,
 
 cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jobs,
                               const TileInfo* chunks, const int* n_chunks, int max_chunks,
-                              const int32_t* chunk_start, const int32_t* sorted_pairs, int k,
-                              cudaStream_t s) {
+                              const int32_t* chunk_start, cudaStream_t s) {
   if (n_jobs < 1 || n_jobs > 2) return cudaErrorInvalidValue;
   using C0 = WgradCfg<16>;
   CUtensorMap tm[4];      // Big of each problem, then Small of each problem
   WgradParams wp{};
   const uint64_t P = (uint64_t)(g.P > 0 ? g.P : 1);
   bool v = true;
-  for (int j = 0; j < n_jobs; ++j) v = v && (jobs[j].gsrc != nullptr || jobs[j].D % 64 == 0);
+  for (int j = 0; j < n_jobs; ++j) v = v && jobs[j].D % 64 == 0;
   for (int j = 0; j < n_jobs; ++j) {
     const WgradJob& jb = jobs[j];
     const uint64_t ls = (uint64_t)jb.ld_small;
@@ -74,15 +73,11 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
     const uint32_t sb[3] = {8, (uint32_t)C0::BK, (uint32_t)g.rp / 8};
     if (!encode(&tm[2 + j], jb.small, 3, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
-    // Big [P, D] sorted: BK rows x 256 columns per stage (four 64-column atoms); a
-    // gathered Big has no map (the Small map stands in)
-    bool okb = true;
-    if (jb.gsrc != nullptr) tm[j] = tm[2 + j];
-    else okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, C0::BN / 64)
-                 : encode2d(&tm[j], jb.big, P, (uint64_t)jb.D, (uint64_t)jb.D, C0::BK, 64);
+    // Big [P, D] sorted: BK rows x 256 columns per stage (four 64-column atoms)
+    const bool okb = v ? encode_atoms(&tm[j], jb.big, false, 1, P, (uint64_t)jb.D, C0::BK, C0::BN / 64)
+                       : encode2d(&tm[j], jb.big, P, (uint64_t)jb.D, (uint64_t)jb.D, C0::BK, 64);
     if (!okb) return cudaErrorInvalidValue;
     WgradProblem& q = wp.pr[j];
-    q.gsrc = reinterpret_cast<const __nv_bfloat16*>(jb.gsrc);
     q.small = reinterpret_cast<const __nv_bfloat16*>(jb.small);
     q.ld_small = jb.ld_small;
     q.r_small = jb.ld_small;
@@ -104,8 +99,6 @@ cudaError_t launch_lora_wgrad(const GemmShape& g, const WgradJob* jobs, int n_jo
   wp.E = g.E;
   wp.r = g.r;
   wp.scale = g.scale;
-  wp.sorted_pairs = sorted_pairs;
-  wp.k = k;
   wp.err = g.err;
   return v ? wgrad_dispatch<true>(g, tm, wp, max_chunks, s) : wgrad_dispatch<false>(g, tm, wp, max_chunks, s);
 }

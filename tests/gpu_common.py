@@ -66,6 +66,8 @@ def check_full_parity(buf, cpu_inp, cfg, tol=TOL):
     assert np.array_equal(buf.offsets.cpu().numpy(), aux["offsets"]), "offsets"
     assert np.array_equal(buf.sorted_pairs.cpu().numpy(), aux["sorted_pairs"]), "sorted_pairs"
     assert np.array_equal(buf.pair_pos.cpu().numpy(), aux["pair_pos"]), "pair_pos"
+    # the saved sorted input rows are X itself, gathered: bit-exact
+    assert torch.equal(buf.save_Xs.cpu(), cpu_inp["X"][torch.from_numpy(aux["sorted_pairs"] // cfg.k)]), "save_Xs"
     errs = {
         "GU": rel_err(to_np(buf.save_GU), aux["gu"]),
         "H": rel_err(to_np(buf.save_H), aux["h"]),

@@ -85,7 +85,7 @@ def test_host_validation_returns_before_launch(L):
     assert L.moe_permute(fake, 4, 2, 8, fake, fake, fake, fake, fake, 8, null) == ml.MOE_ERR_WORKSPACE
     # forward: bad dims, NULL / misaligned pointers, small workspace
     d = dims()
-    ptrs = [P(4096)] * 15
+    ptrs = [P(4096)] * 16
     assert L.moe_grouped_gemm_lora_fwd(ctypes.byref(dims(m=100)), *ptrs, 1 << 30, null) == ml.MOE_ERR_UNSUPPORTED
     assert L.moe_grouped_gemm_lora_fwd(None, *ptrs, 1 << 30, null) == ml.MOE_ERR_INVALID_ARG
     bad = list(ptrs)
@@ -184,3 +184,19 @@ def test_selftest_bounded_wait_checks_its_arguments(L):
     assert L.moe_selftest_bounded_wait(999, ctypes.c_void_p(16), None) == ml.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_bounded_wait(2_000_000_000, ctypes.c_void_p(16), None) == ml.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_bounded_wait(1_000_000, None, None) == ml.MOE_ERR_INVALID_ARG
+
+
+def test_route_permute_host_validation(L):
+    P = ctypes.c_void_p
+    fake, null = P(256), None
+    args = lambda T, E, k, ws, wsb: (fake, T, E, k, fake, fake, fake, fake, fake, fake, ws, wsb, null)
+    assert L.moe_route_permute(*args(4, 8, 0, fake, 1 << 20)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_route_permute(*args(4, 8, 9, fake, 1 << 20)) == ml.MOE_ERR_UNSUPPORTED
+    assert L.moe_route_permute(*args(-1, 8, 2, fake, 1 << 20)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_route_permute(*args(4, 8, 2, null, 0)) == ml.MOE_ERR_INVALID_ARG
+    assert L.moe_route_permute(*args(4, 8, 2, fake, 8)) == ml.MOE_ERR_WORKSPACE
+    # moe_workspace_bytes covers the routed histogram chunks for any k
+    for k in (1, 3, 5, 8, 32):
+        T, E = 1000, 64
+        chunks = -(-T // (512 // k))
+        assert ml.moe_workspace_bytes(dims(T=T, E=E, k=k)) >= chunks * E * 4 + 4

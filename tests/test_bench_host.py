@@ -32,13 +32,12 @@ def test_roof_entry_rates_and_binding_resource():
 
 
 def test_gate_up_forward_bytes_at_the_qwen_shape():
-    # W_gu, X (its rows are gathered, k per token, from L2: read once), bf16(c XA),
-    # B_gu, and GU and H written, each once, in bf16
+    # W_gu, sorted X, bf16(c XA), B_gu, and GU and H written, each once, in bf16
     cfg = CONFIGS["qwen3_30b_a3b"]
     P = cfg.T * cfg.k
-    want = (cfg.E * cfg.m * 2 * cfg.n + cfg.T * cfg.m + P * 16 + cfg.E * 16 * 2 * cfg.n
+    want = (cfg.E * cfg.m * 2 * cfg.n + P * cfg.m + P * 16 + cfg.E * 16 * 2 * cfg.n
             + P * 2 * cfg.n + P * cfg.n) * 2
-    assert bench.kernel_work(cfg)["gemm_gateup_fwd"]["byte"] == want == 980_418_560
+    assert bench.kernel_work(cfg)["gemm_gateup_fwd"]["byte"] == want == 1_097_859_072
     # only the experts that received tokens have their weights read
     fewer = bench.kernel_work(cfg, active_experts=64)["gemm_gateup_fwd"]["byte"]
     assert want - fewer == 64 * (cfg.m * 2 * cfg.n + 16 * 2 * cfg.n) * 2
@@ -52,7 +51,8 @@ def test_rank_padding_of_the_lora_operands():
     for r, rp in ((8, 16), (16, 16), (24, 32), (48, 64), (64, 64), (96, 128), (128, 128)):
         cfg = LayerConfig("x", T=base.T, m=base.m, n=base.n, E=base.E, k=base.k, r=r, alpha=r)
         w = bench.kernel_work(cfg)
-        assert w["rank_t2"]["byte"] == P * 2 * cfg.n * 2 + cfg.E * r * 2 * cfg.n * 2 + 2 * P * rp * 2
+        assert w["rank_ha"]["byte"] == (P * cfg.n * 2 + cfg.E * cfg.n * r * 2 + P * r * 2
+                                        + P * rp * 2)
 
 
 def test_ncu_traffic_only_while_the_sources_match(tmp_path, monkeypatch):

@@ -64,6 +64,45 @@ def test_permute_bitexact(T, k, E, hot):
     assert np.array_equal(pos.cpu().numpy(), rpos)
 
 
+@pytest.mark.parametrize("T,E,k", [(4096, 128, 8), (300, 64, 3), (64, 1024, 32), (1000, 16, 1),
+                                   (129, 33, 5), (1, 8, 2), (0, 8, 2)])
+def test_route_permute_fused_bitexact(T, E, k):
+    # routing and the counting sort in one call: the same ids, weights and permutation
+    # as the oracle (and as moe_route_topk followed by moe_permute), ties included
+    g = torch.Generator().manual_seed(T * 7 + E + k)
+    logits = (torch.randn(T, E, generator=g) * 2).round() / 2
+    if T > 0:
+        logits[0] = 0.0
+    P = T * k
+    d = lambda *shape, dt=torch.int32: torch.full(shape, -1, dtype=dt, device="cuda")
+    ids, w = d(T, k), d(T, k, dt=torch.float32)
+    counts, offsets, sp, pos = d(E), d(E + 1), d(P), d(P)
+    ws = torch.empty(ml.moe_workspace_bytes(ml.make_dims(max(T, 1), 64, 64, E, k, 16, 1.0)),
+                     dtype=torch.uint8, device="cuda")
+    ml.moe_route_permute(logits.cuda(), k, ids, w, counts, offsets, sp, pos, ws)
+    assert ml.moe_get_device_error() == ml.MOE_OK
+    rid, rw = O.route_topk(logits.numpy(), k) if T > 0 else (np.zeros((0, k), np.int64), np.zeros((0, k)))
+    rc, ro, rsp, rpos = O.permute(rid, E)
+    assert np.array_equal(ids.cpu().numpy(), rid)
+    if T > 0:
+        assert rel_err(to_np(w), rw) <= TOL_W
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(sp.cpu().numpy(), rsp)
+    assert np.array_equal(pos.cpu().numpy(), rpos)
+    # the separate calls give the same bits
+    ids2, w2 = d(T, k), d(T, k, dt=torch.float32)
+    c2, o2, sp2, pos2 = d(E), d(E + 1), d(P), d(P)
+    if T > 0:
+        ml.moe_route_topk(logits.cuda(), k, ids2, w2)
+    ml.moe_permute(ids2, E, c2, o2, sp2, pos2, ws)
+    torch.cuda.synchronize()
+    for a, b in ((ids, ids2), (counts, c2), (offsets, o2), (sp, sp2), (pos, pos2)):
+        assert torch.equal(a, b)
+    if T > 0:
+        assert torch.equal(w, w2)
+
+
 def test_permute_reports_bad_expert_id_without_faulting():
     ids = torch.tensor([[0, 1], [2, 7]], dtype=torch.int32, device="cuda")   # 7 >= E
     E = 4
@@ -248,7 +287,7 @@ def test_graph_replay_matches_eager_bitwise():
     cfg = small_config(T=640, m=256, n=128, E=8, k=2, r=16, alpha=16)
     inp, _ = inputs_on(cfg, seed=11)
     eager = run_layer(inp, cfg)
-    keys = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU", "save_H", "Y_sorted")
+    keys = ("Y", "dX", "dA_gu", "dB_gu", "dA_d", "dB_d", "save_GU", "save_Xs", "save_H", "Y_sorted")
     snap = {k: getattr(eager, k).clone() for k in keys}
     buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale)
     s = torch.cuda.Stream()
