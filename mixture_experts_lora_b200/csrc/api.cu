@@ -126,7 +126,7 @@ Layout make_layout(const moe_dims_t& d) {
   const size_t dmax = m > 2 * n ? m : 2 * n;
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
-  L.hist = take((size_t)L.perm_chunks * E * 4 + 4);
+  L.hist = take(permute_scratch_ints(L.perm_chunks, d.E) * 4);
   L.tiles = take((size_t)L.max_row_tiles * sizeof(TileInfo));
   L.n_tiles = take(4);
   L.gchunks = take((size_t)L.max_gchunks * sizeof(TileInfo));
@@ -375,13 +375,13 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
   if (counts == nullptr || offsets == nullptr || ws == nullptr) return MOE_ERR_INVALID_ARG;
   if (P > 0 && (topk_ids == nullptr || sorted_pairs == nullptr || pair_pos == nullptr))
     return MOE_ERR_INVALID_ARG;
-  const size_t n_hist = (size_t)((P + kPermuteChunk - 1) / kPermuteChunk) * E;
-  if (ws_bytes < align256(n_hist * 4 + 4)) return MOE_ERR_WORKSPACE;
+  const size_t need = permute_scratch_ints((P + kPermuteChunk - 1) / kPermuteChunk, E) * 4;
+  if (ws_bytes < need) return MOE_ERR_WORKSPACE;
   int* err = status_ptr();
   if (err == nullptr) return MOE_ERR_CUDA;
-  int32_t* hist = static_cast<int32_t*>(ws);
-  return cuda_status(launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos, hist,
-                                    hist + n_hist, err, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos,
+                                    static_cast<int32_t*>(ws), err,
+                                    static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_route_permute(const float* logits, int64_t T, int32_t E, int32_t k,
@@ -397,12 +397,10 @@ moe_status_t moe_route_permute(const float* logits, int64_t T, int32_t E, int32_
                 sorted_pairs == nullptr || pair_pos == nullptr))
     return MOE_ERR_INVALID_ARG;
   const int64_t tpb = route_tokens_per_chunk(k);
-  const size_t n_hist = (size_t)((T + tpb - 1) / tpb) * E;
-  if (ws_bytes < align256(n_hist * 4 + 4)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < permute_scratch_ints((T + tpb - 1) / tpb, E) * 4) return MOE_ERR_WORKSPACE;
   if (status_ptr() == nullptr) return MOE_ERR_CUDA;
-  int32_t* hist = static_cast<int32_t*>(ws);
   return cuda_status(launch_route_permute(logits, T, E, k, topk_ids, topk_w, counts, offsets,
-                                          sorted_pairs, pair_pos, hist, hist + n_hist,
+                                          sorted_pairs, pair_pos, static_cast<int32_t*>(ws),
                                           static_cast<cudaStream_t>(stream)));
 }
 

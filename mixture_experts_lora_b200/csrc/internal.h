@@ -67,18 +67,24 @@ void* current_context();
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
-// one block per chunk of kPermuteChunk pairs; hist holds n_chunks * E ints; arrive is
-// an int the call zeroes (the last block of the histogram launch is the one that scans)
+// Counting-sort scratch: per-chunk histograms [n_chunks][E], expert totals [E] and
+// an arrival counter (the last block of the histogram launch is the one that scans).
 constexpr int kPermuteChunk = 512;
+inline size_t permute_scratch_ints(int64_t n_chunks, int E) {
+  return (size_t)n_chunks * E + E + 1;
+}
+// One block per chunk of kPermuteChunk pairs; scratch holds
+// permute_scratch_ints(ceil(P / kPermuteChunk), E) ints (the call zeroes what it needs).
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
-                           int32_t* hist, int* arrive, int* err, cudaStream_t s);
+                           int32_t* scratch, int* err, cudaStream_t s);
 // Routing fused with the permutation's histogram: chunks of route_tokens_per_chunk(k)
-// tokens (their k pairs each), hist holds ceil(T / that) * E ints.
+// tokens (their k pairs each); scratch holds
+// permute_scratch_ints(ceil(T / route_tokens_per_chunk(k)), E) ints.
 int route_tokens_per_chunk(int k);
 cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
                                  float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
-                                 int32_t* pair_pos, int32_t* hist, int* arrive, cudaStream_t s);
+                                 int32_t* pair_pos, int32_t* scratch, cudaStream_t s);
 // From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
 // experts (row kernels), token chunks of at most `gchunk_rows` rows split
 // evenly inside each expert (grouped GEMMs; all but the last chunk of an expert

@@ -18,9 +18,9 @@ namespace moe {
 namespace {
 
 // 2^19 int32 = 2 MiB: room for ceil(T*k / kPermuteChunk) * E histogram entries, then
-// the arrival counter of the histogram launch.
+// the expert totals (E <= 1024) and the arrival counter of the histogram launch.
 constexpr size_t kPermuteScratchInts = size_t(1) << 19;
-__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts + 64];
+__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts + 1024 + 64];
 
 constexpr int kMaxDevices = 64;
 
@@ -64,15 +64,16 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, 
   if (counts == nullptr || offsets == nullptr) return MOE_ERR_INVALID_ARG;
   if (P > 0 && (topk_ids == nullptr || sorted_pairs == nullptr || pair_pos == nullptr))
     return MOE_ERR_INVALID_ARG;
-  // every histogram entry is written before it is read; the arrival counter after them
-  // is zeroed by the call itself
-  const int64_t need = ((P + kPermuteChunk - 1) / kPermuteChunk) * (int64_t)E;
-  if (need > (int64_t)kPermuteScratchInts) return MOE_ERR_WORKSPACE;
+  // every histogram entry is written before it is read; the totals and the arrival
+  // counter after them are zeroed by the call itself
+  const int64_t n_hist = ((P + kPermuteChunk - 1) / kPermuteChunk) * (int64_t)E;
+  if (n_hist > (int64_t)kPermuteScratchInts) return MOE_ERR_WORKSPACE;
+  static_assert(kPermuteScratchInts + 1024 + 1 <= sizeof(g_permute_scratch) / sizeof(int32_t),
+                "histograms, totals and counter");
   int32_t* scratch = permute_scratch();
   int* err = moe_status_word();
   if (scratch == nullptr || err == nullptr) return MOE_ERR_CUDA;
   const cudaError_t st = launch_permute(topk_ids, P, E, counts, offsets, sorted_pairs, pair_pos,
-                                        scratch, scratch + kPermuteScratchInts, err,
-                                        static_cast<cudaStream_t>(stream));
+                                        scratch, err, static_cast<cudaStream_t>(stream));
   return st == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -70,8 +70,10 @@ struct RankCfg {
   static constexpr int L_BYTES = HALVES * L_CHUNK;
   static constexpr int STAGE_BYTES = NT * TILE_BYTES + L_BYTES;
   // RK_GATHER: four stages (two of copies in flight) keep three CTAs on an SM at rank
-  // 16; deeper rings cost that third CTA and were slower
-  static constexpr int STAGES_WANT = 4;
+  // 16; deeper rings cost that third CTA and were slower, three stages were no faster.
+  // RK_DSWIGLU: two stages of three tiles keep two CTAs on an SM (one CTA of three or
+  // four stages was 7-12% slower)
+  static constexpr int STAGES_WANT = MODE == RK_DSWIGLU ? 2 : 4;
   static constexpr int STAGES_FIT = (232448 - 2048) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT < STAGES_WANT ? STAGES_FIT : STAGES_WANT;
   static constexpr int LOOK = MODE == RK_GATHER ? STAGES - 2 : 0;   // gathered stages in flight

@@ -106,16 +106,16 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 
 // ------------------------------------------------------------------ permute
 // Counting sort in two launches.  Pairs are cut into chunks of consecutive pair
-// indices, one block per chunk:
-//   1. each block counts its chunk's pairs per expert (shared-memory atomics) into
-//      hist[c][e]; the block that finishes last (an arrival counter decides which,
-//      never the order of any sum) scans every expert's counts over the chunks,
-//      forms counts and offsets with a block scan over the experts, and turns
-//      hist[c][e] into the sorted position of the first pair of e in chunk c;
-//   2. each block ranks its pairs: __match_any_sync groups the lanes of a warp by
-//      expert (rank = earlier lanes of the group), a shared [warp][expert] table
-//      prefix-summed over the warps orders the warps, hist gives the chunk base;
-//      positions are therefore stable (ascending pair index inside every segment).
+// indices, one block per chunk.  Scratch: hist [n_chunks][E], tot [E], arrive.
+//   1. each block counts its chunk's pairs per expert into hist[c][e] and adds them
+//      to tot[e] (integer atomics: the sums do not depend on their order); the
+//      block that finishes last (an arrival counter decides which) scans tot into
+//      counts and offsets;
+//   2. block c starts expert e's run at offsets[e] + sum over c' < c of hist[c'][e],
+//      then ranks its pairs: __match_any_sync groups the lanes of a warp by expert
+//      (rank = earlier lanes of the group), a shared [warp][expert] table prefix-
+//      summed over the warps orders the warps; positions are therefore stable
+//      (ascending pair index inside every segment).
 // Routing can fill launch 1 as well: in moe_route_permute each routing warp counts
 // its token's pairs.
 // Replaces the per-expert mask lookup of the loop form ("What is
@@ -124,28 +124,13 @@ constexpr int kPermThreads = kPermuteChunk;
 constexpr int kPermWarps = kPermThreads / 32;
 
 // Run by every thread of the last block of a histogram launch (any block size that is
-// a multiple of 32, at most 1024): see step 1 above.  hist is [n_chunks][E]; s_tot
-// holds E ints.  A thread per expert walks the chunks in batches of independent loads.
-__device__ void scan_histograms(int32_t* __restrict__ hist, int n_chunks, int E, int64_t P,
-                                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                int* s_tot, int* s_warp) {
-  constexpr int B = 16;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int c0 = 0; c0 < n_chunks; c0 += B) {
-      int v[B];
-#pragma unroll
-      for (int j = 0; j < B; ++j) v[j] = c0 + j < n_chunks ? __ldcg(hist + (int64_t)(c0 + j) * E + e) : 0;
-#pragma unroll
-      for (int j = 0; j < B; ++j) {
-        if (c0 + j < n_chunks) hist[(int64_t)(c0 + j) * E + e] = run;
-        run += v[j];
-      }
-    }
-    s_tot[e] = run;
-  }
+// a multiple of 32, at most 1024): counts and offsets from the expert totals.
+__device__ void scan_totals(const int32_t* __restrict__ tot, int E, int64_t P,
+                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                            int* s_tot, int* s_warp) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = __ldcg(tot + e);
   __syncthreads();
-  // exclusive scan of the expert totals: each thread owns a run of `per` experts
+  // exclusive scan of the totals: each thread owns a run of `per` experts
   const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
   const int e0 = threadIdx.x * per;
   int mine = 0;
@@ -156,38 +141,18 @@ __device__ void scan_histograms(int32_t* __restrict__ hist, int n_chunks, int E,
     const int t = s_tot[e];
     counts[e] = t;
     offsets[e] = run;
-    s_tot[e] = run;
     run += t;
   }
   if (threadIdx.x == 0) offsets[E] = (int32_t)P;
-  __syncthreads();
-  const int64_t total = (int64_t)n_chunks * E;
-  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) hist[i] += s_tot[i % E];
-}
-
-// The block's histogram is in s_hist: publish it, and let the last block scan.
-__device__ __forceinline__ void publish_histogram(const int* s_hist, int32_t* __restrict__ hist,
-                                                  int n_chunks, int E, int64_t P,
-                                                  int32_t* __restrict__ counts,
-                                                  int32_t* __restrict__ offsets, int* arrive,
-                                                  int* s_tot, int* s_warp, int* s_last) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) *s_last = atomicAdd(arrive, 1) == n_chunks - 1;
-  __syncthreads();
-  if (!*s_last) return;
-  __threadfence();
-  scan_histograms(hist, n_chunks, E, P, counts, offsets, s_tot, s_warp);
-  if (threadIdx.x == 0) *arrive = 0;                 // ready for the next call
 }
 
 __global__ void __launch_bounds__(kPermThreads)
     permute_hist_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
-                        int32_t* __restrict__ hist, int32_t* __restrict__ counts,
-                        int32_t* __restrict__ offsets, int* arrive, int* err) {
+                        int32_t* __restrict__ hist, int32_t* __restrict__ tot,
+                        int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* arrive,
+                        int* err) {
   pdl_begin();
-  __shared__ int s_hist[1024], s_tot[1024], s_warp[33], s_last;
+  __shared__ int s_hist[1024], s_warp[33], s_last;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
   const int64_t p = (int64_t)blockIdx.x * kPermuteChunk + threadIdx.x;
@@ -197,19 +162,31 @@ __global__ void __launch_bounds__(kPermThreads)
     else report_error(err, MOE_ERR_DEVICE_INDEX);
   }
   __syncthreads();
-  publish_histogram(s_hist, hist, n_chunks, E, P, counts, offsets, arrive, s_tot, s_warp, &s_last);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = s_hist[e];
+    hist[(int64_t)blockIdx.x * E + e] = c;
+    if (c != 0) atomicAdd(&tot[e], c);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(arrive, 1) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  scan_totals(tot, E, P, counts, offsets, s_hist, s_warp);
+  if (threadIdx.x == 0) *arrive = 0;                 // ready for the next call
 }
 
 // Routing (a warp per token, as route_topk_kernel, 8 tokens per block) fused with the
 // permutation's histogram: chunk c holds the pairs of tokens [c tpc, (c + 1) tpc), and
-// each warp adds its token's k pairs to hist[c][e] with integer atomics (the counts
-// do not depend on their order); the last block to finish scans.  hist and the
-// arrival counter after it are zero on entry.
+// each warp adds its token's k pairs to hist[c][e] and tot[e] with integer atomics;
+// the last block to finish scans tot.  hist, tot and the arrival counter after them
+// are zero on entry.
 __global__ void __launch_bounds__(256)
     route_hist_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int tpc,
-                      int32_t* __restrict__ ids, float* __restrict__ wout, int n_chunks,
-                      int32_t* __restrict__ hist, int32_t* __restrict__ counts,
-                      int32_t* __restrict__ offsets, int* arrive) {
+                      int32_t* __restrict__ ids, float* __restrict__ wout,
+                      int32_t* __restrict__ hist, int32_t* __restrict__ tot,
+                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* arrive) {
   pdl_begin();
   extern __shared__ float s_logits[];               // [8 warps][E]
   __shared__ int s_tot[1024], s_warp[33], s_last;
@@ -247,6 +224,7 @@ __global__ void __launch_bounds__(256)
       ids[t * k + lane] = my_id;
       wout[t * k + lane] = z / sum;
       atomicAdd(&hist[(t / tpc) * E + my_id], 1);
+      atomicAdd(&tot[my_id], 1);
     }
   }
   __threadfence();
@@ -255,19 +233,42 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  scan_histograms(hist, n_chunks, E, T * k, counts, offsets, s_tot, s_warp);
+  scan_totals(tot, E, T * k, counts, offsets, s_tot, s_warp);
 }
 
 __global__ void __launch_bounds__(kPermThreads)
-    permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int n_chunks,
-                           int chunk_pairs, const int32_t* __restrict__ base,
+    permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int chunk_pairs,
+                           const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
                            int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos) {
   pdl_begin();
-  extern __shared__ int s_cnt[];   // [kPermWarps][E]
+  extern __shared__ int s_cnt[];   // [kPermWarps][E], then the chunk's base per expert [E]
+  int* s_base = s_cnt + kPermWarps * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_cnt[i] = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] = offsets[e];
   __syncthreads();
-  const int64_t p = (int64_t)blockIdx.x * chunk_pairs + threadIdx.x;
+  // the chunk's base: G threads per expert each add every G-th earlier chunk's count,
+  // eight independent loads at a time
+  {
+    const int G = E < kPermThreads ? kPermThreads / E : 1;
+    for (int i = threadIdx.x; i < G * E; i += blockDim.x) {
+      const int e = i % E, part = i / E;
+      int sum = 0;
+      for (int c0 = part; c0 < c; c0 += 8 * G) {
+        int v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int cc = c0 + j * G;
+          v[j] = cc < c ? hist[(int64_t)cc * E + e] : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum += v[j];
+      }
+      if (sum != 0) atomicAdd(&s_base[e], sum);
+    }
+  }
+  const int64_t p = (int64_t)c * chunk_pairs + threadIdx.x;
   const bool in = (int)threadIdx.x < chunk_pairs && p < P;
   int e = -1;
   if (in) e = ids[p];
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kPermThreads)
   if (ok && (31 - __clz(grp)) == lane) s_cnt[warp * E + e] = __popc(grp);
   __syncthreads();
   for (int ee = threadIdx.x; ee < E; ee += blockDim.x) {
-    int run = base[(int64_t)blockIdx.x * E + ee];
+    int run = s_base[ee];
     for (int w = 0; w < kPermWarps; ++w) {
       const int t = s_cnt[w * E + ee];
       s_cnt[w * E + ee] = run;
@@ -294,24 +295,24 @@ __global__ void __launch_bounds__(kPermThreads)
 }
 
 static cudaError_t launch_scatter(const int32_t* ids, int64_t P, int E, int n_chunks, int chunk_pairs,
-                                  const int32_t* hist, int32_t* sorted_pairs, int32_t* pair_pos,
-                                  cudaStream_t s) {
-  const int smem = kPermWarps * E * (int)sizeof(int);
+                                  const int32_t* hist, const int32_t* offsets,
+                                  int32_t* sorted_pairs, int32_t* pair_pos, cudaStream_t s) {
+  const int smem = (kPermWarps + 1) * E * (int)sizeof(int);
   if (smem > 48 * 1024) {
     cudaError_t st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (st != cudaSuccess) return st;
   }
   ProfScope ps(K_PERM_SCATTER, s);
   if (cudaError_t le_ = launch_pdl(permute_scatter_kernel, dim3(n_chunks), dim3(kPermThreads), smem, s, 1, ids,
-                                   P, E, n_chunks, chunk_pairs, hist, sorted_pairs, pair_pos);
+                                   P, E, chunk_pairs, hist, offsets, sorted_pairs, pair_pos);
       le_ != cudaSuccess)
     return le_;
   return cudaGetLastError();
 }
 
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts, int32_t* offsets,
-                           int32_t* sorted_pairs, int32_t* pair_pos, int32_t* hist, int* arrive,
-                           int* err, cudaStream_t s) {
+                           int32_t* sorted_pairs, int32_t* pair_pos, int32_t* scratch, int* err,
+                           cudaStream_t s) {
   const int n_chunks = (int)((P + kPermuteChunk - 1) / kPermuteChunk);
   if (n_chunks == 0) {
     // no pairs: zero counts, offsets all zero
@@ -319,25 +320,29 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
     if (st != cudaSuccess) return st;
     return cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
   }
-  cudaError_t st = cudaMemsetAsync(arrive, 0, sizeof(int), s);
+  int32_t* hist = scratch;
+  int32_t* tot = hist + (size_t)n_chunks * E;
+  int* arrive = tot + E;
+  // every hist entry is written by its block; the totals and the counter start at zero
+  cudaError_t st = cudaMemsetAsync(tot, 0, (size_t)(E + 1) * sizeof(int32_t), s);
   if (st != cudaSuccess) return st;
   {
     ProfScope ps(K_PERM_HIST, s);
     if (cudaError_t le_ = launch_pdl(permute_hist_kernel, dim3(n_chunks), dim3(kPermThreads), 0, s, 1,
-                                     ids, P, E, n_chunks, hist, counts, offsets, arrive, err);
+                                     ids, P, E, n_chunks, hist, tot, counts, offsets, arrive, err);
         le_ != cudaSuccess)
       return le_;
     st = cudaGetLastError();
     if (st != cudaSuccess) return st;
   }
-  return launch_scatter(ids, P, E, n_chunks, kPermuteChunk, hist, sorted_pairs, pair_pos, s);
+  return launch_scatter(ids, P, E, n_chunks, kPermuteChunk, hist, offsets, sorted_pairs, pair_pos, s);
 }
 
 int route_tokens_per_chunk(int k) { return kPermuteChunk / k; }
 
 cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
                                  float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
-                                 int32_t* pair_pos, int32_t* hist, int* arrive, cudaStream_t s) {
+                                 int32_t* pair_pos, int32_t* scratch, cudaStream_t s) {
   const int tpc = route_tokens_per_chunk(k);
   const int n_chunks = (int)((T + tpc - 1) / tpc);
   const int64_t P = T * (int64_t)k;
@@ -346,23 +351,24 @@ cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, i
     if (st != cudaSuccess) return st;
     return cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
   }
-  // the histogram and, right after it, the arrival counter start at zero
-  const size_t n_hist = (size_t)n_chunks * E;
-  if (arrive != hist + n_hist) return cudaErrorInvalidValue;
-  cudaError_t st = cudaMemsetAsync(hist, 0, (n_hist + 1) * sizeof(int32_t), s);
+  // the histograms, the totals and the arrival counter after them start at zero
+  int32_t* hist = scratch;
+  int32_t* tot = hist + (size_t)n_chunks * E;
+  int* arrive = tot + E;
+  cudaError_t st = cudaMemsetAsync(hist, 0, permute_scratch_ints(n_chunks, E) * sizeof(int32_t), s);
   if (st != cudaSuccess) return st;
   {
     const size_t smem = (size_t)8 * E * sizeof(float);
     ProfScope ps(K_ROUTE, s);
     if (cudaError_t le_ = launch_pdl(route_hist_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), smem, s,
-                                     1, logits, T, E, k, tpc, ids, w, n_chunks, hist, counts, offsets,
+                                     1, logits, T, E, k, tpc, ids, w, hist, tot, counts, offsets,
                                      arrive);
         le_ != cudaSuccess)
       return le_;
     st = cudaGetLastError();
     if (st != cudaSuccess) return st;
   }
-  return launch_scatter(ids, P, E, n_chunks, tpc * k, hist, sorted_pairs, pair_pos, s);
+  return launch_scatter(ids, P, E, n_chunks, tpc * k, hist, offsets, sorted_pairs, pair_pos, s);
 }
 
 // ------------------------------------------------------------------ tile tables
