@@ -43,7 +43,7 @@ import numpy as np
 __all__ = [
     "to64", "route_topk", "permute", "silu", "sigmoid",
     "expert_forward", "expert_forward_merged", "expert_backward",
-    "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
+    "unpermute_combine", "moe_forward", "moe_backward", "moe_forward_merged", "moe_forward_base",
     "token_forward", "token_backward_dx", "expert_lora_grads", "router_backward",
     "layer_split_gate_up", "moe_weight_grads", "expert_weight_grads",
 ]
@@ -186,6 +186,22 @@ def _route_and_permute(inp, k):
     return ids, w, counts, offsets, sorted_pairs, pair_pos
 
 
+def unpermute_combine(yp, w, pair_pos, k: int):
+    """Un-permute: Y[t] = sum_j w[t,j] * yp[pair_pos[t*k + j]], j ascending; w None
+    means every weight is 1 (the sum of dX over a token's pairs in the backward).
+    The output of a token is its experts' outputs mixed by the routing weights
+    ([Cookbook] "The Dynamic Dispatch Bottleneck in Mixture-of-Experts
+    Architectures"; [MoE12x] "What is torch._grouped_mm?").
+    """
+    yp = np.asarray(yp, dtype=np.float64)
+    T = pair_pos.shape[0] // k
+    Y = np.zeros((T, yp.shape[1]))
+    for j in range(k):
+        rows = yp[pair_pos[np.arange(T) * k + j]]
+        Y += rows if w is None else np.asarray(w, dtype=np.float64)[:, j:j + 1] * rows
+    return Y
+
+
 def moe_forward(inp, k: int, c: float, keep=True):
     """Whole layer forward: route, permute, experts, weighted combine.
 
@@ -218,10 +234,7 @@ def moe_forward(inp, k: int, c: float, keep=True):
             for name in ("gu", "h", "xa", "ha"):
                 aux[name][lo:hi] = f[name]
     aux["yp"] = Yp
-    Y = np.zeros((T, m))
-    for j in range(k):
-        Y += w[:, j:j + 1] * Yp[pair_pos[np.arange(T) * k + j]]
-    return Y, aux
+    return unpermute_combine(Yp, w, pair_pos, k), aux
 
 
 def moe_backward(inp, aux, dY, k: int, c: float):
@@ -266,10 +279,7 @@ def moe_backward(inp, aux, dY, k: int, c: float):
         out["t1"][lo:hi] = b["t1"]
         out["t2"][lo:hi] = b["t2"]
         out["dxp"][lo:hi] = b["dx"]
-    dX = np.zeros((T, m))
-    for j in range(k):
-        dX += out["dxp"][pair_pos[np.arange(T) * k + j]]
-    out["dX"] = dX
+    out["dX"] = unpermute_combine(out["dxp"], None, pair_pos, k)
     return out
 
 

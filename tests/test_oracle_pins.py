@@ -215,6 +215,27 @@ def test_permute_matches_bruteforce():
     assert counts[5] >= 0 and offsets[E] == T * k
 
 
+def test_unpermute_combine_matches_per_token_bruteforce():
+    # Y[t] is token t's routing-weighted sum of its k expert outputs, wherever the
+    # permutation put those rows; the plain form sums them with weight 1
+    rng = np.random.default_rng(11)
+    T, k, m = 9, 3, 5
+    yp = rng.standard_normal((T * k, m))
+    w = rng.random((T, k))
+    pos = rng.permutation(T * k)
+    for weights in (w, None):
+        Y = O.unpermute_combine(yp, weights, pos, k)
+        for t in range(T):
+            want = np.zeros(m)
+            for j in range(k):
+                want = want + (1.0 if weights is None else w[t, j]) * yp[pos[t * k + j]]
+            assert np.allclose(Y[t], want, rtol=1e-15, atol=1e-15)
+    # the identity permutation with one-hot weights picks a single row
+    one = np.zeros((T, k))
+    one[:, 1] = 1.0
+    assert np.array_equal(O.unpermute_combine(yp, one, np.arange(T * k), k), yp[1::k])
+
+
 def test_permute_rejects_bad_ids():
     with pytest.raises(ValueError):
         O.permute(np.array([[0, 9]]), 4)

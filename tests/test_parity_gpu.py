@@ -128,12 +128,8 @@ def test_unpermute_combine(weighted):
     y = torch.empty(T, m, dtype=torch.bfloat16, device="cuda")
     ml.moe_unpermute_combine(ys.cuda(), w.cuda() if weighted else None, pos.cuda(), T, k, m, y)
     torch.cuda.synchronize()
-    ys64 = ys.double().numpy()
-    pos_n = pos.numpy().astype(np.int64)
-    ref = np.zeros((T, m))
-    for j in range(k):
-        wj = w[:, j].double().numpy()[:, None] if weighted else 1.0
-        ref += wj * ys64[pos_n[np.arange(T) * k + j]]
+    ref = O.unpermute_combine(ys.double().numpy(), w.double().numpy() if weighted else None,
+                              pos.numpy().astype(np.int64), k)
     # one bf16 rounding of an fp32 sum: within one bf16 ulp of the value
     assert np.all(np.abs(to_np(y) - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
 
