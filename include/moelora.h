@@ -107,9 +107,9 @@ moe_status_t moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k
  * offsets      int32 [E+1]  (written) exclusive prefix sum of counts, offsets[E] = P
  * sorted_pairs int32 [P]    (written) pair index p at sorted position q
  * pair_pos     int32 [P]    (written) sorted position of pair p (inverse of sorted_pairs)
- * ws, ws_bytes              scratch: (ceil(T*k / 512) * E + E + 1) int32 (per-chunk
- *                           histograms, expert totals, one counter); contents on entry
- *                           do not matter
+ * ws, ws_bytes              scratch: (ceil(T*k / 512) * E + 32 * E + 1) int32
+ *                           (per-chunk histograms, expert totals 128 bytes apart, one
+ *                           counter); contents on entry do not matter
  * An id outside [0, E) sets MOE_ERR_DEVICE_INDEX in the device error word; that
  * pair is left out and the outputs are then incomplete.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
@@ -122,7 +122,7 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
  * block's pairs per expert, so routing and the counting sort take two launches
  * instead of three.  Same definitions and outputs as the two calls (stable order,
  * ties to the lower expert index).
- * ws, ws_bytes: scratch of at least (ceil(T / floor(512 / k)) * E + E + 1) int32
+ * ws, ws_bytes: scratch of at least (ceil(T / floor(512 / k)) * E + 32 * E + 1) int32
  * (per-chunk histograms of whole-token chunks, expert totals, one counter);
  * moe_workspace_bytes() for any dims with this T, E, k is enough.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
@@ -224,8 +224,8 @@ moe_status_t moe_grouped_gemm_full_bwd(
  * memory: plug-ins hosted inside another framework that owns all device memory
  * and hands them no allocator, or code that must run with a fixed device-memory
  * footprint decided before it starts.  It takes no workspace; its scratch (the
- * per-chunk histograms) is a 2 MiB array built into the library (with room for the
- * expert totals and one counter after it), which every GPU that loads the library
+ * per-chunk histograms) is a 2 MiB array built into the library (with 128 KiB more
+ * for the expert totals and one counter), which every GPU that loads the library
  * holds until the process exits.  There is no
  * counterpart on the pages: this is an interface convenience.
  * Limit: ceil(T*k / 512) * E <= 524288 (e.g. T*k <= 2^21 pairs at E = 128);

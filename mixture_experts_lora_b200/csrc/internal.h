@@ -67,11 +67,12 @@ void* current_context();
 // ---- SIMT kernels (simt_kernels.cu)
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids,
                               float* w, int* err, cudaStream_t s);
-// Counting-sort scratch: per-chunk histograms [n_chunks][E], expert totals [E] and
-// an arrival counter (the last block of the histogram launch is the one that scans).
+// Counting-sort scratch: per-chunk histograms [n_chunks][E], expert totals (one per
+// kTotStride ints) and an arrival counter (the last block of the histogram launch is the one that scans).
 constexpr int kPermuteChunk = 512;
+constexpr int kTotStride = 32;            // ints between two experts' totals (128 bytes)
 inline size_t permute_scratch_ints(int64_t n_chunks, int E) {
-  return (size_t)n_chunks * E + E + 1;
+  return (size_t)n_chunks * E + (size_t)E * kTotStride + 1;
 }
 // One block per chunk of kPermuteChunk pairs; scratch holds
 // permute_scratch_ints(ceil(P / kPermuteChunk), E) ints (the call zeroes what it needs).

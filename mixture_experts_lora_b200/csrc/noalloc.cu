@@ -18,9 +18,11 @@ namespace moe {
 namespace {
 
 // 2^19 int32 = 2 MiB: room for ceil(T*k / kPermuteChunk) * E histogram entries, then
-// the expert totals (E <= 1024) and the arrival counter of the histogram launch.
+// the expert totals (E <= 1024, one per kTotStride ints) and the arrival counter of
+// the histogram launch.
 constexpr size_t kPermuteScratchInts = size_t(1) << 19;
-__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts + 1024 + 64];
+constexpr size_t kTotalsInts = size_t(1024) * kTotStride;
+__device__ __align__(256) int32_t g_permute_scratch[kPermuteScratchInts + kTotalsInts + 64];
 
 constexpr int kMaxDevices = 64;
 
@@ -68,7 +70,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t* topk_ids, int64_t T, 
   // counter after them are zeroed by the call itself
   const int64_t n_hist = ((P + kPermuteChunk - 1) / kPermuteChunk) * (int64_t)E;
   if (n_hist > (int64_t)kPermuteScratchInts) return MOE_ERR_WORKSPACE;
-  static_assert(kPermuteScratchInts + 1024 + 1 <= sizeof(g_permute_scratch) / sizeof(int32_t),
+  static_assert(kPermuteScratchInts + kTotalsInts + 1 <= sizeof(g_permute_scratch) / sizeof(int32_t),
                 "histograms, totals and counter");
   int32_t* scratch = permute_scratch();
   int* err = moe_status_word();

@@ -39,34 +39,73 @@ __device__ __forceinline__ T block_exclusive_scan_1024(T v, T* s_warp, T* total_
 }
 
 // ------------------------------------------------------------------ routing
-// One warp per token; the token's logits are staged in shared memory.  Each of
-// the k rounds picks the largest remaining logit, lower expert id on ties: every
-// lane proposes its best untaken candidate as (order-preserving key of the
-// value, lower id wins), two warp max-reductions (redux.sync) pick the winner.
-// The weights are a softmax over the k picked logits.  Router equation:
-// "Accelerating Mixture-of-Experts Fine-Tuning", section "The Dynamic Dispatch
-// Bottleneck in Mixture-of-Experts Architectures".
+// One warp per token.  The k rounds each pick the largest remaining logit, lower
+// expert id on ties, and the weights are a softmax over the k picked logits.  Router
+// equation: "Accelerating Mixture-of-Experts Fine-Tuning", section "The Dynamic
+// Dispatch Bottleneck in Mixture-of-Experts Architectures".
+//
+// Values are compared through an order-preserving unsigned key.  Lane l holds the
+// logits of experts l, l + 32, ...; up to 256 experts these PL <= 8 logits are sorted
+// once in registers (largest first, lower id first on ties: a total order, so any
+// sorting network gives the same list), and each round is two warp max-reductions
+// (redux.sync) over the lanes' list heads, after which the winning lane drops its
+// head.  Wider rows stage the logits in shared memory and every lane rescans its
+// untaken candidates each round.
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;                       // -0 ties with +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // larger float -> larger key
 }
 
-__global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
-                                  int32_t* __restrict__ ids, float* __restrict__ wout) {
-  pdl_begin();
-  extern __shared__ float s_logits[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
-  if (t >= T) return;
-  float* row = s_logits + warp * E;
-  const float* src = logits + t * E;
-  for (int e = lane; e < E; e += 32) row[e] = src[e];
-  __syncwarp();
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// Lane j < k receives the j-th pick: its expert id and logit.
+template <int PL>
+__device__ __forceinline__ void warp_topk_sorted(const float* __restrict__ src, int E, int k,
+                                                 int lane, float& my_val, int& my_id) {
+  uint32_t key[PL];
+  int id[PL];
+#pragma unroll
+  for (int q = 0; q < PL; ++q) {
+    id[q] = lane + 32 * q;
+    key[q] = id[q] < E ? order_key(__ldg(src + id[q])) : 0u;
+  }
+  // odd-even transposition sort, best first; ids >= E (no expert) sort last
+#pragma unroll
+  for (int rnd = 0; rnd < PL; ++rnd) {
+#pragma unroll
+    for (int q = rnd & 1; q + 1 < PL; q += 2) {
+      const bool vq = id[q] < E, vn = id[q + 1] < E;
+      const bool swap =
+          vn && (!vq || key[q + 1] > key[q] || (key[q + 1] == key[q] && id[q + 1] < id[q]));
+      if (swap) {
+        const uint32_t tk = key[q]; key[q] = key[q + 1]; key[q + 1] = tk;
+        const int ti = id[q]; id[q] = id[q + 1]; id[q + 1] = ti;
+      }
+    }
+  }
+  for (int j = 0; j < k; ++j) {
+    const bool has = id[0] < E;
+    const uint32_t wkey = __reduce_max_sync(0xffffffffu, has ? key[0] : 0u);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, (has && key[0] == wkey) ? ~(uint32_t)id[0] : 0u);
+    const int bi = (int)(~wlo);
+    if (lane == j) { my_val = key_value(wkey); my_id = bi; }
+    if (has && id[0] == bi) {
+#pragma unroll
+      for (int q = 0; q + 1 < PL; ++q) { key[q] = key[q + 1]; id[q] = id[q + 1]; }
+      key[PL - 1] = 0u;
+      id[PL - 1] = E;
+    }
+  }
+}
+
+// Rows of more than 256 experts: `row` is the token's logits in shared memory.
+__device__ __forceinline__ void warp_topk_scan(const float* row, int E, int k, int lane,
+                                               float& my_val, int& my_id) {
   const int per_lane = (E + 31) >> 5;
   uint32_t taken = 0;
-  float my_val = 0.f;
-  int my_id = 0;
   for (int j = 0; j < k; ++j) {
     uint32_t bkey = 0, blo = 0;          // blo = ~e of the lane's candidate (0: none)
     for (int i = 0; i < per_lane; ++i) {
@@ -79,16 +118,48 @@ __global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, i
     const uint32_t wlo = __reduce_max_sync(0xffffffffu, (blo != 0 && bkey == wkey) ? blo : 0u);
     const int bi = (int)(~wlo);
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == j) { my_val = row[bi]; my_id = bi; }
+    if (lane == j) { my_val = key_value(wkey); my_id = bi; }
+  }
+}
+
+// Token t's top k (lane j < k gets pick j) and its softmax weight.  s_row: this
+// warp's E floats of shared memory, used for rows of more than 256 experts.
+__device__ __forceinline__ void warp_route(const float* __restrict__ logits, int64_t t, int E,
+                                           int k, int lane, float* s_row, int& my_id,
+                                           float& my_w) {
+  const float* src = logits + t * E;
+  float my_val = 0.f;
+  my_id = 0;
+  if (E <= 32) warp_topk_sorted<1>(src, E, k, lane, my_val, my_id);
+  else if (E <= 64) warp_topk_sorted<2>(src, E, k, lane, my_val, my_id);
+  else if (E <= 128) warp_topk_sorted<4>(src, E, k, lane, my_val, my_id);
+  else if (E <= 256) warp_topk_sorted<8>(src, E, k, lane, my_val, my_id);
+  else {
+    for (int e = lane; e < E; e += 32) s_row[e] = src[e];
+    __syncwarp();
+    warp_topk_scan(s_row, E, k, lane, my_val, my_id);
   }
   const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
   const float z = lane < k ? expf(my_val - vmax) : 0.f;
   float sum = z;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  my_w = z / sum;
+}
+
+__global__ void route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+                                  int32_t* __restrict__ ids, float* __restrict__ wout) {
+  pdl_begin();
+  extern __shared__ float s_logits[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;
+  int my_id;
+  float my_w;
+  warp_route(logits, t, E, k, lane, s_logits + (E > 256 ? warp * E : 0), my_id, my_w);
   if (lane < k) {
     ids[t * k + lane] = my_id;
-    wout[t * k + lane] = z / sum;
+    wout[t * k + lane] = my_w;
   }
 }
 
@@ -98,7 +169,7 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
   if (T == 0) return cudaSuccess;
   const int warps = 8;
   const int64_t blocks = (T + warps - 1) / warps;
-  const size_t smem = (size_t)warps * E * sizeof(float);
+  const size_t smem = E > 256 ? (size_t)warps * E * sizeof(float) : 0;
   ProfScope ps(K_ROUTE, s);
   if (cudaError_t le_ = launch_pdl(route_topk_kernel, dim3((unsigned)blocks), dim3(warps * 32), smem, s, 1, logits, T, E, k, ids, w); le_ != cudaSuccess) return le_;
   return cudaGetLastError();
@@ -106,7 +177,9 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 
 // ------------------------------------------------------------------ permute
 // Counting sort in two launches.  Pairs are cut into chunks of consecutive pair
-// indices, one block per chunk.  Scratch: hist [n_chunks][E], tot [E], arrive.
+// indices, one block per chunk.  Scratch: hist [n_chunks][E], the expert totals tot
+// (one per 128-byte line, so that the atomics of different experts do not queue on
+// one line), arrive.
 //   1. each block counts its chunk's pairs per expert into hist[c][e] and adds them
 //      to tot[e] (integer atomics: the sums do not depend on their order); the
 //      block that finishes last (an arrival counter decides which) scans tot into
@@ -128,7 +201,7 @@ constexpr int kPermWarps = kPermThreads / 32;
 __device__ void scan_totals(const int32_t* __restrict__ tot, int E, int64_t P,
                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                             int* s_tot, int* s_warp) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = __ldcg(tot + e);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = __ldcg(tot + (int64_t)e * kTotStride);
   __syncthreads();
   // exclusive scan of the totals: each thread owns a run of `per` experts
   const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
@@ -165,11 +238,14 @@ __global__ void __launch_bounds__(kPermThreads)
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = s_hist[e];
     hist[(int64_t)blockIdx.x * E + e] = c;
-    if (c != 0) atomicAdd(&tot[e], c);
+    if (c != 0) atomicAdd(&tot[(int64_t)e * kTotStride], c);
   }
-  __threadfence();
+  // the block's writes are ordered before its arrival by the barrier and one fence
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(arrive, 1) == n_chunks - 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(arrive, 1) == n_chunks - 1;
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -188,48 +264,28 @@ __global__ void __launch_bounds__(256)
                       int32_t* __restrict__ hist, int32_t* __restrict__ tot,
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* arrive) {
   pdl_begin();
-  extern __shared__ float s_logits[];               // [8 warps][E]
+  extern __shared__ float s_logits[];               // [8 warps][E] when E > 256
   __shared__ int s_tot[1024], s_warp[33], s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * 8 + warp;
   if (t < T) {
-    float* row = s_logits + warp * E;
-    const float* src = logits + t * E;
-    for (int e = lane; e < E; e += 32) row[e] = src[e];
-    __syncwarp();
-    const int per_lane = (E + 31) >> 5;
-    uint32_t taken = 0;
-    float my_val = 0.f;
-    int my_id = 0;
-    for (int j = 0; j < k; ++j) {
-      uint32_t bkey = 0, blo = 0;
-      for (int q = 0; q < per_lane; ++q) {
-        const int e = lane + 32 * q;
-        if (e >= E || ((taken >> q) & 1u)) continue;
-        const uint32_t key = order_key(row[e]);
-        if (blo == 0 || key > bkey) { bkey = key; blo = ~(uint32_t)e; }
-      }
-      const uint32_t wkey = __reduce_max_sync(0xffffffffu, blo != 0 ? bkey : 0u);
-      const uint32_t wlo = __reduce_max_sync(0xffffffffu, (blo != 0 && bkey == wkey) ? blo : 0u);
-      const int bi = (int)(~wlo);
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (lane == j) { my_val = row[bi]; my_id = bi; }
-    }
-    const float vmax = __shfl_sync(0xffffffffu, my_val, 0);
-    const float z = lane < k ? expf(my_val - vmax) : 0.f;
-    float sum = z;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    int my_id;
+    float my_w;
+    warp_route(logits, t, E, k, lane, s_logits + (E > 256 ? warp * E : 0), my_id, my_w);
     if (lane < k) {
       ids[t * k + lane] = my_id;
-      wout[t * k + lane] = z / sum;
+      wout[t * k + lane] = my_w;
       atomicAdd(&hist[(t / tpc) * E + my_id], 1);
-      atomicAdd(&tot[my_id], 1);
+      atomicAdd(&tot[(int64_t)my_id * kTotStride], 1);
     }
   }
-  __threadfence();
+  // the block's writes are ordered before its arrival by the barrier and one fence (a
+  // fence in every thread made each wait for its own atomics: most of the launch)
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(arrive, 1) == (int)gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(arrive, 1) == (int)gridDim.x - 1;
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -322,9 +378,9 @@ cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts
   }
   int32_t* hist = scratch;
   int32_t* tot = hist + (size_t)n_chunks * E;
-  int* arrive = tot + E;
+  int* arrive = tot + (size_t)E * kTotStride;
   // every hist entry is written by its block; the totals and the counter start at zero
-  cudaError_t st = cudaMemsetAsync(tot, 0, (size_t)(E + 1) * sizeof(int32_t), s);
+  cudaError_t st = cudaMemsetAsync(tot, 0, ((size_t)E * kTotStride + 1) * sizeof(int32_t), s);
   if (st != cudaSuccess) return st;
   {
     ProfScope ps(K_PERM_HIST, s);
@@ -354,11 +410,11 @@ cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, i
   // the histograms, the totals and the arrival counter after them start at zero
   int32_t* hist = scratch;
   int32_t* tot = hist + (size_t)n_chunks * E;
-  int* arrive = tot + E;
+  int* arrive = tot + (size_t)E * kTotStride;
   cudaError_t st = cudaMemsetAsync(hist, 0, permute_scratch_ints(n_chunks, E) * sizeof(int32_t), s);
   if (st != cudaSuccess) return st;
   {
-    const size_t smem = (size_t)8 * E * sizeof(float);
+    const size_t smem = E > 256 ? (size_t)8 * E * sizeof(float) : 0;
     ProfScope ps(K_ROUTE, s);
     if (cudaError_t le_ = launch_pdl(route_hist_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), smem, s,
                                      1, logits, T, E, k, tpc, ids, w, hist, tot, counts, offsets,
