@@ -13,6 +13,7 @@ cudaError_t launch_gemm_down_bwd(const GemmShape& g, const LayerPtrs& w, const u
                     encode_atoms(&mp.m[1], dys, false, 1, P, m, 128, 2)
               : encode3d(&mp.m[0], w.W_d, E, n, m, 128, 64) && encode2d(&mp.m[1], dys, P, m, m, 128, 64);
   ok = ok && encode_lora(mp, g, false, w.A_d, g.n, T1c) && encode_out(&mp.m[4], dH, g, n, n);
+  ok = ok && encode_act_boxes(mp, dys, P, m, v);
   if (!ok) return cudaErrorInvalidValue;
   mp.m[5] = mp.m[4];
   mp.m[6] = mp.m[4];

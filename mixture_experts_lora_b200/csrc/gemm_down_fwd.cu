@@ -13,6 +13,7 @@ cudaError_t launch_gemm_down_fwd(const GemmShape& g, const LayerPtrs& w, const u
                     encode_atoms(&mp.m[1], H, false, 1, P, n, 128, 2)
               : encode3d(&mp.m[0], w.W_d, E, n, m, 128, 64) && encode2d(&mp.m[1], H, P, n, n, 128, 64);
   ok = ok && encode_lora(mp, g, true, w.B_d, g.m, HAc) && encode_out(&mp.m[4], Yp, g, m, m);
+  ok = ok && encode_act_boxes(mp, H, P, n, v);
   if (!ok) return cudaErrorInvalidValue;
   mp.m[5] = mp.m[4];
   mp.m[6] = mp.m[4];

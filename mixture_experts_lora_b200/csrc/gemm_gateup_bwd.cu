@@ -14,6 +14,7 @@ cudaError_t launch_gemm_gateup_bwd(const GemmShape& g, const LayerPtrs& w, const
               : encode3d(&mp.m[0], w.W_gu, E, m, 2 * n, 128, 64) &&
                     encode2d(&mp.m[1], dGU, P, 2 * n, 2 * n, 128, 64);
   ok = ok && encode_lora(mp, g, false, w.A_gu, g.m, T2c) && encode_out(&mp.m[4], dXp, g, m, m);
+  ok = ok && encode_act_boxes(mp, dGU, P, 2 * n, v);
   if (!ok) return cudaErrorInvalidValue;
   mp.m[5] = mp.m[4];
   mp.m[6] = mp.m[4];

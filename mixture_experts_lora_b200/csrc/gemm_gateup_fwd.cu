@@ -25,6 +25,7 @@ cudaError_t launch_gemm_gateup_fwd(const GemmShape& g, const LayerPtrs& w, const
   ok = ok && encode_lora(mp, g, true, w.B_gu, 2 * g.n, XAc) &&
        encode_out(&mp.m[4], GU, g, n, 2 * n) && encode_out(&mp.m[5], GU + n, g, n, 2 * n) &&
        encode_out(&mp.m[6], H, g, n, n);
+  ok = ok && encode_act_boxes(mp, Xs, P, m, v);
   if (!ok) return cudaErrorInvalidValue;
   GemmParams p{};
   p.chunks = g.gchunks;

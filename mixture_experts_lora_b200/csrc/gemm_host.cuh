@@ -8,11 +8,25 @@
 
 namespace moe {
 
-// Tensor maps of one GEMM launch: weights, token operand, the LoRA block's two
-// operands, and up to three output maps (unused ones repeat a valid map).
+// Tensor maps of one GEMM launch: weights, token operand (boxes of 128 rows), the
+// LoRA block's two operands, up to three output maps (unused ones repeat a valid
+// map), and the token operand in boxes of 32, 64 and 96 rows.
 struct GemmMaps {
-  CUtensorMap m[7];
+  CUtensorMap m[10];
 };
+
+// The token operand's narrower boxes (atom views only; otherwise copies of the
+// 128-row map, which the kernel then does not use).
+inline bool encode_act_boxes(GemmMaps& mp, const uint16_t* act, uint64_t P, uint64_t K, bool v) {
+  for (int i = 0; i < 3; ++i) {
+    if (!v) {
+      mp.m[7 + i] = mp.m[1];
+    } else if (!encode_atoms(&mp.m[7 + i], act, false, 1, P, K, 32u * (i + 1), 2)) {
+      return false;
+    }
+  }
+  return true;
+}
 
 template <class C>
 cudaError_t launch_gemm_cfg(int kind, const GemmShape& g, const GemmMaps& mp, const GemmParams& p,
@@ -25,7 +39,7 @@ cudaError_t launch_gemm_cfg(int kind, const GemmShape& g, const GemmMaps& mp, co
   const int pairs = (int)(tiles < pairs_max ? (tiles > 0 ? tiles : 1) : pairs_max);
   ProfScope ps(kind, s);
   st = launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM_BYTES, s, 2, mp.m[0], mp.m[1],
-                  mp.m[2], mp.m[3], mp.m[4], mp.m[5], mp.m[6], p);
+                  mp.m[2], mp.m[3], mp.m[4], mp.m[5], mp.m[6], mp.m[7], mp.m[8], mp.m[9], p);
   if (st != cudaSuccess) return st;
   return cudaGetLastError();
 }

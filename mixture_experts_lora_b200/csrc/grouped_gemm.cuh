@@ -164,12 +164,23 @@ __device__ __forceinline__ int feat_box(int w, int r, int i, int n) {
   else return w * 256 + r * 128 + i * 64;
 }
 
+// Token rows each CTA of the pair copies per K atom for a chunk whose half (rows per
+// CTA, rounded up to 8) is `half`: with atom views the copy is cut to the chunk in
+// steps of 32 rows (the MMA reads only the chunk's columns), else whole 128-row boxes.
+template <class C>
+__device__ __forceinline__ int act_box_rows(int half) {
+  if constexpr (C::V) return half > 96 ? 128 : (half + 31) & ~31;
+  else return C::NHALF;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmAct,
                     const __grid_constant__ CUtensorMap tmLW, const __grid_constant__ CUtensorMap tmLR,
                     const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmOut2,
-                    const __grid_constant__ CUtensorMap tmOut3, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmOut3, const __grid_constant__ CUtensorMap tmAct32,
+                    const __grid_constant__ CUtensorMap tmAct64, const __grid_constant__ CUtensorMap tmAct96,
+                    const GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -212,6 +223,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmLW);
     tma_prefetch_desc(&tmLR);
+    if constexpr (C::V) {
+      tma_prefetch_desc(&tmAct32);
+      tma_prefetch_desc(&tmAct64);
+      tma_prefetch_desc(&tmAct96);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -257,6 +273,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int nbh = (half + C::BOXR - 1) / C::BOXR;
       const int r0 = ch.row0 + (int)rank * half;
       const uint32_t lbytes = C::LA_BYTES + C::LK_ATOMS * nbh * C::LR_BOX_BYTES;
+      const int brows = act_box_rows<C>(half);
+      const CUtensorMap* tact = brows == 32 ? &tmAct32 : brows == 64 ? &tmAct64
+                              : brows == 96 ? &tmAct96 : &tmAct;
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       if constexpr (C::LSIDE) {
         // LoRA operands of this tile into side buffer it & 1
@@ -278,11 +297,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const uint32_t sa = s_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
           if (ks < p.nk) {
-            // every copy is full-size (rows past the chunk are loaded and ignored,
-            // rows past P and K past the end read as zero)
+            // the token copy covers the CTA's half of the chunk rounded up to its box
+            // (rows past the chunk are loaded and ignored, rows past P and K past the
+            // end read as zero)
             const int k0 = ks * C::BK;
             if (rank == 0)
-              mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + C::B_BYTES));
+              mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * (C::A_BYTES + brows * C::BK * 2));
             if constexpr (C::V) {
               if constexpr (C::EPI == EPI_SWIGLU)
                 tma_load_5d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, 0, ch.e);
@@ -290,7 +310,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tma_load_4d_pair(&tmW, fb, sa, 0, k0, feat_box<C>(w, rank, 0, p.n) / 64, ch.e);
               else
                 tma_load_4d_pair(&tmW, fb, sa, 0, feat_box<C>(w, rank, 0, p.n), k0 / C::KA, ch.e);
-              tma_load_3d_pair(&tmAct, fb, sb, 0, r0, k0 / C::KA);
+              tma_load_3d_pair(tact, fb, sb, 0, r0, k0 / C::KA);
             } else {
               if constexpr (C::A_MN) {
                 tma_load_3d_pair(&tmW, fb, sa, feat_box<C>(w, rank, 0, p.n), k0, ch.e);
@@ -344,6 +364,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const TileInfo ch = p.chunks[c];
         const int ncols = ((ch.row_end - ch.row0) + 15) & ~15;
         const uint32_t idesc = idesc_bf16(256, ncols, C::A_MN ? 1 : 0, 0);
+        const int atom_b = act_box_rows<C>(ncols >> 1) * C::KA * 2;   // bytes between B's K atoms
         const int b = it & 1;
         const bool aok = mbar_wait(smem_u32(&acc_empty[b]), ((it >> 1) & 1) ^ 1, p.err);
         if (!__all_sync(0xffffffffu, aok)) { ok = false; break; }
@@ -378,7 +399,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 // K step kk: MN-major A advances 16 rows of 128 B; K-major operands
                 // advance 32 B inside a K atom, atoms ATOM_* bytes apart
                 const uint32_t ka = (uint32_t)((kk >> 2) * C::ATOM_A + (kk & 3) * 32) >> 4;
-                const uint32_t kb = (uint32_t)((kk >> 2) * C::ATOM_B + (kk & 3) * 32) >> 4;
+                const uint32_t kb = (uint32_t)((kk >> 2) * atom_b + (kk & 3) * 32) >> 4;
                 umma_bf16_pair(d, a_desc0 + so + (C::A_MN ? kk * (2048 / 16) : ka), b_desc0 + so + kb,
                                idesc, (C::LSIDE || (ks | kk)) ? 1u : 0u);
               }
