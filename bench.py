@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=0,
                     help="tokens per oracle sample (0: sized for ~15 s)")
+    ap.add_argument("--plain", action="store_true",
+                    help="run W + K layer steps with host launches and no timing, tracing or "
+                         "JSON line, then exit (a short command for profilers; one GPU)")
     return ap.parse_args()
 
 
@@ -753,10 +756,26 @@ def run_ours(args, cfg):
     print(json.dumps(line), flush=True)
 
 
+def run_plain(args, cfg):
+    """W + K steps of the layer through the public API, nothing else."""
+    import mixture_experts_lora_b200 as ml
+    torch.cuda.set_device(0)
+    inp = generate(cfg, seed=0, device="cuda")
+    buf = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, cfg.r, cfg.scale)
+    for _ in range(args.warmup + args.steps):
+        ml.layer_step(inp, cfg.k, cfg.scale, buf)
+    torch.cuda.synchronize()
+    st = ml.moe_get_device_error()
+    if st != ml.MOE_OK:
+        raise SystemExit(f"device error: {ml.status_string(st)}")
+
+
 def main():
     args = parse_args()
     cfg = CONFIGS[args.config]
-    if args.impl == "reference":
+    if args.plain:
+        run_plain(args, cfg)
+    elif args.impl == "reference":
         run_reference(args, cfg)
     else:
         run_ours(args, cfg)

@@ -16,7 +16,7 @@ cudaError_t launch_rank_cfg(int kind, const GemmShape& g, const CUtensorMap* tm,
   if (st != cudaSuccess) return st;
   ProfScope ps(kind, s);
   st = launch_pdl(kern, dim3(g.max_row_tiles), dim3(C::THREADS), C::SMEM_BYTES, s, 1, tm[0], tm[1],
-                  tm[2], p);
+                  tm[2], tm[3], tm[4], p);
   if (st != cudaSuccess) return st;
   return cudaGetLastError();
 }
@@ -64,10 +64,12 @@ cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* s
                                  uint16_t* rows_out, const uint16_t* L, bool l_mn,
                                  uint16_t* out_save, int ld_save, int r_save, uint16_t* out_c,
                                  cudaStream_t s) {
-  CUtensorMap tm[3];
-  if (!encode_l(&tm[0], g, L, K, l_mn)) return cudaErrorInvalidValue;
-  tm[1] = tm[0];   // rows gathered, no map
-  tm[2] = tm[0];
+  CUtensorMap tm[5];
+  // tm[1]: the sorted rows written out, [P, K] in 128-row x 64-column swizzled boxes
+  if (!encode_l(&tm[0], g, L, K, l_mn) ||
+      !encode2d(&tm[1], rows_out, (uint64_t)g.P, (uint64_t)K, (uint64_t)K, 128, 64))
+    return cudaErrorInvalidValue;
+  tm[2] = tm[3] = tm[4] = tm[0];
   RankParams p = base_params(g, K, out_save, ld_save, r_save, out_c);
   p.src = reinterpret_cast<const __nv_bfloat16*>(src);
   p.sorted_pairs = sorted_pairs;
@@ -81,11 +83,11 @@ cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* s
 cudaError_t launch_rank_sorted(int kind, const GemmShape& g, const uint16_t* rows, int K,
                                const uint16_t* L, bool l_mn, uint16_t* out_save, int ld_save,
                                int r_save, uint16_t* out_c, cudaStream_t s) {
-  CUtensorMap tm[3];
+  CUtensorMap tm[5];
   if (!encode_l(&tm[0], g, L, K, l_mn) ||
       !encode2d(&tm[1], rows, (uint64_t)g.P, (uint64_t)K, (uint64_t)K, 128, 64))
     return cudaErrorInvalidValue;
-  tm[2] = tm[1];
+  tm[2] = tm[3] = tm[4] = tm[1];
   RankParams p = base_params(g, K, out_save, ld_save, r_save, out_c);
   return l_mn ? dispatch_rank<RK_SORTED, true>(kind, g, tm, p, s)
               : dispatch_rank<RK_SORTED, false>(kind, g, tm, p, s);
@@ -94,10 +96,13 @@ cudaError_t launch_rank_sorted(int kind, const GemmShape& g, const uint16_t* row
 cudaError_t launch_rank_dswiglu(const GemmShape& g, const uint16_t* dH, const uint16_t* GU,
                                 const uint16_t* B_gu, uint16_t* dGU, uint16_t* out_save,
                                 int ld_save, int r_save, uint16_t* out_c, cudaStream_t s) {
-  CUtensorMap tm[3];
+  CUtensorMap tm[5];
   const uint64_t P = (uint64_t)g.P, n = (uint64_t)g.n;
+  // tm[3], tm[4]: the dg and du halves of dGU [P, 2n] (each n wide, so a box past n is
+  // clipped at the half's end)
   if (!encode_l(&tm[0], g, B_gu, 2 * g.n, false) || !encode2d(&tm[1], dH, P, n, n, 128, 64) ||
-      !encode2d(&tm[2], GU, P, 2 * n, 2 * n, 128, 64))
+      !encode2d(&tm[2], GU, P, 2 * n, 2 * n, 128, 64) ||
+      !encode2d(&tm[3], dGU, P, n, 2 * n, 128, 64) || !encode2d(&tm[4], dGU + n, P, n, 2 * n, 128, 64))
     return cudaErrorInvalidValue;
   RankParams p = base_params(g, g.n, out_save, ld_save, r_save, out_c);
   p.rows_out = reinterpret_cast<__nv_bfloat16*>(dGU);

@@ -20,13 +20,14 @@
 //   * RK_GATHER: 256 worker threads copy 16-byte pieces of the tile's rows with
 //     cp.async straight into the UMMA K-major 128-byte-swizzled layout, LOOK stages
 //     ahead; once its pieces of a stage have landed a worker scales them (weighted
-//     rows), writes them to the sorted output and arrives; thread 0 also loads each
-//     stage's L chunk with TMA;
+//     rows) and arrives; thread 0 also loads each stage's L chunk with TMA.  The
+//     staged rows go to the sorted output as one TMA tensor store per stage (full
+//     tiles; the workers store a ragged tile's rows themselves);
 //   * RK_SORTED: one thread loads each stage's row tile and L chunk with TMA;
 //   * RK_DSWIGLU: a loader thread brings each stage's dH, g and u tiles and the two
 //     L chunks (gate and up columns) with TMA; the workers compute dg and du in place
-//     in the swizzled tiles, which thereby become the MMA operands, and write them
-//     to dGU;
+//     in the swizzled tiles, which thereby become the MMA operands and go to dGU as
+//     two TMA tensor stores (the workers store a ragged tile's rows themselves);
 //   * the control thread waits for the stage, issues the MMAs
 //     LR[128 x RP] += Rows[128 x 64] L[64 x RP] into TMEM and commits them, which
 //     frees the slot.
@@ -97,7 +98,8 @@ struct RankCfg {
 template <class C>
 __global__ void __launch_bounds__(C::THREADS)
     rank_r_kernel(const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmRows,
-                  const __grid_constant__ CUtensorMap tmGU, const RankParams p) {
+                  const __grid_constant__ CUtensorMap tmGU, const __grid_constant__ CUtensorMap tmOutG,
+                  const __grid_constant__ CUtensorMap tmOutU, const RankParams p) {
   constexpr int RP = C::RP, S = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -119,8 +121,12 @@ __global__ void __launch_bounds__(C::THREADS)
     mbar_init(smem_u32(acc_done), 1);
     mbar_fence_init();
     tma_prefetch_desc(&tmL);
-    if constexpr (C::MODE != RK_GATHER) tma_prefetch_desc(&tmRows);
-    if constexpr (C::MODE == RK_DSWIGLU) tma_prefetch_desc(&tmGU);
+    tma_prefetch_desc(&tmRows);
+    if constexpr (C::MODE == RK_DSWIGLU) {
+      tma_prefetch_desc(&tmGU);
+      tma_prefetch_desc(&tmOutG);
+      tma_prefetch_desc(&tmOutU);
+    }
   }
   if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -137,6 +143,11 @@ __global__ void __launch_bounds__(C::THREADS)
   if (active) ti = p.tiles[tile];
   const int n_it = p.n_it;
   bool ok = true;
+  // RK_GATHER and RK_DSWIGLU: a full tile's stages go out to rows_out as TMA tensor
+  // stores issued by the control thread (the staged tiles are already in the store's
+  // swizzled layout); the rows of a ragged last tile, whose neighbours belong to the
+  // next tile, are stored by the workers
+  const bool tma_rows = C::MODE != RK_SORTED && ti.row_end - ti.row0 == C::BM;
 
   // TMA bytes of stage it into slot it % S: the L chunk(s), plus the row tile(s) in the
   // TMA-fed modes
@@ -238,7 +249,8 @@ __global__ void __launch_bounds__(C::THREADS)
             v = pack8(x);
             *sp = v;
           }
-          if (col < p.K) *reinterpret_cast<uint4*>(p.rows_out + (size_t)qrow[j] * p.K + col) = v;
+          if (!tma_rows && col < p.K)
+            *reinterpret_cast<uint4*>(p.rows_out + (size_t)qrow[j] * p.K + col) = v;
         }
         fence_proxy_async_smem();                 // generic-proxy writes -> tcgen05 reads
         mbar_arrive(smem_u32(&rfull[it % S]));
@@ -278,7 +290,7 @@ __global__ void __launch_bounds__(C::THREADS)
           const uint4 o0 = pack8(dg), o1 = pack8(du);
           *pg = o0;
           *pu = o1;
-          if (in_n) {
+          if (in_n && !tma_rows) {
             *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * n + col) = o0;
             *reinterpret_cast<uint4*>(p.rows_out + (size_t)q * 2 * n + n + col) = o1;
           }
@@ -310,6 +322,16 @@ __global__ void __launch_bounds__(C::THREADS)
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
       const uint32_t sl = sa + C::NT * C::TILE_BYTES;
+      if (tma_rows) {
+        // columns past K (past n in each half of dGU) are clipped by the maps
+        if constexpr (C::MODE == RK_GATHER) {
+          tma_store_2d(&tmRows, sa, it * C::BK, ti.row0);
+        } else if constexpr (C::MODE == RK_DSWIGLU) {
+          tma_store_2d(&tmOutG, sa, it * C::BK, ti.row0);
+          tma_store_2d(&tmOutU, sa + C::TILE_BYTES, it * C::BK, ti.row0);
+        }
+        bulk_commit_group();
+      }
 #pragma unroll
       for (int h = 0; h < C::HALVES; ++h) {
 #pragma unroll
@@ -323,9 +345,12 @@ __global__ void __launch_bounds__(C::THREADS)
           umma_bf16(tmem, ad, bd, idesc, (it | h | kk) ? 1u : 0u);
         }
       }
+      // the slot is refilled once sfree fires: the store must have read it by then
+      if (tma_rows) bulk_wait_read<0>();
       umma_commit(smem_u32(&sfree[s]));
     }
     umma_commit(smem_u32(acc_done));
+    if (tma_rows) bulk_wait<0>();
   }
 
   // ---- epilogue: warps 0-3 read their TMEM lane quarter (row = tile row)
