@@ -162,20 +162,30 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
     if (e_ != cudaSuccess) return MOE_ERR_CUDA;        \
   } while (0)
 
-// Common set-up of the grouped GEMMs: tables and operand pointers.  Adapters are used
-// as given: ranks r .. rp - 1 read as zero through the tensor maps.
+// Common set-up of the grouped GEMMs: operand pointers, and the description of the
+// tables that the first kernel of the call builds from the offsets (tb).  Adapters are
+// used as given: ranks r .. rp - 1 read as zero through the tensor maps.
 moe_status_t prepare(const moe_dims_t& d, const Layout& L, void* ws, const int32_t* offsets,
                      const uint16_t* W_gu, const uint16_t* W_d, const uint16_t* A_gu,
                      const uint16_t* B_gu, const uint16_t* A_d, const uint16_t* B_d,
-                     bool with_chunks, cudaStream_t s, GemmShape* g, LayerPtrs* w) {
+                     bool with_chunks, GemmShape* g, LayerPtrs* w, TableBuild* tb) {
   int* err = status_ptr();
   if (err == nullptr) return MOE_ERR_CUDA;
-  MOE_TRY(launch_build_tables(offsets, d.E, kTileRows, at<TileInfo>(ws, L.tiles),
-                              at<int>(ws, L.n_tiles), kGemmChunkRows, at<TileInfo>(ws, L.gchunks),
-                              at<int>(ws, L.n_gchunks), L.chunk_rows,
-                              with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr,
-                              at<int>(ws, L.n_chunks), at<int32_t>(ws, L.chunk_start),
-                              at<int>(ws, L.counters), with_chunks ? 4 * d.E * L.max_dtiles : 0, s));
+  *tb = TableBuild{};
+  tb->offsets = offsets;
+  tb->E = d.E;
+  tb->tile_rows = kTileRows;
+  tb->tiles = at<TileInfo>(ws, L.tiles);
+  tb->n_tiles = at<int>(ws, L.n_tiles);
+  tb->gchunk_rows = kGemmChunkRows;
+  tb->gchunks = at<TileInfo>(ws, L.gchunks);
+  tb->n_gchunks = at<int>(ws, L.n_gchunks);
+  tb->chunk_rows = L.chunk_rows;
+  tb->chunks = with_chunks ? at<TileInfo>(ws, L.chunks) : nullptr;
+  tb->n_chunks = at<int>(ws, L.n_chunks);
+  tb->chunk_start = at<int32_t>(ws, L.chunk_start);
+  tb->zero = at<int>(ws, L.counters);
+  tb->n_zero = with_chunks ? 4 * d.E * L.max_dtiles : 0;
   w->W_gu = W_gu;
   w->W_d = W_d;
   w->A_gu = A_gu; w->B_gu = B_gu; w->A_d = A_d; w->B_d = B_d;
@@ -241,7 +251,8 @@ moe_status_t backward(
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   GemmShape g;
   LayerPtrs w;
-  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, s, &g, &w);
+  TableBuild tb;
+  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, true, &g, &w, &tb);
   if (st != MOE_OK) return st;
   uint16_t* rows = at<uint16_t>(ws, L.rows);
   uint16_t* dh = at<uint16_t>(ws, L.dh);
@@ -259,9 +270,9 @@ moe_status_t backward(
   const size_t cstride = (size_t)d.E * L.max_dtiles;
   const int rp = L.rp;
   // dy = w dY[t] in expert order (the row buffer), T1 = dy B_d^T (kept for dA_d) and
-  // bf16(c T1)
+  // bf16(c T1); this first kernel also builds the call's tables
   MOE_TRY(launch_rank_gathered(K_RANK_T1, g, dY, d.m, sorted_pairs, d.k, topk_w, rows, w.B_d,
-                               false, t1, rp, rp, lrc1, s));
+                               false, t1, rp, rp, lrc1, &tb, s));
   // dH = dy W_d^T + (c T1) A_d^T
   MOE_TRY(launch_gemm_down_bwd(g, w, rows, lrc1, dh, s));
   // dA_d = c H^T T1 and dB_d = c HA^T dy, one launch
@@ -446,13 +457,15 @@ moe_status_t moe_grouped_gemm_lora_fwd(const moe_dims_t* dims, const moe_bf16_t*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   GemmShape g;
   LayerPtrs w;
-  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, s, &g, &w);
+  TableBuild tb;
+  st = prepare(d, L, ws, offsets, W_gu, W_d, A_gu, B_gu, A_d, B_d, false, &g, &w, &tb);
   if (st != MOE_OK) return st;
   uint16_t* xac = at<uint16_t>(ws, L.lrc1);
   uint16_t* hac = at<uint16_t>(ws, L.lrc2);
-  // X rows in expert order (saved), XA = X A_gu (saved) and bf16(c XA)
+  // X rows in expert order (saved), XA = X A_gu (saved) and bf16(c XA); this first
+  // kernel also builds the call's tables
   MOE_TRY(launch_rank_gathered(K_RANK_XA, g, X, d.m, sorted_pairs, d.k, nullptr, save_Xs, w.A_gu,
-                               true, save_XA, d.r, d.r, xac, s));
+                               true, save_XA, d.r, d.r, xac, &tb, s));
   // GU = X W_gu + (c XA) B_gu and H = silu(g) u, fused
   MOE_TRY(launch_gemm_gateup_fwd(g, w, save_Xs, xac, save_GU, save_H, s));
   // HA = H A_d (saved) and bf16(c HA)

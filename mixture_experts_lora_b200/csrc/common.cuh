@@ -448,4 +448,146 @@ struct TileInfo {
   int pad;
 };
 
+// ---------------------------------------------------------------- block scan
+// Exclusive scan of one value per thread (int or 64-bit) over a block of up to 1024
+// threads; *total_out receives the block total.  s_warp holds 33 values.
+template <class T>
+__device__ __forceinline__ T block_exclusive_scan_1024(T v, T* s_warp, T* total_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const T u = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += u;
+  }
+  __syncthreads();
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const T w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : T(0);
+    T inc2 = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const T u = __shfl_up_sync(0xffffffffu, inc2, off);
+      if (lane >= off) inc2 += u;
+    }
+    s_warp[lane] = inc2 - w;
+    if (lane == 31) s_warp[32] = inc2;
+  }
+  __syncthreads();
+  *total_out = s_warp[32];
+  return incl - v + s_warp[warp];
+}
+
+// ---------------------------------------------------------------- layer tables
+// The tables of one layer call, derived from the permutation's offsets:
+//   tiles    128-row tiles that never straddle two experts (rank-r kernels): every
+//            expert's full tiles in expert order, then the short last tiles in four
+//            size classes from the largest to the smallest (expert order inside a
+//            class), so that a launch of one CTA per tile, dispatched in tile order,
+//            gives the smallest tiles to the CTAs that share an SM with two others;
+//   gchunks  token chunks of the grouped GEMMs: ceil(cnt / gchunk_rows) chunks per
+//            expert of equal size rounded up to 16 rows;
+//   chunks   row chunks of chunk_rows rows for the adapter gradients, with
+//            chunk_start[e] the first chunk of expert e (optional);
+//   zero     arrival counters set to zero (optional).
+struct TableBuild {
+  const int32_t* offsets;   // [E + 1]; nullptr: the tables are built already
+  int E;
+  int tile_rows;
+  TileInfo* tiles;
+  int* n_tiles;
+  int gchunk_rows;
+  TileInfo* gchunks;
+  int* n_gchunks;
+  int chunk_rows;
+  TileInfo* chunks;         // nullptr: no gradient chunks
+  int* n_chunks;
+  int32_t* chunk_start;     // [E + 1]
+  int* zero;
+  int n_zero;
+};
+
+// Run by every thread of every CTA of the first kernel of a call (a grid of at least
+// E CTAs): each CTA finds its own tile b among the tiles and writes it, CTA e writes
+// expert e's token and gradient chunks, CTA 0 the counts, and each CTA a slice of the
+// zeroed counters.  Returns the number of tiles; *my receives tile b (unchanged when
+// b is past the last tile).
+static __device__ int build_tables_cta(const TableBuild& tb, int b, int nb, TileInfo* my, int* s_warp,
+                                unsigned long long* s_warp64, TileInfo* s_tile) {
+  const int E = tb.E, R = tb.tile_rows;
+  const int per = (E + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
+  int my_full = 0, my_ng = 0, my_nc = 0;
+  unsigned long long my_cls = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int cnt = tb.offsets[e + 1] - tb.offsets[e];
+    const int rag = cnt % R;
+    my_full += cnt / R;
+    if (rag > 0) my_cls += 1ull << (16 * (3 - (rag * 4) / R));
+    my_ng += (cnt + tb.gchunk_rows - 1) / tb.gchunk_rows;
+    if (tb.chunks != nullptr) my_nc += (cnt + tb.chunk_rows - 1) / tb.chunk_rows;
+  }
+  int total_full, gtotal, ctotal = 0;
+  unsigned long long ctot;
+  int f = block_exclusive_scan_1024(my_full, s_warp, &total_full);
+  unsigned long long cr = block_exclusive_scan_1024(my_cls, s_warp64, &ctot);
+  int g = block_exclusive_scan_1024(my_ng, s_warp, &gtotal);
+  int cc = tb.chunks != nullptr ? block_exclusive_scan_1024(my_nc, s_warp, &ctotal) : 0;
+  int cbase[4];
+  int n_tiles = total_full;
+  for (int c = 0; c < 4; ++c) {
+    cbase[c] = n_tiles;
+    n_tiles += (int)((ctot >> (16 * c)) & 0xffffu);
+  }
+  if (threadIdx.x == 0) s_tile->e = -1;
+  __syncthreads();
+  for (int e = e0; e < e1; ++e) {
+    const int lo = tb.offsets[e], hi = tb.offsets[e + 1], cnt = hi - lo;
+    const int nf = cnt / R, rag = cnt - nf * R;
+    if (b >= f && b < f + nf) *s_tile = TileInfo{e, lo + (b - f) * R, lo + (b - f + 1) * R, 0};
+    f += nf;
+    if (rag > 0) {
+      const int c = 3 - (rag * 4) / R;
+      if (cbase[c] + (int)((cr >> (16 * c)) & 0xffffu) == b) *s_tile = TileInfo{e, lo + nf * R, hi, 0};
+      cr += 1ull << (16 * c);
+    }
+    const int ng = (cnt + tb.gchunk_rows - 1) / tb.gchunk_rows;
+    if (e == b) {
+      const int sz = ng > 0 ? (((cnt + ng - 1) / ng + 15) & ~15) : 0;
+      for (int i = 0; i < ng; ++i)
+        tb.gchunks[g + i] = TileInfo{e, lo + i * sz, min(hi, lo + (i + 1) * sz), 0};
+    }
+    g += ng;
+    if (tb.chunks != nullptr) {
+      const int nc = (cnt + tb.chunk_rows - 1) / tb.chunk_rows;
+      if (e == b) {
+        for (int i = 0; i < nc; ++i)
+          tb.chunks[cc + i] = TileInfo{e, lo + i * tb.chunk_rows, min(hi, lo + (i + 1) * tb.chunk_rows), 0};
+        tb.chunk_start[e] = cc;
+      }
+      cc += nc;
+    }
+  }
+  if (b == 0 && threadIdx.x == 0) {
+    *tb.n_tiles = n_tiles;
+    *tb.n_gchunks = gtotal;
+    if (tb.chunks != nullptr) {
+      *tb.n_chunks = ctotal;
+      tb.chunk_start[E] = ctotal;
+    }
+  }
+  if (tb.n_zero > 0) {
+    const int zper = (tb.n_zero + nb - 1) / nb;
+    for (int i = b * zper + (int)threadIdx.x; i < min(tb.n_zero, (b + 1) * zper); i += blockDim.x)
+      tb.zero[i] = 0;
+  }
+  __syncthreads();
+  if (s_tile->e >= 0) {
+    *my = *s_tile;
+    if (threadIdx.x == 0) tb.tiles[b] = *s_tile;
+  }
+  return n_tiles;
+}
+
 }  // namespace moe

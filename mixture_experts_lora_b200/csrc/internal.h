@@ -10,6 +10,7 @@
 namespace moe {
 
 struct TileInfo;
+struct TableBuild;
 
 // Launch with programmatic stream serialization (the kernel calls pdl_begin() before
 // touching global memory; see common.cuh), plus an optional cluster size.
@@ -40,7 +41,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // ---- kernel timing (profile.cu): while enabled, each launch is bracketed by
 // CUDA events on its stream and attributed to one of these kinds.
 enum KernelKind : int {
-  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCATTER, K_TABLES,
+  K_ROUTE = 0, K_PERM_HIST, K_PERM_SCATTER,
   K_GEMM_GATEUP_FWD, K_GEMM_DOWN_FWD, K_GEMM_DOWN_BWD, K_GEMM_GATEUP_BWD, K_WGRAD,
   K_COMBINE, K_MEMSET, K_RANK_XA, K_RANK_HA, K_RANK_T1, K_RANK_T2,
   K_ROUTER_BWD, K_GEMM_DW_GU, K_GEMM_DW_D, K_NUM_KINDS
@@ -86,16 +87,6 @@ int route_tokens_per_chunk(int k);
 cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
                                  float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                                  int32_t* pair_pos, int32_t* scratch, cudaStream_t s);
-// From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
-// experts (row kernels), token chunks of at most `gchunk_rows` rows split
-// evenly inside each expert (grouped GEMMs; all but the last chunk of an expert
-// are multiples of 16), and row chunks of `chunk_rows` rows (adapter gradients)
-// with chunk_start[e] = first chunk of expert e.
-cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
-                                int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
-                                int chunk_rows, TileInfo* chunks, int* n_chunks,
-                                int32_t* chunk_start, int* zero, int n_zero,
-                                cudaStream_t s);
 // dlogits [T, E] fp32 = router backward (see simt_kernels.cu); m % 8 == 0
 cudaError_t launch_router_backward(const uint16_t* dY, const uint16_t* ys, const int32_t* ids,
                                    const float* w, const int32_t* pos, int64_t T, int k, int E,
@@ -155,7 +146,7 @@ cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* s
                                  const int32_t* sorted_pairs, int k, const float* w,
                                  uint16_t* rows_out, const uint16_t* L, bool l_mn,
                                  uint16_t* out_save, int ld_save, int r_save, uint16_t* out_c,
-                                 cudaStream_t s);
+                                 const TableBuild* tb, cudaStream_t s);
 // Sorted rows [P, K].
 cudaError_t launch_rank_sorted(int kind, const GemmShape& g, const uint16_t* rows, int K,
                                const uint16_t* L, bool l_mn, uint16_t* out_save, int ld_save,

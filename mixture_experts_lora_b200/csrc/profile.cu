@@ -15,7 +15,7 @@
 namespace moe {
 
 const char* const kKernelNames[K_NUM_KINDS] = {
-    "route_topk",        "permute_hist",      "permute_scatter",  "build_tables",
+    "route_topk",        "permute_hist",      "permute_scatter",
     "gemm_gateup_fwd",   "gemm_down_fwd",     "gemm_down_bwd",
     "gemm_gateup_bwd",   "lora_wgrad",        "unpermute_combine", "memset",
     "rank_xa",           "rank_ha",           "rank_t1",          "rank_t2",

@@ -63,7 +63,7 @@ cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* s
                                  const int32_t* sorted_pairs, int k, const float* w,
                                  uint16_t* rows_out, const uint16_t* L, bool l_mn,
                                  uint16_t* out_save, int ld_save, int r_save, uint16_t* out_c,
-                                 cudaStream_t s) {
+                                 const TableBuild* tb, cudaStream_t s) {
   CUtensorMap tm[5];
   // tm[1]: the sorted rows written out, [P, K] in 128-row x 64-column swizzled boxes
   if (!encode_l(&tm[0], g, L, K, l_mn) ||
@@ -76,6 +76,7 @@ cudaError_t launch_rank_gathered(int kind, const GemmShape& g, const uint16_t* s
   p.k = k;
   p.w = w;
   p.rows_out = reinterpret_cast<__nv_bfloat16*>(rows_out);
+  if (tb != nullptr) p.tb = *tb;
   return l_mn ? dispatch_rank<RK_GATHER, true>(kind, g, tm, p, s)
               : dispatch_rank<RK_GATHER, false>(kind, g, tm, p, s);
 }

@@ -57,6 +57,8 @@ struct RankParams {
   __nv_bfloat16* out_c;         // [P, RP]
   float scale;
   int* err;
+  TableBuild tb;                // RK_GATHER: tb.offsets set when this launch builds the
+                                // call's tables (then its own tile comes from them)
 };
 
 template <int RP_, int MODE_, bool L_MN_>
@@ -136,11 +138,19 @@ __global__ void __launch_bounds__(C::THREADS)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_begin();          // predecessors' outputs (tile table, rows) visible from here
+  pdl_begin();          // predecessors' outputs (offsets, tile table, rows) visible from here
   const int tile = blockIdx.x;
-  const bool active = tile < *p.n_tiles;
+  bool active;
   TileInfo ti{};
-  if (active) ti = p.tiles[tile];
+  if (C::MODE == RK_GATHER && p.tb.offsets != nullptr) {
+    __shared__ int s_scan[33];
+    __shared__ unsigned long long s_scan64[33];
+    __shared__ TileInfo s_tile;
+    active = tile < build_tables_cta(p.tb, tile, (int)gridDim.x, &ti, s_scan, s_scan64, &s_tile);
+  } else {
+    active = tile < *p.n_tiles;
+    if (active) ti = p.tiles[tile];
+  }
   const int n_it = p.n_it;
   bool ok = true;
   // RK_GATHER and RK_DSWIGLU: a full tile's stages go out to rows_out as TMA tensor

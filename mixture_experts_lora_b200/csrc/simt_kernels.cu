@@ -7,37 +7,6 @@
 
 namespace moe {
 
-// ------------------------------------------------------------------ block scan
-// Exclusive scan of one value per thread (int or 64-bit) over a block of up to 1024
-// threads; *total_out receives the block total.  s_warp holds 33 values.
-template <class T>
-__device__ __forceinline__ T block_exclusive_scan_1024(T v, T* s_warp, T* total_out) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  T incl = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const T u = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += u;
-  }
-  __syncthreads();
-  if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const T w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : T(0);
-    T inc2 = w;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const T u = __shfl_up_sync(0xffffffffu, inc2, off);
-      if (lane >= off) inc2 += u;
-    }
-    s_warp[lane] = inc2 - w;
-    if (lane == 31) s_warp[32] = inc2;
-  }
-  __syncthreads();
-  *total_out = s_warp[32];
-  return incl - v + s_warp[warp];
-}
-
 // ------------------------------------------------------------------ routing
 // One warp per token.  The k rounds each pick the largest remaining logit, lower
 // expert id on ties, and the weights are a softmax over the k picked logits.  Router
@@ -425,98 +394,6 @@ cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, i
     if (st != cudaSuccess) return st;
   }
   return launch_scatter(ids, P, E, n_chunks, tpc * k, hist, offsets, sorted_pairs, pair_pos, s);
-}
-
-// ------------------------------------------------------------------ tile tables
-// From offsets[E+1]: row tiles of `tile_rows` rows that never straddle two
-// experts (row kernels), token chunks of at most `gchunk_rows` rows (grouped
-// GEMMs), and row chunks of `chunk_rows` rows (adapter
-// gradients) with chunk_start[e] = first chunk of expert e.
-__global__ void build_tables_kernel(const int32_t* __restrict__ offsets, int E, int tile_rows,
-                                    TileInfo* __restrict__ tiles, int* __restrict__ n_tiles,
-                                    int gchunk_rows, TileInfo* __restrict__ gchunks,
-                                    int* __restrict__ n_gchunks, int chunk_rows,
-                                    TileInfo* __restrict__ chunks, int* __restrict__ n_chunks,
-                                    int32_t* __restrict__ chunk_start, int* __restrict__ zero,
-                                    int n_zero) {
-  pdl_begin();
-  for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
-  __shared__ int s_warp[33];
-  __shared__ unsigned long long s_warp64[33];
-  const int e = threadIdx.x;
-  int lo = 0, hi = 0;
-  if (e < E) { lo = offsets[e]; hi = offsets[e + 1]; }
-  const int cnt = hi - lo;
-  int total;
-  // row tiles of tile_rows rows: every expert's full tiles in expert order, then its
-  // short last tile in four size classes from the largest to the smallest (expert
-  // order inside a class).  A launch of one CTA per tile is dispatched in tile
-  // order, breadth-first over the SMs, so the smallest tiles become the CTAs that
-  // share an SM with two others.
-  const int nfull = cnt / tile_rows, rag = cnt - nfull * tile_rows;
-  const int f0 = block_exclusive_scan_1024(nfull, s_warp, &total);
-  for (int i = 0; i < nfull; ++i) {
-    TileInfo ti;
-    ti.e = e; ti.row0 = lo + i * tile_rows; ti.row_end = lo + (i + 1) * tile_rows; ti.pad = 0;
-    tiles[f0 + i] = ti;
-  }
-  {
-    // one scan of the four class flags packed 16 bits apart (E <= 1024 per class)
-    const int cls = rag > 0 ? 3 - (rag * 4) / tile_rows : -1;   // 0: largest class
-    unsigned long long ctot;
-    const unsigned long long r = block_exclusive_scan_1024(
-        cls >= 0 ? 1ull << (16 * cls) : 0ull, s_warp64, &ctot);
-    int base = total;
-    for (int c = 0; c < 4; ++c) {
-      if (c == cls) {
-        TileInfo ti;
-        ti.e = e; ti.row0 = lo + nfull * tile_rows; ti.row_end = hi; ti.pad = 0;
-        tiles[base + (int)((r >> (16 * c)) & 0xffffu)] = ti;
-      }
-      base += (int)((ctot >> (16 * c)) & 0xffffu);
-    }
-    total = base;
-  }
-  if (threadIdx.x == 0) *n_tiles = total;
-  // token chunks: ceil(cnt / gchunk_rows) chunks of equal size rounded up to 16
-  if (gchunks != nullptr) {
-    const int ng = (cnt + gchunk_rows - 1) / gchunk_rows;
-    int gtotal;
-    const int g0 = block_exclusive_scan_1024(ng, s_warp, &gtotal);
-    const int sz = ng > 0 ? (((cnt + ng - 1) / ng + 15) & ~15) : 0;
-    for (int i = 0; i < ng; ++i) {
-      TileInfo ti;
-      ti.e = e; ti.row0 = lo + i * sz; ti.row_end = min(hi, lo + (i + 1) * sz); ti.pad = 0;
-      gchunks[g0 + i] = ti;
-    }
-    if (threadIdx.x == 0) *n_gchunks = gtotal;
-  }
-  if (chunks != nullptr) {
-    const int nc = (cnt + chunk_rows - 1) / chunk_rows;
-    int ctotal;
-    const int c0 = block_exclusive_scan_1024(nc, s_warp, &ctotal);
-    for (int i = 0; i < nc; ++i) {
-      TileInfo ti;
-      ti.e = e;
-      ti.row0 = lo + i * chunk_rows;
-      ti.row_end = min(hi, lo + (i + 1) * chunk_rows);
-      ti.pad = 0;
-      chunks[c0 + i] = ti;
-    }
-    if (e < E) chunk_start[e] = c0;
-    if (threadIdx.x == 0) { *n_chunks = ctotal; chunk_start[E] = ctotal; }
-  }
-}
-
-cudaError_t launch_build_tables(const int32_t* offsets, int E, int tile_rows, TileInfo* tiles,
-                                int* n_tiles, int gchunk_rows, TileInfo* gchunks, int* n_gchunks,
-                                int chunk_rows, TileInfo* chunks, int* n_chunks,
-                                int32_t* chunk_start, int* zero, int n_zero, cudaStream_t s) {
-  ProfScope ps(K_TABLES, s);
-  if (cudaError_t le_ = launch_pdl(build_tables_kernel, dim3(1), dim3(1024), 0, s, 1, offsets, E, tile_rows, tiles, n_tiles, gchunk_rows, gchunks,
-                                         n_gchunks, chunk_rows, chunks, n_chunks, chunk_start,
-                                         zero, n_zero); le_ != cudaSuccess) return le_;
-  return cudaGetLastError();
 }
 
 static int g_num_sms_cache = 0;

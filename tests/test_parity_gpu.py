@@ -277,6 +277,24 @@ def test_expert_spanning_several_chunks():
     assert buf.counts.cpu().tolist()[0] == 1500
 
 
+@pytest.mark.parametrize("r", [16, 32, 64])
+def test_multi_chunk_experts_at_every_rank_width(r):
+    # Experts of more than 256 rows are cut into several balanced token chunks of the
+    # grouped GEMMs: 257 rows (the smallest cut), 300, 513 (three chunks), 600, next to
+    # an expert of one chunk and an empty one.  Rank 16 keeps the GEMMs' LoRA block in
+    # its side buffer; ranks 32 and 64 take a ring stage per tile.
+    counts = [600, 257, 513, 100, 0, 300]
+    cfg = small_config(T=sum(counts), m=128, n=64, E=len(counts), k=1, r=r, alpha=r)
+    owner = np.repeat(np.arange(len(counts)), counts)
+    owner = owner[np.random.default_rng(5).permutation(len(owner))]
+
+    def mutate(cpu):
+        cpu["logits"][torch.arange(cfg.T), torch.from_numpy(owner)] += 30.0
+    errs, buf = _layer_case(cfg, mutate)
+    assert buf.counts.cpu().tolist() == counts
+    print(r, errs)
+
+
 def test_graph_replay_matches_eager_bitwise():
     # bench.py times CUDA-graph replays of the step (every kernel launched with
     # programmatic dependent launch): a replay must give the eager results bit for bit
