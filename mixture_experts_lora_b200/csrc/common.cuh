@@ -69,10 +69,6 @@ __device__ __forceinline__ void unpack8(uint4 v, float (&x)[8]) {
   x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z);
   x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
 }
-// Round an fp32 value to bf16 and back (round to nearest even).
-__device__ __forceinline__ float round_bf16(float x) {
-  return __bfloat162float(__float2bfloat16_rn(x));
-}
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -108,30 +104,6 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, int
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0 && globaltimer_ns() - t0 > limit_ns) {
-      report_error(err, MOE_ERR_TIMEOUT);
-      return false;
-    }
-  }
-}
-// try_wait with acquire at cluster scope: pairs with arrivals released at cluster
-// scope by the other CTA of a pair (its threads' shared-memory writes become visible).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, int* err) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 31u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
       report_error(err, MOE_ERR_TIMEOUT);
       return false;
     }
@@ -181,11 +153,6 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-// One arrival on `bar` once every prior cp.async of this thread has landed
-// (counted in the barrier's expected arrivals).
-__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -362,10 +329,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t cta_mask
       " [%0], %1;" ::"r"(bar),
       "h"(cta_mask)
       : "memory");
-}
-__device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
 }
 
 // ---------------------------------------------------------------- TMA stores
