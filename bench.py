@@ -569,6 +569,27 @@ def run_ours(args, cfg):
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
 
+    # the same step at LoRA rank 64, the rank the pages work their numbers at
+    # (adapters drawn with the same distributions; alpha = r, so c = 1)
+    if cfg.r != 64:
+        g64 = torch.Generator(device=dev).manual_seed(7)
+        r64 = dict(inp)
+        for name, shape, std in (("A_gu", (cfg.E, cfg.m, 64), cfg.m ** -0.5),
+                                 ("B_gu", (cfg.E, 64, 2 * cfg.n), 0.02),
+                                 ("A_d", (cfg.E, cfg.n, 64), cfg.n ** -0.5),
+                                 ("B_d", (cfg.E, 64, cfg.m), 0.02)):
+            r64[name] = (torch.randn(shape, generator=g64, device=dev) * std).to(torch.bfloat16)
+        b64 = ml.alloc_buffers(cfg.T, cfg.m, cfg.n, cfg.E, cfg.k, 64, 1.0, device=dev)
+        r64_ms = extra_ms(lambda: ml.layer_step(r64, cfg.k, 1.0, b64), min(args.steps, 50))
+        if ml.moe_get_device_error() != ml.MOE_OK:
+            raise SystemExit("device error in the rank-64 timing")
+        r64_flops = acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, 64)
+        extras["rank_64"] = {
+            "what": "the step at LoRA rank 64 (alpha 64) on the same workload",
+            "ms_per_step": r64_ms, "tokens_per_s": world * cfg.T / (r64_ms / 1e3),
+            "tflops": r64_flops / (r64_ms / 1e3) / 1e12}
+        del b64, r64
+
     # full fine-tuning (NEXT-3): forward, then the backward with the expert-weight
     # gradients dW_gu, dW_d and no adapter gradients
     dWg = torch.empty(cfg.E, cfg.m, 2 * cfg.n, dtype=torch.bfloat16, device=dev)
