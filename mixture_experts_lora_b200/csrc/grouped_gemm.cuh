@@ -371,21 +371,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
         const uint32_t d = tmem + b * C::NMAX;
         if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-        if constexpr (C::LSIDE) {
-          // the LoRA block first (it starts the accumulation), from side buffer it & 1
-          const int lb = it & 1;
-          const bool lok = mbar_wait(smem_u32(&lfull[lb]), (it >> 1) & 1, p.err);
-          if (!__all_sync(0xffffffffu, lok)) { ok = false; break; }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
-            const uint64_t la0 = C::A_MN ? smem_desc(la, C::LA_BOX_BYTES, 1024, kSw128)
-                                         : smem_desc(la, 16, C::LK_SBO, C::LK_SW);
-            lora_mmas(d, la0, smem_desc(la + C::LA_BYTES, 16, C::LK_SBO, C::LK_SW), idesc, true);
-            umma_commit_pair(smem_u32(&lempty[lb]), 0x3);
-          }
-          __syncwarp();
-        }
         for (int ks = 0; ks < p.nk + NST; ++ks) {
           const bool fok = mbar_wait(smem_u32(&full[stage]), phase, p.err);
           if (!__all_sync(0xffffffffu, fok)) { ok = false; break; }
@@ -401,7 +386,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const uint32_t ka = (uint32_t)((kk >> 2) * C::ATOM_A + (kk & 3) * 32) >> 4;
                 const uint32_t kb = (uint32_t)((kk >> 2) * atom_b + (kk & 3) * 32) >> 4;
                 umma_bf16_pair(d, a_desc0 + so + (C::A_MN ? kk * (2048 / 16) : ka), b_desc0 + so + kb,
-                               idesc, (C::LSIDE || (ks | kk)) ? 1u : 0u);
+                               idesc, (ks | kk) ? 1u : 0u);
               }
             } else {
               lora_mmas(d, la_desc0 + so, lr_desc0 + so, idesc, false);
@@ -413,6 +398,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
+        if constexpr (C::LSIDE) {
+          // the LoRA block last, from side buffer it & 1 (loaded when the tile's copies
+          // began, so the tile starts on K stages already in the ring)
+          const int lb = it & 1;
+          const bool lok = mbar_wait(smem_u32(&lfull[lb]), (it >> 1) & 1, p.err);
+          if (!__all_sync(0xffffffffu, lok)) { ok = false; break; }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t la = s_base + side_off + lb * C::LS_BYTES;
+            const uint64_t la0 = C::A_MN ? smem_desc(la, C::LA_BOX_BYTES, 1024, kSw128)
+                                         : smem_desc(la, 16, C::LK_SBO, C::LK_SW);
+            lora_mmas(d, la0, smem_desc(la + C::LA_BYTES, 16, C::LK_SBO, C::LK_SW), idesc, false);
+            umma_commit_pair(smem_u32(&lempty[lb]), 0x3);
+          }
+          __syncwarp();
+        }
         if (lane == 0) umma_commit_pair(smem_u32(&acc_full[b]), 0x3);
         __syncwarp();
       }
