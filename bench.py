@@ -569,6 +569,18 @@ def run_ours(args, cfg):
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
 
+    # routing and the counting sort alone (moe_route_permute: two launches, logits to
+    # sorted pairs), one event pair around the call: the per-kernel table's event nodes
+    # around each of its two small launches add several us to each
+    rp_ms = extra_ms(lambda: ml.moe_route_permute(inp["logits"], cfg.k, buf.ids, buf.w, buf.counts,
+                                                  buf.offsets, buf.sorted_pairs, buf.pair_pos, buf.ws),
+                     min(args.steps, 50))
+    if ml.moe_get_device_error() != ml.MOE_OK:
+        raise SystemExit("device error in the routing timing")
+    extras["route_permute"] = {
+        "what": "routing and the counting-sort permutation (2 launches) timed as one call",
+        "ms_per_call": rp_ms}
+
     # the same step at LoRA rank 64, the rank the pages work their numbers at
     # (adapters drawn with the same distributions; alpha = r, so c = 1)
     if cfg.r != 64:
