@@ -164,7 +164,9 @@ def kernel_work(cfg, active_experts=None):
         # two launches: (H, w dY) -> dA_d, dB_d; (dGU, X) -> dB_gu, dA_gu
         "lora_wgrad": {"byte": P * n * 2 + rows + lrc + P * r * 2 + E * r * (n + m) * 2
                                + P * 2 * n * 2 + rows + P * r * 2 + lrc + E * r * (m + 2 * n) * 2},
-        "route_topk": {"byte": acc.bytes_route(T, E, k)},
+        # routing with the whole counting sort (one launch): logits read, ids and
+        # weights written, ids read back, sorted_pairs and pair_pos written
+        "route_topk": {"byte": acc.bytes_route(T, E, k) + P * 12},
         "unpermute_combine": {"byte": 2 * acc.bytes_combine(T, m, k)},  # Y and dX
         # full fine-tuning only: the expert-weight gradients (sorted operands read once,
         # every expert's gradient written once)
@@ -569,17 +571,28 @@ def run_ours(args, cfg):
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
 
-    # routing and the counting sort alone (moe_route_permute: two launches, logits to
-    # sorted pairs), one event pair around the call: the per-kernel table's event nodes
-    # around each of its two small launches add several us to each
-    rp_ms = extra_ms(lambda: ml.moe_route_permute(inp["logits"], cfg.k, buf.ids, buf.w, buf.counts,
-                                                  buf.offsets, buf.sorted_pairs, buf.pair_pos, buf.ws),
-                     min(args.steps, 50))
+    # routing and the counting sort alone (moe_route_permute: a memset and one cooperative
+    # launch, logits to sorted pairs), one event pair around the call; the per-kernel
+    # table's event nodes around the launch add several us.  A single replayed call also
+    # carries the graph's launch latency, so the call is timed a second way too: a graph
+    # of 20 calls back to back, divided by 20 (logits, 2 MB at this shape, stay in L2
+    # between those calls, as they do after the router GEMM that writes them)
+    def route_call():
+        ml.moe_route_permute(inp["logits"], cfg.k, buf.ids, buf.w, buf.counts, buf.offsets,
+                             buf.sorted_pairs, buf.pair_pos, buf.ws)
+
+    def route_20():
+        for _ in range(20):
+            route_call()
+
+    rp_ms = extra_ms(route_call, min(args.steps, 50))
+    rp20_ms = extra_ms(route_20, min(args.steps, 20)) / 20
     if ml.moe_get_device_error() != ml.MOE_OK:
         raise SystemExit("device error in the routing timing")
     extras["route_permute"] = {
-        "what": "routing and the counting-sort permutation (2 launches) timed as one call",
-        "ms_per_call": rp_ms}
+        "what": "routing and the counting-sort permutation (a memset and one cooperative "
+                "launch) timed as one call, and per call in a graph of 20 calls",
+        "ms_per_call": rp_ms, "ms_per_call_in_sequence": rp20_ms}
 
     # the same step at LoRA rank 64, the rank the pages work their numbers at
     # (adapters drawn with the same distributions; alpha = r, so c = 1)

@@ -118,9 +118,10 @@ moe_status_t moe_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t 
                          int32_t* pair_pos, void* ws, size_t ws_bytes, void* stream);
 
 /* moe_route_topk() and moe_permute() in one call, for the common case where the
- * permutation follows the routing directly: the routing kernel also counts each
- * block's pairs per expert, so routing and the counting sort take two launches
- * instead of three.  Same definitions and outputs as the two calls (stable order,
+ * permutation follows the routing directly: one cooperative kernel routes the tokens,
+ * counts their pairs per expert, and after a grid barrier (its wait bounded) scans the
+ * counts and scatters the pairs; a memset of the scratch comes first.  Same definitions
+ * and outputs as the two calls (stable order,
  * ties to the lower expert index).
  * ws, ws_bytes: scratch of at least (ceil(T / floor(512 / k)) * E + 32 * E + 1) int32
  * (per-chunk histograms of whole-token chunks, expert totals, one counter);

@@ -149,7 +149,7 @@ def moe_permute(topk_ids, E, counts, offsets, sorted_pairs, pair_pos, ws, stream
 
 def moe_route_permute(logits, k, topk_ids, topk_w, counts, offsets, sorted_pairs, pair_pos, ws,
                       stream=None):
-    """moe_route_topk and moe_permute in one call (two launches)."""
+    """moe_route_topk and moe_permute in one call (one cooperative launch)."""
     T, E = logits.shape
     _check("moe_route_permute", lib().moe_route_permute(
         _ptr(logits), T, E, int(k), _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(offsets),

@@ -80,9 +80,9 @@ inline size_t permute_scratch_ints(int64_t n_chunks, int E) {
 cudaError_t launch_permute(const int32_t* ids, int64_t P, int E, int32_t* counts,
                            int32_t* offsets, int32_t* sorted_pairs, int32_t* pair_pos,
                            int32_t* scratch, int* err, cudaStream_t s);
-// Routing fused with the permutation's histogram: chunks of route_tokens_per_chunk(k)
-// tokens (their k pairs each); scratch holds
-// permute_scratch_ints(ceil(T / route_tokens_per_chunk(k)), E) ints.
+// Routing and the counting sort in one cooperative launch (after a memset of the
+// scratch): chunks of route_tokens_per_chunk(k) tokens (their k pairs each); scratch
+// holds permute_scratch_ints(ceil(T / route_tokens_per_chunk(k)), E) ints.
 int route_tokens_per_chunk(int k);
 cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, int32_t* ids,
                                  float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,

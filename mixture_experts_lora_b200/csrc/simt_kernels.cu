@@ -144,6 +144,17 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
   return cudaGetLastError();
 }
 
+static int g_num_sms_cache = 0;
+static int num_sms() {
+  if (g_num_sms_cache == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms_cache, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms_cache <= 0) g_num_sms_cache = 148;
+  }
+  return g_num_sms_cache;
+}
+
 // ------------------------------------------------------------------ permute
 // Counting sort in two launches.  Pairs are cut into chunks of consecutive pair
 // indices, one block per chunk.  Scratch: hist [n_chunks][E], the expert totals tot
@@ -158,8 +169,9 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 //      (rank = earlier lanes of the group), a shared [warp][expert] table prefix-
 //      summed over the warps orders the warps; positions are therefore stable
 //      (ascending pair index inside every segment).
-// Routing can fill launch 1 as well: in moe_route_permute each routing warp counts
-// its token's pairs.
+// moe_route_permute does routing and all of this in one cooperative launch
+// (route_permute_kernel below): its routing warps fill the histogram, grid barriers
+// separate the three phases.
 // Replaces the per-expert mask lookup of the loop form ("What is
 // torch._grouped_mm?", Unsloth faster-moe docs).
 constexpr int kPermThreads = kPermuteChunk;
@@ -167,9 +179,11 @@ constexpr int kPermWarps = kPermThreads / 32;
 
 // Run by every thread of the last block of a histogram launch (any block size that is
 // a multiple of 32, at most 1024): counts and offsets from the expert totals.
+// The expert totals tot[e * kTotStride] scanned into counts and offsets (written when
+// write_out) by one block; on return s_tot[e] holds offsets[e] for every e < E.
 __device__ void scan_totals(const int32_t* __restrict__ tot, int E, int64_t P,
                             int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                            int* s_tot, int* s_warp) {
+                            int* s_tot, int* s_warp, bool write_out = true) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = __ldcg(tot + (int64_t)e * kTotStride);
   __syncthreads();
   // exclusive scan of the totals: each thread owns a run of `per` experts
@@ -181,11 +195,15 @@ __device__ void scan_totals(const int32_t* __restrict__ tot, int E, int64_t P,
   int run = block_exclusive_scan_1024(mine, s_warp, &all);
   for (int e = e0; e < e0 + per && e < E; ++e) {
     const int t = s_tot[e];
-    counts[e] = t;
-    offsets[e] = run;
+    s_tot[e] = run;                   // (each thread owns its run of entries)
+    if (write_out) {
+      counts[e] = t;
+      offsets[e] = run;
+    }
     run += t;
   }
-  if (threadIdx.x == 0) offsets[E] = (int32_t)P;
+  if (write_out && threadIdx.x == 0) offsets[E] = (int32_t)P;
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kPermThreads)
@@ -222,56 +240,21 @@ __global__ void __launch_bounds__(kPermThreads)
   if (threadIdx.x == 0) *arrive = 0;                 // ready for the next call
 }
 
-// Routing (a warp per token, as route_topk_kernel, 8 tokens per block) fused with the
-// permutation's histogram: chunk c holds the pairs of tokens [c tpc, (c + 1) tpc), and
-// each warp adds its token's k pairs to hist[c][e] and tot[e] with integer atomics;
-// the last block to finish scans tot.  hist, tot and the arrival counter after them
-// are zero on entry.
-__global__ void __launch_bounds__(256)
-    route_hist_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int tpc,
-                      int32_t* __restrict__ ids, float* __restrict__ wout,
-                      int32_t* __restrict__ hist, int32_t* __restrict__ tot,
-                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int* arrive) {
-  pdl_begin();
-  extern __shared__ float s_logits[];               // [8 warps][E] when E > 256
-  __shared__ int s_tot[1024], s_warp[33], s_last;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-  if (t < T) {
-    int my_id;
-    float my_w;
-    warp_route(logits, t, E, k, lane, s_logits + (E > 256 ? warp * E : 0), my_id, my_w);
-    if (lane < k) {
-      ids[t * k + lane] = my_id;
-      wout[t * k + lane] = my_w;
-      atomicAdd(&hist[(t / tpc) * E + my_id], 1);
-      atomicAdd(&tot[(int64_t)my_id * kTotStride], 1);
-    }
-  }
-  // the block's writes are ordered before its arrival by the barrier and one fence (a
-  // fence in every thread made each wait for its own atomics: most of the launch)
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(arrive, 1) == (int)gridDim.x - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  scan_totals(tot, E, T * k, counts, offsets, s_tot, s_warp);
-}
-
-__global__ void __launch_bounds__(kPermThreads)
-    permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int chunk_pairs,
-                           const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
-                           int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos) {
-  pdl_begin();
-  extern __shared__ int s_cnt[];   // [kPermWarps][E], then the chunk's base per expert [E]
+// Chunk c of the counting sort's scatter (a block of kPermThreads threads): its base per
+// expert from the offsets and the earlier chunks' counts, then the ranks of its pairs.
+// The offsets come from global memory, or from shared memory when s_off is given.
+// s_cnt holds (kPermWarps + 1) * E ints.
+__device__ void scatter_chunk(const int32_t* __restrict__ ids, int64_t P, int E, int chunk_pairs,
+                              int c, const int32_t* __restrict__ hist,
+                              const int32_t* __restrict__ offsets, const int* s_off,
+                              int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos,
+                              int* s_cnt) {
   int* s_base = s_cnt + kPermWarps * E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x;
+  __syncthreads();                    // the previous chunk's reads of s_cnt are done
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) s_cnt[i] = 0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_base[e] = offsets[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    s_base[e] = s_off != nullptr ? s_off[e] : __ldcg(offsets + e);
   __syncthreads();
   // the chunk's base: G threads per expert each add every G-th earlier chunk's count,
   // eight independent loads at a time
@@ -285,7 +268,7 @@ __global__ void __launch_bounds__(kPermThreads)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int cc = c0 + j * G;
-          v[j] = cc < c ? hist[(int64_t)cc * E + e] : 0;
+          v[j] = cc < c ? __ldcg(hist + (int64_t)cc * E + e) : 0;
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) sum += v[j];
@@ -296,7 +279,7 @@ __global__ void __launch_bounds__(kPermThreads)
   const int64_t p = (int64_t)c * chunk_pairs + threadIdx.x;
   const bool in = (int)threadIdx.x < chunk_pairs && p < P;
   int e = -1;
-  if (in) e = ids[p];
+  if (in) e = __ldcg(ids + p);       // (written by other CTAs of the same launch)
   const bool ok = in && e >= 0 && e < E;
   const int key = ok ? e : -1 - lane;  // invalid lanes never group
   const unsigned grp = __match_any_sync(0xffffffffu, key);
@@ -317,6 +300,78 @@ __global__ void __launch_bounds__(kPermThreads)
     sorted_pairs[pos] = (int32_t)p;
     pair_pos[p] = pos;
   }
+}
+
+__global__ void __launch_bounds__(kPermThreads)
+    permute_scatter_kernel(const int32_t* __restrict__ ids, int64_t P, int E, int chunk_pairs,
+                           const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets,
+                           int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos) {
+  pdl_begin();
+  extern __shared__ int s_cnt[];   // [kPermWarps][E], then the chunk's base per expert [E]
+  scatter_chunk(ids, P, E, chunk_pairs, blockIdx.x, hist, offsets, nullptr, sorted_pairs, pair_pos,
+                s_cnt);
+}
+
+// Routing and the whole counting sort in one cooperative launch (all CTAs resident):
+//   1. every warp routes tokens (warp_route) and adds its token's k pairs to the chunk
+//      histogram hist[c][e] and the expert totals with integer atomics;
+//   2. after a grid barrier, every CTA that has a chunk to scatter scans the totals into
+//      its own copy of the offsets (CTA 0 also writes counts and offsets), then scatters
+//      its chunks (scatter_chunk).
+// hist, tot and the barrier counter after them are zero on entry.  The barrier's wait is
+// bounded (MOE_ERR_TIMEOUT, then the CTA leaves).
+__device__ __forceinline__ bool grid_barrier(int* ctr, int target, int* err, int* s_fail) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1);
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1; *reinterpret_cast<volatile int*>(ctr) < target; ++i) {
+      if ((i & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+        report_error(err, MOE_ERR_TIMEOUT);
+        *s_fail = 1;
+        break;
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *s_fail == 0;
+}
+
+__global__ void __launch_bounds__(kPermThreads)
+    route_permute_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int tpc,
+                         int n_chunks, int32_t* __restrict__ ids, float* __restrict__ wout,
+                         int32_t* __restrict__ hist, int32_t* __restrict__ tot,
+                         int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ sorted_pairs, int32_t* __restrict__ pair_pos,
+                         int* bar, int* err) {
+  pdl_begin();
+  extern __shared__ int s_dyn[];    // routing: [kPermWarps][E] logits when E > 256;
+                                    // scatter: (kPermWarps + 1) * E ints
+  __shared__ int s_tot[1024], s_warp[33], s_fail;
+  if (threadIdx.x == 0) s_fail = 0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t P = T * k;
+  for (int64_t t = ((int64_t)blockIdx.x * kPermWarps) + warp; t < T;
+       t += (int64_t)gridDim.x * kPermWarps) {
+    int my_id;
+    float my_w;
+    warp_route(logits, t, E, k, lane, reinterpret_cast<float*>(s_dyn) + (E > 256 ? warp * E : 0),
+               my_id, my_w);
+    if (lane < k) {
+      ids[t * k + lane] = my_id;
+      wout[t * k + lane] = my_w;
+      atomicAdd(&hist[(t / tpc) * E + my_id], 1);
+      atomicAdd(&tot[(int64_t)my_id * kTotStride], 1);
+    }
+    __syncwarp();                   // the warp's logits row is reused by its next token
+  }
+  if (!grid_barrier(bar, (int)gridDim.x, err, &s_fail)) return;
+  if ((int)blockIdx.x >= n_chunks) return;
+  scan_totals(tot, E, P, counts, offsets, s_tot, s_warp, blockIdx.x == 0);
+  for (int c = blockIdx.x; c < n_chunks; c += gridDim.x)
+    scatter_chunk(ids, P, E, tpc * k, c, hist, offsets, s_tot, sorted_pairs, pair_pos, s_dyn);
 }
 
 static cudaError_t launch_scatter(const int32_t* ids, int64_t P, int E, int n_chunks, int chunk_pairs,
@@ -370,41 +425,50 @@ cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, i
                                  int32_t* pair_pos, int32_t* scratch, cudaStream_t s) {
   const int tpc = route_tokens_per_chunk(k);
   const int n_chunks = (int)((T + tpc - 1) / tpc);
-  const int64_t P = T * (int64_t)k;
   if (n_chunks == 0) {
     cudaError_t st = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s);
     if (st != cudaSuccess) return st;
     return cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s);
   }
-  // the histograms, the totals and the arrival counter after them start at zero
+  // the histograms, the totals and the barrier counter after them start at zero
   int32_t* hist = scratch;
   int32_t* tot = hist + (size_t)n_chunks * E;
-  int* arrive = tot + (size_t)E * kTotStride;
+  int* bar = tot + (size_t)E * kTotStride;
+  int* err = moe_status_word();
+  if (err == nullptr) return cudaErrorInvalidValue;
   cudaError_t st = cudaMemsetAsync(hist, 0, permute_scratch_ints(n_chunks, E) * sizeof(int32_t), s);
   if (st != cudaSuccess) return st;
-  {
-    const size_t smem = E > 256 ? (size_t)8 * E * sizeof(float) : 0;
-    ProfScope ps(K_ROUTE, s);
-    if (cudaError_t le_ = launch_pdl(route_hist_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), smem, s,
-                                     1, logits, T, E, k, tpc, ids, w, hist, tot, counts, offsets,
-                                     arrive);
-        le_ != cudaSuccess)
-      return le_;
-    st = cudaGetLastError();
+  const int lsm = E > 256 ? kPermWarps * E * (int)sizeof(float) : 0;
+  const int ssm = (kPermWarps + 1) * E * (int)sizeof(int);
+  const int smem = lsm > ssm ? lsm : ssm;
+  if (smem > 48 * 1024) {
+    st = cudaFuncSetAttribute(route_permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (st != cudaSuccess) return st;
   }
-  return launch_scatter(ids, P, E, n_chunks, tpc * k, hist, offsets, sorted_pairs, pair_pos, s);
-}
-
-static int g_num_sms_cache = 0;
-static int num_sms() {
-  if (g_num_sms_cache == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms_cache, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms_cache <= 0) g_num_sms_cache = 148;
-  }
-  return g_num_sms_cache;
+  // every CTA must be resident at once (the grid barriers): at most the occupancy bound
+  int per_sm = 0;
+  st = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_permute_kernel, kPermThreads, smem);
+  if (st != cudaSuccess) return st;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int64_t want_route = (T + kPermWarps - 1) / kPermWarps;
+  const int64_t want = want_route > n_chunks ? want_route : n_chunks;
+  const int64_t cap = (int64_t)per_sm * num_sms();
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPermThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfScope ps(K_ROUTE, s);
+  st = cudaLaunchKernelEx(&cfg, route_permute_kernel, logits, T, E, k, tpc, n_chunks, ids, w, hist, tot,
+                          counts, offsets, sorted_pairs, pair_pos, bar, err);
+  if (st != cudaSuccess) return st;
+  return cudaGetLastError();
 }
 
 static unsigned grid_for(int64_t work, int threads) {

@@ -65,10 +65,14 @@ def test_permute_bitexact(T, k, E, hot):
 
 
 @pytest.mark.parametrize("T,E,k", [(4096, 128, 8), (300, 64, 3), (64, 1024, 32), (1000, 16, 1),
-                                   (129, 33, 5), (1, 8, 2), (0, 8, 2)])
+                                   (129, 33, 5), (1, 8, 2), (0, 8, 2),
+                                   (40000, 128, 8), (20000, 512, 4)])
 def test_route_permute_fused_bitexact(T, E, k):
     # routing and the counting sort in one call: the same ids, weights and permutation
-    # as the oracle (and as moe_route_topk followed by moe_permute), ties included
+    # as the oracle (and as moe_route_topk followed by moe_permute), ties included.
+    # The two large cases need more chunks than resident CTAs (a CTA scatters several)
+    # and more tokens than routing warps (a warp routes several, E > 256 reusing its
+    # shared logits row).
     g = torch.Generator().manual_seed(T * 7 + E + k)
     logits = (torch.randn(T, E, generator=g) * 2).round() / 2
     if T > 0:
