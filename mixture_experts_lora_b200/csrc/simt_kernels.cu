@@ -170,8 +170,8 @@ static int num_sms() {
 //      summed over the warps orders the warps; positions are therefore stable
 //      (ascending pair index inside every segment).
 // moe_route_permute does routing and all of this in one cooperative launch
-// (route_permute_kernel below): its routing warps fill the histogram, grid barriers
-// separate the three phases.
+// (route_permute_kernel below): its routing warps fill the histogram, and one grid
+// barrier separates that from the scan and the scatter.
 // Replaces the per-expert mask lookup of the loop form ("What is
 // torch._grouped_mm?", Unsloth faster-moe docs).
 constexpr int kPermThreads = kPermuteChunk;
@@ -350,23 +350,44 @@ __global__ void __launch_bounds__(kPermThreads)
   extern __shared__ int s_dyn[];    // routing: [kPermWarps][E] logits when E > 256;
                                     // scatter: (kPermWarps + 1) * E ints
   __shared__ int s_tot[1024], s_warp[33], s_fail;
+  __shared__ int s_grp[2 * 1024];   // a group's pair counts in its (at most two) chunks
   if (threadIdx.x == 0) s_fail = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t P = T * k;
-  for (int64_t t = ((int64_t)blockIdx.x * kPermWarps) + warp; t < T;
-       t += (int64_t)gridDim.x * kPermWarps) {
-    int my_id;
-    float my_w;
-    warp_route(logits, t, E, k, lane, reinterpret_cast<float*>(s_dyn) + (E > 256 ? warp * E : 0),
-               my_id, my_w);
-    if (lane < k) {
-      ids[t * k + lane] = my_id;
-      wout[t * k + lane] = my_w;
-      atomicAdd(&hist[(t / tpc) * E + my_id], 1);
-      atomicAdd(&tot[(int64_t)my_id * kTotStride], 1);
+  // Groups of kPermWarps consecutive tokens, a warp per token.  A group spans at most two
+  // chunks (tpc >= kPermWarps): its counts are summed in shared memory first, so a hot
+  // expert costs one global atomic per group and chunk instead of one per pair, and the
+  // expert totals one per CTA.
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = 0;
+  const int64_t n_groups = (T + kPermWarps - 1) / kPermWarps;
+  for (int64_t g = blockIdx.x; g < n_groups; g += gridDim.x) {
+    for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) s_grp[i] = 0;
+    __syncthreads();
+    const int64_t t0 = g * kPermWarps, t = t0 + warp, c0 = t0 / tpc;
+    if (t < T) {
+      int my_id;
+      float my_w;
+      warp_route(logits, t, E, k, lane, reinterpret_cast<float*>(s_dyn) + (E > 256 ? warp * E : 0),
+                 my_id, my_w);
+      if (lane < k) {
+        ids[t * k + lane] = my_id;
+        wout[t * k + lane] = my_w;
+        atomicAdd(&s_grp[(int)(t / tpc - c0) * E + my_id], 1);
+      }
     }
-    __syncwarp();                   // the warp's logits row is reused by its next token
+    __syncthreads();
+    for (int i = threadIdx.x; i < 2 * E; i += blockDim.x) {
+      const int cnt = s_grp[i];
+      if (cnt != 0) {
+        const int half = i >= E ? 1 : 0, e = i - half * E;
+        atomicAdd(&hist[(c0 + half) * E + e], cnt);
+        atomicAdd(&s_tot[e], cnt);
+      }
+    }
+    __syncthreads();                // s_grp and the warps' logits rows are reused
   }
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (s_tot[e] != 0) atomicAdd(&tot[(int64_t)e * kTotStride], s_tot[e]);
   if (!grid_barrier(bar, (int)gridDim.x, err, &s_fail)) return;
   if ((int)blockIdx.x >= n_chunks) return;
   scan_totals(tot, E, P, counts, offsets, s_tot, s_warp, blockIdx.x == 0);
@@ -424,6 +445,7 @@ cudaError_t launch_route_permute(const float* logits, int64_t T, int E, int k, i
                                  float* w, int32_t* counts, int32_t* offsets, int32_t* sorted_pairs,
                                  int32_t* pair_pos, int32_t* scratch, cudaStream_t s) {
   const int tpc = route_tokens_per_chunk(k);
+  if (tpc < kPermWarps || E > 1024) return cudaErrorInvalidValue;   // (k <= 32 by the API)
   const int n_chunks = (int)((T + tpc - 1) / tpc);
   if (n_chunks == 0) {
     cudaError_t st = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s);

@@ -64,17 +64,23 @@ def test_permute_bitexact(T, k, E, hot):
     assert np.array_equal(pos.cpu().numpy(), rpos)
 
 
-@pytest.mark.parametrize("T,E,k", [(4096, 128, 8), (300, 64, 3), (64, 1024, 32), (1000, 16, 1),
-                                   (129, 33, 5), (1, 8, 2), (0, 8, 2),
-                                   (40000, 128, 8), (20000, 512, 4)])
-def test_route_permute_fused_bitexact(T, E, k):
+@pytest.mark.parametrize("T,E,k,hot", [(4096, 128, 8, False), (300, 64, 3, False),
+                                       (64, 1024, 32, False), (1000, 16, 1, False),
+                                       (129, 33, 5, False), (1, 8, 2, False), (0, 8, 2, False),
+                                       (40000, 128, 8, False), (20000, 512, 4, False),
+                                       (16384, 128, 8, True), (3001, 96, 3, True)])
+def test_route_permute_fused_bitexact(T, E, k, hot):
     # routing and the counting sort in one call: the same ids, weights and permutation
     # as the oracle (and as moe_route_topk followed by moe_permute), ties included.
     # The two large cases need more chunks than resident CTAs (a CTA scatters several)
     # and more tokens than routing warps (a warp routes several, E > 256 reusing its
-    # shared logits row).
+    # shared logits row).  The hot cases bias the logits towards the low experts, so
+    # nearly every token picks the same few (the counts of a token group pile up on
+    # one expert; tpc = 170 at k = 3 puts group boundaries inside chunks).
     g = torch.Generator().manual_seed(T * 7 + E + k)
     logits = (torch.randn(T, E, generator=g) * 2).round() / 2
+    if hot:
+        logits = logits + 8.0 / (1.0 + torch.arange(E, dtype=torch.float32))
     if T > 0:
         logits[0] = 0.0
     P = T * k
