@@ -477,7 +477,7 @@ def run_ours(args, cfg):
     P = cfg.T * cfg.k
     rb_bytes = P * cfg.m * 2 + cfg.T * cfg.m * 2 + cfg.T * cfg.E * 4 + P * 12
     extras["router_backward"] = {
-        "what": "dlogits [T, E] from dY and the expert outputs (NEXT-1 row; not part of the step)",
+        "what": "dlogits [T, E] from dY and the expert outputs (router backward; not part of the step)",
         "ms_per_launch": rb_ms, "algorithmic_bytes": rb_bytes,
         "achieved": rb_bytes / (rb_ms / 1e3) / 1e9, "unit": "GB/s"}
 
@@ -509,7 +509,7 @@ def run_ours(args, cfg):
         del gph
         return statistics.mean(a.elapsed_time(b) for a, b in xevs)
 
-    # the shared expert (dense MLP + LoRA on every token, NEXT-4): the layer with one
+    # the shared expert (dense MLP + LoRA on every token): the layer with one
     # expert at the same token count and dimensions
     from moe_inputs import LayerConfig
     scfg = LayerConfig("shared_expert", T=cfg.T, m=cfg.m, n=cfg.n, E=1, k=1, r=cfg.r, alpha=cfg.alpha)
@@ -520,7 +520,7 @@ def run_ours(args, cfg):
         raise SystemExit("device error in the shared-expert timing")
     se_flops = acc.flops_step(scfg.T, scfg.m, scfg.n, 1, scfg.r)
     extras["shared_expert"] = {
-        "what": f"dense SwiGLU MLP + LoRA on all {scfg.T} tokens, fwd+bwd (NEXT-4 row; not part of the step)",
+        "what": f"dense SwiGLU MLP + LoRA on all {scfg.T} tokens, fwd+bwd (shared expert; not part of the step)",
         "ms_per_step": se_ms, "tokens_per_s": scfg.T / (se_ms / 1e3),
         "tflops": se_flops / (se_ms / 1e3) / 1e12}
 
@@ -548,7 +548,7 @@ def run_ours(args, cfg):
         "tflops": (acc.flops_step(cfg.T, cfg.m, cfg.n, cfg.k, cfg.r) + se_flops) / (both_ms / 1e3) / 1e12}
     del sinp, sbuf
 
-    # separate gate/up adapters of rank r (NEXT-2): the same workload run as the fused
+    # separate gate/up adapters of rank r: the same workload run as the fused
     # rank-2r adapter (skipped when 2r > 128)
     if 2 * cfg.r <= 128:
         ad = ml.SplitGateUpAdapters(cfg.E, cfg.m, cfg.n, cfg.r, device=dev)
@@ -566,8 +566,7 @@ def run_ours(args, cfg):
         if ml.moe_get_device_error() != ml.MOE_OK:
             raise SystemExit("device error in the separate-adapter timing")
         extras["separate_gate_up_adapters"] = {
-            "what": f"the step with separate gate and up adapters of rank {cfg.r} (fused rank {2 * cfg.r}; "
-                    "NEXT-2 row)",
+            "what": f"the step with separate gate and up adapters of rank {cfg.r} (fused rank {2 * cfg.r})",
             "ms_per_step": sp_ms, "tokens_per_s": world * cfg.T / (sp_ms / 1e3)}
         del sp_buf, sp_inp, ad
 
@@ -615,7 +614,7 @@ def run_ours(args, cfg):
             "tflops": r64_flops / (r64_ms / 1e3) / 1e12}
         del b64, r64
 
-    # full fine-tuning (NEXT-3): forward, then the backward with the expert-weight
+    # full fine-tuning: forward, then the backward with the expert-weight
     # gradients dW_gu, dW_d and no adapter gradients
     dWg = torch.empty(cfg.E, cfg.m, 2 * cfg.n, dtype=torch.bfloat16, device=dev)
     dWd = torch.empty(cfg.E, cfg.n, cfg.m, dtype=torch.bfloat16, device=dev)
@@ -647,7 +646,7 @@ def run_ours(args, cfg):
                              **roof_entry(ft_work[name], tot / launches, 1, ft_peaks)}
     extras["full_fine_tuning"] = {
         "what": "forward + backward with the expert-weight gradients dW_gu, dW_d (no adapter "
-                "gradients; NEXT-3 row; not part of the step)",
+                "gradients; not part of the step)",
         "ms_per_step": ft_ms, "tokens_per_s": world * cfg.T / (ft_ms / 1e3),
         "tflops": ft_flops / (ft_ms / 1e3) / 1e12, "kernels": ft_kern}
     del dWg, dWd
